@@ -1,0 +1,257 @@
+/*
+ * ssd_oracle.c -- plain, slow fp64 CPU evaluation of the Mamba-2 SSD
+ * selective-state-space recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or helper with the CUDA path in state_space_sequence_scan_b200/
+ * and the CUDA path never calls it.
+ *
+ * What it computes (nnterp guide "Mamba-2", opening paragraph and the table
+ * in "The values"):
+ *   per head h, with state S an N x P matrix (state_dim rows, head_dim cols,
+ *   "key side first"), for every token t in order:
+ *     dt  = clamp(softplus(dt_raw[t,h] + dt_bias[h]), dt_lo, dt_hi)
+ *     a   = exp(dt * A[h])                       (A*dt is the log decay)
+ *     S   = a * S + dt * B[t,g] (outer) x[t,h]   (B is the key, x the value)
+ *     y[t,h] = S^T C[t,g] + D[h] * x[t,h]        (C reads the state)
+ *   where g = h / (H / G) is the group whose B and C head h uses ("one per
+ *   group of heads"), S starts from init_state (zeros when absent, as for a
+ *   fresh prompt) and final_state is S after the last token.
+ * The decode step (nnterp guide "Mamba-2", section "The state between
+ * steps") is the same loop body for one token with the state updated in
+ * place.
+ *
+ * Readings where the pages are silent: softplus in its exact stable form;
+ * the clamp is applied after the softplus; groups are contiguous blocks of
+ * heads; D is one scalar per head.
+ *
+ * Inputs are float32 arrays holding exactly the values given to the GPU
+ * (bf16 inputs widened to float32, which is exact); all arithmetic is double.
+ * Layouts (row-major, contiguous):
+ *   x [b,L,H,P]  dt_raw [b,L,H]  dt_bias [H]  A [H]  B,C [b,L,G,N]  D [H]
+ *   init_state [b,H,N,P] (may be NULL)   y [b,L,H,P]  final_state [b,H,N,P]
+ *
+ * Parity: pinned by tests/test_oracle.py (closed form, invariants, special
+ * cases, hand-computed golden example).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+static double sp_exact(double z)
+{
+    /* softplus(z) = log(1 + e^z), written so neither branch overflows */
+    return (z > 0.0 ? z : 0.0) + log1p(exp(-fabs(z)));
+}
+
+static double clamp_dt(double v, double lo, double hi)
+{
+    if (v < lo) v = lo;
+    if (v > hi) v = hi;
+    return v;
+}
+
+double ssd_oracle_softplus(double z) { return sp_exact(z); }
+
+typedef struct {
+    const float *x, *dt_raw, *dt_bias, *A, *B, *C, *D, *init_state;
+    double *y, *final_state;
+    int64_t b, L, H, P, N, G;
+    double dt_lo, dt_hi;
+    int64_t next;             /* next chain to claim */
+    pthread_mutex_t lock;
+    int status;
+} scan_job;
+
+static int64_t claim(scan_job *J)
+{
+    int64_t c;
+    pthread_mutex_lock(&J->lock);
+    c = J->next++;
+    pthread_mutex_unlock(&J->lock);
+    return c;
+}
+
+/* One (batch, head) chain of the recurrence, token by token. */
+static int run_chain(scan_job *J, int64_t bi, int64_t h, double *S, double *yacc)
+{
+    const int64_t L = J->L, H = J->H, P = J->P, N = J->N, G = J->G;
+    const int64_t g = h / (H / G);
+    const double A = J->A[h], Dh = J->D[h], bias = J->dt_bias[h];
+    int64_t n, p, t;
+
+    if (J->init_state) {
+        const float *s0 = J->init_state + (bi * H + h) * N * P;
+        for (n = 0; n < N * P; ++n) S[n] = (double)s0[n];
+    } else {
+        memset(S, 0, sizeof(double) * (size_t)(N * P));
+    }
+
+    for (t = 0; t < L; ++t) {
+        const double z = (double)J->dt_raw[(bi * L + t) * H + h] + bias;
+        const double dt = clamp_dt(sp_exact(z), J->dt_lo, J->dt_hi);
+        const double a = exp(dt * A);
+        const float *xr = J->x + ((bi * L + t) * H + h) * P;
+        const float *Br = J->B + ((bi * L + t) * G + g) * N;
+        const float *Cr = J->C + ((bi * L + t) * G + g) * N;
+        double *yr = J->y + ((bi * L + t) * H + h) * P;
+
+        /* S <- a S + dt B x^T */
+        for (n = 0; n < N; ++n) {
+            const double w = dt * (double)Br[n];
+            double *Sn = S + n * P;
+            for (p = 0; p < P; ++p) Sn[p] = a * Sn[p] + w * (double)xr[p];
+        }
+        /* y <- S^T C + D x */
+        for (p = 0; p < P; ++p) yacc[p] = 0.0;
+        for (n = 0; n < N; ++n) {
+            const double c = (double)Cr[n];
+            const double *Sn = S + n * P;
+            for (p = 0; p < P; ++p) yacc[p] += c * Sn[p];
+        }
+        for (p = 0; p < P; ++p) yr[p] = yacc[p] + Dh * (double)xr[p];
+    }
+
+    if (J->final_state) {
+        double *sf = J->final_state + (bi * H + h) * N * P;
+        memcpy(sf, S, sizeof(double) * (size_t)(N * P));
+    }
+    return 0;
+}
+
+static void *scan_worker(void *arg)
+{
+    scan_job *J = (scan_job *)arg;
+    double *S = (double *)malloc(sizeof(double) * (size_t)(J->N * J->P));
+    double *yacc = (double *)malloc(sizeof(double) * (size_t)J->P);
+    int64_t c;
+    if (!S || !yacc) {
+        J->status = -2;
+        free(S);
+        free(yacc);
+        return NULL;
+    }
+    while ((c = claim(J)) < J->b * J->H) run_chain(J, c / J->H, c % J->H, S, yacc);
+    free(S);
+    free(yacc);
+    return NULL;
+}
+
+static int pick_threads(int nthreads, int64_t chains)
+{
+    if (nthreads <= 0) {
+        long nc = sysconf(_SC_NPROCESSORS_ONLN);
+        nthreads = nc > 0 ? (int)nc : 1;
+    }
+    if (nthreads > chains) nthreads = (int)chains;
+    if (nthreads < 1) nthreads = 1;
+    return nthreads;
+}
+
+static int run_threads(void *(*fn)(void *), void *job, int nthreads)
+{
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    int i, started = 0;
+    if (!tid) {
+        fn(job);               /* run on the calling thread alone */
+        return 0;
+    }
+    for (i = 0; i < nthreads - 1; ++i)
+        if (pthread_create(&tid[started], NULL, fn, job) == 0) ++started;
+    fn(job);
+    for (i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+    free(tid);
+    return 0;
+}
+
+/* Whole-sequence recurrence.  Returns 0, or -1 on bad dimensions, -2 when out
+ * of memory.  nthreads <= 0 uses every online core. */
+int ssd_oracle_scan(const float *x, const float *dt_raw, const float *dt_bias,
+                    const float *A, const float *B, const float *C, const float *D,
+                    const float *init_state, double *y, double *final_state,
+                    int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                    double dt_lo, double dt_hi, int nthreads)
+{
+    scan_job J;
+    if (b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0) return -1;
+    if (b == 0) return 0;
+    memset(&J, 0, sizeof J);
+    J.x = x; J.dt_raw = dt_raw; J.dt_bias = dt_bias; J.A = A; J.B = B; J.C = C; J.D = D;
+    J.init_state = init_state; J.y = y; J.final_state = final_state;
+    J.b = b; J.L = L; J.H = H; J.P = P; J.N = N; J.G = G;
+    J.dt_lo = dt_lo; J.dt_hi = dt_hi;
+    pthread_mutex_init(&J.lock, NULL);
+    run_threads(scan_worker, &J, pick_threads(nthreads, b * H));
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
+}
+
+typedef struct {
+    const float *x, *dt_raw, *dt_bias, *A, *B, *C, *D;
+    double *state, *y;
+    int64_t b, H, P, N, G;
+    double dt_lo, dt_hi;
+    int64_t next;
+    pthread_mutex_t lock;
+} step_job;
+
+static void *step_worker(void *arg)
+{
+    step_job *J = (step_job *)arg;
+    const int64_t H = J->H, P = J->P, N = J->N, G = J->G;
+    int64_t c, n, p;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        c = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (c >= J->b * H) break;
+        {
+            const int64_t bi = c / H, h = c % H, g = h / (H / G);
+            const double z = (double)J->dt_raw[bi * H + h] + (double)J->dt_bias[h];
+            const double dt = clamp_dt(sp_exact(z), J->dt_lo, J->dt_hi);
+            const double a = exp(dt * (double)J->A[h]);
+            const float *xr = J->x + (bi * H + h) * P;
+            const float *Br = J->B + (bi * G + g) * N;
+            const float *Cr = J->C + (bi * G + g) * N;
+            double *S = J->state + (bi * H + h) * N * P;
+            double *yr = J->y + (bi * H + h) * P;
+            for (n = 0; n < N; ++n) {
+                const double w = dt * (double)Br[n];
+                for (p = 0; p < P; ++p) S[n * P + p] = a * S[n * P + p] + w * (double)xr[p];
+            }
+            for (p = 0; p < P; ++p) yr[p] = 0.0;
+            for (n = 0; n < N; ++n) {
+                const double cn = (double)Cr[n];
+                for (p = 0; p < P; ++p) yr[p] += cn * S[n * P + p];
+            }
+            for (p = 0; p < P; ++p) yr[p] += (double)J->D[h] * (double)xr[p];
+        }
+    }
+    return NULL;
+}
+
+/* One decode token: state [b,H,N,P] (double) updated in place, y [b,H,P].
+ * x [b,H,P], dt_raw [b,H], B,C [b,G,N]. */
+int ssd_oracle_step(const float *x, const float *dt_raw, const float *dt_bias,
+                    const float *A, const float *B, const float *C, const float *D,
+                    double *state, double *y,
+                    int64_t b, int64_t H, int64_t P, int64_t N, int64_t G,
+                    double dt_lo, double dt_hi, int nthreads)
+{
+    step_job J;
+    if (b < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0) return -1;
+    if (b == 0) return 0;
+    memset(&J, 0, sizeof J);
+    J.x = x; J.dt_raw = dt_raw; J.dt_bias = dt_bias; J.A = A; J.B = B; J.C = C; J.D = D;
+    J.state = state; J.y = y;
+    J.b = b; J.H = H; J.P = P; J.N = N; J.G = G;
+    J.dt_lo = dt_lo; J.dt_hi = dt_hi;
+    pthread_mutex_init(&J.lock, NULL);
+    run_threads(step_worker, &J, pick_threads(nthreads, b * H));
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}

@@ -1,0 +1,85 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a private copy of the oracle's C source (a
+dropped term, a wrong sign or index, swapped operands), compiles it on the
+CPU, and checks that the closed-form pin rejects it.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+from test_oracle import _closed_form, _rand_case, _rel
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "ssd_oracle.c")
+
+MUTANTS = {
+    "drop_D_skip": ("yr[p] = yacc[p] + Dh * (double)xr[p];", "yr[p] = yacc[p];"),
+    "decay_sign": ("const double a = exp(dt * A);", "const double a = exp(-dt * A);"),
+    "no_dt_on_write": ("const double w = dt * (double)Br[n];\n            double *Sn",
+                       "const double w = (double)Br[n];\n            double *Sn"),
+    "group_index": ("const int64_t g = h / (H / G);", "const int64_t g = h % G;"),
+    "B_C_swapped": ("const float *Br = J->B + ((bi * L + t) * G + g) * N;\n        const float *Cr = J->C",
+                    "const float *Br = J->C + ((bi * L + t) * G + g) * N;\n        const float *Cr = J->B"),
+    "no_bias": ("const double z = (double)J->dt_raw[(bi * L + t) * H + h] + bias;",
+                "const double z = (double)J->dt_raw[(bi * L + t) * H + h];"),
+    "decay_on_new_write": ("Sn[p] = a * Sn[p] + w * (double)xr[p];", "Sn[p] = a * (Sn[p] + w * (double)xr[p]);"),
+    "state_transposed_read": ("const double *Sn = S + n * P;\n            for (p = 0; p < P; ++p) yacc[p] += c * Sn[p];",
+                              "for (p = 0; p < P; ++p) yacc[p] += c * S[(p % N) * P + (n % P)];"),
+    "no_init_state": ("for (n = 0; n < N * P; ++n) S[n] = (double)s0[n];",
+                      "for (n = 0; n < N * P; ++n) S[n] = 0.0 * s0[n];"),
+}
+
+
+def _build(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert old in src, name
+    src = src.replace(old, new)
+    c = tmp_path / (name + ".c")
+    c.write_text(src)
+    so = tmp_path / (name + ".so")
+    subprocess.check_call(["gcc", "-O1", "-fPIC", "-shared", "-std=c99", "-D_POSIX_C_SOURCE=200809L",
+                           "-o", str(so), str(c), "-lm", "-lpthread"])
+    return str(so)
+
+
+def _scan_with(lib_path, case):
+    lib = ctypes.CDLL(lib_path)
+    f32p = ctypes.POINTER(ctypes.c_float)
+    f64p = ctypes.POINTER(ctypes.c_double)
+    lib.ssd_oracle_scan.restype = ctypes.c_int
+    lib.ssd_oracle_scan.argtypes = [f32p] * 8 + [f64p, f64p] + [ctypes.c_int64] * 6 + [
+        ctypes.c_double, ctypes.c_double, ctypes.c_int]
+    arr = {k: (np.ascontiguousarray(v, np.float32) if v is not None else None) for k, v in case.items()}
+    b, L, H, P = arr["x"].shape
+    G, N = arr["B"].shape[2:]
+    y = np.empty((b, L, H, P))
+    fs = np.empty((b, H, N, P))
+    p = lambda a: a.ctypes.data_as(f32p)
+    rc = lib.ssd_oracle_scan(p(arr["x"]), p(arr["dt_raw"]), p(arr["dt_bias"]), p(arr["A"]), p(arr["B"]),
+                             p(arr["C"]), p(arr["D"]),
+                             p(arr["init_state"]) if arr["init_state"] is not None else f32p(),
+                             y.ctypes.data_as(f64p), fs.ctypes.data_as(f64p), b, L, H, P, N, G,
+                             0.0, float("inf"), 1)
+    assert rc == 0
+    return y, fs
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_planted_mistake(tmp_path, name):
+    old, new = MUTANTS[name]
+    so = _build(tmp_path, name, old, new)
+    case = _rand_case(21, b=1, L=9, H=4, P=3, N=5, G=2, init=True)
+    y, fs = _scan_with(so, case)
+    y_ref, fs_ref = _closed_form(case)
+    assert max(_rel(y, y_ref), _rel(fs, fs_ref)) > 1e-6, "planted mistake went unnoticed"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    so = _build(tmp_path, "clean", "/* S <- a S + dt B x^T */", "/* S <- a S + dt B x^T */")
+    case = _rand_case(21, b=1, L=9, H=4, P=3, N=5, G=2, init=True)
+    y, fs = _scan_with(so, case)
+    y_ref, fs_ref = _closed_form(case)
+    assert max(_rel(y, y_ref), _rel(fs, fs_ref)) < 1e-12
