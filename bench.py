@@ -1,0 +1,561 @@
+#!/usr/bin/env python
+"""Throughput of the B200 SSD scan (and decode step) on synthetic workloads.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A "step" is one chunked forward scan (every stage of the hot path: dt
+preparation, chunk cumsum, intra-chunk C.B^T, chunk states, state passing,
+chunk output) over one batch of the workload; the decode workload's step is
+one single-token state update.  Rank 0 prints ONE JSON line.  With N > 1 each
+rank runs its own copy of the workload (independent batches, no collective on
+the data path: weak scaling); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from state_space_sequence_scan_b200.inputs import (  # noqa: E402
+    SCAN_CONFIGS, STEP_CONFIGS, make_scan_inputs, make_step_inputs)
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "SSD chunked-scan Mtokens/s & % roofline; decode state-update HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------
+# algorithmic work (bytes every implementation must move, flops of the causal
+# chunked form with C.B^T counted once per group)
+
+def scan_bytes(cfg) -> float:
+    b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
+    e = 4 if cfg.dtype == "f32" else 2
+    tok = b * L
+    byt = tok * H * P * e + 2 * tok * G * N * e + tok * H * 4   # x, B, C, dt_raw
+    byt += tok * H * P * 4                                      # y (fp32)
+    byt += b * H * N * P * 4 * (2 if cfg.init == "normal" else 1)  # init (if any) + final state
+    byt += 3 * H * 4
+    return float(byt)
+
+
+def scan_flops(cfg) -> float:
+    b, L, H, P, N, G, Q = (cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups,
+                           cfg.chunk_size)
+    nc = math.ceil(L / Q)
+    per_chunk = G * Q * (Q + 1) * N + H * (Q * (Q + 1) * P + 4 * Q * N * P)
+    return float(b * nc * per_chunk)
+
+
+def step_bytes(cfg) -> float:
+    b, H, P, N, G = cfg.batch, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
+    e = 4 if cfg.dtype == "f32" else 2
+    return float(2 * b * H * N * P * 4 + b * H * P * e + 2 * b * G * N * e + b * H * 4 + b * H * P * 4 + 3 * H * 4)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------
+
+def init_dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _dev_sets(inp, nsets, device):
+    """nsets device copies of the inputs (rotated so timed steps never hit L2)."""
+    sets = []
+    for _ in range(nsets):
+        sets.append({k: (v.to(device) if v is not None else None) for k, v in inp.items()})
+    return sets
+
+
+def bench_scan(cfg, args, ws, rank, local):
+    from state_space_sequence_scan_b200 import ssd
+    dev = torch.device("cuda", local)
+    inp = make_scan_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    one = scan_bytes(cfg)
+    nsets = max(1, min(8, math.ceil(3 * L2_BYTES / one)))
+    sets = _dev_sets(inp, nsets, dev)
+    b, L, H, P, N, G, Q = (cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups,
+                           cfg.chunk_size)
+    outs = [(torch.empty(b, L, H, P, device=dev), torch.empty(b, H, N, P, device=dev)) for _ in range(nsets)]
+    wsz = ssd.workspace_size(b, L, H, P, N, G, Q, sets[0]["x"].dtype, args.path)
+    work = ssd.alloc_workspace(wsz, dev)
+
+    def step(k):
+        s = sets[k % nsets]
+        y, fs = outs[k % nsets]
+        ssd.chunk_scan_fwd(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"],
+                           init_state=s["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
+                           final_state=fs)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    if ssd.read_device_status(work) != 0:
+        raise RuntimeError("device status %d after warm-up" % ssd.read_device_status(work))
+
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for k in range(args.steps):
+        step(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, ws)
+
+    # per-kernel device times: the same K steps again with event brackets
+    ssd.trace_enable(min(8192, 8 * args.steps + 8))
+    for k in range(args.steps):
+        step(k)
+    torch.cuda.synchronize()
+    trace = ssd.trace_read()
+    ssd.trace_enable(0)
+    launches_per_step = sum(n for n, _ in trace.values()) / max(args.steps, 1)
+
+    res = dict(ms=ms_max, tokens=cfg.tokens, bytes=one, flops=scan_flops(cfg), clocks=clk, trace=trace,
+               launches=int(round(launches_per_step * args.steps)), nsets=nsets)
+    res["e2e"] = e2e_scan(inp, cfg, args, dev, work)
+    return res
+
+
+def e2e_scan(inp, cfg, args, dev, work):
+    """Same metric through the public call with host buffers: pinned host
+    inputs copied in, the scan, y and final_state copied back, every step."""
+    from state_space_sequence_scan_b200 import ssd
+    host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+    d = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in inp.items()}
+    b, L, H, P, N, Q = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.chunk_size
+    y = torch.empty(b, L, H, P, device=dev)
+    fs = torch.empty(b, H, N, P, device=dev)
+    y_h = torch.empty(b, L, H, P).pin_memory()
+    fs_h = torch.empty(b, H, N, P).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = y_h.numel() * 4 + fs_h.numel() * 4
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        for k, v in host.items():
+            if v is not None:
+                d[k].copy_(v, non_blocking=True)
+        ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                           init_state=d["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
+                           final_state=fs)
+        y_h.copy_(y, non_blocking=True)
+        fs_h.copy_(fs, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return dict(ms_per_step=ms, h2d=h2d, d2h=d2h, steps=steps)
+
+
+def bench_step(cfg, args, ws, rank, local):
+    from state_space_sequence_scan_b200 import ssd
+    dev = torch.device("cuda", local)
+    ntok = 32
+    inp = make_step_inputs(cfg, steps=ntok, seed=cfg.seed + 1000 * rank)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    state = d["state"].clone()
+    b, H, P = cfg.batch, cfg.nheads, cfg.head_dim
+    y = torch.empty(b, H, P, device=dev)
+
+    def step(k):
+        t = k % ntok
+        ssd.step(d["x"][t], d["dt_raw"][t], d["dt_bias"], d["A"], d["B"][t], d["C"][t], d["D"], state, y=y)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for k in range(args.steps):
+        step(k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    ms_max = max_over_ranks(e0.elapsed_time(e1), ws)
+    ssd.trace_enable(min(8192, args.steps + 8))
+    for k in range(args.steps):
+        step(k)
+    torch.cuda.synchronize()
+    trace = ssd.trace_read()
+    ssd.trace_enable(0)
+
+    # e2e: pinned host token inputs in, y out, state resident (it is the cache)
+    host = {k: inp[k][0].contiguous().pin_memory() for k in ("x", "dt_raw", "B", "C")}
+    dd = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    y_h = torch.empty(b, H, P).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y_h.numel() * 4
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n2 = max(3, min(args.steps, 50))
+    f0.record()
+    for _ in range(n2):
+        for k, v in host.items():
+            dd[k].copy_(v, non_blocking=True)
+        ssd.step(dd["x"], dd["dt_raw"], d["dt_bias"], d["A"], dd["B"], dd["C"], d["D"], state, y=y)
+        y_h.copy_(y, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    e2e = dict(ms_per_step=f0.elapsed_time(f1) / n2, h2d=h2d, d2h=d2h, steps=n2)
+    return dict(ms=ms_max, bytes=step_bytes(cfg), clocks=clk, trace=trace,
+                launches=sum(n for n, _ in trace.values()), e2e=e2e)
+
+
+def dominant(trace):
+    if not trace:
+        return None, 0, 0.0
+    name = max(trace, key=lambda k: trace[k][1])
+    n, ms = trace[name]
+    return name, n, ms
+
+
+# algorithmic bytes each traced kernel must move (per launch), as fractions of the call
+def kernel_bytes(cfg, name) -> float:
+    b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
+    e = 4 if cfg.dtype == "f32" else 2
+    tok = b * L
+    x, bc, dt, y = tok * H * P * e, tok * G * N * e, tok * H * 4, tok * H * P * 4
+    st = b * H * N * P * 4
+    if name.endswith("chunk_out"):
+        return float(x + 2 * bc + y)
+    if name.endswith("chunk_state") or name.endswith("unit_state"):
+        return float(x + bc + dt)
+    if name.endswith("state_pass"):
+        return float(st * (2 if cfg.init == "normal" else 1))
+    return scan_bytes(cfg)
+
+
+def cpu_baseline_scan(cfg, budget_s=12.0):
+    """The oracle as it stands, on this host's cores, on a bounded sample:
+    whole sequences of a subset of (batch, head) chains, repeated until the
+    budget is used.  Returned in the metric's unit (tokens of all heads)."""
+    import numpy as np
+    import oracle
+    inp = make_scan_inputs(cfg)
+    cores = os.cpu_count() or 1
+    H = cfg.nheads
+    G = cfg.ngroups
+    # a sample of heads of batch 0 (each chain is independent)
+    nh = min(H, max(1, cores))
+    heads = list(range(nh))
+    sub = dict(x=inp["x"][:1, :, :nh], dt_raw=inp["dt_raw"][:1, :, :nh], dt_bias=inp["dt_bias"][:nh],
+               A=inp["A"][:nh], D=inp["D"][:nh])
+    gsel = [h // (H // G) for h in heads]
+    sub["B"] = inp["B"][:1, :, gsel]
+    sub["C"] = inp["C"][:1, :, gsel]
+    sub["init_state"] = None if inp["init_state"] is None else inp["init_state"][:1, :nh]
+    # G' = nh: every sampled head reads its own group's B, C
+    t0 = time.time()
+    reps = 0
+    while True:
+        oracle.scan(sub["x"], sub["dt_raw"], sub["dt_bias"], sub["A"], sub["B"], sub["C"], sub["D"],
+                    init_state=sub["init_state"], nthreads=cores)
+        reps += 1
+        if time.time() - t0 >= budget_s or reps >= 200:
+            break
+    el = time.time() - t0
+    token_heads = reps * cfg.seqlen * nh
+    mtok = token_heads / H / el / 1e6
+    return dict(value=mtok, unit="Mtokens/s", cores=cores, kind="oracle",
+                sample="%d of %d heads of batch 0, full seqlen %d, x%d repeats (%.1f s); tokens counted as "
+                       "token-heads / heads" % (nh, H, cfg.seqlen, reps, el), seconds=el)
+
+
+def cpu_baseline_step(cfg, budget_s=12.0):
+    import numpy as np
+    import oracle
+    cores = os.cpu_count() or 1
+    rows = max(1, min(cfg.batch, 16))
+    c2 = cfg.with_(batch=rows)
+    inp = make_step_inputs(c2, steps=8)
+    st = inp["state"].double().numpy().copy()
+    t0 = time.time()
+    n = 0
+    while True:
+        t = n % 8
+        oracle.step(inp["x"][t], inp["dt_raw"][t], inp["dt_bias"], inp["A"], inp["B"][t], inp["C"][t], inp["D"],
+                    st, nthreads=cores)
+        n += 1
+        if time.time() - t0 >= budget_s or n >= 2000:
+            break
+    el = time.time() - t0
+    gbs = step_bytes(c2) * n / el / 1e9
+    return dict(value=gbs, unit="GB/s", cores=cores, kind="oracle",
+                sample="%d of %d batch rows, %d steps (%.1f s); algorithmic state bytes per step" %
+                       (rows, cfg.batch, n, el), seconds=el)
+
+
+def run_reference(args, ws, rank):
+    """--impl reference: the fp64 CPU oracle (this method has no other
+    reference implementation) timed on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    cfg, is_step = pick(args.workload)
+    steps, warm = args.steps, args.warmup
+    budget = max(2.0, min(60.0, 6.0 * steps / max(steps + warm, 1)))
+    if is_step:
+        cb = cpu_baseline_step(cfg, budget_s=budget)
+        value, unit, hib = cb["value"], "GB/s", True
+        ms = step_bytes(cfg) / (cb["value"] * 1e9) * 1e3
+        dtype = "f64"
+    else:
+        cb = cpu_baseline_scan(cfg, budget_s=budget)
+        value, unit, hib = cb["value"], "Mtokens/s", True
+        ms = cfg.tokens / (cb["value"] * 1e6) * 1e3
+        dtype = "f64"
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": steps, "warmup": warm,
+            "ms_per_step": ms, "higher_is_better": hib, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+            "data": "synthetic", "impl": "reference", "config": workload_config(cfg, is_step),
+            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def pick(name):
+    if name in SCAN_CONFIGS:
+        return SCAN_CONFIGS[name], False
+    if name in STEP_CONFIGS:
+        return STEP_CONFIGS[name], True
+    raise SystemExit("unknown workload %s (scan: %s; decode: %s)" % (name, list(SCAN_CONFIGS), list(STEP_CONFIGS)))
+
+
+def workload_config(cfg, is_step, nsets=None):
+    if is_step:
+        c = {"workload": cfg.name, "batch": cfg.batch, "heads": cfg.nheads, "head_dim": cfg.head_dim,
+             "state_dim": cfg.state_dim, "groups": cfg.ngroups, "state_dtype": "f32", "in_dtype": cfg.dtype,
+             "l2": "state %.0f MB > L2, streamed every step" % (cfg.batch * cfg.nheads * cfg.state_dim *
+                                                              cfg.head_dim * 4 / 1e6)}
+    else:
+        c = {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen, "heads": cfg.nheads,
+             "head_dim": cfg.head_dim, "state_dim": cfg.state_dim, "groups": cfg.ngroups,
+             "chunk_size": cfg.chunk_size, "in_dtype": cfg.dtype, "y_dtype": "f32",
+             "init_state": cfg.init != "zero"}
+        if nsets is not None:
+            c["l2"] = ("rotating %d input/output sets (%.0f MB > 2x L2)" % (nsets, nsets * scan_bytes(cfg) / 1e6)
+                       if nsets > 1 else "inputs %.0f MB > L2" % (scan_bytes(cfg) / 1e6))
+    return c
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c1_130m")
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode figure on the scan line")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    ws, rank, local = init_dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+            return
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+        from state_space_sequence_scan_b200 import ssd
+        ssd.load_library()
+        peaks, peak_kind = load_peaks()
+        cfg, is_step = pick(args.workload)
+        if is_step:
+            r = bench_step(cfg, args, ws, rank, local)
+        else:
+            r = bench_scan(cfg, args, ws, rank, local)
+        out = finish(cfg, is_step, r, args, ws, rank, peaks, peak_kind)
+        if not is_step and not args.no_decode:
+            dcfg = STEP_CONFIGS["c4_decode"]
+            dr = bench_step(dcfg, args, ws, rank, local)
+            dline = finish(dcfg, True, dr, args, ws, rank, peaks, peak_kind, sub=True)
+            if out is not None:
+                out["decode"] = dline
+        if rank == 0 and out is not None:
+            if ws == 1 and not args.no_cpu_baseline:
+                cb = cpu_baseline_step(cfg) if is_step else cpu_baseline_scan(cfg)
+                out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            print(json.dumps(out), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def finish(cfg, is_step, r, args, ws, rank, peaks, peak_kind, sub=False):
+    ms_step = r["ms"] / args.steps
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    name, n, kms = dominant(r["trace"])
+    avg = kms / max(n, 1)
+    if is_step:
+        value = ws * r["bytes"] / (ms_step * 1e-3) / 1e9
+        unit = "GB/s"
+        kb = r["bytes"]
+        dtype = "f32"
+        e2e_val = ws * r["bytes"] / (r["e2e"]["ms_per_step"] * 1e-3) / 1e9
+    else:
+        value = ws * r["tokens"] / (ms_step * 1e-3) / 1e6
+        unit = "Mtokens/s"
+        kb = kernel_bytes(cfg, name) if name else r["bytes"]
+        dtype = "f32" if cfg.dtype == "f32" else "bf16-in/f32"
+        e2e_val = ws * r["tokens"] / (r["e2e"]["ms_per_step"] * 1e-3) / 1e6
+    achieved = kb / (avg * 1e-3) / 1e9 if avg > 0 else None
+    roof = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": (achieved / hbm) if achieved else None, "traffic": None,
+            "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+            else "fallback 6.65 TB/s",
+            "kernel_ms_avg": avg, "kernel_bytes": kb,
+            "shares": {k: round(v[1] / max(sum(x[1] for x in r["trace"].values()), 1e-12), 4)
+                       for k, v in r["trace"].items()}}
+    if not is_step:
+        t_mem = r["bytes"] / (hbm * 1e9)
+        t_flop = r["flops"] / (float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) * 1e12)
+        t_roof = max(t_mem, t_flop)
+        roof["path"] = {"roofline_ms": t_roof * 1e3, "ms_per_step": ms_step,
+                        "frac": t_roof * 1e3 / ms_step, "bound": "hbm" if t_mem >= t_flop else "tensor",
+                        "algorithmic_bytes": r["bytes"], "algorithmic_flops": r["flops"]}
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded; shapes/distributions of the workload)",
+            "config": workload_config(cfg, is_step, r.get("nsets")), "roofline": roof, "clocks": r["clocks"],
+            "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": r["e2e"]["h2d"],
+                    "d2h_bytes_per_step": r["e2e"]["d2h"]},
+            "gpu_launches": r["launches"]}
+    if sub:
+        for k in ("metric", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "vs_baseline", "data"):
+            line.pop(k, None)
+    return line if rank == 0 else None
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,160 @@
+/*
+ * ssd.h -- C ABI of libssd.so, the B200 (sm_100a) Mamba-2 SSD scan.
+ *
+ * The operation (nnterp guide "Mamba-2", opening paragraph and the table in
+ * "The values"): per head h, with state S an N x P matrix stored state_dim
+ * first ("key side first"), for every token t
+ *     dt  = clamp(softplus(dt_raw[t,h] + dt_bias[h]), dt_lo, dt_hi)
+ *     S   = exp(dt * A[h]) * S + dt * B[t,g] (outer) x[t,h]
+ *     y   = S^T C[t,g] + D[h] * x[t,h]
+ * where head h reads the B and C of group g = h / (H / G) (B and C are "one
+ * per group of heads").  A * dt is the log decay and must be <= 0.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers unless stated; the caller allocates and
+ *     owns every buffer, workspace included.  The library never allocates,
+ *     frees or synchronises on the compute calls; work is enqueued on
+ *     `stream` (a cudaStream_t; NULL is the legacy default stream) and the
+ *     call returns before it finishes.
+ *   - Layouts are contiguous, row-major, with these shapes:
+ *       x            [batch, seqlen, nheads, head_dim]     in_dtype
+ *       dt_raw       [batch, seqlen, nheads]               float32
+ *       dt_bias, A, D [nheads]                             float32
+ *       B, C         [batch, seqlen, ngroups, state_dim]   in_dtype
+ *       init_state, final_state, state
+ *                    [batch, nheads, state_dim, head_dim]  float32
+ *       y            [batch, seqlen, nheads, head_dim]     float32
+ *     (the decode step drops the seqlen axis).
+ *   - x, B, C, y and every state pointer must be 16-byte aligned.
+ *   - Errors come back as an ssd_status; nothing is thrown across the ABI.
+ *     Argument errors are detected on the host before anything is enqueued.
+ *     Conditions only the GPU can see (a positive A in the chunked scan) are
+ *     recorded in a status word at the start of the workspace and read back
+ *     with ssd_read_device_status().
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ssd_status {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,    /* null pointer, size <= 0, H % G != 0, bad dt limits */
+    SSD_ERR_UNSUPPORTED = 2,    /* dtype, path or size outside what is implemented */
+    SSD_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
+    SSD_ERR_WORKSPACE = 4,      /* workspace null or smaller than ssd_chunk_scan_workspace_size() */
+    SSD_ERR_CUDA = 5,           /* a CUDA call failed; see ssd_last_cuda_error() */
+    SSD_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait gave up */
+    SSD_ERR_PRECONDITION = 7    /* the GPU saw A > 0 (the log decay must be non-positive), or on the
+                                   tensor path an operand outside the fp16 range (|v| > 65504) */
+} ssd_status;
+
+typedef enum ssd_dtype {
+    SSD_F32 = 0,   /* float32 x, B, C */
+    SSD_BF16 = 1   /* bfloat16 x, B, C */
+} ssd_dtype;
+
+typedef enum ssd_path {
+    SSD_PATH_AUTO = 0,    /* tensor-core path when the shape allows it, else SIMT */
+    SSD_PATH_SIMT = 1,    /* fp32 CUDA-core kernels: any chunk size, fp32 or bf16 inputs */
+    SSD_PATH_TENSOR = 2   /* tcgen05 kernels: bf16 inputs, state_dim 128, head_dim 64,
+                             chunk size 64, 128 or 256; fp16 operands, fp32 accumulate */
+} ssd_path;
+
+/* Bytes of device workspace ssd_chunk_scan_fwd needs for these sizes and
+ * this path (SSD_PATH_AUTO resolves as the forward call would).  Host only;
+ * enqueues nothing.  Returns SSD_ERR_INVALID_ARG / SSD_ERR_UNSUPPORTED for
+ * sizes the forward call would reject. */
+SSD_API ssd_status ssd_chunk_scan_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads,
+                                         int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                                         int64_t chunk_size, int in_dtype, int path,
+                                         size_t *bytes);
+
+/* Chunked forward scan over whole sequences (the prompt path: nnterp guide
+ * "Mamba-2", sections "The values" and "The state after every token";
+ * chunked two-stage evaluation as on the "Mamba2" knowledge page).
+ *
+ * Evaluates the recurrence above for every (batch, head) from init_state
+ * (NULL means zeros, a fresh prompt) and writes y for every token and
+ * final_state, the state after the last token (final_state may be NULL when
+ * not wanted).  The work is split into chunks of chunk_size tokens: within a
+ * chunk a masked, decay-weighted C.B^T contraction; between chunks a serial
+ * pass of the chunk states.  The result equals the token-by-token recurrence
+ * up to rounding, whatever the chunk size.
+ *   dt_lo, dt_hi  the time-step limit applied after the softplus
+ *                 (0 and +INFINITY for no limit); 0 <= dt_lo <= dt_hi.
+ *   in_dtype      ssd_dtype of x, B and C.
+ *   path          ssd_path.
+ *   workspace     device scratch of at least ssd_chunk_scan_workspace_size()
+ *                 bytes, 256-byte aligned; its first 256 bytes hold the
+ *                 device status word.  It is overwritten by every call, so
+ *                 two calls in flight at once need two workspaces.
+ * Inputs are never modified.  y, final_state and the workspace must not
+ * overlap the inputs. */
+SSD_API ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const float *dt_bias,
+                              const float *A, const void *B, const void *C, const float *D,
+                              const float *init_state, float *y, float *final_state,
+                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                              int64_t state_dim, int64_t ngroups, int64_t chunk_size,
+                              float dt_lo, float dt_hi, int in_dtype, int path,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* One decode token (nnterp guide "Mamba-2", section "The state between
+ * steps": the update writes the new state into the cache and returns only y;
+ * there is no sequence axis).
+ *   x [batch, nheads, head_dim], dt_raw [batch, nheads],
+ *   B, C [batch, ngroups, state_dim], state [batch, nheads, state_dim, head_dim]
+ *   float32, updated IN PLACE; y [batch, nheads, head_dim] float32 out.
+ *   dt_lo, dt_hi  as for the scan; pass 0 and +INFINITY for the pages'
+ *                 decode semantics (no clamp).
+ * head_dim must be a multiple of 4 with head_dim / 4 dividing 256.  A > 0 is
+ * evaluated as written (nothing in the step depends on its sign). */
+SSD_API ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
+                    const void *B, const void *C, const float *D, float *state, float *y,
+                    int64_t batch, int64_t nheads, int64_t head_dim, int64_t state_dim,
+                    int64_t ngroups, float dt_lo, float dt_hi, int in_dtype, void *stream);
+
+/* Waits for `stream`, then reads the device status word that the last
+ * ssd_chunk_scan_fwd on this workspace left: SSD_OK, SSD_ERR_PRECONDITION or
+ * SSD_ERR_DEVICE_TIMEOUT.  `workspace` is a device pointer. */
+SSD_API ssd_status ssd_read_device_status(const void *workspace, void *stream);
+
+/* Text for a status code (static storage; never NULL). */
+SSD_API const char *ssd_status_string(int status);
+
+/* The cudaError_t behind the last SSD_ERR_CUDA returned on this host thread. */
+SSD_API int ssd_last_cuda_error(void);
+
+/* Kernel tracing, off by default.  ssd_trace_enable(n) creates 2n CUDA
+ * events once (n <= 8192), clears earlier records and from then on brackets
+ * each kernel the library launches with an event pair recorded on the
+ * launching stream, for the first n launches; ssd_trace_enable(0) stops
+ * recording (records are kept).  ssd_trace_read() waits for the recorded
+ * events of kernel id `kernel` (0 <= kernel < ssd_trace_kernel_count()) and
+ * returns how many launches were recorded and their summed device time in
+ * milliseconds.  ssd_trace_kernel_name() names a kernel id.  Not
+ * thread-safe against concurrent compute calls from other host threads. */
+SSD_API ssd_status ssd_trace_enable(int max_launches);
+SSD_API ssd_status ssd_trace_read(int kernel, int *launches, double *total_ms);
+SSD_API const char *ssd_trace_kernel_name(int kernel);
+SSD_API int ssd_trace_kernel_count(void);
+
+/* ABI version: (major << 16) | minor. */
+SSD_API int ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

@@ -1,0 +1,192 @@
+// C ABI of libssd.so: argument checks, path selection, workspace carve-up and
+// launches.  Declared in include/ssd.h, which documents every argument.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/ssd.h"
+#include "ssd_common.cuh"
+#include "ssd_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+ssd_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return SSD_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dtype_ok(int t) { return t == SSD_F32 || t == SSD_BF16; }
+
+bool limits_ok(float lo, float hi) {
+    return !isnan(lo) && !isnan(hi) && lo >= 0.0f && hi >= lo;
+}
+
+ssd_status check_scan_dims(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                           int64_t Q, int in_dtype, int path) {
+    if (b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || Q <= 0) return SSD_ERR_INVALID_ARG;
+    if (H % G != 0) return SSD_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return SSD_ERR_UNSUPPORTED;
+    if (path != SSD_PATH_AUTO && path != SSD_PATH_SIMT && path != SSD_PATH_TENSOR)
+        return SSD_ERR_INVALID_ARG;
+    // every flat index fits comfortably in 63 bits; per-launch grid limits are
+    // checked by the path's own support test
+    if (b > (1ll << 20) || L > (1ll << 31) || H > 65535 || P > 65535 || N > 65535) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+// SSD_PATH_AUTO picks the tensor-core path when this is set and the shape fits.
+constexpr bool kAutoTensor = false;
+
+// Resolves `path` for these sizes; SSD_ERR_UNSUPPORTED when nothing fits.
+ssd_status resolve_path(const ssd::ScanDims &d, int in_dtype, int path, int *chosen) {
+    const bool tc = ssd::tc_supported(d, in_dtype == SSD_BF16);
+    const bool simt = ssd::simt_supported(d);
+    if (path == SSD_PATH_TENSOR) {
+        if (!tc) return SSD_ERR_UNSUPPORTED;
+        *chosen = SSD_PATH_TENSOR;
+    } else if (path == SSD_PATH_SIMT) {
+        if (!simt) return SSD_ERR_UNSUPPORTED;
+        *chosen = SSD_PATH_SIMT;
+    } else if (tc && kAutoTensor) {
+        *chosen = SSD_PATH_TENSOR;
+    } else if (simt) {
+        *chosen = SSD_PATH_SIMT;
+    } else {
+        return SSD_ERR_UNSUPPORTED;
+    }
+    return SSD_OK;
+}
+
+ssd::ScanDims make_dims(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, int64_t Q) {
+    ssd::ScanDims d;
+    d.b = b; d.L = L; d.H = H; d.P = P; d.N = N; d.G = G; d.Q = Q;
+    d.nc = (L + Q - 1) / Q;
+    return d;
+}
+
+size_t path_ws(const ssd::ScanDims &d, int chosen) {
+    return chosen == SSD_PATH_TENSOR ? ssd::tc_workspace_bytes(d) : ssd::simt_workspace_bytes(d);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssd_version(void) { return (1 << 16) | 0; }
+
+int ssd_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *ssd_status_string(int s) {
+    switch (s) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_INVALID_ARG: return "invalid argument";
+        case SSD_ERR_UNSUPPORTED: return "unsupported dtype, path or size";
+        case SSD_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSD_ERR_CUDA: return "CUDA error";
+        case SSD_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case SSD_ERR_PRECONDITION:
+            return "precondition violated on device (A > 0, or a tensor-path operand outside the fp16 range)";
+        default: return "unknown status";
+    }
+}
+
+ssd_status ssd_chunk_scan_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads,
+                                         int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                                         int64_t chunk_size, int in_dtype, int path, size_t *bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size,
+                                    in_dtype, path);
+    if (st != SSD_OK) return st;
+    const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
+    int chosen = 0;
+    if ((st = resolve_path(d, in_dtype, path, &chosen)) != SSD_OK) return st;
+    *bytes = path_ws(d, chosen);
+    return SSD_OK;
+}
+
+ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const float *dt_bias,
+                              const float *A, const void *B, const void *C, const float *D,
+                              const float *init_state, float *y, float *final_state,
+                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                              int64_t state_dim, int64_t ngroups, int64_t chunk_size,
+                              float dt_lo, float dt_hi, int in_dtype, int path,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size,
+                                    in_dtype, path);
+    if (st != SSD_OK) return st;
+    if (!limits_ok(dt_lo, dt_hi)) return SSD_ERR_INVALID_ARG;
+    if (!dt_bias || !A || !D) return SSD_ERR_INVALID_ARG;
+    const bool has_tokens = batch > 0 && seqlen > 0;
+    if (has_tokens && (!x || !dt_raw || !B || !C || !y)) return SSD_ERR_INVALID_ARG;
+    if ((x && !aligned16(x)) || (B && !aligned16(B)) || (C && !aligned16(C)) || (y && !aligned16(y)) ||
+        (init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
+        return SSD_ERR_ALIGNMENT;
+    const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
+    int chosen = 0;
+    if ((st = resolve_path(d, in_dtype, path, &chosen)) != SSD_OK) return st;
+    if (!workspace || workspace_bytes < path_ws(d, chosen)) return SSD_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, ssd::kStatusBytes, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (batch == 0) return SSD_OK;
+    const size_t state_bytes = (size_t)batch * nheads * state_dim * head_dim * sizeof(float);
+    if (seqlen == 0) {
+        // no tokens: the state leaves as it came in
+        if (final_state) {
+            e = init_state ? cudaMemcpyAsync(final_state, init_state, state_bytes, cudaMemcpyDeviceToDevice, s)
+                           : cudaMemsetAsync(final_state, 0, state_bytes, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return SSD_OK;
+    }
+
+    ssd::ScanArgs a;
+    a.x = x; a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.init_state = init_state; a.y = y; a.final_state = final_state;
+    a.dt_lo = dt_lo; a.dt_hi = dt_hi; a.bf16 = in_dtype == SSD_BF16;
+    e = chosen == SSD_PATH_TENSOR ? ssd::tc_scan(a, d, workspace, s) : ssd::simt_scan(a, d, workspace, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return SSD_OK;
+}
+
+ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
+                    const void *B, const void *C, const float *D, float *state, float *y,
+                    int64_t batch, int64_t nheads, int64_t head_dim, int64_t state_dim,
+                    int64_t ngroups, float dt_lo, float dt_hi, int in_dtype, void *stream) {
+    if (batch < 0 || nheads <= 0 || head_dim <= 0 || state_dim <= 0 || ngroups <= 0) return SSD_ERR_INVALID_ARG;
+    if (nheads % ngroups != 0 || !limits_ok(dt_lo, dt_hi)) return SSD_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return SSD_ERR_UNSUPPORTED;
+    if (!ssd::step_supported(head_dim, state_dim) || batch * nheads > 0x7fffffffll) return SSD_ERR_UNSUPPORTED;
+    if (batch == 0) return SSD_OK;
+    if (!x || !dt_raw || !dt_bias || !A || !B || !C || !D || !state || !y) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(B) || !aligned16(C) || !aligned16(state) || !aligned16(y))
+        return SSD_ERR_ALIGNMENT;
+    ssd::StepArgs a;
+    a.x = x; a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.state = state; a.y = y;
+    a.b = batch; a.H = nheads; a.P = head_dim; a.N = state_dim; a.G = ngroups;
+    a.dt_lo = dt_lo; a.dt_hi = dt_hi; a.bf16 = in_dtype == SSD_BF16;
+    cudaError_t e = ssd::step_launch(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return SSD_OK;
+}
+
+ssd_status ssd_read_device_status(const void *workspace, void *stream) {
+    if (!workspace) return SSD_ERR_INVALID_ARG;
+    unsigned word = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word & ssd::kStatusTimeout) return SSD_ERR_DEVICE_TIMEOUT;
+    if (word & (ssd::kStatusPrecondition | ssd::kStatusRange)) return SSD_ERR_PRECONDITION;
+    return SSD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// Device helpers shared by the SSD kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// Device status word bits (first word of the scan workspace).
+enum : unsigned {
+    kStatusPrecondition = 1u,   // A > 0 seen
+    kStatusTimeout = 2u,        // a bounded wait gave up
+    kStatusRange = 4u,          // tensor path: a value outside the fp16 operand range
+};
+
+constexpr size_t kStatusBytes = 256;   // status region at the start of the workspace
+
+__device__ __forceinline__ float softplus_f(float z) {
+    // log(1 + e^z) in the stable form max(z,0) + log1p(e^-|z|)
+    return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
+}
+
+__device__ __forceinline__ float dt_of(float raw, float bias, float lo, float hi) {
+    return fminf(fmaxf(softplus_f(raw + bias), lo), hi);
+}
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {
+    return __bfloat162float(v);
+}
+
+__device__ __forceinline__ void flag_status(unsigned *status, unsigned bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// Inclusive scan of one float per thread across a block of up to 1024 threads
+// (blockDim.x a multiple of 32); `total` receives the block-wide sum.
+// `warp_tot` is shared scratch of 32 floats.  Fixed combination order:
+// deterministic run to run.
+__device__ __forceinline__ float block_inclusive_scan(float v, float *warp_tot, float &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        float t = lane < nw ? warp_tot[lane] : 0.0f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            float u = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += u;
+        }
+        if (lane < nw) warp_tot[lane] = t;
+    }
+    __syncthreads();
+    if (warp > 0) v += warp_tot[warp - 1];
+    total = warp_tot[nw - 1];
+    __syncthreads();
+    return v;
+}
+
+}  // namespace ssd

@@ -1,0 +1,53 @@
+// Internal launcher interface between the C ABI (ssd_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssd {
+
+struct ScanDims {
+    int64_t b, L, H, P, N, G, Q;   // batch, seqlen, heads, head_dim, state_dim, groups, chunk
+    int64_t nc;                    // ceil(L / Q)
+};
+
+struct ScanArgs {
+    const void *x;
+    const float *dt_raw, *dt_bias, *A;
+    const void *B, *C;
+    const float *D, *init_state;
+    float *y, *final_state;
+    float dt_lo, dt_hi;
+    int bf16;                      // 1: x/B/C are bfloat16, 0: float32
+};
+
+struct StepArgs {
+    const void *x;
+    const float *dt_raw, *dt_bias, *A;
+    const void *B, *C;
+    const float *D;
+    float *state, *y;
+    int64_t b, H, P, N, G;
+    float dt_lo, dt_hi;
+    int bf16;
+};
+
+// Workspace carve-up: [status | per-path regions], every region 256-byte aligned.
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// ---- SIMT fp32 path (any chunk size) --------------------------------------
+bool simt_supported(const ScanDims &d);
+size_t simt_workspace_bytes(const ScanDims &d);
+cudaError_t simt_scan(const ScanArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
+
+// ---- tcgen05 tensor-core path -----------------------------------------------
+bool tc_supported(const ScanDims &d, int bf16);
+size_t tc_workspace_bytes(const ScanDims &d);
+cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
+
+// ---- decode step ------------------------------------------------------------
+bool step_supported(int64_t P, int64_t N);
+cudaError_t step_launch(const StepArgs &a, cudaStream_t s);
+
+}  // namespace ssd

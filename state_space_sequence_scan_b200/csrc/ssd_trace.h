@@ -1,0 +1,32 @@
+// Internal tracing hooks (see ssd_trace.cu and ssd_trace_enable in ssd.h).
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace ssd {
+
+enum TraceKernel {
+    kTrSimtChunkState = 0,
+    kTrSimtStatePass = 1,
+    kTrSimtChunkOut = 2,
+    kTrDecodeStep = 3,
+    kTrTcUnitState = 4,
+    kTrTcStatePass = 5,
+    kTrTcChunkOut = 6,
+    kTrTcDtPrep = 7,
+    kKernelCount = 8,
+};
+
+bool trace_on();
+int trace_begin(cudaStream_t s, int kernel);   // returns a slot, or -1 when tracing is off/full
+void trace_end(cudaStream_t s, int slot);
+
+// RAII bracket: `TraceScope t(stream, kTrX); launch...;`
+struct TraceScope {
+    cudaStream_t s;
+    int slot;
+    TraceScope(cudaStream_t st, int kernel) : s(st), slot(trace_begin(st, kernel)) {}
+    ~TraceScope() { trace_end(s, slot); }
+};
+
+}  // namespace ssd

@@ -1,0 +1,222 @@
+"""Python binding of libssd.so (argument marshalling only).
+
+Every step of the scan and of the decode update runs in the CUDA library; this
+module checks tensor shapes/dtypes/devices, allocates outputs and workspace
+through PyTorch (device memory is the only thing PyTorch provides here), and
+passes raw pointers plus the current CUDA stream across the C ABI declared in
+include/ssd.h.  There is no CPU fallback: without the built library, or
+without a CUDA device, every compute call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd.so")
+
+SSD_OK = 0
+STATUS_NAMES = {
+    0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "SSD_ERR_ALIGNMENT",
+    4: "SSD_ERR_WORKSPACE", 5: "SSD_ERR_CUDA", 6: "SSD_ERR_DEVICE_TIMEOUT", 7: "SSD_ERR_PRECONDITION",
+}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+PATHS = {"auto": 0, "simt": 1, "tensor": 2}
+
+EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_step",
+            "ssd_read_device_status", "ssd_status_string", "ssd_last_cuda_error", "ssd_version",
+            "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count")
+
+_lib = None
+
+
+class SSDError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        name = STATUS_NAMES.get(status, str(status))
+        super().__init__("%s failed: %s%s" % (fn, name, (" (" + detail + ")") if detail else ""))
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libssd.so and declares the C signatures.  Raises if it is missing:
+    there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("libssd.so is not built (%s); run python -m state_space_sequence_scan_b200.build"
+                           % path)
+    lib = ctypes.CDLL(path)
+    vp, i64, f32, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int, ctypes.c_size_t
+    lib.ssd_chunk_scan_workspace_size.restype = i32
+    lib.ssd_chunk_scan_workspace_size.argtypes = [i64] * 7 + [i32, i32, ctypes.POINTER(sz)]
+    lib.ssd_chunk_scan_fwd.restype = i32
+    lib.ssd_chunk_scan_fwd.argtypes = [vp] * 10 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
+    lib.ssd_step.restype = i32
+    lib.ssd_step.argtypes = [vp] * 9 + [i64] * 5 + [f32, f32, i32, vp]
+    lib.ssd_read_device_status.restype = i32
+    lib.ssd_read_device_status.argtypes = [vp, vp]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_status_string.argtypes = [i32]
+    lib.ssd_last_cuda_error.restype = i32
+    lib.ssd_last_cuda_error.argtypes = []
+    lib.ssd_version.restype = i32
+    lib.ssd_version.argtypes = []
+    lib.ssd_trace_enable.restype = i32
+    lib.ssd_trace_enable.argtypes = [i32]
+    lib.ssd_trace_read.restype = i32
+    lib.ssd_trace_read.argtypes = [i32, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_double)]
+    lib.ssd_trace_kernel_name.restype = ctypes.c_char_p
+    lib.ssd_trace_kernel_name.argtypes = [i32]
+    lib.ssd_trace_kernel_count.restype = i32
+    lib.ssd_trace_kernel_count.argtypes = []
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, st: int):
+    if st != SSD_OK:
+        detail = ""
+        if st == 5:
+            detail = "cudaError %d" % load_library().ssd_last_cuda_error()
+        raise SSDError(fn, st, detail)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def workspace_size(batch: int, seqlen: int, nheads: int, head_dim: int, state_dim: int, ngroups: int,
+                   chunk_size: int, dtype: torch.dtype = torch.bfloat16, path: str = "auto") -> int:
+    lib = load_library()
+    out = ctypes.c_size_t(0)
+    _check("ssd_chunk_scan_workspace_size", lib.ssd_chunk_scan_workspace_size(
+        batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, DTYPES[dtype], PATHS[path],
+        ctypes.byref(out)))
+    return int(out.value)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """Workspace as a uint8 CUDA tensor (PyTorch allocations are 256-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def chunk_scan_fwd(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor, A: torch.Tensor,
+                   B: torch.Tensor, C: torch.Tensor, D: torch.Tensor,
+                   init_state: Optional[torch.Tensor] = None, chunk_size: int = 256,
+                   dt_limit: Tuple[float, float] = (0.0, math.inf), path: str = "auto",
+                   workspace: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                   final_state: Optional[torch.Tensor] = None,
+                   want_final_state: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked forward scan.  Shapes as in include/ssd.h:
+    x [b,L,H,P], dt_raw [b,L,H] f32, dt_bias/A/D [H] f32, B/C [b,L,G,N] (same
+    dtype as x, f32 or bf16), init_state [b,H,N,P] f32 or None.
+    Returns (y [b,L,H,P] f32, final_state [b,H,N,P] f32 or None)."""
+    lib = load_library()
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    _need_cuda("x", x)
+    if x.dtype not in DTYPES:
+        raise ValueError("x/B/C must be float32 or bfloat16")
+    _need_cuda("B", B, x.dtype, (b, L, G, N))
+    _need_cuda("C", C, x.dtype, (b, L, G, N))
+    _need_cuda("dt_raw", dt_raw, torch.float32, (b, L, H))
+    for nm, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need_cuda(nm, t, torch.float32, (H,))
+    if init_state is not None:
+        _need_cuda("init_state", init_state, torch.float32, (b, H, N, P))
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
+    else:
+        _need_cuda("y", y, torch.float32, (b, L, H, P))
+    if want_final_state and final_state is None:
+        final_state = torch.empty((b, H, N, P), dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _need_cuda("final_state", final_state, torch.float32, (b, H, N, P))
+    need = workspace_size(b, L, H, P, N, G, chunk_size, x.dtype, path)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    st = lib.ssd_chunk_scan_fwd(
+        _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+        _ptr(y), _ptr(final_state), b, L, H, P, N, G, int(chunk_size),
+        float(dt_limit[0]), float(dt_limit[1]), DTYPES[x.dtype], PATHS[path],
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _check("ssd_chunk_scan_fwd", st)
+    return y, final_state
+
+
+def read_device_status(workspace: torch.Tensor) -> int:
+    """Synchronises the current stream and returns the device status code."""
+    lib = load_library()
+    return int(lib.ssd_read_device_status(_ptr(workspace), _stream(workspace.device)))
+
+
+def step(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor, A: torch.Tensor,
+         B: torch.Tensor, C: torch.Tensor, D: torch.Tensor, state: torch.Tensor,
+         dt_limit: Tuple[float, float] = (0.0, math.inf),
+         y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One decode token: x [b,H,P], dt_raw [b,H] f32, B/C [b,G,N], state
+    [b,H,N,P] f32 updated in place.  Returns y [b,H,P] f32."""
+    lib = load_library()
+    if x.dim() != 3 or B.dim() != 3:
+        raise ValueError("x must be [b,H,P] and B, C [b,G,N]")
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    _need_cuda("x", x)
+    if x.dtype not in DTYPES:
+        raise ValueError("x/B/C must be float32 or bfloat16")
+    _need_cuda("B", B, x.dtype, (b, G, N))
+    _need_cuda("C", C, x.dtype, (b, G, N))
+    _need_cuda("dt_raw", dt_raw, torch.float32, (b, H))
+    for nm, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need_cuda(nm, t, torch.float32, (H,))
+    _need_cuda("state", state, torch.float32, (b, H, N, P))
+    if y is None:
+        y = torch.empty((b, H, P), dtype=torch.float32, device=x.device)
+    else:
+        _need_cuda("y", y, torch.float32, (b, H, P))
+    st = lib.ssd_step(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                      _ptr(state), _ptr(y), b, H, P, N, G, float(dt_limit[0]), float(dt_limit[1]),
+                      DTYPES[x.dtype], _stream(x.device))
+    _check("ssd_step", st)
+    return y
+
+
+def trace_enable(max_launches: int) -> None:
+    """Start (max_launches > 0) or stop (0) per-kernel event tracing."""
+    _check("ssd_trace_enable", load_library().ssd_trace_enable(int(max_launches)))
+
+
+def trace_read() -> dict:
+    """{kernel name: (launches, total device ms)} for every traced kernel."""
+    lib = load_library()
+    out = {}
+    for k in range(lib.ssd_trace_kernel_count()):
+        n = ctypes.c_int(0)
+        ms = ctypes.c_double(0.0)
+        _check("ssd_trace_read", lib.ssd_trace_read(k, ctypes.byref(n), ctypes.byref(ms)))
+        if n.value:
+            out[lib.ssd_trace_kernel_name(k).decode()] = (int(n.value), float(ms.value))
+    return out

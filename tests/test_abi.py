@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry
+point include/ssd.h declares, and rejects bad arguments before touching the
+GPU (no compute call is made here)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from state_space_sequence_scan_b200 import ssd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"SSD_API\s+[\w\s\*]*?\b(ssd_\w+)\s*\(", txt)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from state_space_sequence_scan_b200 import build
+    build.build_library()
+    return ssd.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(ssd.EXPORTED) <= set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.ssd_version() >> 16 == 1
+    for code in range(8):
+        s = lib.ssd_status_string(code)
+        assert s and s != b"unknown status"
+    assert lib.ssd_status_string(99) == b"unknown status"
+
+
+def _ws(lib, *dims, dtype=1, path=0):
+    out = ctypes.c_size_t(0)
+    st = lib.ssd_chunk_scan_workspace_size(*dims, dtype, path, ctypes.byref(out))
+    return st, out.value
+
+
+def test_workspace_size_validation(lib):
+    assert _ws(lib, 1, 64, 4, 16, 16, 1, 16, dtype=0)[0] == 0
+    assert _ws(lib, 1, 64, 4, 16, 16, 1, 16, dtype=0)[1] >= 256
+    assert _ws(lib, 1, 64, 4, 16, 16, 3, 16)[0] == 1          # H % G != 0
+    assert _ws(lib, 1, 64, 0, 16, 16, 1, 16)[0] == 1          # no heads
+    assert _ws(lib, 1, 64, 4, 16, 16, 1, 0)[0] == 1           # chunk 0
+    assert _ws(lib, -1, 64, 4, 16, 16, 1, 16)[0] == 1
+    assert _ws(lib, 1, 64, 4, 16, 16, 1, 16, dtype=7)[0] == 2  # unknown dtype
+    assert _ws(lib, 1, 64, 4, 16, 16, 1, 16, path=9)[0] == 1   # unknown path
+    assert _ws(lib, 1, 64, 4, 24, 16, 1, 16)[0] == 2          # head_dim must divide 256 (SIMT)
+    st = lib.ssd_chunk_scan_workspace_size(1, 64, 4, 16, 16, 1, 16, 0, 0, None)
+    assert st == 1
+
+
+def test_workspace_grows_with_chunks(lib):
+    _, small = _ws(lib, 2, 1024, 4, 64, 128, 1, 256, path=1)
+    _, big = _ws(lib, 2, 1024, 4, 64, 128, 1, 16, path=1)
+    assert big > small > 0
+
+
+def _fwd(lib, **kw):
+    a = dict(x=None, dt_raw=None, dt_bias=None, A=None, B=None, C=None, D=None, init=None, y=None, fs=None,
+             b=1, L=8, H=2, P=16, N=16, G=1, Q=4, lo=0.0, hi=math.inf, dtype=0, path=0, ws=None, wsb=0,
+             stream=None)
+    a.update(kw)
+    return lib.ssd_chunk_scan_fwd(a["x"], a["dt_raw"], a["dt_bias"], a["A"], a["B"], a["C"], a["D"], a["init"],
+                                  a["y"], a["fs"], a["b"], a["L"], a["H"], a["P"], a["N"], a["G"], a["Q"],
+                                  a["lo"], a["hi"], a["dtype"], a["path"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_forward_rejects_bad_arguments_on_host(lib):
+    fake = 0x10000          # aligned non-null stand-in; never dereferenced (calls fail validation first)
+    ok = dict(x=fake, dt_raw=fake, dt_bias=fake, A=fake, B=fake, C=fake, D=fake, y=fake, fs=fake)
+    assert _fwd(lib) == 1                                     # null pointers
+    assert _fwd(lib, **ok, H=3, G=2) == 1                     # H % G
+    assert _fwd(lib, **ok, lo=0.5, hi=0.1) == 1               # dt limits reversed
+    assert _fwd(lib, **ok, lo=-1.0) == 1                      # negative lower limit
+    assert _fwd(lib, **ok, lo=float("nan")) == 1
+    assert _fwd(lib, **dict(ok, x=fake + 4)) == 3             # misaligned
+    assert _fwd(lib, **ok) == 4                               # no workspace
+    assert _fwd(lib, **ok, ws=fake, wsb=16) == 4              # workspace too small
+    assert _fwd(lib, **ok, ws=fake + 16, wsb=1 << 30) == 3    # workspace not 256-aligned
+    assert _fwd(lib, **ok, dtype=5) == 2
+    assert _fwd(lib, **ok, path=2, dtype=0) == 2              # tensor path needs bf16
+
+
+def test_step_rejects_bad_arguments_on_host(lib):
+    fake = 0x10000
+    f = lambda **kw: lib.ssd_step(*([kw.get("p", fake)] * 9), kw.get("b", 2), kw.get("H", 4), kw.get("P", 16),
+                                 kw.get("N", 16), kw.get("G", 2), kw.get("lo", 0.0), kw.get("hi", math.inf),
+                                 kw.get("dtype", 1), None)
+    assert f(p=None) == 1
+    assert f(H=3) == 1
+    assert f(P=6) == 2
+    assert f(P=12) == 2                                       # 12/4 = 3 does not divide 256
+    assert f(dtype=3) == 2
+    assert f(lo=2.0, hi=1.0) == 1
+    assert f(b=0) == 0                                        # empty batch: nothing to do
+    assert lib.ssd_step(*([fake + 8] * 9), 2, 4, 16, 16, 2, 0.0, math.inf, 1, None) == 3
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 2, 16)
+    with pytest.raises(ValueError):
+        ssd.chunk_scan_fwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(2), torch.zeros(1, 4, 1, 16),
+                           torch.zeros(1, 4, 1, 16), torch.zeros(2), chunk_size=4)

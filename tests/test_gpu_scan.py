@@ -1,0 +1,213 @@
+"""GPU parity of the chunked scan (through the C ABI) against the fp64 oracle.
+
+Bar: max|gpu - oracle| / RMS(oracle) <= 1e-4 for fp32 inputs and <= 2e-2 for
+bf16 inputs (oracle fed the same bf16-rounded values), separately for y and
+for final_state.  Small cases span several chunks/tiles and a ragged tail;
+the full-size workloads are checked on sampled (batch, head) chains, each of
+which the oracle evaluates alone (chains are independent).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import TOL_BF16, TOL_F32, compare, run_scan, sample_chains, tol_for
+from state_space_sequence_scan_b200 import ssd
+from state_space_sequence_scan_b200.inputs import SCAN_CONFIGS, ScanConfig, make_scan_inputs
+
+pytestmark = pytest.mark.gpu
+
+PATHS = ["auto", "simt"]
+
+
+def _oracle(inp, dt_limit=(0.0, math.inf)):
+    return oracle.scan(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"],
+                       init_state=inp["init_state"], dt_limit=dt_limit)
+
+
+def _check(inp, Q, path, dt_limit=(0.0, math.inf), what=""):
+    y, fs = run_scan(inp, Q, path=path, dt_limit=dt_limit)
+    yr, fr = _oracle(inp, dt_limit)
+    tol = tol_for(inp["x"].dtype)
+    compare(y, yr, tol, what + " y")
+    compare(fs, fr, tol, what + " final_state")
+    return y, fs
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_tiny_fp32_config(path):
+    cfg = SCAN_CONFIGS["c0_tiny_fp32"]
+    _check(make_scan_inputs(cfg), cfg.chunk_size, path, what=cfg.name)
+
+
+CASES = [
+    # b, L, H, P, N, G, Q, dtype, init
+    (2, 3 * 64 + 5, 4, 64, 128, 2, 64, "f32", "normal"),
+    (2, 3 * 64 + 5, 4, 64, 128, 2, 64, "bf16", "normal"),
+    (1, 2 * 256 + 37, 8, 64, 128, 1, 256, "bf16", "normal"),
+    (2, 700, 6, 64, 128, 3, 128, "bf16", "zero"),
+    (1, 300, 4, 32, 64, 4, 100, "f32", "normal"),        # G = H, odd chunk
+    (3, 77, 2, 16, 16, 1, 7, "f32", "normal"),
+    (1, 50, 2, 8, 4, 2, 1, "f32", "normal"),             # chunk 1: every token a boundary
+    (1, 129, 2, 64, 128, 1, 128, "bf16", "normal"),      # one token past a chunk
+    (2, 1, 4, 64, 128, 1, 256, "bf16", "normal"),        # one token
+]
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "b%d_L%d_H%d_P%d_N%d_G%d_Q%d_%s_%s" % c)
+def test_small_parity(case, path):
+    b, L, H, P, N, G, Q, dt, init = case
+    cfg = ScanConfig("case", b, L, H, P, N, G, Q, dt, "normal", init, seed=sum(c for c in case if isinstance(c, int)) % 997)
+    _check(make_scan_inputs(cfg), Q, path, what=str(case))
+
+
+def test_dt_limit_clamp():
+    cfg = ScanConfig("clamp", 2, 300, 4, 64, 128, 2, 64, "bf16", "ones", "normal", seed=11)
+    inp = make_scan_inputs(cfg)
+    _check(inp, 64, "auto", dt_limit=(0.02, 0.3), what="clamp")
+
+
+def test_c1_130m_full():
+    cfg = SCAN_CONFIGS["c1_130m"]
+    _check(make_scan_inputs(cfg), cfg.chunk_size, "auto", what=cfg.name)
+
+
+@pytest.mark.parametrize("name,chains", [
+    ("c2_2p7b", [(0, 0), (3, 41), (7, 79), (5, 17)]),
+    ("c3_long", [(0, 0), (0, 37), (0, 79)]),
+])
+def test_full_size_sampled_chains(name, chains):
+    """The kernels run on the whole workload (the launch the benchmark times);
+    the oracle evaluates the sampled chains alone."""
+    cfg = SCAN_CONFIGS[name]
+    inp = make_scan_inputs(cfg)
+    y, fs = run_scan(inp, cfg.chunk_size, path="auto")
+    assert np.isfinite(y).all() and np.isfinite(fs).all()
+    H, G = cfg.nheads, cfg.ngroups
+    for (bi, h), sub in zip(chains, sample_chains(inp, chains)):
+        yr, fr = _oracle(sub)
+        compare(y[bi:bi + 1, :, h:h + 1], yr, TOL_BF16, "%s chain %s y" % (name, (bi, h)))
+        compare(fs[bi:bi + 1, h:h + 1], fr, TOL_BF16, "%s chain %s final_state" % (name, (bi, h)))
+
+
+def test_chunk_size_invariance_fp32():
+    cfg = ScanConfig("inv", 1, 512, 4, 64, 128, 2, 64, "f32", "normal", "normal", seed=5)
+    inp = make_scan_inputs(cfg)
+    ys = [run_scan(inp, Q, path="simt") for Q in (1, 16, 64, 200, 512)]
+    yr, fr = _oracle(inp)
+    y0, f0 = ys[2]
+    for y, f in ys:
+        compare(y, yr, TOL_F32, "y vs oracle")
+        compare(f, fr, TOL_F32, "final_state vs oracle")
+        compare(y, y0, TOL_F32, "y across chunk sizes")
+        compare(f, f0, TOL_F32, "final_state across chunk sizes")
+
+
+def test_split_and_carry():
+    cfg = ScanConfig("split", 2, 1000, 4, 64, 128, 1, 128, "bf16", "ones", "normal", seed=6)
+    inp = make_scan_inputs(cfg)
+    y, fs = run_scan(inp, 128)
+    T1 = 389
+    first = {k: (v[:, :T1] if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
+    y1, h1 = run_scan(first, 128)
+    second = {k: (v[:, T1:] if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
+    second["init_state"] = torch.from_numpy(h1).float()
+    y2, h2 = run_scan(second, 128)
+    yr, fr = _oracle(inp)
+    compare(np.concatenate([y1, y2], axis=1), yr, TOL_BF16, "split y")
+    compare(h2, fr, TOL_BF16, "split final_state")
+    compare(y, yr, TOL_BF16, "whole y")
+
+
+def test_skip_token():
+    """dt = 0 exactly (softplus underflow): the token writes nothing and decays
+    nothing, so the rest of the sequence sees what it would without it."""
+    cfg = ScanConfig("skip", 1, 300, 4, 64, 128, 1, 64, "f32", "ones", "normal", seed=7)
+    inp = make_scan_inputs(cfg)
+    t = 130
+    inp["dt_raw"][:, t] = -1.0e4
+    y, fs = run_scan(inp, 64)
+    cut = {k: (torch.cat([v[:, :t], v[:, t + 1:]], 1) if k in ("x", "dt_raw", "B", "C") else v)
+           for k, v in inp.items()}
+    yc, fc = run_scan(cut, 64)
+    compare(np.delete(y, t, axis=1), yc, TOL_F32, "skip y")
+    compare(fs, fc, TOL_F32, "skip final_state")
+
+
+def test_memoryless_and_nonfinite_guard():
+    """Huge |A| and dt >= 0.01: every exponent underflows to 0; output must
+    stay finite and equal dt_t (C_t.B_t) x_t + D x_t."""
+    cfg = ScanConfig("memless", 1, 600, 4, 64, 128, 1, 256, "bf16", "ones", "normal", seed=8)
+    inp = make_scan_inputs(cfg)
+    inp["A"][:] = -1.0e5
+    y, fs = run_scan(inp, 256, dt_limit=(0.01, math.inf))
+    yr, fr = _oracle(inp, (0.01, math.inf))
+    compare(y, yr, TOL_BF16, "memoryless y")
+    compare(fs, fr, TOL_BF16, "memoryless final")
+
+
+def test_deterministic():
+    cfg = SCAN_CONFIGS["c1_130m"].with_(seqlen=1024)
+    inp = make_scan_inputs(cfg)
+    a = run_scan(inp, cfg.chunk_size)
+    b = run_scan(inp, cfg.chunk_size)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_groups_replicated_equal():
+    cfg = ScanConfig("grp", 1, 400, 4, 64, 128, 1, 128, "bf16", "ones", "normal", seed=9)
+    inp = make_scan_inputs(cfg)
+    y1, f1 = run_scan(inp, 128)
+    rep = dict(inp)
+    rep["B"] = inp["B"].repeat_interleave(4, dim=2).contiguous()
+    rep["C"] = inp["C"].repeat_interleave(4, dim=2).contiguous()
+    y4, f4 = run_scan(rep, 128)
+    compare(y4, y1, 1e-6, "G=H vs G=1 y")
+    compare(f4, f1, 1e-6, "G=H vs G=1 final")
+
+
+def test_positive_A_is_reported():
+    cfg = ScanConfig("posA", 1, 64, 2, 16, 16, 1, 16, "f32", "ones", "zero", seed=10)
+    inp = make_scan_inputs(cfg)
+    inp["A"][1] = 0.5
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    ws = ssd.alloc_workspace(ssd.workspace_size(1, 64, 2, 16, 16, 1, 16, torch.float32), "cuda")
+    ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], chunk_size=16,
+                       workspace=ws)
+    assert ssd.read_device_status(ws) == 7
+    inp["A"][1] = -0.5
+    d["A"] = inp["A"].cuda()
+    ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], chunk_size=16,
+                       workspace=ws)
+    assert ssd.read_device_status(ws) == 0                 # the status word is cleared per call
+
+
+def test_empty_sequence_and_batch():
+    H, P, N = 4, 64, 128
+    init = torch.randn(2, H, N, P, device="cuda")
+    x = torch.zeros(2, 0, H, P, device="cuda", dtype=torch.bfloat16)
+    B = torch.zeros(2, 0, 1, N, device="cuda", dtype=torch.bfloat16)
+    z = torch.zeros(H, device="cuda")
+    y, fs = ssd.chunk_scan_fwd(x, torch.zeros(2, 0, H, device="cuda"), z, -torch.ones(H, device="cuda"), B, B.clone(),
+                               torch.ones(H, device="cuda"), init_state=init, chunk_size=256)
+    torch.cuda.synchronize()
+    assert y.shape == (2, 0, H, P) and torch.equal(fs, init)
+    x0 = torch.zeros(0, 10, H, P, device="cuda", dtype=torch.bfloat16)
+    B0 = torch.zeros(0, 10, 1, N, device="cuda", dtype=torch.bfloat16)
+    y0, f0 = ssd.chunk_scan_fwd(x0, torch.zeros(0, 10, H, device="cuda"), z, -torch.ones(H, device="cuda"), B0,
+                                B0.clone(), torch.ones(H, device="cuda"), chunk_size=256)
+    assert y0.shape == (0, 10, H, P) and f0.shape == (0, H, N, P)
+
+
+def test_130m_shapes_match_pages():
+    """Shapes the nnterp guide prints for mamba2-130m on a 10-token prompt."""
+    cfg = ScanConfig("shapes", 1, 10, 24, 64, 128, 1, 256, "bf16", "ones", "zero", seed=12)
+    inp = make_scan_inputs(cfg)
+    y, fs = run_scan(inp, 256)
+    assert y.shape == (1, 10, 24, 64) and fs.shape == (1, 24, 128, 64)
+    yr, fr = _oracle(inp)
+    compare(y, yr, TOL_BF16, "130m 10-token y")
+    compare(fs, fr, TOL_BF16, "130m 10-token final")
