@@ -6,7 +6,9 @@
 A "step" is one chunked forward scan (every stage of the hot path: dt
 preparation, chunk cumsum, intra-chunk C.B^T, chunk states, state passing,
 chunk output) over one batch of the workload; the decode workload's step is
-one single-token state update.  Rank 0 prints ONE JSON line.  With N > 1 each
+one single-token state update.  The K timed steps are captured once into a
+CUDA graph and launched as one graph, so the number is device time, not
+Python call overhead; per-kernel times come from an eager traced pass.  Rank 0 prints ONE JSON line.  With N > 1 each
 rank runs its own copy of the workload (independent batches, no collective on
 the data path: weak scaling); the time is the max over ranks.
 
@@ -200,6 +202,7 @@ def bench_scan(cfg, args, ws, rank, local):
     if ssd.read_device_status(work) != 0:
         raise RuntimeError("device status %d after warm-up" % ssd.read_device_status(work))
 
+    graph = capture_steps(step, args.steps)
     stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -208,16 +211,16 @@ def bench_scan(cfg, args, ws, rank, local):
     barrier(ws)
     torch.cuda.synchronize()
     e0.record(stream)
-    for k in range(args.steps):
-        step(k)
+    graph.replay()                     # exactly K steps, launched as one CUDA graph
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     ms_max = max_over_ranks(ms, ws)
+    del graph
 
-    # per-kernel device times: the same K steps again with event brackets
+    # per-kernel device times: the same K steps again, eagerly, with event brackets
     ssd.trace_enable(min(8192, 8 * args.steps + 8))
     for k in range(args.steps):
         step(k)
@@ -230,6 +233,23 @@ def bench_scan(cfg, args, ws, rank, local):
                launches=int(round(launches_per_step * args.steps)), nsets=nsets)
     res["e2e"] = e2e_scan(inp, cfg, args, dev, work)
     return res
+
+
+def capture_steps(step, steps):
+    """A CUDA graph holding exactly `steps` calls of step(k): the timed
+    region then costs one launch instead of `steps` Python/ctypes calls."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(0)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for k in range(steps):
+            step(k)
+    torch.cuda.synchronize()
+    return g
 
 
 def e2e_scan(inp, cfg, args, dev, work):
@@ -287,6 +307,7 @@ def bench_step(cfg, args, ws, rank, local):
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize()
+    graph = capture_steps(step, args.steps)
     stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -295,13 +316,13 @@ def bench_step(cfg, args, ws, rank, local):
     barrier(ws)
     torch.cuda.synchronize()
     e0.record(stream)
-    for k in range(args.steps):
-        step(k)
+    graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
     clk = clocks.stop()
     ms_max = max_over_ranks(e0.elapsed_time(e1), ws)
+    del graph
     ssd.trace_enable(min(8192, args.steps + 8))
     for k in range(args.steps):
         step(k)

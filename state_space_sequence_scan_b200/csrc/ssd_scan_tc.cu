@@ -1,31 +1,33 @@
-// Chunked SSD forward scan on the sm_100a tensor cores (tcgen05 + TMEM).
+// Chunked SSD forward scan on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // Scope: bf16 x/B/C, state_dim N = 128, head_dim P = 64, fp32 dt/A/D/state,
-// fp32 y.  Every contraction runs as a kind::f16 MMA with fp16 operands
-// (bf16 inputs are widened exactly; the decay-weighted operands need fp16's
-// 11-bit significand, bf16's 8 bits are not enough for the 2e-2 bar) and
-// fp32 accumulation in TMEM.
+// fp32 y.  Every contraction runs as a kind::f16 MMA with fp16 operands and
+// fp32 accumulation in TMEM: the bf16 tiles arrive by TMA already in the
+// 128-byte-swizzled operand layout and are widened to fp16 in place (exact);
+// the decay-weighted operands are formed in fp16, whose 11-bit significand
+// the 2e-2 bar needs (bf16's 8 bits are not enough).
 //
 // The sequence of every (batch, head) is cut into 128-token blocks (the MMA
 // M extent) and the blocks into `units` of consecutive blocks.  Four
-// launches, no kernel waits on another CTA:
+// launches; no CTA ever waits on another CTA:
 //   dt_prep     dt = clamp(softplus(dt_raw + dt_bias)), dA = dt*A, and the
 //               inclusive cumsum `cum` of dA inside every 128-token block
 //               (warp shuffles, fixed order), transposed to [b, H, L].
-//   unit_state  per (unit u, head, batch), units 0..U-2: the state the unit
-//               leaves when it starts from zero,
-//                 S'_u = sum_{j in u} exp(sum_{r=j+1..end(u)} dA_r) dt_j B_j x_j^T
-//               as ONE accumulated MMA over the unit's tokens:
-//               D[n,p] += B^T[n,j] (w x)[j,p]  (M=128 n, N=64 p, K=16 per step).
+//   unit_state  per (head, unit u < U-1, batch): the state the unit leaves
+//               when it starts from zero,
+//                 S'_u = sum_{j in u} exp(sum_{r=j+1..end(u)} dA_r) dt_j B_j x_j^T,
+//               as ONE accumulated MMA over the unit's tokens,
+//               D[n,p] += B^T[n,j] (w x)[j,p]  (M=128 n, N=64 p, K=16 per
+//               instruction), with a two-stage TMA pipeline.
 //   state_pass  per (b, h, state element), serial over units:
 //               H_in(0) = init (or 0),  H_in(u+1) = exp(ell_u) H_in(u) + S'_u.
-//   chunk_out   per (unit, head, batch): starting from H_in(u), for each
-//               128-token block in order (state H fp32 in TMEM):
+//   chunk_out   per (head, unit, batch): from H_in(u), for each 128-token
+//               block in order (state H fp32 in TMEM):
 //                 Z   = C H                    (M=128 i, N=64 p, K=128 n)
 //                 CB  = C B^T                  (M=128 i, N=128 j, K=128 n)
 //                 W   = CB .* exp(cum_i - cum_j) dt_j on j <= i, 0 above
 //                 Y   = W X                    (M=128 i, N=64 p, K=128 j)
-//                 y_i = Y_i + exp(cum_i) Z_i + D x_i
+//                 y_i = Y_i + exp(cum_i) Z_i + D x_i      (TMA store)
 //                 H   = exp(cum_last) H + B^T (w X),  w_j = exp(cum_last - cum_j) dt_j
 //               and the last unit writes final_state.
 // This is the chunked form of the scan ("Mamba2" knowledge page: intra-chunk
@@ -40,6 +42,7 @@
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
 #include "ssd_tc.cuh"
+#include "ssd_tmap.h"
 #include "ssd_trace.h"
 
 namespace ssd {
@@ -51,10 +54,11 @@ constexpr int kBlk = 128;                       // tokens per block
 constexpr int kN = 128;                         // state_dim
 constexpr int kP = 64;                          // head_dim
 constexpr int kNP = kN * kP;
-constexpr int kTcThreads = 128;
-constexpr long long kWaitBudget = 1ll << 32;    // clock cycles before an MMA wait gives up (~2 s)
+constexpr int kThreads = 256;                   // 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..
+constexpr long long kWaitBudget = 1ll << 32;    // clock cycles before a wait gives up (~2 s)
 constexpr float kF16Max = 65504.0f;
 constexpr int kUnitTarget = 8 * 148;            // aim for ~8 units per SM across the grid
+constexpr uint32_t kTileBytes = 16384;          // one 128-row x 128-byte swizzled tile
 
 struct TcWs {
     unsigned *status;
@@ -68,13 +72,22 @@ struct TcPlan {
     int64_t nblk, U, bpu;
 };
 
+struct TcMaps {
+    CUtensorMap x, B, C, y;
+};
+
 TcPlan make_plan(const ScanDims &d) {
     TcPlan p;
     p.nblk = (d.L + kBlk - 1) / kBlk;
+    if (p.nblk < 1 || d.b < 1) {          // no tokens: nothing is launched
+        p.nblk = 0;
+        p.U = 1;
+        p.bpu = 1;
+        return p;
+    }
     int64_t U = 1;
     while (d.b * d.H * U < kUnitTarget && U < p.nblk) U *= 2;
     if (U > p.nblk) U = p.nblk;
-    if (U < 1) U = 1;
     p.bpu = (p.nblk + U - 1) / U;
     p.U = (p.nblk + p.bpu - 1) / p.bpu;
     return p;
@@ -99,34 +112,55 @@ size_t ws_bytes(const ScanDims &d, const TcPlan &p) {
            align256((size_t)d.b * d.H * p.U * kNP * sizeof(float));
 }
 
+// Tensor maps over [b, L, H|G, P|N] with 128-token boxes (4-D, innermost
+// first).  x, B, C: bf16 boxes of 64 x 1 x 128 x 1 (one 16 KB swizzled tile);
+// y: fp32 boxes of 32 x 1 x 128 x 1.
+bool make_maps(const ScanArgs &a, const ScanDims &d, TcMaps *m) {
+    const uint64_t b = d.b, L = d.L, H = d.H, G = d.G;
+    const uint32_t box_h[4] = {64, 1, kBlk, 1};
+    const uint32_t box_y[4] = {32, 1, kBlk, 1};
+    {
+        const uint64_t dims[4] = {kP, H, L, b};
+        const uint64_t st[3] = {kP * 2, H * kP * 2, L * H * kP * 2};
+        if (!tmap_encode_4d(&m->x, a.x, 2, dims, st, box_h)) return false;
+    }
+    {
+        const uint64_t dims[4] = {kN, G, L, b};
+        const uint64_t st[3] = {kN * 2, G * kN * 2, L * G * kN * 2};
+        if (!tmap_encode_4d(&m->B, a.B, 2, dims, st, box_h)) return false;
+        if (!tmap_encode_4d(&m->C, a.C, 2, dims, st, box_h)) return false;
+    }
+    {
+        const uint64_t dims[4] = {kP, H, L, b};
+        const uint64_t st[3] = {kP * 4, H * kP * 4, L * H * kP * 4};
+        if (!tmap_encode_4d(&m->y, a.y, 4, dims, st, box_y)) return false;
+    }
+    return true;
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ uint4 ldg16(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
-
-// 8 bf16 (one 16-byte chunk) -> 8 fp16; flags values outside the fp16 range
-__device__ __forceinline__ uint4 cvt_chunk(uint4 v, bool &range_ok) {
-    const float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
-                        bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) range_ok &= fabsf(f[i]) <= kF16Max;
-    return make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
-}
-
-// 8 bf16 scaled by w -> 8 fp16
-__device__ __forceinline__ uint4 cvt_chunk_scaled(uint4 v, float w, bool &range_ok) {
-    const float f[8] = {w * bf16lo(v.x), w * bf16hi(v.x), w * bf16lo(v.y), w * bf16hi(v.y),
-                        w * bf16lo(v.z), w * bf16hi(v.z), w * bf16lo(v.w), w * bf16hi(v.w)};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) range_ok &= fabsf(f[i]) <= kF16Max;
-    return make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
 }
 
 __device__ __forceinline__ uint4 pack8(const float *f, bool &range_ok) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) range_ok &= fabsf(f[i]) <= kF16Max;
     return make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
+}
+
+// In place: one 16-byte chunk of 8 bf16, scaled by w, -> 8 fp16.
+__device__ __forceinline__ void widen_chunk(uint8_t *p, float w, bool &range_ok) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(p);
+    const float f[8] = {w * bf16lo(v.x), w * bf16hi(v.x), w * bf16lo(v.y), w * bf16hi(v.y),
+                        w * bf16lo(v.z), w * bf16hi(v.z), w * bf16lo(v.w), w * bf16hi(v.w)};
+    *reinterpret_cast<uint4 *>(p) = pack8(f, range_ok);
+}
+
+__device__ __forceinline__ void widen_chunk(uint8_t *p, bool &range_ok) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(p);
+    const float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
+                        bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
+    *reinterpret_cast<uint4 *>(p) = pack8(f, range_ok);
 }
 
 // ---------------------------------------------------------------------------
@@ -173,26 +207,26 @@ dt_prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bi
 }
 
 // ---------------------------------------------------------------------------
-// unit_state: grid (H, U-1, b), 128 threads.
-constexpr size_t kUsSmem = 1024 + 32768 + 16384 + 128 * 4 + 4096 * 4 + 64;
+// unit_state: grid (H, U-1, b), 256 threads, two TMA stages of (B, X).
+// Units 0..U-2 never hold the sequence's ragged tail (it is in the last
+// unit), so every block here is a full 128 tokens.
+constexpr uint32_t kUsStage = 3 * kTileBytes;                 // B (2 tiles) + X (1 tile)
+constexpr size_t kUsSmem = 1024 + 2 * kUsStage + 2 * kBlk * 4 + 64;
 
-__global__ void __launch_bounds__(kTcThreads)
-unit_state_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Bm, TcWs ws, int L,
-                  int H, int G, int nblk, int U, int bpu) {
+__global__ void __launch_bounds__(kThreads, 2)
+unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, int nblk, int U, int bpu) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint8_t *sB = sm;                                          // [128 j][128 n] fp16
-    uint8_t *sWX = sm + 32768;                                 // [128 j][64 p] fp16
-    float *s_w = reinterpret_cast<float *>(sm + 49152);        // 128
-    float *s_suf = s_w + kBlk;                                 // bpu (<= 4096)
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_suf + 4096);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);
+    float *s_w = reinterpret_cast<float *>(sm + 2 * kUsStage);   // [2][128]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(s_w + 2 * kBlk); // tma[2], mma[2]
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 4);
 
     const int h = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int g = h / (H / G);
     const int tid = threadIdx.x, warp = tid >> 5;
     const size_t bh = (size_t)b * H + h;
     const int kb0 = u * bpu, kb1 = min(nblk, kb0 + bpu);
+    const int nk = kb1 - kb0;
     const float *cum = ws.cum + bh * (size_t)nblk * kBlk;
     const float *dtv = ws.dt + bh * (size_t)nblk * kBlk;
 
@@ -201,73 +235,93 @@ unit_state_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__re
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(mbar, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(bar + i, 1);
         fence_mbar_init();
-        float acc = 0.f;
-        for (int k = kb1 - 1; k >= kb0; --k) {    // suffix sums of the block totals
-            s_suf[k - kb0] = acc;
-            acc += cum[(size_t)k * kBlk + kBlk - 1];
+        for (int i = 0; i < 2 && i < nk; ++i) {
+            uint8_t *st = sm + i * kUsStage;
+            const int t0 = (kb0 + i) * kBlk;
+            mbar_arrive_expect_tx(bar + i, kUsStage);
+            tma_load_4d(st, &maps.B, bar + i, 0, g, t0, b);
+            tma_load_4d(st + kTileBytes, &maps.B, bar + i, 64, g, t0, b);
+            tma_load_4d(st + 2 * kTileBytes, &maps.x, bar + i, 0, h, t0, b);
         }
-        ws.ell[bh * U + u] = acc;
     }
+    // suffix: the unit's log decay after the current block (sum of later block totals)
+    float suffix = 0.f;
+    for (int k = kb0 + 1; k < kb1; ++k) suffix += cum[(size_t)k * kBlk + kBlk - 1];
+    if (tid == 0) ws.ell[bh * U + u] = suffix + cum[(size_t)kb0 * kBlk + kBlk - 1];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
     bool ok = true, range_ok = true;
-    uint32_t phase = 0;
+    uint32_t tma_par = 0, mma_par = 0;              // per-stage phase bits
     const uint32_t idesc = idesc_f16(128, 64, 1, 1);
     for (int k = kb0; k < kb1; ++k) {
-        const int t0 = k * kBlk;
-        {
-            const float e = cum[t0 + kBlk - 1] - cum[t0 + tid] + s_suf[k - kb0];
-            s_w[tid] = expf(fminf(e, 0.f)) * dtv[t0 + tid];
+        const int i = k - kb0, s = i & 1;
+        uint8_t *st = sm + s * kUsStage;
+        float *w = s_w + s * kBlk;
+        if (tid < kBlk) {
+            const float e = cum[(size_t)k * kBlk + kBlk - 1] - cum[(size_t)k * kBlk + tid] + suffix;
+            w[tid] = expf(fminf(e, 0.f)) * dtv[(size_t)k * kBlk + tid];
         }
-        __syncthreads();
-        for (int c = tid; c < kBlk * 16; c += kTcThreads) {
-            const int r = c >> 4, kk = c & 15, t = t0 + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < L) v = ldg16(Bm + (((size_t)b * L + t) * G + g) * kN + kk * 8);
-            *reinterpret_cast<uint4 *>(sB + (kk >> 3) * 16384 + sw128_off(r, kk & 7)) = cvt_chunk(v, range_ok);
-        }
-        for (int c = tid; c < kBlk * 8; c += kTcThreads) {
-            const int r = c >> 3, kk = c & 7, t = t0 + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < L) v = ldg16(x + (((size_t)b * L + t) * H + h) * kP + kk * 8);
-            *reinterpret_cast<uint4 *>(sWX + sw128_off(r, kk)) = cvt_chunk_scaled(v, s_w[r], range_ok);
+        if (k + 1 < kb1) suffix -= cum[(size_t)(k + 1) * kBlk + kBlk - 1];
+        ok = mbar_wait(bar + s, (tma_par >> s) & 1u, kWaitBudget);
+        tma_par ^= 1u << s;
+        __syncthreads();                            // w[] visible
+        // widen in place: B (2 tiles), X scaled by the w of its row (row = offset / 128)
+        for (int c = tid; c < 3 * 1024; c += kThreads) {
+            uint8_t *p = st + c * 16;
+            if (c < 2048) widen_chunk(p, range_ok);
+            else widen_chunk(p, w[(c - 2048) >> 3], range_ok);
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        ok = __syncthreads_and(ok);
         tc_fence_after();
-        if (tid == 0) {
-            const uint32_t b_base = smem_u32(sB), w_base = smem_u32(sWX);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                mma_f16(tmem, sdesc_sw128(b_base + s * 2048, 16384, 1024), sdesc_sw128(w_base + s * 2048, 16384, 1024),
-                        idesc, (k > kb0 || s > 0) ? 1u : 0u);
-            mma_commit(mbar);
-        }
-        ok = __syncthreads_and(mbar_wait(mbar, phase, kWaitBudget));
-        phase ^= 1u;
         if (!ok) break;
-        tc_fence_after();
+        if (tid == 0) {
+            const uint32_t b_base = smem_u32(st), x_base = smem_u32(st + 2 * kTileBytes);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                mma_f16(tmem, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
+                        sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc, (i > 0 || q > 0) ? 1u : 0u);
+            mma_commit(bar + 2 + s);
+            // refill this stage with block k+2 once these MMAs have read it
+            if (k + 2 < kb1) {
+                const bool done = mbar_wait(bar + 2 + s, (mma_par >> s) & 1u, kWaitBudget);
+                mma_par ^= 1u << s;
+                if (done) {
+                    const int t0 = (k + 2) * kBlk;
+                    mbar_arrive_expect_tx(bar + s, kUsStage);
+                    tma_load_4d(st, &maps.B, bar + s, 0, g, t0, b);
+                    tma_load_4d(st + kTileBytes, &maps.B, bar + s, 64, g, t0, b);
+                    tma_load_4d(st + 2 * kTileBytes, &maps.x, bar + s, 0, h, t0, b);
+                } else {
+                    flag_status(ws.status, kStatusTimeout);
+                }
+            }
+        }
     }
+    // wait for the last block's MMAs (the stage it used still has that commit pending)
+    if (ok && tid == 0 && nk > 0) {
+        const int s = (nk - 1) & 1;
+        ok = mbar_wait(bar + 2 + s, (mma_par >> s) & 1u, kWaitBudget);
+    }
+    ok = __syncthreads_and(ok);
+    tc_fence_after();
     if (!ok) {
         if (tid == 0) flag_status(ws.status, kStatusTimeout);
     } else {
-        float *dst = ws.states + (bh * U + u) * (size_t)kNP + (size_t)tid * kP;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        // 8 warps: lanes 32*(warp%4).., columns 32*(warp/4)..
+        const int n = 32 * (warp & 3) + (tid & 31), ch = warp >> 2;
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ch * 32, v);
+        float *dst = ws.states + (bh * U + u) * (size_t)kNP + (size_t)n * kP + ch * 32;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(lane_addr + half * 32, v);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4 *>(dst + half * 32 + 4 * q) =
-                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
     if (!__syncthreads_and(range_ok) && tid == 0) flag_status(ws.status, kStatusRange);
     tc_fence_before();
@@ -276,45 +330,68 @@ unit_state_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__re
 }
 
 // ---------------------------------------------------------------------------
-// state_pass: grid (N*P/256, H, b), 256 threads.
+// state_pass: grid (N*P/4/256, H, b), 256 threads; each thread owns one
+// float4 of the state and issues its loads for a batch of units before the
+// serial combine.
+constexpr int kSpBatch = 8;
+
 __global__ void __launch_bounds__(256)
 tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
-    const int e = blockIdx.x * 256 + threadIdx.x;
+    const int e4 = blockIdx.x * 256 + threadIdx.x;
     const size_t bh = (size_t)blockIdx.z * H + blockIdx.y;
-    float hs = init ? init[bh * kNP + e] : 0.f;
-    float *S = ws.states + bh * (size_t)U * kNP + e;
+    float4 hs = init ? reinterpret_cast<const float4 *>(init + bh * kNP)[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 *S = reinterpret_cast<float4 *>(ws.states + bh * (size_t)U * kNP) + e4;
     const float *ell = ws.ell + bh * U;
-    for (int u = 0; u + 1 < U; ++u) {
-        const float s = S[(size_t)u * kNP];
-        S[(size_t)u * kNP] = hs;                  // state entering unit u
-        hs = fmaf(expf(fminf(ell[u], 0.f)), hs, s);
+    for (int u0 = 0; u0 + 1 < U; u0 += kSpBatch) {
+        const int n = min(kSpBatch, U - 1 - u0);
+        float4 s[kSpBatch];
+        float a[kSpBatch];
+#pragma unroll
+        for (int i = 0; i < kSpBatch; ++i) {
+            if (i < n) {
+                s[i] = S[(size_t)(u0 + i) * (kNP / 4)];
+                a[i] = expf(fminf(ell[u0 + i], 0.f));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kSpBatch; ++i) {
+            if (i < n) {
+                S[(size_t)(u0 + i) * (kNP / 4)] = hs;   // state entering unit u0+i
+                hs.x = fmaf(a[i], hs.x, s[i].x);
+                hs.y = fmaf(a[i], hs.y, s[i].y);
+                hs.z = fmaf(a[i], hs.z, s[i].z);
+                hs.w = fmaf(a[i], hs.w, s[i].w);
+            }
+        }
     }
-    S[(size_t)(U - 1) * kNP] = hs;
+    S[(size_t)(U - 1) * (kNP / 4)] = hs;
 }
 
 // ---------------------------------------------------------------------------
-// chunk_out: grid (H, U, b), 128 threads, 2 CTAs per SM.
-constexpr size_t kCoSmem = 1024 + 32768 * 2 + 16384 * 2 + 2 * kBlk * 4 + 64;
+// chunk_out: grid (H, U, b), 256 threads, 2 CTAs per SM.
+constexpr size_t kCoSmem = 1024 + 6 * kTileBytes + 3 * kBlk * 4 + 64;
 
-__global__ void __launch_bounds__(kTcThreads, 2)
-chunk_out_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Bm,
-                 const __nv_bfloat16 *__restrict__ Cm, const float *__restrict__ D,
-                 const float *__restrict__ init, float *__restrict__ y, float *__restrict__ final_state, TcWs ws,
-                 int L, int H, int G, int nblk, int U, int bpu, int states_from_ws) {
+__global__ void __launch_bounds__(kThreads, 2)
+chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
+                 const float *__restrict__ init, float *__restrict__ final_state, TcWs ws, int L, int H, int G,
+                 int nblk, int U, int bpu, int states_from_ws) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint8_t *sCW = sm;                      // C tile [128 i][128 n], then W tile [128 i][128 j]
-    uint8_t *sB = sm + 32768;               // B tile [128 j][128 n]
-    uint8_t *sX = sm + 65536;               // X tile [128 j][64 p]
-    uint8_t *sHW = sm + 81920;              // fp16 state [128 n][64 p], then w.X [128 j][64 p]
-    float *s_dt = reinterpret_cast<float *>(sm + 98304);
+    uint8_t *sCW = sm;                              // C tile -> W tile -> y staging (2 tiles)
+    uint8_t *sB = sm + 2 * kTileBytes;              // B tile (2 tiles)
+    uint8_t *sX = sm + 4 * kTileBytes;              // X tile
+    uint8_t *sHW = sm + 5 * kTileBytes;             // fp16 state [n][p], then w.X [j][p]
+    float *s_dt = reinterpret_cast<float *>(sm + 6 * kTileBytes);
     float *s_cum = s_dt + kBlk;
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_cum + kBlk);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(mbar + 1);
+    float *s_w = s_cum + kBlk;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(s_w + kBlk);    // [0] TMA, [1] MMA
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 2);
 
     const int h = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int g = h / (H / G);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row = 32 * (warp & 3) + lane;         // TMEM lane / tile row of this thread
+    const int ch = warp >> 2;                       // which 32-column half it handles
     const size_t bh = (size_t)b * H + h;
     const int kb0 = u * bpu, kb1 = min(nblk, kb0 + bpu);
     const float *cum = ws.cum + bh * (size_t)nblk * kBlk;
@@ -325,102 +402,101 @@ chunk_out_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__res
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(mbar, 1);
+        mbar_init(bar, 1);
+        mbar_init(bar + 1, 1);
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const uint32_t tH = 0, tZ = 64, tCB = 128;   // TMEM columns: state, C.H, C.B^T then Y
     bool range_ok = true;
 
-    // state entering the unit -> TMEM (fp32) and sHW (fp16); thread tid owns row n = tid
+    // state entering the unit -> TMEM (fp32) and sHW (fp16): row n = `row`, columns 32*ch..
     {
         const float *src = states_from_ws ? ws.states + (bh * U + u) * (size_t)kNP
                                           : (init ? init + bh * kNP : nullptr);
+        float v[32];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float v[32];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float4 f = src ? *reinterpret_cast<const float4 *>(src + (size_t)tid * kP + half * 32 + 4 * q)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
-            }
-            tmem_st32(lane_addr + tH + half * 32, v);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(sHW + sw128_off(tid, half * 4 + q)) = pack8(v + 8 * q, range_ok);
+        for (int q = 0; q < 8; ++q) {
+            const float4 f = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kP + ch * 32 + 4 * q)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
         }
+        tmem_st32(lane_addr + tH + ch * 32, v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, range_ok);
     }
 
     bool ok = true;
-    uint32_t phase = 0;
+    uint32_t tma_par = 0, mma_par = 0;
     const uint32_t idesc_z = idesc_f16(128, 64, 0, 1);    // A=C K-major, B=H MN-major
     const uint32_t idesc_cb = idesc_f16(128, 128, 0, 0);  // A=C K-major, B=B K-major
     const uint32_t idesc_y = idesc_f16(128, 64, 0, 1);    // A=W K-major, B=X MN-major
     const uint32_t idesc_s = idesc_f16(128, 64, 1, 1);    // A=B^T MN-major, B=wX MN-major
     const float Dh = D[h];
 
-    for (int k = kb0; k < kb1 && ok; ++k) {
+    for (int k = kb0; k < kb1; ++k) {
         const int t0 = k * kBlk;
-        s_dt[tid] = dtv[t0 + tid];
-        s_cum[tid] = cum[t0 + tid];
-        for (int c = tid; c < kBlk * 16; c += kTcThreads) {
-            const int r = c >> 4, kk = c & 15, t = t0 + r;
-            uint4 vc = make_uint4(0u, 0u, 0u, 0u), vb = vc;
-            if (t < L) {
-                const size_t off = (((size_t)b * L + t) * G + g) * kN + kk * 8;
-                vc = ldg16(Cm + off);
-                vb = ldg16(Bm + off);
-            }
-            const uint32_t o = (kk >> 3) * 16384 + sw128_off(r, kk & 7);
-            *reinterpret_cast<uint4 *>(sCW + o) = cvt_chunk(vc, range_ok);
-            *reinterpret_cast<uint4 *>(sB + o) = cvt_chunk(vb, range_ok);
+        if (tid == 0) {
+            tma_store_wait_read();                 // the previous y store has left sCW
+            mbar_arrive_expect_tx(bar, 5 * kTileBytes);
+            tma_load_4d(sCW, &maps.C, bar, 0, g, t0, b);
+            tma_load_4d(sCW + kTileBytes, &maps.C, bar, 64, g, t0, b);
+            tma_load_4d(sB, &maps.B, bar, 0, g, t0, b);
+            tma_load_4d(sB + kTileBytes, &maps.B, bar, 64, g, t0, b);
+            tma_load_4d(sX, &maps.x, bar, 0, h, t0, b);
         }
-        for (int c = tid; c < kBlk * 8; c += kTcThreads) {
-            const int r = c >> 3, kk = c & 7, t = t0 + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < L) v = ldg16(x + (((size_t)b * L + t) * H + h) * kP + kk * 8);
-            *reinterpret_cast<uint4 *>(sX + sw128_off(r, kk)) = cvt_chunk(v, range_ok);
-        }
+        if (tid < kBlk) s_dt[tid] = dtv[(size_t)t0 + tid];
+        else s_cum[tid - kBlk] = cum[(size_t)t0 + tid - kBlk];
+        ok = mbar_wait(bar, tma_par, kWaitBudget);
+        tma_par ^= 1u;
+        __syncthreads();                           // s_dt, s_cum visible
+        // decay to the block's last real token (padding carries dA = 0 but its
+        // cumsum may round differently)
+        const float clast = s_cum[min(kBlk - 1, L - 1 - t0)];
+        if (tid < kBlk) s_w[tid] = expf(fminf(clast - s_cum[tid], 0.f)) * s_dt[tid];
+        for (int c = tid; c < 5 * 1024; c += kThreads) widen_chunk(sm + c * 16, range_ok);
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        ok = __syncthreads_and(ok);
         tc_fence_after();
+        if (!ok) break;
 
         if (tid == 0) {
             const uint32_t c_base = smem_u32(sCW), b_base = smem_u32(sB), h_base = smem_u32(sHW);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint64_t ad = sdesc_sw128(c_base + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024);
-                mma_f16(tmem + tZ, ad, sdesc_sw128(h_base + s * 2048, 16384, 1024), idesc_z, s > 0);
-                mma_f16(tmem + tCB, ad, sdesc_sw128(b_base + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), idesc_cb,
-                        s > 0);
+            for (int q = 0; q < 8; ++q) {
+                const uint64_t ad = sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024);
+                mma_f16(tmem + tZ, ad, sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_z, q > 0);
+                mma_f16(tmem + tCB, ad, sdesc_sw128(b_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
+                        idesc_cb, q > 0);
             }
-            mma_commit(mbar);
+            mma_commit(bar + 1);
         }
-        ok = __syncthreads_and(mbar_wait(mbar, phase, kWaitBudget));
-        phase ^= 1u;
+        ok = __syncthreads_and(mbar_wait(bar + 1, mma_par, kWaitBudget));
+        mma_par ^= 1u;
         if (!ok) break;
         tc_fence_after();
 
-        // W row i = tid (K-major over j), w.X row j = tid, state scaled by the block decay
+        // W (row `row`, columns 64*ch..64*ch+63) into sCW; w.X into sHW; the
+        // state scaled by the block decay
         {
-            const int i = tid;
-            const float ci = s_cum[i];
+            const float ci = s_cum[row];
 #pragma unroll
-            for (int c32 = 0; c32 < 4; ++c32) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c32 = 2 * ch + cc;
                 uint4 out[4];
-                if (c32 <= warp) {                       // warp-uniform: rows 32w.. see columns < 32(w+1)
+                if (c32 <= (warp & 3)) {                 // warp-uniform causal skip
                     float v[32];
                     tmem_ld32(lane_addr + tCB + c32 * 32, v);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = c32 * 32 + jj;
-                        v[jj] = (j <= i) ? v[jj] * expf(fminf(ci - s_cum[j], 0.f)) * s_dt[j] : 0.f;
+                        v[jj] = (j <= row) ? v[jj] * expf(fminf(ci - s_cum[j], 0.f)) * s_dt[j] : 0.f;
                     }
 #pragma unroll
                     for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, range_ok);
@@ -430,28 +506,25 @@ chunk_out_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__res
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(sCW + (c32 >> 1) * 16384 + sw128_off(i, (c32 & 1) * 4 + q)) = out[q];
+                    *reinterpret_cast<uint4 *>(sCW + ch * kTileBytes + sw128_off(row, cc * 4 + q)) = out[q];
             }
-            const float clast = s_cum[kBlk - 1];
-            const float wj = expf(fminf(clast - s_cum[tid], 0.f)) * s_dt[tid];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(tid, q));
-                float f[8];
+            for (int r = 0; r < 4; ++r) {                // 1024 chunks of w.X
+                const int c = tid + r * kThreads;
+                const int j = c >> 3, q = c & 7;
+                const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(j, q));
+                const float wj = s_w[j];
                 const float2 a0 = unpack_h2(xv.x), a1 = unpack_h2(xv.y), a2 = unpack_h2(xv.z), a3 = unpack_h2(xv.w);
-                f[0] = wj * a0.x; f[1] = wj * a0.y; f[2] = wj * a1.x; f[3] = wj * a1.y;
-                f[4] = wj * a2.x; f[5] = wj * a2.y; f[6] = wj * a3.x; f[7] = wj * a3.y;
-                *reinterpret_cast<uint4 *>(sHW + sw128_off(tid, q)) = pack8(f, range_ok);
+                const float f[8] = {wj * a0.x, wj * a0.y, wj * a1.x, wj * a1.y,
+                                    wj * a2.x, wj * a2.y, wj * a3.x, wj * a3.y};
+                *reinterpret_cast<uint4 *>(sHW + sw128_off(j, q)) = pack8(f, range_ok);
             }
             const float decay = expf(fminf(clast, 0.f));
+            float v[32];
+            tmem_ld32(lane_addr + tH + ch * 32, v);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-                tmem_ld32(lane_addr + tH + half * 32, v);
-#pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] *= decay;
-                tmem_st32(lane_addr + tH + half * 32, v);
-            }
+            for (int q = 0; q < 32; ++q) v[q] *= decay;
+            tmem_st32(lane_addr + tH + ch * 32, v);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -462,71 +535,67 @@ chunk_out_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__res
             const uint32_t w_base = smem_u32(sCW), x_base = smem_u32(sX), b_base = smem_u32(sB),
                            wx_base = smem_u32(sHW);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                mma_f16(tmem + tCB, sdesc_sw128(w_base + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                        sdesc_sw128(x_base + s * 2048, 16384, 1024), idesc_y, s > 0);
-                mma_f16(tmem + tH, sdesc_sw128(b_base + s * 2048, 16384, 1024),
-                        sdesc_sw128(wx_base + s * 2048, 16384, 1024), idesc_s, 1u);
+            for (int q = 0; q < 8; ++q) {
+                mma_f16(tmem + tCB, sdesc_sw128(w_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
+                        sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc_y, q > 0);
+                mma_f16(tmem + tH, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
+                        sdesc_sw128(wx_base + q * 2048, kTileBytes, 1024), idesc_s, 1u);
             }
-            mma_commit(mbar);
+            mma_commit(bar + 1);
         }
-        ok = __syncthreads_and(mbar_wait(mbar, phase, kWaitBudget));
-        phase ^= 1u;
+        ok = __syncthreads_and(mbar_wait(bar + 1, mma_par, kWaitBudget));
+        mma_par ^= 1u;
         if (!ok) break;
         tc_fence_after();
 
-        // y_i = Y_i + exp(cum_i) Z_i + D x_i ; next block's fp16 state
+        // y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging (sCW, two 32-column
+        // fp32 tiles) -> TMA store; the next block's fp16 state into sHW
         {
-            const int i = tid, t = t0 + i;
-            const float ei = expf(fminf(s_cum[i], 0.f));
-            float *yrow = y + (((size_t)b * L + t) * H + h) * kP;
+            const float ei = expf(fminf(s_cum[row], 0.f));
+            float yv[32], zv[32];
+            tmem_ld32(lane_addr + tCB + ch * 32, yv);
+            tmem_ld32(lane_addr + tZ + ch * 32, zv);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float yv[32], zv[32];
-                tmem_ld32(lane_addr + tCB + half * 32, yv);
-                tmem_ld32(lane_addr + tZ + half * 32, zv);
+            for (int q = 0; q < 4; ++q) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(row, ch * 4 + q));
+                const float2 a0 = unpack_h2(xv.x), a1 = unpack_h2(xv.y), a2 = unpack_h2(xv.z), a3 = unpack_h2(xv.w);
+                const float xs[8] = {a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(i, half * 4 + q));
-                    const float2 a0 = unpack_h2(xv.x), a1 = unpack_h2(xv.y), a2 = unpack_h2(xv.z),
-                                 a3 = unpack_h2(xv.w);
-                    const float xs[8] = {a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int p = q * 8 + e;
-                        yv[p] = fmaf(Dh, xs[e], fmaf(ei, zv[p], yv[p]));
-                    }
-                }
-                if (t < L) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        *reinterpret_cast<float4 *>(yrow + half * 32 + 4 * q) =
-                            make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
+                for (int e = 0; e < 8; ++e) {
+                    const int p = q * 8 + e;
+                    yv[p] = fmaf(Dh, xs[e], fmaf(ei, zv[p], yv[p]));
                 }
             }
+            uint8_t *stg = sCW + ch * kTileBytes;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4 *>(stg + sw128_off(row, q)) =
+                    make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
             const bool last = (k + 1 == kb1);
+            float v[32];
+            tmem_ld32(lane_addr + tH + ch * 32, v);
+            if (!last) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-                tmem_ld32(lane_addr + tH + half * 32, v);
-                if (!last) {
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, range_ok);
+            } else if (final_state && u == U - 1) {
+                float *dst = final_state + bh * kNP + (size_t)row * kP + ch * 32;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4 *>(sHW + sw128_off(tid, half * 4 + q)) = pack8(v + 8 * q, range_ok);
-                } else if (final_state && u == U - 1) {
-                    float *dst = final_state + bh * kNP + (size_t)tid * kP + half * 32;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        *reinterpret_cast<float4 *>(dst + 4 * q) =
-                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                }
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == 0) {
+            tma_store_4d(&maps.y, sCW, 0, h, t0, b);
+            tma_store_4d(&maps.y, sCW + kTileBytes, 32, h, t0, b);
+            tma_store_commit();
+        }
     }
+    if (tid == 0) tma_store_wait_all();
     if (!ok && tid == 0) flag_status(ws.status, kStatusTimeout);
     if (!__syncthreads_and(range_ok) && tid == 0) flag_status(ws.status, kStatusRange);
     tc_fence_before();
@@ -539,16 +608,19 @@ chunk_out_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__res
 bool tc_supported(const ScanDims &d, int bf16) {
     if (!bf16 || d.N != kN || d.P != kP) return false;
     if (d.Q != 64 && d.Q != 128 && d.Q != 256) return false;
-    if (d.H > 65535 || d.b > 65535) return false;
+    if (d.H > 65535 || d.b > 65535 || d.L > 0x7fffffffll - kBlk) return false;
     const TcPlan p = make_plan(d);
-    return p.U <= 65535 && p.nblk <= 0x7fffffff && p.bpu <= 4096;
+    return p.U <= 65535;
 }
 
 size_t tc_workspace_bytes(const ScanDims &d) { return ws_bytes(d, make_plan(d)); }
 
 cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) {
     const TcPlan p = make_plan(d);
+    if (p.nblk == 0) return cudaSuccess;
     TcWs ws = carve(d, p, wsp);
+    TcMaps maps;
+    if (!make_maps(a, d, &maps)) return cudaErrorInvalidValue;
     cudaError_t e;
     static bool attr_done = false;
     if (!attr_done) {
@@ -560,9 +632,6 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
             return e;
         attr_done = true;
     }
-    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(a.x);
-    const __nv_bfloat16 *Bm = static_cast<const __nv_bfloat16 *>(a.B);
-    const __nv_bfloat16 *Cm = static_cast<const __nv_bfloat16 *>(a.C);
     {
         TraceScope tr(s, kTrTcDtPrep);
         dt_prep_kernel<<<dim3((unsigned)p.nblk, (unsigned)((d.H + 31) / 32), (unsigned)d.b), 256, 0, s>>>(
@@ -572,22 +641,22 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     if (p.U > 1) {
         {
             TraceScope tr(s, kTrTcUnitState);
-            unit_state_kernel<<<dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kTcThreads, kUsSmem, s>>>(
-                x, Bm, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu);
+            unit_state_kernel<<<dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kThreads, kUsSmem, s>>>(
+                maps, ws, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         {
             TraceScope tr(s, kTrTcStatePass);
-            tc_state_pass_kernel<<<dim3(kNP / 256, (unsigned)d.H, (unsigned)d.b), 256, 0, s>>>(ws, a.init_state,
-                                                                                               (int)d.H, (int)p.U);
+            tc_state_pass_kernel<<<dim3(kNP / 4 / 256, (unsigned)d.H, (unsigned)d.b), 256, 0, s>>>(
+                ws, a.init_state, (int)d.H, (int)p.U);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
         TraceScope tr(s, kTrTcChunkOut);
-        chunk_out_kernel<<<dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kTcThreads, kCoSmem, s>>>(
-            x, Bm, Cm, a.D, a.init_state, a.y, a.final_state, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk,
-            (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0);
+        chunk_out_kernel<<<dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kThreads, kCoSmem, s>>>(
+            maps, a.D, a.init_state, a.final_state, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U,
+            (int)p.bpu, p.U > 1 ? 1 : 0);
     }
     return cudaGetLastError();
 }

@@ -16,6 +16,17 @@ def tol_for(dtype) -> float:
     return TOL_F32 if dtype in (torch.float32, "f32") else TOL_BF16
 
 
+def path_supported(inp, chunk_size, path) -> bool:
+    """Whether the library accepts this shape on this path (host-side query)."""
+    b, L, H, P = inp["x"].shape
+    G, N = inp["B"].shape[2], inp["B"].shape[3]
+    try:
+        ssd.workspace_size(b, L, H, P, N, G, chunk_size, inp["x"].dtype, path)
+        return True
+    except ssd.SSDError:
+        return False
+
+
 def to_dev(inp, device="cuda"):
     return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
 

@@ -13,13 +13,14 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import TOL_BF16, TOL_F32, compare, run_scan, sample_chains, tol_for
+from gpu_helpers import TOL_BF16, TOL_F32, compare, path_supported, run_scan, sample_chains, tol_for
 from state_space_sequence_scan_b200 import ssd
 from state_space_sequence_scan_b200.inputs import SCAN_CONFIGS, ScanConfig, make_scan_inputs
 
 pytestmark = pytest.mark.gpu
 
-PATHS = ["auto", "simt"]
+PATHS = ["auto", "simt", "tensor"]
+BF16_PATHS = ["simt", "tensor"]
 
 
 def _oracle(inp, dt_limit=(0.0, math.inf)):
@@ -28,6 +29,8 @@ def _oracle(inp, dt_limit=(0.0, math.inf)):
 
 
 def _check(inp, Q, path, dt_limit=(0.0, math.inf), what=""):
+    if not path_supported(inp, Q, path):
+        pytest.skip("the %s path does not cover this shape/dtype" % path)
     y, fs = run_scan(inp, Q, path=path, dt_limit=dt_limit)
     yr, fr = _oracle(inp, dt_limit)
     tol = tol_for(inp["x"].dtype)
@@ -64,27 +67,30 @@ def test_small_parity(case, path):
     _check(make_scan_inputs(cfg), Q, path, what=str(case))
 
 
-def test_dt_limit_clamp():
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_dt_limit_clamp(path):
     cfg = ScanConfig("clamp", 2, 300, 4, 64, 128, 2, 64, "bf16", "ones", "normal", seed=11)
     inp = make_scan_inputs(cfg)
-    _check(inp, 64, "auto", dt_limit=(0.02, 0.3), what="clamp")
+    _check(inp, 64, path, dt_limit=(0.02, 0.3), what="clamp")
 
 
-def test_c1_130m_full():
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_c1_130m_full(path):
     cfg = SCAN_CONFIGS["c1_130m"]
-    _check(make_scan_inputs(cfg), cfg.chunk_size, "auto", what=cfg.name)
+    _check(make_scan_inputs(cfg), cfg.chunk_size, path, what=cfg.name)
 
 
+@pytest.mark.parametrize("path", BF16_PATHS)
 @pytest.mark.parametrize("name,chains", [
     ("c2_2p7b", [(0, 0), (3, 41), (7, 79), (5, 17)]),
     ("c3_long", [(0, 0), (0, 37), (0, 79)]),
 ])
-def test_full_size_sampled_chains(name, chains):
+def test_full_size_sampled_chains(name, chains, path):
     """The kernels run on the whole workload (the launch the benchmark times);
     the oracle evaluates the sampled chains alone."""
     cfg = SCAN_CONFIGS[name]
     inp = make_scan_inputs(cfg)
-    y, fs = run_scan(inp, cfg.chunk_size, path="auto")
+    y, fs = run_scan(inp, cfg.chunk_size, path=path)
     assert np.isfinite(y).all() and np.isfinite(fs).all()
     H, G = cfg.nheads, cfg.ngroups
     for (bi, h), sub in zip(chains, sample_chains(inp, chains)):
@@ -106,16 +112,17 @@ def test_chunk_size_invariance_fp32():
         compare(f, f0, TOL_F32, "final_state across chunk sizes")
 
 
-def test_split_and_carry():
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_split_and_carry(path):
     cfg = ScanConfig("split", 2, 1000, 4, 64, 128, 1, 128, "bf16", "ones", "normal", seed=6)
     inp = make_scan_inputs(cfg)
-    y, fs = run_scan(inp, 128)
+    y, fs = run_scan(inp, 128, path=path)
     T1 = 389
     first = {k: (v[:, :T1] if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
-    y1, h1 = run_scan(first, 128)
+    y1, h1 = run_scan(first, 128, path=path)
     second = {k: (v[:, T1:] if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
     second["init_state"] = torch.from_numpy(h1).float()
-    y2, h2 = run_scan(second, 128)
+    y2, h2 = run_scan(second, 128, path=path)
     yr, fr = _oracle(inp)
     compare(np.concatenate([y1, y2], axis=1), yr, TOL_BF16, "split y")
     compare(h2, fr, TOL_BF16, "split final_state")
@@ -137,34 +144,37 @@ def test_skip_token():
     compare(fs, fc, TOL_F32, "skip final_state")
 
 
-def test_memoryless_and_nonfinite_guard():
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_memoryless_and_nonfinite_guard(path):
     """Huge |A| and dt >= 0.01: every exponent underflows to 0; output must
     stay finite and equal dt_t (C_t.B_t) x_t + D x_t."""
     cfg = ScanConfig("memless", 1, 600, 4, 64, 128, 1, 256, "bf16", "ones", "normal", seed=8)
     inp = make_scan_inputs(cfg)
     inp["A"][:] = -1.0e5
-    y, fs = run_scan(inp, 256, dt_limit=(0.01, math.inf))
+    y, fs = run_scan(inp, 256, path=path, dt_limit=(0.01, math.inf))
     yr, fr = _oracle(inp, (0.01, math.inf))
     compare(y, yr, TOL_BF16, "memoryless y")
     compare(fs, fr, TOL_BF16, "memoryless final")
 
 
-def test_deterministic():
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_deterministic(path):
     cfg = SCAN_CONFIGS["c1_130m"].with_(seqlen=1024)
     inp = make_scan_inputs(cfg)
-    a = run_scan(inp, cfg.chunk_size)
-    b = run_scan(inp, cfg.chunk_size)
+    a = run_scan(inp, cfg.chunk_size, path=path)
+    b = run_scan(inp, cfg.chunk_size, path=path)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
-def test_groups_replicated_equal():
+@pytest.mark.parametrize("path", BF16_PATHS)
+def test_groups_replicated_equal(path):
     cfg = ScanConfig("grp", 1, 400, 4, 64, 128, 1, 128, "bf16", "ones", "normal", seed=9)
     inp = make_scan_inputs(cfg)
-    y1, f1 = run_scan(inp, 128)
+    y1, f1 = run_scan(inp, 128, path=path)
     rep = dict(inp)
     rep["B"] = inp["B"].repeat_interleave(4, dim=2).contiguous()
     rep["C"] = inp["C"].repeat_interleave(4, dim=2).contiguous()
-    y4, f4 = run_scan(rep, 128)
+    y4, f4 = run_scan(rep, 128, path=path)
     compare(y4, y1, 1e-6, "G=H vs G=1 y")
     compare(f4, f1, 1e-6, "G=H vs G=1 final")
 
@@ -211,3 +221,29 @@ def test_130m_shapes_match_pages():
     yr, fr = _oracle(inp)
     compare(y, yr, TOL_BF16, "130m 10-token y")
     compare(fs, fr, TOL_BF16, "130m 10-token final")
+
+
+@pytest.mark.parametrize("Q", [64, 128, 256])
+def test_tensor_path_chunk_sizes(Q):
+    """The tensor path over each chunk size it accepts, against the oracle."""
+    cfg = ScanConfig("tcq", 2, 3 * 256 + 77, 4, 64, 128, 2, Q, "bf16", "normal", "normal", seed=30 + Q)
+    _check(make_scan_inputs(cfg), Q, "tensor", what="tensor Q=%d" % Q)
+
+
+def test_tensor_path_units():
+    """Long sequences split into several units per (batch, head): the state
+    passed between units must equal the oracle's."""
+    cfg = ScanConfig("units", 1, 8192 + 45, 2, 64, 128, 1, 256, "bf16", "ones", "normal", seed=40)
+    _check(make_scan_inputs(cfg), 256, "tensor", what="tensor units")
+
+
+def test_tensor_path_range_guard():
+    """An input outside the fp16 operand range is reported, not silently wrong."""
+    cfg = ScanConfig("range", 1, 256, 2, 64, 128, 1, 128, "bf16", "ones", "zero", seed=41)
+    inp = make_scan_inputs(cfg)
+    inp["x"][0, 10, 0, 3] = 1.0e6
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    ws = ssd.alloc_workspace(ssd.workspace_size(1, 256, 2, 64, 128, 1, 128, torch.bfloat16, "tensor"), "cuda")
+    ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], chunk_size=128,
+                       path="tensor", workspace=ws)
+    assert ssd.read_device_status(ws) == 7
