@@ -125,6 +125,35 @@ SSD_API ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_
                     int64_t batch, int64_t nheads, int64_t head_dim, int64_t state_dim,
                     int64_t ngroups, float dt_lo, float dt_hi, int in_dtype, void *stream);
 
+/* ssd_chunk_scan_fwd without a caller-provided workspace.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- code that runs where cudaMalloc is forbidden or unsafe
+ * (inside a host callback, a plug-in of another runtime that owns every
+ * allocation, a memory-capped sandbox) or that is handed only its input and
+ * output buffers.  The scratch it needs lives in a fixed 32 MiB device array
+ * inside libssd.so, which every GPU that loads the library holds until the
+ * process exits.  Arguments are those of ssd_chunk_scan_fwd minus the
+ * workspace; inputs and outputs are still the caller's.
+ *   - Sizes whose workspace (ssd_chunk_scan_workspace_size) exceeds 32 MiB
+ *     are rejected with SSD_ERR_UNSUPPORTED before anything is enqueued.
+ *   - It never calls cudaMalloc, cudaFree or any allocating routine.
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents
+ *     (each call clears the part that must start at zero).  Calls whose work
+ *     overlaps on the GPU -- two streams, or two host threads -- race on it;
+ *     serialise them.
+ *   - The device status word sits in that array and is not read back here:
+ *     host-side errors come back as usual, device-side conditions
+ *     (SSD_ERR_PRECONDITION) are only visible through ssd_chunk_scan_fwd. */
+SSD_API ssd_status ssd_chunk_scan_fwd_noalloc(const void *x, const float *dt_raw, const float *dt_bias,
+                                      const float *A, const void *B, const void *C, const float *D,
+                                      const float *init_state, float *y, float *final_state,
+                                      int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                                      int64_t state_dim, int64_t ngroups, int64_t chunk_size,
+                                      float dt_lo, float dt_hi, int in_dtype, int path, void *stream);
+
 /* Waits for `stream`, then reads the device status word that the last
  * ssd_chunk_scan_fwd on this workspace left: SSD_OK, SSD_ERR_PRECONDITION or
  * SSD_ERR_DEVICE_TIMEOUT.  `workspace` is a device pointer. */

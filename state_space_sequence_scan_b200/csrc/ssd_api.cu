@@ -67,6 +67,14 @@ ssd::ScanDims make_dims(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, i
     return d;
 }
 
+}  // namespace
+
+namespace ssd {
+int record_cuda_error(cudaError_t e) { return (int)cuda_fail(e); }
+}  // namespace ssd
+
+namespace {
+
 size_t path_ws(const ssd::ScanDims &d, int chosen) {
     return chosen == SSD_PATH_TENSOR ? ssd::tc_workspace_bytes(d) : ssd::simt_workspace_bytes(d);
 }

@@ -33,6 +33,9 @@ struct StepArgs {
     int bf16;
 };
 
+// Records `e` as the last CUDA error of this host thread; returns SSD_ERR_CUDA (5).
+int record_cuda_error(cudaError_t e);
+
 // Workspace carve-up: [status | per-path regions], every region 256-byte aligned.
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
