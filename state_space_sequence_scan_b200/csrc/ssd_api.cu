@@ -38,7 +38,7 @@ ssd_status check_scan_dims(int64_t b, int64_t L, int64_t H, int64_t P, int64_t N
 }
 
 // SSD_PATH_AUTO picks the tensor-core path when this is set and the shape fits.
-constexpr bool kAutoTensor = false;
+constexpr bool kAutoTensor = true;
 
 // Resolves `path` for these sizes; SSD_ERR_UNSUPPORTED when nothing fits.
 ssd_status resolve_path(const ssd::ScanDims &d, int in_dtype, int path, int *chosen) {
