@@ -2,17 +2,19 @@
 //
 // Scope: bf16 x/B/C, state_dim N = 128, head_dim P = 64, fp32 dt/A/D/state,
 // fp32 y.  Every contraction runs as a kind::f16 MMA with fp16 operands and
-// fp32 accumulation in TMEM: the bf16 tiles arrive by TMA already in the
-// 128-byte-swizzled operand layout and are widened to fp16 in place (exact);
-// the decay-weighted operands are formed in fp16, whose 11-bit significand
-// the 2e-2 bar needs (bf16's 8 bits are not enough).
+// fp32 accumulation in TMEM.  bf16 -> fp16 is exact for inputs within fp16
+// range; the decay-weighted operands are formed in fp16, whose 11-bit
+// significand the 2e-2 bar needs (bf16's 8 bits are not enough).  Tiles
+// arrive by TMA already in the 128-byte-swizzled operand layout.
 //
 // The sequence of every (batch, head) is cut into 128-token blocks (the MMA
 // M extent) and the blocks into `units` of consecutive blocks.  Four
 // launches; no CTA ever waits on another CTA:
-//   dt_prep     dt = clamp(softplus(dt_raw + dt_bias)), dA = dt*A, and the
+//   prep        dt = clamp(softplus(dt_raw + dt_bias)), dA = dt*A, and the
 //               inclusive cumsum `cum` of dA inside every 128-token block
-//               (warp shuffles, fixed order), transposed to [b, H, L].
+//               (warp shuffles, fixed order), transposed to [b, H, L]; and an
+//               fp16 copy of B and C (zero-padded to whole blocks), made once
+//               per call because every head of a group reads them.
 //   unit_state  per (head, unit u < U-1, batch): the state the unit leaves
 //               when it starts from zero,
 //                 S'_u = sum_{j in u} exp(sum_{r=j+1..end(u)} dA_r) dt_j B_j x_j^T,
@@ -35,8 +37,11 @@
 // intra-chunk quadratic term evaluated on 128-token blocks and the state
 // carried on chip between them; it equals the token recurrence up to
 // rounding for any chunk size (nnterp guide "Mamba-2", "The state after every
-// token").  Exponents are only taken of min(., 0) after the causal select,
-// so none can overflow.
+// token").  Every exponent is of min(., 0), taken after the causal select,
+// so none can overflow.  Below the diagonal 32x32 sub-blocks the decay
+// factors through the row group's first row m:
+//   exp(cum_i - cum_j) = exp(cum_i - cum_m) * exp(cum_m - cum_j),  j <= m <= i,
+// both factors <= 1, so W there costs two multiplies instead of an exp.
 #include <stdint.h>
 
 #include "ssd_common.cuh"
@@ -62,10 +67,12 @@ constexpr uint32_t kTileBytes = 16384;          // one 128-row x 128-byte swizzl
 
 struct TcWs {
     unsigned *status;
-    float *dt;      // [b, H, nblk*128]
-    float *cum;     // [b, H, nblk*128]
-    float *ell;     // [b, H, U]
-    float *states;  // [b, H, U, N, P]
+    float *dt;       // [b, H, nblk*128]
+    float *cum;      // [b, H, nblk*128]
+    float *ell;      // [b, H, U]
+    float *states;   // [b, H, U, N, P]
+    __half *Bh;      // [b, nblk*128, G, N]  fp16 copy of B, zero rows past L
+    __half *Ch;      // [b, nblk*128, G, N]  fp16 copy of C
 };
 
 struct TcPlan {
@@ -93,6 +100,10 @@ TcPlan make_plan(const ScanDims &d) {
     return p;
 }
 
+size_t bc_bytes(const ScanDims &d, const TcPlan &p) {
+    return (size_t)d.b * p.nblk * kBlk * d.G * kN * sizeof(__half);
+}
+
 TcWs carve(const ScanDims &d, const TcPlan &p, void *ws) {
     char *c = static_cast<char *>(ws);
     TcWs w;
@@ -102,38 +113,40 @@ TcWs carve(const ScanDims &d, const TcPlan &p, void *ws) {
     w.dt = reinterpret_cast<float *>(c + off); off += align256(tok);
     w.cum = reinterpret_cast<float *>(c + off); off += align256(tok);
     w.ell = reinterpret_cast<float *>(c + off); off += align256((size_t)d.b * d.H * p.U * sizeof(float));
-    w.states = reinterpret_cast<float *>(c + off);
+    w.states = reinterpret_cast<float *>(c + off); off += align256((size_t)d.b * d.H * p.U * kNP * sizeof(float));
+    w.Bh = reinterpret_cast<__half *>(c + off); off += align256(bc_bytes(d, p));
+    w.Ch = reinterpret_cast<__half *>(c + off);
     return w;
 }
 
 size_t ws_bytes(const ScanDims &d, const TcPlan &p) {
     const size_t tok = (size_t)d.b * d.H * p.nblk * kBlk * sizeof(float);
     return kStatusBytes + 2 * align256(tok) + align256((size_t)d.b * d.H * p.U * sizeof(float)) +
-           align256((size_t)d.b * d.H * p.U * kNP * sizeof(float));
+           align256((size_t)d.b * d.H * p.U * kNP * sizeof(float)) + 2 * align256(bc_bytes(d, p));
 }
 
-// Tensor maps over [b, L, H|G, P|N] with 128-token boxes (4-D, innermost
-// first).  x, B, C: bf16 boxes of 64 x 1 x 128 x 1 (one 16 KB swizzled tile);
-// y: fp32 boxes of 32 x 1 x 128 x 1.
-bool make_maps(const ScanArgs &a, const ScanDims &d, TcMaps *m) {
-    const uint64_t b = d.b, L = d.L, H = d.H, G = d.G;
+// Tensor maps (4-D, innermost first) with 128-token boxes: x bf16 [b,L,H,P]
+// and the fp16 B/C copies [b,Lp,G,N] in 64 x 1 x 128 x 1 boxes (one 16 KB
+// swizzled tile); y fp32 [b,L,H,P] in 32 x 1 x 128 x 1 boxes.
+bool make_maps(const ScanArgs &a, const ScanDims &d, const TcPlan &p, const TcWs &w, TcMaps *m) {
+    const uint64_t b = d.b, L = d.L, H = d.H, G = d.G, Lp = p.nblk * kBlk;
     const uint32_t box_h[4] = {64, 1, kBlk, 1};
     const uint32_t box_y[4] = {32, 1, kBlk, 1};
     {
         const uint64_t dims[4] = {kP, H, L, b};
         const uint64_t st[3] = {kP * 2, H * kP * 2, L * H * kP * 2};
-        if (!tmap_encode_4d(&m->x, a.x, 2, dims, st, box_h)) return false;
+        if (!tmap_encode_4d(&m->x, a.x, kTmapBF16, dims, st, box_h)) return false;
     }
     {
-        const uint64_t dims[4] = {kN, G, L, b};
-        const uint64_t st[3] = {kN * 2, G * kN * 2, L * G * kN * 2};
-        if (!tmap_encode_4d(&m->B, a.B, 2, dims, st, box_h)) return false;
-        if (!tmap_encode_4d(&m->C, a.C, 2, dims, st, box_h)) return false;
+        const uint64_t dims[4] = {kN, G, Lp, b};
+        const uint64_t st[3] = {kN * 2, G * kN * 2, Lp * G * kN * 2};
+        if (!tmap_encode_4d(&m->B, w.Bh, kTmapF16, dims, st, box_h)) return false;
+        if (!tmap_encode_4d(&m->C, w.Ch, kTmapF16, dims, st, box_h)) return false;
     }
     {
         const uint64_t dims[4] = {kP, H, L, b};
         const uint64_t st[3] = {kP * 4, H * kP * 4, L * H * kP * 4};
-        if (!tmap_encode_4d(&m->y, a.y, 4, dims, st, box_y)) return false;
+        if (!tmap_encode_4d(&m->y, a.y, kTmapF32, dims, st, box_y)) return false;
     }
     return true;
 }
@@ -142,35 +155,55 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-__device__ __forceinline__ uint4 pack8(const float *f, bool &range_ok) {
+// 8 floats -> 8 fp16 (one 16-byte chunk); `amax` tracks the largest magnitude
+__device__ __forceinline__ uint4 pack8(const float *f, float &amax) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) range_ok &= fabsf(f[i]) <= kF16Max;
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
     return make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
 }
 
-// In place: one 16-byte chunk of 8 bf16, scaled by w, -> 8 fp16.
-__device__ __forceinline__ void widen_chunk(uint8_t *p, float w, bool &range_ok) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(p);
-    const float f[8] = {w * bf16lo(v.x), w * bf16hi(v.x), w * bf16lo(v.y), w * bf16hi(v.y),
-                        w * bf16lo(v.z), w * bf16hi(v.z), w * bf16lo(v.w), w * bf16hi(v.w)};
-    *reinterpret_cast<uint4 *>(p) = pack8(f, range_ok);
+__device__ __forceinline__ void bf16_chunk_to_f32(uint4 v, float *f) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
 }
 
-__device__ __forceinline__ void widen_chunk(uint8_t *p, bool &range_ok) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(p);
-    const float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
-                        bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
-    *reinterpret_cast<uint4 *>(p) = pack8(f, range_ok);
+__device__ __forceinline__ void f16_chunk_to_f32(uint4 v, float *f) {
+    const float2 a0 = unpack_h2(v.x), a1 = unpack_h2(v.y), a2 = unpack_h2(v.z), a3 = unpack_h2(v.w);
+    f[0] = a0.x; f[1] = a0.y; f[2] = a1.x; f[3] = a1.y; f[4] = a2.x; f[5] = a2.y; f[6] = a3.x; f[7] = a3.y;
 }
 
 // ---------------------------------------------------------------------------
-// dt_prep: grid (nblk, ceil(H/32), b), 256 threads.
+// prep: grid (nblk, ceil(H/32) + G, b), 256 threads.  y-slices below
+// ceil(H/32) do dt/cum for 32 heads; the rest convert B and C of one group.
 __global__ void __launch_bounds__(256)
-dt_prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
-               const float *__restrict__ A, TcWs ws, int L, int H, int nblk, float lo, float hi) {
+prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias, const float *__restrict__ A,
+            const __nv_bfloat16 *__restrict__ Bm, const __nv_bfloat16 *__restrict__ Cm, TcWs ws, int L, int H,
+            int G, int nblk, float lo, float hi) {
     __shared__ float s_dt[kBlk][33];
     __shared__ float s_da[kBlk][33];
-    const int blk = blockIdx.x, h0 = blockIdx.y * 32, b = blockIdx.z;
+    const int blk = blockIdx.x, b = blockIdx.z;
+    const int nhy = (H + 31) / 32;
+    if ((int)blockIdx.y >= nhy) {
+        const int g = blockIdx.y - nhy;
+        const int t0 = blk * kBlk;
+        const size_t Lp = (size_t)nblk * kBlk;
+        float amax = 0.f;
+#pragma unroll 4
+        for (int c = threadIdx.x; c < 2 * kBlk * 16; c += 256) {
+            const int which = c >> 11, r = (c >> 4) & (kBlk - 1), kk = c & 15;
+            const int t = t0 + r;
+            const __nv_bfloat16 *src = which ? Cm : Bm;
+            __half *dst = which ? ws.Ch : ws.Bh;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (t < L) v = __ldg(reinterpret_cast<const uint4 *>(src + (((size_t)b * L + t) * G + g) * kN + kk * 8));
+            float f[8];
+            bf16_chunk_to_f32(v, f);
+            *reinterpret_cast<uint4 *>(dst + (((size_t)b * Lp + t) * G + g) * kN + kk * 8) = pack8(f, amax);
+        }
+        if (!(amax <= kF16Max)) flag_status(ws.status, kStatusRange);
+        return;
+    }
+    const int h0 = blockIdx.y * 32;
     const int nh = min(32, H - h0);
     for (int e = threadIdx.x; e < kBlk * 32; e += 256) {
         const int tok = e >> 5, hh = e & 31;
@@ -207,7 +240,7 @@ dt_prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bi
 }
 
 // ---------------------------------------------------------------------------
-// unit_state: grid (H, U-1, b), 256 threads, two TMA stages of (B, X).
+// unit_state: grid (H, U-1, b), 256 threads, two TMA stages of (B fp16, X bf16).
 // Units 0..U-2 never hold the sequence's ragged tail (it is in the last
 // unit), so every block here is a full 128 tokens.
 constexpr uint32_t kUsStage = 3 * kTileBytes;                 // B (2 tiles) + X (1 tile)
@@ -255,7 +288,8 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    bool ok = true, range_ok = true;
+    bool ok = true;
+    float amax = 0.f;
     uint32_t tma_par = 0, mma_par = 0;              // per-stage phase bits
     const uint32_t idesc = idesc_f16(128, 64, 1, 1);
     for (int k = kb0; k < kb1; ++k) {
@@ -270,11 +304,18 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
         ok = mbar_wait(bar + s, (tma_par >> s) & 1u, kWaitBudget);
         tma_par ^= 1u << s;
         __syncthreads();                            // w[] visible
-        // widen in place: B (2 tiles), X scaled by the w of its row (row = offset / 128)
-        for (int c = tid; c < 3 * 1024; c += kThreads) {
-            uint8_t *p = st + c * 16;
-            if (c < 2048) widen_chunk(p, range_ok);
-            else widen_chunk(p, w[(c - 2048) >> 3], range_ok);
+        // X (bf16) -> w.X (fp16) in place; the row of a chunk is offset / 128
+        uint8_t *sx = st + 2 * kTileBytes;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int c = tid + r * kThreads;
+            uint4 *p = reinterpret_cast<uint4 *>(sx + c * 16);
+            float f[8];
+            bf16_chunk_to_f32(*p, f);
+            const float wr = w[c >> 3];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= wr;
+            *p = pack8(f, amax);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -282,7 +323,7 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
         tc_fence_after();
         if (!ok) break;
         if (tid == 0) {
-            const uint32_t b_base = smem_u32(st), x_base = smem_u32(st + 2 * kTileBytes);
+            const uint32_t b_base = smem_u32(st), x_base = smem_u32(sx);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 mma_f16(tmem, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
@@ -323,7 +364,7 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
         for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
-    if (!__syncthreads_and(range_ok) && tid == 0) flag_status(ws.status, kStatusRange);
+    if (!__syncthreads_and(amax <= kF16Max) && tid == 0) flag_status(ws.status, kStatusRange);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
@@ -369,7 +410,7 @@ tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
 
 // ---------------------------------------------------------------------------
 // chunk_out: grid (H, U, b), 256 threads, 2 CTAs per SM.
-constexpr size_t kCoSmem = 1024 + 6 * kTileBytes + 3 * kBlk * 4 + 64;
+constexpr size_t kCoSmem = 1024 + 6 * kTileBytes + (3 * kBlk + 3 * kBlk) * 4 + 64;
 
 __global__ void __launch_bounds__(kThreads, 2)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
@@ -384,13 +425,15 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     float *s_dt = reinterpret_cast<float *>(sm + 6 * kTileBytes);
     float *s_cum = s_dt + kBlk;
     float *s_w = s_cum + kBlk;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(s_w + kBlk);    // [0] TMA, [1] MMA
+    float *s_v = s_w + kBlk;                        // [3][128] pivot factors for row groups 1..3
+    uint64_t *bar = reinterpret_cast<uint64_t *>(s_v + 3 * kBlk);  // [0] TMA, [1] MMA
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 2);
 
     const int h = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int g = h / (H / G);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int row = 32 * (warp & 3) + lane;         // TMEM lane / tile row of this thread
+    const int w4 = warp & 3;                        // row group: rows 32*w4 .. 32*w4+31
+    const int row = 32 * w4 + lane;                 // TMEM lane / tile row of this thread
     const int ch = warp >> 2;                       // which 32-column half it handles
     const size_t bh = (size_t)b * H + h;
     const int kb0 = u * bpu, kb1 = min(nblk, kb0 + bpu);
@@ -410,9 +453,9 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * w4) << 16);
     const uint32_t tH = 0, tZ = 64, tCB = 128;   // TMEM columns: state, C.H, C.B^T then Y
-    bool range_ok = true;
+    float amax = 0.f;
 
     // state entering the unit -> TMEM (fp32) and sHW (fp16): row n = `row`, columns 32*ch..
     {
@@ -428,7 +471,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         tmem_st32(lane_addr + tH + ch * 32, v);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, range_ok);
+            *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, amax);
     }
 
     bool ok = true;
@@ -452,14 +495,26 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         }
         if (tid < kBlk) s_dt[tid] = dtv[(size_t)t0 + tid];
         else s_cum[tid - kBlk] = cum[(size_t)t0 + tid - kBlk];
-        ok = mbar_wait(bar, tma_par, kWaitBudget);
-        tma_par ^= 1u;
         __syncthreads();                           // s_dt, s_cum visible
         // decay to the block's last real token (padding carries dA = 0 but its
         // cumsum may round differently)
         const float clast = s_cum[min(kBlk - 1, L - 1 - t0)];
         if (tid < kBlk) s_w[tid] = expf(fminf(clast - s_cum[tid], 0.f)) * s_dt[tid];
-        for (int c = tid; c < 5 * 1024; c += kThreads) widen_chunk(sm + c * 16, range_ok);
+        for (int idx = tid; idx < 3 * kBlk; idx += kThreads) {   // pivot factors, row groups 1..3
+            const int gm = idx >> 7, j = idx & (kBlk - 1);
+            const int m = 32 * (gm + 1) - 1;
+            if (j <= m) s_v[idx] = expf(fminf(s_cum[m] - s_cum[j], 0.f)) * s_dt[j];
+        }
+        ok = mbar_wait(bar, tma_par, kWaitBudget);
+        tma_par ^= 1u;
+        // X: bf16 -> fp16 in place (C and B arrive as fp16)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            uint4 *p = reinterpret_cast<uint4 *>(sX + (tid + r * kThreads) * 16);
+            float f[8];
+            bf16_chunk_to_f32(*p, f);
+            *p = pack8(f, amax);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok);
@@ -486,20 +541,35 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         // state scaled by the block decay
         {
             const float ci = s_cum[row];
+            const float ui = w4 > 0 ? expf(fminf(ci - s_cum[32 * w4 - 1], 0.f)) : 0.f;
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int c32 = 2 * ch + cc;
                 uint4 out[4];
-                if (c32 <= (warp & 3)) {                 // warp-uniform causal skip
+                if (c32 < w4) {                          // below the diagonal: factored decay
+                    float v[32];
+                    tmem_ld32(lane_addr + tCB + c32 * 32, v);
+                    const float4 *vf = reinterpret_cast<const float4 *>(s_v + (w4 - 1) * kBlk + c32 * 32);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 f = vf[q];
+                        v[4 * q] *= f.x * ui;
+                        v[4 * q + 1] *= f.y * ui;
+                        v[4 * q + 2] *= f.z * ui;
+                        v[4 * q + 3] *= f.w * ui;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, amax);
+                } else if (c32 == w4) {                  // diagonal 32x32: masked, exact exponent
                     float v[32];
                     tmem_ld32(lane_addr + tCB + c32 * 32, v);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = c32 * 32 + jj;
-                        v[jj] = (j <= row) ? v[jj] * expf(fminf(ci - s_cum[j], 0.f)) * s_dt[j] : 0.f;
+                        v[jj] = (jj <= lane) ? v[jj] * expf(fminf(ci - s_cum[j], 0.f)) * s_dt[j] : 0.f;
                     }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, range_ok);
+                    for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, amax);
                 } else {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) out[q] = make_uint4(0u, 0u, 0u, 0u);
@@ -512,12 +582,12 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             for (int r = 0; r < 4; ++r) {                // 1024 chunks of w.X
                 const int c = tid + r * kThreads;
                 const int j = c >> 3, q = c & 7;
-                const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(j, q));
+                float f[8];
+                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(sX + sw128_off(j, q)), f);
                 const float wj = s_w[j];
-                const float2 a0 = unpack_h2(xv.x), a1 = unpack_h2(xv.y), a2 = unpack_h2(xv.z), a3 = unpack_h2(xv.w);
-                const float f[8] = {wj * a0.x, wj * a0.y, wj * a1.x, wj * a1.y,
-                                    wj * a2.x, wj * a2.y, wj * a3.x, wj * a3.y};
-                *reinterpret_cast<uint4 *>(sHW + sw128_off(j, q)) = pack8(f, range_ok);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] *= wj;
+                *reinterpret_cast<uint4 *>(sHW + sw128_off(j, q)) = pack8(f, amax);
             }
             const float decay = expf(fminf(clast, 0.f));
             float v[32];
@@ -557,9 +627,8 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             tmem_ld32(lane_addr + tZ + ch * 32, zv);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(row, ch * 4 + q));
-                const float2 a0 = unpack_h2(xv.x), a1 = unpack_h2(xv.y), a2 = unpack_h2(xv.z), a3 = unpack_h2(xv.w);
-                const float xs[8] = {a0.x, a0.y, a1.x, a1.y, a2.x, a2.y, a3.x, a3.y};
+                float xs[8];
+                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(sX + sw128_off(row, ch * 4 + q)), xs);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int p = q * 8 + e;
@@ -577,7 +646,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             if (!last) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, range_ok);
+                    *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, amax);
             } else if (final_state && u == U - 1) {
                 float *dst = final_state + bh * kNP + (size_t)row * kP + ch * 32;
 #pragma unroll
@@ -597,7 +666,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     }
     if (tid == 0) tma_store_wait_all();
     if (!ok && tid == 0) flag_status(ws.status, kStatusTimeout);
-    if (!__syncthreads_and(range_ok) && tid == 0) flag_status(ws.status, kStatusRange);
+    if (!__syncthreads_and(amax <= kF16Max) && tid == 0) flag_status(ws.status, kStatusRange);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
@@ -610,7 +679,7 @@ bool tc_supported(const ScanDims &d, int bf16) {
     if (d.Q != 64 && d.Q != 128 && d.Q != 256) return false;
     if (d.H > 65535 || d.b > 65535 || d.L > 0x7fffffffll - kBlk) return false;
     const TcPlan p = make_plan(d);
-    return p.U <= 65535;
+    return p.U <= 65535 && (d.H + 31) / 32 + d.G <= 65535;
 }
 
 size_t tc_workspace_bytes(const ScanDims &d) { return ws_bytes(d, make_plan(d)); }
@@ -620,7 +689,7 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     if (p.nblk == 0) return cudaSuccess;
     TcWs ws = carve(d, p, wsp);
     TcMaps maps;
-    if (!make_maps(a, d, &maps)) return cudaErrorInvalidValue;
+    if (!make_maps(a, d, p, ws, &maps)) return cudaErrorInvalidValue;
     cudaError_t e;
     static bool attr_done = false;
     if (!attr_done) {
@@ -634,8 +703,10 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     }
     {
         TraceScope tr(s, kTrTcDtPrep);
-        dt_prep_kernel<<<dim3((unsigned)p.nblk, (unsigned)((d.H + 31) / 32), (unsigned)d.b), 256, 0, s>>>(
-            a.dt_raw, a.dt_bias, a.A, ws, (int)d.L, (int)d.H, (int)p.nblk, a.dt_lo, a.dt_hi);
+        const unsigned ny = (unsigned)((d.H + 31) / 32 + d.G);
+        prep_kernel<<<dim3((unsigned)p.nblk, ny, (unsigned)d.b), 256, 0, s>>>(
+            a.dt_raw, a.dt_bias, a.A, static_cast<const __nv_bfloat16 *>(a.B), static_cast<const __nv_bfloat16 *>(a.C),
+            ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, a.dt_lo, a.dt_hi);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.U > 1) {

@@ -24,12 +24,13 @@ void resolve() {
 
 }  // namespace
 
-bool tmap_encode_4d(CUtensorMap *map, const void *base, int elem_bytes, const uint64_t dims[4],
+bool tmap_encode_4d(CUtensorMap *map, const void *base, TmapElem elem, const uint64_t dims[4],
                     const uint64_t strides_bytes[3], const uint32_t box[4]) {
     std::call_once(g_once, resolve);
     if (!g_encode) return false;
-    const CUtensorMapDataType dt =
-        elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapDataType dt = elem == kTmapBF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : elem == kTmapF16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
     cuuint64_t gs[3] = {strides_bytes[0], strides_bytes[1], strides_bytes[2]};
     cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
