@@ -155,11 +155,19 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// 8 floats -> 8 fp16 (one 16-byte chunk); `amax` tracks the largest magnitude
-__device__ __forceinline__ uint4 pack8(const float *f, float &amax) {
+// 8 floats -> 8 fp16 (one 16-byte chunk).  `hmax` tracks the largest packed
+// magnitude as a half2 (an out-of-range value rounds to inf and stays there).
+__device__ __forceinline__ uint4 pack8(const float *f, __half2 &hmax) {
+    const uint4 o = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
+    const uint32_t w[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-    return make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
+    for (int i = 0; i < 4; ++i) hmax = __hmax2(hmax, __habs2(*reinterpret_cast<const __half2 *>(&w[i])));
+    return o;
+}
+
+__device__ __forceinline__ bool in_f16_range(__half2 hmax) {
+    const float2 m = __half22float2(hmax);
+    return m.x <= kF16Max && m.y <= kF16Max;
 }
 
 __device__ __forceinline__ void bf16_chunk_to_f32(uint4 v, float *f) {
@@ -187,7 +195,7 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
         const int g = blockIdx.y - nhy;
         const int t0 = blk * kBlk;
         const size_t Lp = (size_t)nblk * kBlk;
-        float amax = 0.f;
+        __half2 amax = __float2half2_rn(0.f);
 #pragma unroll 4
         for (int c = threadIdx.x; c < 2 * kBlk * 16; c += 256) {
             const int which = c >> 11, r = (c >> 4) & (kBlk - 1), kk = c & 15;
@@ -200,7 +208,7 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
             bf16_chunk_to_f32(v, f);
             *reinterpret_cast<uint4 *>(dst + (((size_t)b * Lp + t) * G + g) * kN + kk * 8) = pack8(f, amax);
         }
-        if (!(amax <= kF16Max)) flag_status(ws.status, kStatusRange);
+        if (!in_f16_range(amax)) flag_status(ws.status, kStatusRange);
         return;
     }
     const int h0 = blockIdx.y * 32;
@@ -240,133 +248,144 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
 }
 
 // ---------------------------------------------------------------------------
-// unit_state: grid (H, U-1, b), 256 threads, two TMA stages of (B fp16, X bf16).
-// Units 0..U-2 never hold the sequence's ragged tail (it is in the last
-// unit), so every block here is a full 128 tokens.
-constexpr uint32_t kUsStage = 3 * kTileBytes;                 // B (2 tiles) + X (1 tile)
-constexpr size_t kUsSmem = 1024 + 2 * kUsStage + 2 * kBlk * 4 + 64;
+// unit_state: grid (H, U-1, b), 8 compute warps + 1 control warp, 2 CTAs per
+// SM, two TMA stages of (B fp16, X bf16, dt, cum).  The control warp's lane 0
+// issues the TMA copies and the MMAs; the compute warps only widen X (scaled
+// by w) and signal.  Units 0..U-2 never hold the sequence's ragged tail (it
+// is in the last unit), so every block here is a full 128 tokens.
+constexpr int kUsCompute = 256;
+constexpr int kUsThreads = kUsCompute + 32;
+constexpr uint32_t kUsStage = 3 * kTileBytes + 2 * kBlk * 4;  // B (2 tiles) + X (1 tile) + dt + cum
+constexpr uint32_t kUsOffW = 2 * kUsStage;                     // w [2][128]
+constexpr uint32_t kUsOffBar = kUsOffW + 2 * kBlk * 4;         // tma[2], mma[2], converted[2]
+constexpr size_t kUsSmem = 1024 + kUsOffBar + 6 * 8 + 16;
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kUsThreads, 2)
 unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, int nblk, int U, int bpu) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    float *s_w = reinterpret_cast<float *>(sm + 2 * kUsStage);   // [2][128]
-    uint64_t *bar = reinterpret_cast<uint64_t *>(s_w + 2 * kBlk); // tma[2], mma[2]
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 4);
+    // per stage: [0,1] TMA landed, [2,3] MMAs done, [4,5] X converted.  One barrier of
+    // each kind per stage keeps every waiter within one phase of its signaller.
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kUsOffBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 6);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
     const int h = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int g = h / (H / G);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t bh = (size_t)b * H + h;
     const int kb0 = u * bpu, kb1 = min(nblk, kb0 + bpu);
     const int nk = kb1 - kb0;
-    const float *cum = ws.cum + bh * (size_t)nblk * kBlk;
-    const float *dtv = ws.dt + bh * (size_t)nblk * kBlk;
+    const float *cumg = ws.cum + bh * (size_t)nblk * kBlk;
+    const float *dtg = ws.dt + bh * (size_t)nblk * kBlk;
+    auto stage = [&](int s) { return sm + s * kUsStage; };
 
     if (warp == 0) {
         tmem_alloc(tslot, 64);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(bar + i, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(bar + i, 1);
+        *abort_flag = 0;
         fence_mbar_init();
-        for (int i = 0; i < 2 && i < nk; ++i) {
-            uint8_t *st = sm + i * kUsStage;
-            const int t0 = (kb0 + i) * kBlk;
-            mbar_arrive_expect_tx(bar + i, kUsStage);
-            tma_load_4d(st, &maps.B, bar + i, 0, g, t0, b);
-            tma_load_4d(st + kTileBytes, &maps.B, bar + i, 64, g, t0, b);
-            tma_load_4d(st + 2 * kTileBytes, &maps.x, bar + i, 0, h, t0, b);
-        }
     }
-    // suffix: the unit's log decay after the current block (sum of later block totals)
-    float suffix = 0.f;
-    for (int k = kb0 + 1; k < kb1; ++k) suffix += cum[(size_t)k * kBlk + kBlk - 1];
-    if (tid == 0) ws.ell[bh * U + u] = suffix + cum[(size_t)kb0 * kBlk + kBlk - 1];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    bool ok = true;
-    float amax = 0.f;
-    uint32_t tma_par = 0, mma_par = 0;              // per-stage phase bits
-    const uint32_t idesc = idesc_f16(128, 64, 1, 1);
-    for (int k = kb0; k < kb1; ++k) {
-        const int i = k - kb0, s = i & 1;
-        uint8_t *st = sm + s * kUsStage;
-        float *w = s_w + s * kBlk;
-        if (tid < kBlk) {
-            const float e = cum[(size_t)k * kBlk + kBlk - 1] - cum[(size_t)k * kBlk + tid] + suffix;
-            w[tid] = expf(fminf(e, 0.f)) * dtv[(size_t)k * kBlk + tid];
-        }
-        if (k + 1 < kb1) suffix -= cum[(size_t)(k + 1) * kBlk + kBlk - 1];
-        ok = mbar_wait(bar + s, (tma_par >> s) & 1u, kWaitBudget);
-        tma_par ^= 1u << s;
-        __syncthreads();                            // w[] visible
-        // X (bf16) -> w.X (fp16) in place; the row of a chunk is offset / 128
-        uint8_t *sx = st + 2 * kTileBytes;
+    if (warp == kUsCompute / 32) {
+        // ------------------------------ control warp --------------------------
+        if (lane == 0) {
+            auto load = [&](int s, int k) {
+                uint8_t *st = stage(s);
+                const int t0 = k * kBlk;
+                mbar_arrive_expect_tx(bar + s, kUsStage);
+                tma_load_4d(st, &maps.B, bar + s, 0, g, t0, b);
+                tma_load_4d(st + kTileBytes, &maps.B, bar + s, 64, g, t0, b);
+                tma_load_4d(st + 2 * kTileBytes, &maps.x, bar + s, 0, h, t0, b);
+                bulk_load(st + 3 * kTileBytes, dtg + (size_t)t0, kBlk * 4, bar + s);
+                bulk_load(st + 3 * kTileBytes + kBlk * 4, cumg + (size_t)t0, kBlk * 4, bar + s);
+            };
+            const uint32_t idesc = idesc_f16(128, 64, 1, 1);
+            bool ok = true;
+            for (int i = 0; i < 2 && i < nk; ++i) load(i, kb0 + i);
+            for (int i = 0; i < nk && ok; ++i) {
+                const int s = i & 1;
+                ok = mbar_wait_abortable(bar + 4 + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t b_base = smem_u32(stage(s)), x_base = smem_u32(stage(s) + 2 * kTileBytes);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int c = tid + r * kThreads;
-            uint4 *p = reinterpret_cast<uint4 *>(sx + c * 16);
-            float f[8];
-            bf16_chunk_to_f32(*p, f);
-            const float wr = w[c >> 3];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] *= wr;
-            *p = pack8(f, amax);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(ok);
-        tc_fence_after();
-        if (!ok) break;
-        if (tid == 0) {
-            const uint32_t b_base = smem_u32(st), x_base = smem_u32(sx);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                mma_f16(tmem, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
-                        sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc, (i > 0 || q > 0) ? 1u : 0u);
-            mma_commit(bar + 2 + s);
-            // refill this stage with block k+2 once these MMAs have read it
-            if (k + 2 < kb1) {
-                const bool done = mbar_wait(bar + 2 + s, (mma_par >> s) & 1u, kWaitBudget);
-                mma_par ^= 1u << s;
-                if (done) {
-                    const int t0 = (k + 2) * kBlk;
-                    mbar_arrive_expect_tx(bar + s, kUsStage);
-                    tma_load_4d(st, &maps.B, bar + s, 0, g, t0, b);
-                    tma_load_4d(st + kTileBytes, &maps.B, bar + s, 64, g, t0, b);
-                    tma_load_4d(st + 2 * kTileBytes, &maps.x, bar + s, 0, h, t0, b);
-                } else {
-                    flag_status(ws.status, kStatusTimeout);
+                for (int q = 0; q < 8; ++q)
+                    mma_f16(tmem, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
+                            sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc, (i > 0 || q > 0) ? 1u : 0u);
+                mma_commit(bar + 2 + s);
+                if (i + 2 < nk) {       // refill stage s once these MMAs have read it
+                    ok = mbar_wait_abortable(bar + 2 + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
+                    if (ok) load(s, kb0 + i + 2);
                 }
             }
         }
-    }
-    // wait for the last block's MMAs (the stage it used still has that commit pending)
-    if (ok && tid == 0 && nk > 0) {
-        const int s = (nk - 1) & 1;
-        ok = mbar_wait(bar + 2 + s, (mma_par >> s) & 1u, kWaitBudget);
-    }
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-    if (!ok) {
-        if (tid == 0) flag_status(ws.status, kStatusTimeout);
+        __syncwarp();
     } else {
-        // 8 warps: lanes 32*(warp%4).., columns 32*(warp/4)..
-        const int n = 32 * (warp & 3) + (tid & 31), ch = warp >> 2;
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ch * 32, v);
-        float *dst = ws.states + (bh * U + u) * (size_t)kNP + (size_t)n * kP + ch * 32;
+        // ------------------------------ compute warps -------------------------
+        __half2 amax = __float2half2_rn(0.f);
+        bool ok = true;
+        // the unit's log decay after the current block (sum of later block totals)
+        float suffix = 0.f;
+        if (tid < kBlk)
+            for (int k = kb0 + 1; k < kb1; ++k) suffix += cumg[(size_t)k * kBlk + kBlk - 1];
+        if (tid == 0) ws.ell[bh * U + u] = suffix + cumg[(size_t)kb0 * kBlk + kBlk - 1];
+        for (int i = 0; i < nk; ++i) {
+            const int s = i & 1;
+            uint8_t *st = stage(s);
+            const float *dt = reinterpret_cast<const float *>(st + 3 * kTileBytes);
+            const float *cum = dt + kBlk;
+            float *w = reinterpret_cast<float *>(sm + kUsOffW) + s * kBlk;
+            ok = ok && mbar_wait_abortable(bar + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
+            if (ok && tid < kBlk) w[tid] = expf(fminf(cum[kBlk - 1] - cum[tid] + suffix, 0.f)) * dt[tid];
+            if (tid < kBlk && kb0 + i + 1 < kb1) suffix -= cumg[(size_t)(kb0 + i + 1) * kBlk + kBlk - 1];
+            named_bar_sync(kUsCompute);                 // w[] visible
+            if (ok) {
+                uint8_t *sx = st + 2 * kTileBytes;      // X (bf16) -> w.X (fp16); row = offset / 128
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                for (int r = 0; r < 4; ++r) {
+                    const int c = tid + r * kUsCompute;
+                    uint4 *p = reinterpret_cast<uint4 *>(sx + c * 16);
+                    float f[8];
+                    bf16_chunk_to_f32(*p, f);
+                    const float wr = w[c >> 3];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] *= wr;
+                    *p = pack8(f, amax);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(kUsCompute);
+            if (tid == 0) mbar_arrive(bar + 4 + s);
+        }
+        // the accumulated state: wait for the last block's MMAs
+        const int sl = (nk - 1) & 1;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_abortable(bar + 2 + sl, ((uint32_t)(nk - 1) >> 1) & 1u,
+                                                                   kWaitBudget, abort_flag));
+        tc_fence_after();
+        if (ok) {
+            // 8 warps: lanes 32*(warp%4).., columns 32*(warp/4)..
+            const int n = 32 * (warp & 3) + lane, ch = warp >> 2;
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ch * 32, v);
+            float *dst = ws.states + (bh * U + u) * (size_t)kNP + (size_t)n * kP + ch * 32;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4 *>(dst + 4 * q) =
+                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        if (__any_sync(0xffffffffu, !in_f16_range(amax)) && lane == 0) flag_status(ws.status, kStatusRange);
     }
-    if (!__syncthreads_and(amax <= kF16Max) && tid == 0) flag_status(ws.status, kStatusRange);
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && *abort_flag) flag_status(ws.status, kStatusTimeout);
     if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
@@ -409,147 +428,306 @@ tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
 }
 
 // ---------------------------------------------------------------------------
-// chunk_out: grid (H, U, b), 256 threads, 2 CTAs per SM.
-constexpr size_t kCoSmem = 1024 + 6 * kTileBytes + (3 * kBlk + 3 * kBlk) * 4 + 64;
+// chunk_out: grid (H, U, b), one CTA per SM: 16 compute warps + 1 control warp.
+//
+// The control warp's lane 0 issues every TMA copy and every MMA, driven by
+// mbarriers, so the compute warps never wait on issue.  Per 128-token block k
+// (two TMA stages; tiles of block k+2 stream in meanwhile), each MMA runs
+// while the compute warps do independent work:
+//   compute: [1] C.B^T(k), C.H(k) done -> W, w.X, state*decay     -> w_ready
+//            [2] tiles(k+1) landed -> decay factors, X widened     -> ops_ready
+//            [3] W.X(k), state update done -> fp16 state for k+1   -> h16_ready
+//            [4] y(k) staged in block k's C tiles (dead once C.B^T(k)
+//                and C.H(k) are done)                              -> epi_done
+//   control: w_ready -> W.X(k), B^T.(wX)(k);  ops_ready -> C.B^T(k+1);
+//            h16_ready -> C.H(k+1);  epi_done -> y(k) TMA store, tiles(k+2)
+//            (the C tiles of k+2 once the store has read the staging).
+// Compute warp w owns TMEM lanes 32*(w%4).. (its rows) and column slice w/4
+// of each TMEM region: 32 of the 128 C.B^T columns, 16 of the 64 Y/Z/state
+// columns.
+constexpr int kCoCompute = 512;                                 // 16 compute warps
+constexpr int kCoThreads = kCoCompute + 32;                     // + control warp
+constexpr uint32_t kCoStage = 5 * kTileBytes + 2 * kBlk * 4;   // C(2) B(2) X(1) tiles, dt, cum
+constexpr uint32_t kCoFactors = 640;                            // w[128], v[3][128], vd[128]
+constexpr uint32_t kCoOffW = 2 * kCoStage;                      // W tile (2 tiles)
+constexpr uint32_t kCoOffHW = kCoOffW + 2 * kTileBytes;         // fp16 state, then w.X
+constexpr uint32_t kCoOffF = kCoOffHW + kTileBytes;             // factors [2][640] floats
+constexpr uint32_t kCoOffG = kCoOffF + 2 * kCoFactors * 4;      // diagonal fast-path flags [2][4]
+constexpr uint32_t kCoOffBar = kCoOffG + 8 * 4;                 // 8 mbarriers, TMEM slot, abort flag
+constexpr size_t kCoSmem = 1024 + kCoOffBar + 8 * 8 + 16;
+constexpr float kDiagExpCap = 64.0f;                            // largest exponent on the diagonal fast path
 
-__global__ void __launch_bounds__(kThreads, 2)
+enum CoBar { kBarTma0 = 0, kBarTma1 = 1, kBarCBZ = 2, kBarYS = 3, kBarOps = 4, kBarW = 5, kBarEpi = 6,
+             kBarH16 = 7 };
+
+struct CoSmem {
+    uint8_t *base;
+    __device__ uint8_t *C(int s) const { return base + s * kCoStage; }
+    __device__ uint8_t *B(int s) const { return base + s * kCoStage + 2 * kTileBytes; }
+    __device__ uint8_t *X(int s) const { return base + s * kCoStage + 4 * kTileBytes; }
+    __device__ float *dt(int s) const { return reinterpret_cast<float *>(base + s * kCoStage + 5 * kTileBytes); }
+    __device__ float *cum(int s) const { return dt(s) + kBlk; }
+    __device__ uint8_t *W() const { return base + kCoOffW; }
+    __device__ uint8_t *HW() const { return base + kCoOffHW; }
+    __device__ float *F(int s) const { return reinterpret_cast<float *>(base + kCoOffF) + s * kCoFactors; }
+    __device__ int *G(int s) const { return reinterpret_cast<int *>(base + kCoOffG) + s * 4; }
+    __device__ uint64_t *bar(int i) const { return reinterpret_cast<uint64_t *>(base + kCoOffBar) + i; }
+    __device__ uint32_t *tslot() const { return reinterpret_cast<uint32_t *>(bar(8)); }
+    __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(bar(8)) + 1; }
+};
+
+// TMA for block k into stage s, in two parts on one barrier (which expects
+// the bytes of both): B (fp16 copy), X (bf16), dt and cum rows first, then the
+// C tiles (fp16 copy), which may have to wait for a y store out of them.
+__device__ __forceinline__ void co_load_bx(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
+                                           int s, int k, int g, int h, int b) {
+    const int t0 = k * kBlk;
+    uint64_t *bar = S.bar(kBarTma0 + s);
+    mbar_arrive_expect_tx(bar, 5 * kTileBytes + 2 * kBlk * 4);
+    tma_load_4d(S.B(s), &maps.B, bar, 0, g, t0, b);
+    tma_load_4d(S.B(s) + kTileBytes, &maps.B, bar, 64, g, t0, b);
+    tma_load_4d(S.X(s), &maps.x, bar, 0, h, t0, b);
+    bulk_load(S.dt(s), dtv + (size_t)t0, kBlk * 4, bar);
+    bulk_load(S.cum(s), cum + (size_t)t0, kBlk * 4, bar);
+}
+
+__device__ __forceinline__ void co_load_c(const CoSmem &S, const TcMaps &maps, int s, int k, int g, int b) {
+    const int t0 = k * kBlk;
+    uint64_t *bar = S.bar(kBarTma0 + s);
+    tma_load_4d(S.C(s), &maps.C, bar, 0, g, t0, b);
+    tma_load_4d(S.C(s) + kTileBytes, &maps.C, bar, 64, g, t0, b);
+}
+
+__device__ __forceinline__ void co_load(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
+                                        int s, int k, int g, int h, int b) {
+    co_load_bx(S, maps, dtv, cum, s, k, g, h, b);
+    co_load_c(S, maps, s, k, g, b);
+}
+
+// Per-block decay factors (all exponents clamped as stated):
+//   w[j]        = exp(min(cum_last - cum_j, 0)) dt_j               (state update)
+//   v[g-1][j]   = exp(min(cum_m - cum_j, 0)) dt_j, m = 32g-1, j<=m (below the diagonal, row group g)
+//   vd[j]       = exp(min(cum_s0 - cum_j, cap)) dt_j, s0 = 32*(j/32) (diagonal sub-blocks)
+// and flags: the diagonal sub-block of row group g may use vd (its decay is
+// below exp(-cap), so no factor there exceeds exp(cap)).
+__device__ __forceinline__ void co_factors(const CoSmem &S, int s, int last_valid, int tid) {
+    const float *cum = S.cum(s), *dt = S.dt(s);
+    float *F = S.F(s);
+    const float clast = cum[last_valid];
+    for (int idx = tid; idx < (int)kCoFactors; idx += kCoCompute) {
+        float f = 0.f;
+        if (idx < kBlk) {
+            f = expf(fminf(clast - cum[idx], 0.f)) * dt[idx];
+        } else if (idx < 4 * kBlk) {
+            const int q = idx - kBlk, gm = q >> 7, j = q & (kBlk - 1), m = 32 * (gm + 1) - 1;
+            if (j <= m) f = expf(fminf(cum[m] - cum[j], 0.f)) * dt[j];
+        } else {
+            const int j = idx - 4 * kBlk;
+            f = expf(fminf(cum[j & ~31] - cum[j], kDiagExpCap)) * dt[j];
+        }
+        F[idx] = f;
+    }
+    if (tid < 4) S.G(s)[tid] = (cum[32 * tid] - cum[32 * tid + 31]) <= kDiagExpCap ? 1 : 0;
+}
+
+// X tile of stage s: bf16 -> fp16 in place (two 16-byte chunks per thread).
+__device__ __forceinline__ void co_widen_x(const CoSmem &S, int s, int tid, __half2 &amax) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        uint4 *p = reinterpret_cast<uint4 *>(S.X(s) + (tid + r * kCoCompute) * 16);
+        float f[8];
+        bf16_chunk_to_f32(*p, f);
+        *p = pack8(f, amax);
+    }
+}
+
+// TMEM column of the C.H accumulator of the block in stage s (two buffers:
+// block k+1's is written while block k's is still being read).
+__device__ __forceinline__ uint32_t co_tz(int s) { return s ? 384u : 64u; }
+
+// Compute warps: publish this step's smem/TMEM writes, sync the 512 compute
+// threads, and let one of them arrive on `bar` for the control thread.
+__device__ __forceinline__ void co_signal(uint64_t *bar, int tid) {
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar_sync(kCoCompute);
+    if (tid == 0) mbar_arrive(bar);
+}
+
+__global__ void __launch_bounds__(kCoThreads)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
-                 const float *__restrict__ init, float *__restrict__ final_state, TcWs ws, int L, int H, int G,
-                 int nblk, int U, int bpu, int states_from_ws) {
+                 const float *__restrict__ init, float *__restrict__ final_state, TcWs ws,
+                 int L, int H, int G, int nblk, int U, int bpu, int states_from_ws) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = align1024(smem_raw);
-    uint8_t *sCW = sm;                              // C tile -> W tile -> y staging (2 tiles)
-    uint8_t *sB = sm + 2 * kTileBytes;              // B tile (2 tiles)
-    uint8_t *sX = sm + 4 * kTileBytes;              // X tile
-    uint8_t *sHW = sm + 5 * kTileBytes;             // fp16 state [n][p], then w.X [j][p]
-    float *s_dt = reinterpret_cast<float *>(sm + 6 * kTileBytes);
-    float *s_cum = s_dt + kBlk;
-    float *s_w = s_cum + kBlk;
-    float *s_v = s_w + kBlk;                        // [3][128] pivot factors for row groups 1..3
-    uint64_t *bar = reinterpret_cast<uint64_t *>(s_v + 3 * kBlk);  // [0] TMA, [1] MMA
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 2);
+    CoSmem S;
+    S.base = align1024(smem_raw);
+    volatile int *abort_flag = S.abort_flag();
 
     const int h = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int g = h / (H / G);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int w4 = warp & 3;                        // row group: rows 32*w4 .. 32*w4+31
-    const int row = 32 * w4 + lane;                 // TMEM lane / tile row of this thread
-    const int ch = warp >> 2;                       // which 32-column half it handles
     const size_t bh = (size_t)b * H + h;
     const int kb0 = u * bpu, kb1 = min(nblk, kb0 + bpu);
-    const float *cum = ws.cum + bh * (size_t)nblk * kBlk;
-    const float *dtv = ws.dt + bh * (size_t)nblk * kBlk;
+    const float *cumg = ws.cum + bh * (size_t)nblk * kBlk;
+    const float *dtg = ws.dt + bh * (size_t)nblk * kBlk;
 
     if (warp == 0) {
-        tmem_alloc(tslot, 256);
+        tmem_alloc(S.tslot(), 512);
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(bar, 1);
-        mbar_init(bar + 1, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(S.bar(i), 1);
+        *abort_flag = 0;
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tslot;
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * w4) << 16);
-    const uint32_t tH = 0, tZ = 64, tCB = 128;   // TMEM columns: state, C.H, C.B^T then Y
-    float amax = 0.f;
+    const uint32_t tmem = *S.tslot();
+    const uint32_t tH = 0;                           // TMEM columns: state; C.H at co_tz(s); C.B^T/Y at 128, 256
 
-    // state entering the unit -> TMEM (fp32) and sHW (fp16): row n = `row`, columns 32*ch..
-    {
-        const float *src = states_from_ws ? ws.states + (bh * U + u) * (size_t)kNP
-                                          : (init ? init + bh * kNP : nullptr);
-        float v[32];
+    if (warp == kCoCompute / 32) {
+        // ------------------------------ control warp --------------------------
+        if (lane == 0) {
+            const uint32_t idesc_z = idesc_f16(128, 64, 0, 1);    // A=C K-major, B=H MN-major
+            const uint32_t idesc_cb = idesc_f16(128, 128, 0, 0);  // A=C K-major, B=B K-major
+            const uint32_t idesc_y = idesc_f16(128, 64, 0, 1);    // A=W K-major, B=X MN-major
+            const uint32_t idesc_s = idesc_f16(128, 64, 1, 1);    // A=B^T MN-major, B=wX MN-major
+            const uint32_t h_base = smem_u32(S.HW()), w_base = smem_u32(S.W());
+            bool ok = true;
+            co_load(S, maps, dtg, cumg, 0, kb0, g, h, b);
+            if (kb0 + 1 < kb1) co_load(S, maps, dtg, cumg, 1, kb0 + 1, g, h, b);
+            // block kb0: C.B^T and C.H once its operands are ready
+            ok = mbar_wait_abortable(S.bar(kBarOps), 0, kWaitBudget, abort_flag);
+            tc_fence_after();
+            if (ok) {
+                const uint32_t c_base = smem_u32(S.C(0)), b_base = smem_u32(S.B(0));
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float4 f = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kP + ch * 32 + 4 * q)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
-        }
-        tmem_st32(lane_addr + tH + ch * 32, v);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, amax);
-    }
-
-    bool ok = true;
-    uint32_t tma_par = 0, mma_par = 0;
-    const uint32_t idesc_z = idesc_f16(128, 64, 0, 1);    // A=C K-major, B=H MN-major
-    const uint32_t idesc_cb = idesc_f16(128, 128, 0, 0);  // A=C K-major, B=B K-major
-    const uint32_t idesc_y = idesc_f16(128, 64, 0, 1);    // A=W K-major, B=X MN-major
-    const uint32_t idesc_s = idesc_f16(128, 64, 1, 1);    // A=B^T MN-major, B=wX MN-major
-    const float Dh = D[h];
-
-    for (int k = kb0; k < kb1; ++k) {
-        const int t0 = k * kBlk;
-        if (tid == 0) {
-            tma_store_wait_read();                 // the previous y store has left sCW
-            mbar_arrive_expect_tx(bar, 5 * kTileBytes);
-            tma_load_4d(sCW, &maps.C, bar, 0, g, t0, b);
-            tma_load_4d(sCW + kTileBytes, &maps.C, bar, 64, g, t0, b);
-            tma_load_4d(sB, &maps.B, bar, 0, g, t0, b);
-            tma_load_4d(sB + kTileBytes, &maps.B, bar, 64, g, t0, b);
-            tma_load_4d(sX, &maps.x, bar, 0, h, t0, b);
-        }
-        if (tid < kBlk) s_dt[tid] = dtv[(size_t)t0 + tid];
-        else s_cum[tid - kBlk] = cum[(size_t)t0 + tid - kBlk];
-        __syncthreads();                           // s_dt, s_cum visible
-        // decay to the block's last real token (padding carries dA = 0 but its
-        // cumsum may round differently)
-        const float clast = s_cum[min(kBlk - 1, L - 1 - t0)];
-        if (tid < kBlk) s_w[tid] = expf(fminf(clast - s_cum[tid], 0.f)) * s_dt[tid];
-        for (int idx = tid; idx < 3 * kBlk; idx += kThreads) {   // pivot factors, row groups 1..3
-            const int gm = idx >> 7, j = idx & (kBlk - 1);
-            const int m = 32 * (gm + 1) - 1;
-            if (j <= m) s_v[idx] = expf(fminf(s_cum[m] - s_cum[j], 0.f)) * s_dt[j];
-        }
-        ok = mbar_wait(bar, tma_par, kWaitBudget);
-        tma_par ^= 1u;
-        // X: bf16 -> fp16 in place (C and B arrive as fp16)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            uint4 *p = reinterpret_cast<uint4 *>(sX + (tid + r * kThreads) * 16);
-            float f[8];
-            bf16_chunk_to_f32(*p, f);
-            *p = pack8(f, amax);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(ok);
-        tc_fence_after();
-        if (!ok) break;
-
-        if (tid == 0) {
-            const uint32_t c_base = smem_u32(sCW), b_base = smem_u32(sB), h_base = smem_u32(sHW);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint64_t ad = sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024);
-                mma_f16(tmem + tZ, ad, sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_z, q > 0);
-                mma_f16(tmem + tCB, ad, sdesc_sw128(b_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
-                        idesc_cb, q > 0);
+                for (int q = 0; q < 8; ++q) {
+                    const uint64_t ad = sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024);
+                    mma_f16(tmem + 128u, ad, sdesc_sw128(b_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
+                            idesc_cb, q > 0);
+                    mma_f16(tmem + co_tz(0), ad, sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_z, q > 0);
+                }
+                mma_commit(S.bar(kBarCBZ));
             }
-            mma_commit(bar + 1);
-        }
-        ok = __syncthreads_and(mbar_wait(bar + 1, mma_par, kWaitBudget));
-        mma_par ^= 1u;
-        if (!ok) break;
-        tc_fence_after();
-
-        // W (row `row`, columns 64*ch..64*ch+63) into sCW; w.X into sHW; the
-        // state scaled by the block decay
-        {
-            const float ci = s_cum[row];
-            const float ui = w4 > 0 ? expf(fminf(ci - s_cum[32 * w4 - 1], 0.f)) : 0.f;
+            for (int k = kb0; k < kb1 && ok; ++k) {
+                const int i = k - kb0, s = i & 1, s1 = s ^ 1;
+                const uint32_t par = (uint32_t)i & 1u, par1 = (uint32_t)(i + 1) & 1u;
+                const uint32_t tcb = 128u + 128u * s, tcb1 = 128u + 128u * s1;
+                // W.X(k) and the state update once W and w.X are in place
+                ok = mbar_wait_abortable(S.bar(kBarW), par, kWaitBudget, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                {
+                    const uint32_t x_base = smem_u32(S.X(s)), b_base = smem_u32(S.B(s));
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c32 = 2 * ch + cc;
+                    for (int q = 0; q < 8; ++q) {
+                        mma_f16(tmem + tcb, sdesc_sw128(w_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
+                                sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc_y, q > 0);
+                        mma_f16(tmem + tH, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
+                                sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_s, 1u);
+                    }
+                    mma_commit(S.bar(kBarYS));
+                }
+                if (k + 1 < kb1) {
+                    // C.B^T of block k+1 as soon as its operands are ready
+                    ok = mbar_wait_abortable(S.bar(kBarOps), par1, kWaitBudget, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t c_base = smem_u32(S.C(s1)), b_base = smem_u32(S.B(s1));
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        mma_f16(tmem + tcb1, sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
+                                sdesc_sw128(b_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024), idesc_cb,
+                                q > 0);
+                    // C.H of block k+1 once its fp16 entering state is in HW; one commit for both
+                    ok = mbar_wait_abortable(S.bar(kBarH16), par, kWaitBudget, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        mma_f16(tmem + co_tz(s1), sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
+                                sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_z, q > 0);
+                    mma_commit(S.bar(kBarCBZ));
+                }
+                // y(k) staged: store it, then refill stage s with block k+2
+                ok = mbar_wait_abortable(S.bar(kBarEpi), par, kWaitBudget, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                tma_store_4d(&maps.y, S.C(s), 0, h, k * kBlk, b);
+                tma_store_4d(&maps.y, S.C(s) + kTileBytes, 32, h, k * kBlk, b);
+                tma_store_commit();
+                if (k + 2 < kb1) {
+                    // every MMA of block k has completed (the compute warps waited on
+                    // them) and its epilogue is done: only the y store still reads
+                    // stage s, from its C tiles
+                    co_load_bx(S, maps, dtg, cumg, s, k + 2, g, h, b);
+                    tma_store_wait_read();
+                    co_load_c(S, maps, s, k + 2, g, b);
+                }
+            }
+            tma_store_wait_all();
+            if (!ok) *abort_flag = 1;
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------ compute warps -------------------------
+        const int lg = warp & 3;                    // row group: rows 32*lg .. 32*lg+31
+        const int row = 32 * lg + lane;             // TMEM lane / tile row of this thread
+        const int cq = warp >> 2;                   // column slice 0..3
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * lg) << 16);
+        const float Dh = D[h];
+        __half2 amax = __float2half2_rn(0.f);
+        bool ok = true;
+
+        // state entering the unit -> TMEM (fp32) and HW (fp16): row `row`, columns 16*cq..
+        {
+            const float *src = states_from_ws ? ws.states + (bh * U + u) * (size_t)kNP
+                                              : (init ? init + bh * kNP : nullptr);
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 f = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kP + cq * 16 + 4 * q)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+            }
+            tmem_st16(lane_addr + tH + cq * 16, v);
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                *reinterpret_cast<uint4 *>(S.HW() + sw128_off(row, cq * 2 + q)) = pack8(v + 8 * q, amax);
+        }
+        // block kb0: tiles landed -> factors, widened X -> ops_ready
+        ok = mbar_wait_abortable(S.bar(kBarTma0), 0, kWaitBudget, abort_flag);
+        if (ok) {
+            co_factors(S, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
+            co_widen_x(S, 0, tid, amax);
+        }
+        co_signal(S.bar(kBarOps), tid);
+
+        // every compute thread runs every iteration (and so every named barrier);
+        // after an abort the waits return at once and the work is skipped
+        for (int k = kb0; k < kb1; ++k) {
+            const int i = k - kb0, s = i & 1, s1 = s ^ 1;
+            const uint32_t par = (uint32_t)i & 1u;
+            const uint32_t tcb = 128u + 128u * s;
+            const int t0 = k * kBlk;
+            const float *cum = S.cum(s);
+            const float *F = S.F(s);
+
+            // [1] C.B^T(k), C.H(k) done -> W, w.X, state * decay -> w_ready
+            ok = ok && mbar_wait_abortable(S.bar(kBarCBZ), par, kWaitBudget, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);        // warp-uniform before tcgen05.ld
+            tc_fence_after();
+            if (ok) {
+                const int c32 = cq;
+                const float ci = cum[row];
                 uint4 out[4];
-                if (c32 < w4) {                          // below the diagonal: factored decay
+                if (c32 < lg) {                          // below the diagonal: factored decay
                     float v[32];
-                    tmem_ld32(lane_addr + tCB + c32 * 32, v);
-                    const float4 *vf = reinterpret_cast<const float4 *>(s_v + (w4 - 1) * kBlk + c32 * 32);
+                    tmem_ld32(lane_addr + tcb + c32 * 32, v);
+                    const float ui = expf(fminf(ci - cum[32 * lg - 1], 0.f));
+                    const float4 *vf = reinterpret_cast<const float4 *>(F + kBlk * lg + c32 * 32);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 f = vf[q];
@@ -560,13 +738,29 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                     }
 #pragma unroll
                     for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, amax);
-                } else if (c32 == w4) {                  // diagonal 32x32: masked, exact exponent
+                } else if (c32 == lg) {                  // diagonal 32x32: causal select first
                     float v[32];
-                    tmem_ld32(lane_addr + tCB + c32 * 32, v);
+                    tmem_ld32(lane_addr + tcb + c32 * 32, v);
+                    if (S.G(s)[lg]) {
+                        const float ui = expf(fminf(ci - cum[32 * lg], 0.f));
+                        const float4 *vf = reinterpret_cast<const float4 *>(F + 4 * kBlk + c32 * 32);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = c32 * 32 + jj;
-                        v[jj] = (jj <= lane) ? v[jj] * expf(fminf(ci - s_cum[j], 0.f)) * s_dt[j] : 0.f;
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 f = vf[q];
+                            const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int jj = 4 * q + e;
+                                v[jj] = (jj <= lane) ? v[jj] * (fv[e] * ui) : 0.f;
+                            }
+                        }
+                    } else {
+                        const float *dts = S.dt(s);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int j = c32 * 32 + jj;
+                            v[jj] = (jj <= lane) ? v[jj] * expf(fminf(ci - cum[j], 0.f)) * dts[j] : 0.f;
+                        }
                     }
 #pragma unroll
                     for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, amax);
@@ -576,100 +770,85 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(sCW + ch * kTileBytes + sw128_off(row, cc * 4 + q)) = out[q];
+                    *reinterpret_cast<uint4 *>(S.W() + (c32 >> 1) * kTileBytes + sw128_off(row, (c32 & 1) * 4 + q)) =
+                        out[q];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {            // 1024 chunks of w.X
+                    const int c = tid + r * kCoCompute;
+                    const int j = c >> 3, q = c & 7;
+                    float f[8];
+                    f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(j, q)), f);
+                    const float wj = F[j];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] *= wj;
+                    *reinterpret_cast<uint4 *>(S.HW() + sw128_off(j, q)) = pack8(f, amax);
+                }
+                const float decay = expf(fminf(cum[min(kBlk - 1, L - 1 - t0)], 0.f));
+                float hv[16];
+                tmem_ld16(lane_addr + tH + cq * 16, hv);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) hv[q] *= decay;
+                tmem_st16(lane_addr + tH + cq * 16, hv);
             }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {                // 1024 chunks of w.X
-                const int c = tid + r * kThreads;
-                const int j = c >> 3, q = c & 7;
-                float f[8];
-                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(sX + sw128_off(j, q)), f);
-                const float wj = s_w[j];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] *= wj;
-                *reinterpret_cast<uint4 *>(sHW + sw128_off(j, q)) = pack8(f, amax);
-            }
-            const float decay = expf(fminf(clast, 0.f));
-            float v[32];
-            tmem_ld32(lane_addr + tH + ch * 32, v);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] *= decay;
-            tmem_st32(lane_addr + tH + ch * 32, v);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+            co_signal(S.bar(kBarW), tid);
 
-        if (tid == 0) {
-            const uint32_t w_base = smem_u32(sCW), x_base = smem_u32(sX), b_base = smem_u32(sB),
-                           wx_base = smem_u32(sHW);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                mma_f16(tmem + tCB, sdesc_sw128(w_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
-                        sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc_y, q > 0);
-                mma_f16(tmem + tH, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
-                        sdesc_sw128(wx_base + q * 2048, kTileBytes, 1024), idesc_s, 1u);
+            // [2] block k+1: tiles landed -> factors, widened X -> ops_ready (overlaps W.X(k))
+            if (k + 1 < kb1) {
+                ok = ok && mbar_wait_abortable(S.bar(kBarTma0 + s1), ((uint32_t)(i + 1) >> 1) & 1u, kWaitBudget,
+                                               abort_flag);
+                if (ok) {
+                    co_factors(S, s1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
+                    co_widen_x(S, s1, tid, amax);
+                }
+                co_signal(S.bar(kBarOps), tid);
             }
-            mma_commit(bar + 1);
-        }
-        ok = __syncthreads_and(mbar_wait(bar + 1, mma_par, kWaitBudget));
-        mma_par ^= 1u;
-        if (!ok) break;
-        tc_fence_after();
 
-        // y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging (sCW, two 32-column
-        // fp32 tiles) -> TMA store; the next block's fp16 state into sHW
-        {
-            const float ei = expf(fminf(s_cum[row], 0.f));
-            float yv[32], zv[32];
-            tmem_ld32(lane_addr + tCB + ch * 32, yv);
-            tmem_ld32(lane_addr + tZ + ch * 32, zv);
+            // [3] W.X(k), state update done -> fp16 entering state of block k+1 -> h16_ready
+            ok = __all_sync(0xffffffffu, ok && mbar_wait_abortable(S.bar(kBarYS), par, kWaitBudget, abort_flag));
+            tc_fence_after();
+            float yv[16], zv[16];
+            if (ok) {
+                float hv[16];
+                tmem_ld16x3(lane_addr + tH + cq * 16, hv, lane_addr + tcb + cq * 16, yv, lane_addr + co_tz(s) + cq * 16,
+                            zv);
+                if (k + 1 < kb1) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float xs[8];
-                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(sX + sw128_off(row, ch * 4 + q)), xs);
+                    for (int q = 0; q < 2; ++q)
+                        *reinterpret_cast<uint4 *>(S.HW() + sw128_off(row, 2 * cq + q)) = pack8(hv + 8 * q, amax);
+                } else if (final_state && u == U - 1) {
+                    float *dst = final_state + bh * kNP + (size_t)row * kP + cq * 16;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int p = q * 8 + e;
-                    yv[p] = fmaf(Dh, xs[e], fmaf(ei, zv[p], yv[p]));
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<float4 *>(dst + 4 * q) =
+                            make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
                 }
             }
-            uint8_t *stg = sCW + ch * kTileBytes;
+            if (k + 1 < kb1) co_signal(S.bar(kBarH16), tid);
+
+            // [4] y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging (the C tiles of stage s,
+            //     as two 32-column fp32 tiles) -> epi_done; the control warp stores it
+            if (ok) {
+                const float ei = expf(fminf(cum[row], 0.f));
+                float xs[16];
+                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 2 * cq)), xs);
+                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 2 * cq + 1)), xs + 8);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                *reinterpret_cast<float4 *>(stg + sw128_off(row, q)) =
-                    make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
-            const bool last = (k + 1 == kb1);
-            float v[32];
-            tmem_ld32(lane_addr + tH + ch * 32, v);
-            if (!last) {
+                for (int p = 0; p < 16; ++p) yv[p] = fmaf(Dh, xs[p], fmaf(ei, zv[p], yv[p]));
+                uint8_t *stg = S.C(s) + (cq >> 1) * kTileBytes;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(sHW + sw128_off(row, ch * 4 + q)) = pack8(v + 8 * q, amax);
-            } else if (final_state && u == U - 1) {
-                float *dst = final_state + bh * kNP + (size_t)row * kP + ch * 32;
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    *reinterpret_cast<float4 *>(dst + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    *reinterpret_cast<float4 *>(stg + sw128_off(row, (cq & 1) * 4 + q)) =
+                        make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
             }
+            co_signal(S.bar(kBarEpi), tid);
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            tma_store_4d(&maps.y, sCW, 0, h, t0, b);
-            tma_store_4d(&maps.y, sCW + kTileBytes, 32, h, t0, b);
-            tma_store_commit();
-        }
+        named_bar_sync(kCoCompute);
+        if (__any_sync(0xffffffffu, !in_f16_range(amax)) && lane == 0) flag_status(ws.status, kStatusRange);
     }
-    if (tid == 0) tma_store_wait_all();
-    if (!ok && tid == 0) flag_status(ws.status, kStatusTimeout);
-    if (!__syncthreads_and(amax <= kF16Max) && tid == 0) flag_status(ws.status, kStatusRange);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (tid == 0 && *abort_flag) flag_status(ws.status, kStatusTimeout);
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
@@ -712,7 +891,7 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     if (p.U > 1) {
         {
             TraceScope tr(s, kTrTcUnitState);
-            unit_state_kernel<<<dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kThreads, kUsSmem, s>>>(
+            unit_state_kernel<<<dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kUsThreads, kUsSmem, s>>>(
                 maps, ws, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -725,7 +904,7 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     }
     {
         TraceScope tr(s, kTrTcChunkOut);
-        chunk_out_kernel<<<dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kThreads, kCoSmem, s>>>(
+        chunk_out_kernel<<<dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem, s>>>(
             maps, a.D, a.init_state, a.final_state, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U,
             (int)p.bpu, p.U > 1 ? 1 : 0);
     }
