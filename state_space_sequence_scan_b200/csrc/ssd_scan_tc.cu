@@ -59,10 +59,18 @@ constexpr int kBlk = 128;                       // tokens per block
 constexpr int kN = 128;                         // state_dim
 constexpr int kP = 64;                          // head_dim
 constexpr int kNP = kN * kP;
-constexpr int kThreads = 256;                   // 8 warps; warps w and w+4 share TMEM lanes 32*(w%4)..
 constexpr long long kWaitBudget = 1ll << 32;    // clock cycles before a wait gives up (~2 s)
 constexpr float kF16Max = 65504.0f;
-constexpr int kUnitTarget = 8 * 148;            // aim for ~8 units per SM across the grid
+constexpr int kSMs = 148;                       // B200 streaming multiprocessors
+// Relative cost of the unit decomposition, in chunk_out block-times (one
+// 128-token block of one CTA; chunk_out runs one CTA per SM): unit_state runs
+// two CTAs per SM at about this fraction of a chunk_out block, and the
+// state pass costs about this many block-times.
+// A CTA also pays about kCtaStartRel block-times to start its pipeline.
+constexpr double kUnitStateRel = 0.35;
+constexpr double kStatePassRel = 5.0;
+constexpr double kCtaStartRel = 2.0;
+constexpr int64_t kMaxUnits = 4096;
 constexpr uint32_t kTileBytes = 16384;          // one 128-row x 128-byte swizzled tile
 
 struct TcWs {
@@ -92,11 +100,28 @@ TcPlan make_plan(const ScanDims &d) {
         p.bpu = 1;
         return p;
     }
-    int64_t U = 1;
-    while (d.b * d.H * U < kUnitTarget && U < p.nblk) U *= 2;
-    if (U > p.nblk) U = p.nblk;
-    p.bpu = (p.nblk + U - 1) / U;
-    p.U = (p.nblk + p.bpu - 1) / p.bpu;
+    // Split every (batch, head) chain into U units of bpu blocks so that the
+    // grid's waves times the blocks per unit, plus the passes that carry the
+    // state between units, is smallest (ties: fewer units).  A function of
+    // the shape alone, so the workspace size is known before the launch.
+    const int64_t chains = d.b * d.H;
+    double best = 0.0;
+    p.U = 1;
+    p.bpu = p.nblk;
+    for (int64_t U = 1; U <= p.nblk && U <= kMaxUnits; ++U) {
+        const int64_t bpu = (p.nblk + U - 1) / U;
+        if ((p.nblk + bpu - 1) / bpu != U) continue;         // same split as a smaller U
+        double cost = (double)((chains * U + kSMs - 1) / kSMs) * ((double)bpu + kCtaStartRel);
+        if (U > 1)
+            cost += (double)((chains * (U - 1) + 2 * kSMs - 1) / (2 * kSMs)) * ((double)bpu + kCtaStartRel) *
+                        kUnitStateRel +
+                    kStatePassRel;
+        if (U == 1 || cost < best) {
+            best = cost;
+            p.U = U;
+            p.bpu = bpu;
+        }
+    }
     return p;
 }
 
@@ -196,16 +221,25 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
         const int t0 = blk * kBlk;
         const size_t Lp = (size_t)nblk * kBlk;
         __half2 amax = __float2half2_rn(0.f);
-#pragma unroll 4
-        for (int c = threadIdx.x; c < 2 * kBlk * 16; c += 256) {
-            const int which = c >> 11, r = (c >> 4) & (kBlk - 1), kk = c & 15;
-            const int t = t0 + r;
+        // all 16 loads of a thread in flight before any conversion
+        uint4 v[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int c = threadIdx.x + 256 * r;
+            const int which = c >> 11, row = (c >> 4) & (kBlk - 1), kk = c & 15;
+            const int t = t0 + row;
             const __nv_bfloat16 *src = which ? Cm : Bm;
+            v[r] = make_uint4(0u, 0u, 0u, 0u);
+            if (t < L) v[r] = __ldg(reinterpret_cast<const uint4 *>(src + (((size_t)b * L + t) * G + g) * kN + kk * 8));
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int c = threadIdx.x + 256 * r;
+            const int which = c >> 11, row = (c >> 4) & (kBlk - 1), kk = c & 15;
+            const int t = t0 + row;
             __half *dst = which ? ws.Ch : ws.Bh;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < L) v = __ldg(reinterpret_cast<const uint4 *>(src + (((size_t)b * L + t) * G + g) * kN + kk * 8));
             float f[8];
-            bf16_chunk_to_f32(v, f);
+            bf16_chunk_to_f32(v[r], f);
             *reinterpret_cast<uint4 *>(dst + (((size_t)b * Lp + t) * G + g) * kN + kk * 8) = pack8(f, amax);
         }
         if (!in_f16_range(amax)) flag_status(ws.status, kStatusRange);
@@ -213,17 +247,28 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
     }
     const int h0 = blockIdx.y * 32;
     const int nh = min(32, H - h0);
-    for (int e = threadIdx.x; e < kBlk * 32; e += 256) {
-        const int tok = e >> 5, hh = e & 31;
-        const int t = blk * kBlk + tok;
-        float d = 0.f, da = 0.f;
-        if (hh < nh && t < L) {
-            const int h = h0 + hh;
-            d = dt_of(dt_raw[((size_t)b * L + t) * H + h], dt_bias[h], lo, hi);
-            da = d * A[h];
+    {
+        // thread -> head hh = tid % 32 (fixed), tokens tid / 32 + 8 r: all 16
+        // loads in flight before the softplus
+        const int hh = threadIdx.x & 31;
+        const bool hv = hh < nh;
+        const float bias = hv ? dt_bias[h0 + hh] : 0.f, Ah = hv ? A[h0 + hh] : 0.f;
+        float raw[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int tok = (threadIdx.x >> 5) + 8 * r;
+            const int t = blk * kBlk + tok;
+            raw[r] = (hv && t < L) ? dt_raw[((size_t)b * L + t) * H + h0 + hh] : 0.f;
         }
-        s_dt[tok][hh] = d;
-        s_da[tok][hh] = da;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const int tok = (threadIdx.x >> 5) + 8 * r;
+            const int t = blk * kBlk + tok;
+            float d = 0.f;
+            if (hv && t < L) d = dt_of(raw[r], bias, lo, hi);
+            s_dt[tok][hh] = d;
+            s_da[tok][hh] = d * Ah;
+        }
     }
     if (blk == 0 && b == 0 && threadIdx.x < nh && A[h0 + threadIdx.x] > 0.f)
         flag_status(ws.status, kStatusPrecondition);
@@ -428,37 +473,53 @@ tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
 }
 
 // ---------------------------------------------------------------------------
-// chunk_out: grid (H, U, b), one CTA per SM: 16 compute warps + 1 control warp.
+// chunk_out: grid (H, U, b), one CTA per SM: 8 compute warps, an MMA warp and
+// a TMA warp.
 //
-// The control warp's lane 0 issues every TMA copy and every MMA, driven by
-// mbarriers, so the compute warps never wait on issue.  Per 128-token block k
-// (two TMA stages; tiles of block k+2 stream in meanwhile), each MMA runs
-// while the compute warps do independent work:
-//   compute: [1] C.B^T(k), C.H(k) done -> W, w.X, state*decay     -> w_ready
-//            [2] tiles(k+1) landed -> decay factors, X widened     -> ops_ready
-//            [3] W.X(k), state update done -> fp16 state for k+1   -> h16_ready
-//            [4] y(k) staged in block k's C tiles (dead once C.B^T(k)
-//                and C.H(k) are done)                              -> epi_done
-//   control: w_ready -> W.X(k), B^T.(wX)(k);  ops_ready -> C.B^T(k+1);
-//            h16_ready -> C.H(k+1);  epi_done -> y(k) TMA store, tiles(k+2)
-//            (the C tiles of k+2 once the store has read the staging).
-// Compute warp w owns TMEM lanes 32*(w%4).. (its rows) and column slice w/4
-// of each TMEM region: 32 of the 128 C.B^T columns, 16 of the 64 Y/Z/state
-// columns.
-constexpr int kCoCompute = 512;                                 // 16 compute warps
-constexpr int kCoThreads = kCoCompute + 32;                     // + control warp
+// The MMA warp's lane 0 issues every tcgen05.mma, the TMA warp's lane 0
+// every bulk copy; both only wait on mbarriers, so the compute warps never
+// stall on an issue (a tcgen05.mma holds its issuing thread for about as
+// long as it runs).  Per 128-token block k the compute warps run:
+//   [1] C.B^T(k) done -> W(k) into TMEM (fp16, the A operand of W.X)
+//                                                 -> MMA: S(k) = B^T (w.X(k)), Y(k) = W(k) X(k)
+//   [2] tiles(k+1) landed -> decay factors, X(k+1) widened in place and w.X(k+1)
+//                                                 -> MMA: C.B^T(k+1)
+//   [3] S(k), Z(k) done -> H_in(k+1) = a_k H_in(k) + S(k) in registers, fp16 copy
+//                                                 -> MMA: Z(k+1) = C(k+1) H_in(k+1)
+//   [4] Y(k) done -> y(k) = Y + exp(cum) Z(k) + D x, staged in block k's C tiles
+//                                                 -> TMA: store y(k), then tiles(k+2)
+// so the tensor pipe runs S(k), Y(k), C.B^T(k+1), Z(k+1) back to back while
+// the compute warps form operands.  Compute warp w owns TMEM lanes
+// 32*(w%4).. (its rows) and column half w/4: 64 of the 128 C.B^T columns and
+// 32 of the 64 Y/Z/S/state columns.
+constexpr int kCoCompute = 256;                                 // 8 compute warps
+constexpr int kCoWarps = kCoCompute / 32;
+constexpr int kCoMmaWarp = kCoWarps, kCoTmaWarp = kCoWarps + 1;
+constexpr int kCoThreads = kCoCompute + 64;                     // + MMA warp + TMA warp
 constexpr uint32_t kCoStage = 5 * kTileBytes + 2 * kBlk * 4;   // C(2) B(2) X(1) tiles, dt, cum
+constexpr uint32_t kCoOffWX = 2 * kCoStage;                     // w.X fp16, one tile per stage
+constexpr uint32_t kCoOffH16 = kCoOffWX + 2 * kTileBytes;       // fp16 entering state [n][p]
 constexpr uint32_t kCoFactors = 640;                            // w[128], v[3][128], vd[128]
-constexpr uint32_t kCoOffW = 2 * kCoStage;                      // W tile (2 tiles)
-constexpr uint32_t kCoOffHW = kCoOffW + 2 * kTileBytes;         // fp16 state, then w.X
-constexpr uint32_t kCoOffF = kCoOffHW + kTileBytes;             // factors [2][640] floats
+constexpr uint32_t kCoOffF = kCoOffH16 + kTileBytes;            // factors [2][640] floats
 constexpr uint32_t kCoOffG = kCoOffF + 2 * kCoFactors * 4;      // diagonal fast-path flags [2][4]
-constexpr uint32_t kCoOffBar = kCoOffG + 8 * 4;                 // 8 mbarriers, TMEM slot, abort flag
-constexpr size_t kCoSmem = 1024 + kCoOffBar + 8 * 8 + 16;
+constexpr uint32_t kCoOffMask = kCoOffG + 8 * 4;                // causal masks of the diagonal [4][32 lanes] x 16 B
+constexpr uint32_t kCoOffIss = kCoOffMask + 32 * 16 * 4;        // issue counters (drain after an abort)
+constexpr uint32_t kCoOffBar = kCoOffIss + 16 * 4;              // mbarriers, TMEM slot, abort flag
+constexpr int kCoBars = 10;
+constexpr size_t kCoSmem = 1024 + kCoOffBar + kCoBars * 8 + 16;
 constexpr float kDiagExpCap = 64.0f;                            // largest exponent on the diagonal fast path
+static_assert(kCoStage % 1024 == 0, "stage tiles must stay 1024-byte aligned");
+static_assert(kCoSmem <= 232448, "chunk_out shared memory exceeds the per-CTA limit");
 
-enum CoBar { kBarTma0 = 0, kBarTma1 = 1, kBarCBZ = 2, kBarYS = 3, kBarOps = 4, kBarW = 5, kBarEpi = 6,
-             kBarH16 = 7 };
+// TMEM columns (512 allocated)
+constexpr uint32_t kTmCB = 0;      // C.B^T fp32, 128 columns
+constexpr uint32_t kTmW = 128;     // W fp16 pairs, 64 columns
+constexpr uint32_t kTmY = 192;     // W.X fp32, 64 columns
+constexpr uint32_t kTmS = 256;     // B^T.(w.X) fp32, 64 columns
+constexpr uint32_t kTmZ = 320;     // C.H fp32, two buffers of 64 columns (block parity)
+
+enum CoBar { kBarTma0 = 0, kBarTma1 = 1, kBarCB = 2, kBarS = 3, kBarY = 4, kBarZ = 5,   // completion
+             kBarW = 6, kBarOps = 7, kBarH16 = 8, kBarFree = 9 };                       // compute -> issuers
 
 struct CoSmem {
     uint8_t *base;
@@ -467,41 +528,36 @@ struct CoSmem {
     __device__ uint8_t *X(int s) const { return base + s * kCoStage + 4 * kTileBytes; }
     __device__ float *dt(int s) const { return reinterpret_cast<float *>(base + s * kCoStage + 5 * kTileBytes); }
     __device__ float *cum(int s) const { return dt(s) + kBlk; }
-    __device__ uint8_t *W() const { return base + kCoOffW; }
-    __device__ uint8_t *HW() const { return base + kCoOffHW; }
+    __device__ uint8_t *WX(int s) const { return base + kCoOffWX + s * kTileBytes; }
+    __device__ uint8_t *H16() const { return base + kCoOffH16; }
     __device__ float *F(int s) const { return reinterpret_cast<float *>(base + kCoOffF) + s * kCoFactors; }
     __device__ int *G(int s) const { return reinterpret_cast<int *>(base + kCoOffG) + s * 4; }
+    __device__ uint4 *Mask() const { return reinterpret_cast<uint4 *>(base + kCoOffMask); }
+    __device__ int *issued() const { return reinterpret_cast<int *>(base + kCoOffIss); }
     __device__ uint64_t *bar(int i) const { return reinterpret_cast<uint64_t *>(base + kCoOffBar) + i; }
-    __device__ uint32_t *tslot() const { return reinterpret_cast<uint32_t *>(bar(8)); }
-    __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(bar(8)) + 1; }
+    __device__ uint32_t *tslot() const { return reinterpret_cast<uint32_t *>(bar(kCoBars)); }
+    __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(bar(kCoBars)) + 1; }
 };
 
-// TMA for block k into stage s, in two parts on one barrier (which expects
-// the bytes of both): B (fp16 copy), X (bf16), dt and cum rows first, then the
-// C tiles (fp16 copy), which may have to wait for a y store out of them.
-__device__ __forceinline__ void co_load_bx(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
-                                           int s, int k, int g, int h, int b) {
+// Shared-memory descriptors advance by (byte offset >> 4) in their low field
+// (smem addresses stay below 2^18, so the 14-bit field never carries).
+__device__ __forceinline__ uint64_t dadd(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
+// TMA for block k into stage s: C and B (fp16 copies), X (bf16), dt and cum
+// rows, all completing on the stage's barrier.
+__device__ __forceinline__ void co_load(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
+                                        int s, int k, int g, int h, int b) {
     const int t0 = k * kBlk;
     uint64_t *bar = S.bar(kBarTma0 + s);
-    mbar_arrive_expect_tx(bar, 5 * kTileBytes + 2 * kBlk * 4);
+    mbar_arrive_expect_tx(bar, kCoStage);
+    tma_load_4d(S.C(s), &maps.C, bar, 0, g, t0, b);
+    tma_load_4d(S.C(s) + kTileBytes, &maps.C, bar, 64, g, t0, b);
     tma_load_4d(S.B(s), &maps.B, bar, 0, g, t0, b);
     tma_load_4d(S.B(s) + kTileBytes, &maps.B, bar, 64, g, t0, b);
     tma_load_4d(S.X(s), &maps.x, bar, 0, h, t0, b);
     bulk_load(S.dt(s), dtv + (size_t)t0, kBlk * 4, bar);
     bulk_load(S.cum(s), cum + (size_t)t0, kBlk * 4, bar);
-}
-
-__device__ __forceinline__ void co_load_c(const CoSmem &S, const TcMaps &maps, int s, int k, int g, int b) {
-    const int t0 = k * kBlk;
-    uint64_t *bar = S.bar(kBarTma0 + s);
-    tma_load_4d(S.C(s), &maps.C, bar, 0, g, t0, b);
-    tma_load_4d(S.C(s) + kTileBytes, &maps.C, bar, 64, g, t0, b);
-}
-
-__device__ __forceinline__ void co_load(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
-                                        int s, int k, int g, int h, int b) {
-    co_load_bx(S, maps, dtv, cum, s, k, g, h, b);
-    co_load_c(S, maps, s, k, g, b);
+    ++S.issued()[kBarTma0 + s];
 }
 
 // Per-block decay factors (all exponents clamped as stated):
@@ -530,31 +586,105 @@ __device__ __forceinline__ void co_factors(const CoSmem &S, int s, int last_vali
     if (tid < 4) S.G(s)[tid] = (cum[32 * tid] - cum[32 * tid + 31]) <= kDiagExpCap ? 1 : 0;
 }
 
-// X tile of stage s: bf16 -> fp16 in place (two 16-byte chunks per thread).
+// X tile of stage s: bf16 -> fp16 in place, and w.X (fp16) into WX(s) in the
+// same swizzled layout (four 16-byte chunks per thread; a chunk's row is its
+// offset / 128 whatever the swizzle).
 __device__ __forceinline__ void co_widen_x(const CoSmem &S, int s, int tid, __half2 &amax) {
+    const float *w = S.F(s);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        uint4 *p = reinterpret_cast<uint4 *>(S.X(s) + (tid + r * kCoCompute) * 16);
+    for (int r = 0; r < 4; ++r) {
+        const int c = tid + r * kCoCompute;
+        uint4 *p = reinterpret_cast<uint4 *>(S.X(s) + c * 16);
         float f[8];
         bf16_chunk_to_f32(*p, f);
         *p = pack8(f, amax);
+        const float2 wj = make_float2(w[c >> 3], w[c >> 3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 m = __fmul2_rn(make_float2(f[2 * e], f[2 * e + 1]), wj);
+            f[2 * e] = m.x;
+            f[2 * e + 1] = m.y;
+        }
+        *reinterpret_cast<uint4 *>(S.WX(s) + c * 16) = pack8(f, amax);
     }
 }
 
-// TMEM column of the C.H accumulator of the block in stage s (two buffers:
-// block k+1's is written while block k's is still being read).
-__device__ __forceinline__ uint32_t co_tz(int s) { return s ? 384u : 64u; }
-
-// Compute warps: publish this step's smem/TMEM writes, sync the 512 compute
-// threads, and let one of them arrive on `bar` for the control thread.
-__device__ __forceinline__ void co_signal(uint64_t *bar, int tid) {
+// A compute warp hands its shared-memory and TMEM writes to the issuing
+// warps: one arrival per warp on `bar` (initialised with kCoWarps).
+__device__ __forceinline__ void co_arrive(uint64_t *bar, int lane) {
     fence_proxy_async_smem();
     tc_fence_before();
-    named_bar_sync(kCoCompute);
-    if (tid == 0) mbar_arrive(bar);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
 }
 
-__global__ void __launch_bounds__(kCoThreads)
+// 16 floats -> 8 fp16 pairs
+__device__ __forceinline__ void pack16(const float *v, uint32_t *o, __half2 &amax) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        o[q] = pack_h2(v[2 * q], v[2 * q + 1]);
+        amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&o[q])));
+    }
+}
+
+// W for one 32-column slice cq <= lg of this thread's row (see co_factors).
+__device__ __forceinline__ void co_w_slice(const CoSmem &S, int s, uint32_t lane_addr, int lg, int cq, int lane,
+                                           float ci, __half2 &amax) {
+    const float *cum = S.cum(s);
+    const float *F = S.F(s);
+    float v[32];
+    tmem_ld32(lane_addr + kTmCB + cq * 32, v);
+    uint32_t o[16];
+    if (cq < lg) {                                   // below the diagonal: factored decay
+        const float ui = expf(fminf(ci - cum[32 * lg - 1], 0.f));
+        const float2 u2 = make_float2(ui, ui);
+        const float2 *vf = reinterpret_cast<const float2 *>(F + kBlk * lg + cq * 32);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const float2 f = __fmul2_rn(vf[q], u2);
+            const float2 m = __fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), f);
+            v[2 * q] = m.x;
+            v[2 * q + 1] = m.y;
+        }
+        pack16(v, o, amax);
+        pack16(v + 16, o + 8, amax);
+    } else {                                         // diagonal 32x32
+        if (S.G(s)[lg]) {
+            const float ud = expf(fminf(ci - cum[32 * lg], 0.f));
+            const float2 u2 = make_float2(ud, ud);
+            const float2 *vf = reinterpret_cast<const float2 *>(F + 4 * kBlk + cq * 32);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const float2 f = __fmul2_rn(vf[q], u2);
+                const float2 m = __fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), f);
+                v[2 * q] = m.x;
+                v[2 * q + 1] = m.y;
+            }
+        } else {                                     // steep decay: one exp per element
+            const float *dts = S.dt(s) + cq * 32, *cj = cum + cq * 32;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                v[jj] = v[jj] * expf(fminf(ci - cj[jj], 0.f)) * dts[jj];
+                asm volatile("" ::: "memory");       // one element at a time: keeps the loads from piling up
+            }
+        }
+        // causal select on the packed pairs (j <= i kept), before the range check
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 m4 = S.Mask()[q4 * 32 + lane];
+            const uint32_t mw[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int q = 4 * q4 + e;
+                o[q] = pack_h2(v[2 * q], v[2 * q + 1]) & mw[e];
+                amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&o[q])));
+            }
+        }
+    }
+    tmem_st16u(lane_addr + kTmW + 16 * cq, o);
+}
+
+__global__ void __launch_bounds__(kCoThreads, 1)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
                  const float *__restrict__ init, float *__restrict__ final_state, TcWs ws,
                  int L, int H, int G, int nblk, int U, int bpu, int states_from_ws) {
@@ -576,7 +706,10 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(S.bar(i), 1);
+        for (int i = 0; i < kCoBars; ++i) {
+            mbar_init(S.bar(i), i < kBarW ? 1 : kCoWarps);
+            S.issued()[i] = 0;
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -584,271 +717,278 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *S.tslot();
-    const uint32_t tH = 0;                           // TMEM columns: state; C.H at co_tz(s); C.B^T/Y at 128, 256
 
-    if (warp == kCoCompute / 32) {
-        // ------------------------------ control warp --------------------------
+    if (warp == kCoMmaWarp) {
+        // ------------------------------ MMA warp ------------------------------
         if (lane == 0) {
-            const uint32_t idesc_z = idesc_f16(128, 64, 0, 1);    // A=C K-major, B=H MN-major
             const uint32_t idesc_cb = idesc_f16(128, 128, 0, 0);  // A=C K-major, B=B K-major
-            const uint32_t idesc_y = idesc_f16(128, 64, 0, 1);    // A=W K-major, B=X MN-major
+            const uint32_t idesc_z = idesc_f16(128, 64, 0, 1);    // A=C K-major, B=H MN-major
+            const uint32_t idesc_y = idesc_f16(128, 64, 0, 1);    // A=W (TMEM) K-major, B=X MN-major
             const uint32_t idesc_s = idesc_f16(128, 64, 1, 1);    // A=B^T MN-major, B=wX MN-major
-            const uint32_t h_base = smem_u32(S.HW()), w_base = smem_u32(S.W());
-            bool ok = true;
-            co_load(S, maps, dtg, cumg, 0, kb0, g, h, b);
-            if (kb0 + 1 < kb1) co_load(S, maps, dtg, cumg, 1, kb0 + 1, g, h, b);
-            // block kb0: C.B^T and C.H once its operands are ready
-            ok = mbar_wait_abortable(S.bar(kBarOps), 0, kWaitBudget, abort_flag);
-            tc_fence_after();
-            if (ok) {
-                const uint32_t c_base = smem_u32(S.C(0)), b_base = smem_u32(S.B(0));
+            // stage 1's descriptors are stage 0's plus the stage stride (no array:
+            // a dynamically indexed one would live in local memory)
+            const uint64_t dC0 = sdesc_sw128(smem_u32(S.C(0)), 16, 1024);
+            const uint64_t dBk0 = sdesc_sw128(smem_u32(S.B(0)), 16, 1024);
+            const uint64_t dBm0 = sdesc_sw128(smem_u32(S.B(0)), kTileBytes, 1024);
+            const uint64_t dX0 = sdesc_sw128(smem_u32(S.X(0)), kTileBytes, 1024);
+            const uint64_t dWX0 = sdesc_sw128(smem_u32(S.WX(0)), kTileBytes, 1024);
+            const uint64_t dH = sdesc_sw128(smem_u32(S.H16()), kTileBytes, 1024);
+            auto st = [](int s) { return (uint32_t)s * kCoStage; };
+            auto wxs = [](int s) { return (uint32_t)s * kTileBytes; };
+            // K-major K-step q of a 128-wide tile: column block q/4, 32 bytes per step inside it
+            auto kofs = [](int q) { return (uint32_t)((q >> 2) * kTileBytes + (q & 3) * 32); };
+            auto issue_cb = [&](int s) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint64_t ad = sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024);
-                    mma_f16(tmem + 128u, ad, sdesc_sw128(b_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
-                            idesc_cb, q > 0);
-                    mma_f16(tmem + co_tz(0), ad, sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_z, q > 0);
-                }
-                mma_commit(S.bar(kBarCBZ));
-            }
+                for (int q = 0; q < 8; ++q)
+                    mma_f16(tmem + kTmCB, dadd(dC0, st(s) + kofs(q)), dadd(dBk0, st(s) + kofs(q)), idesc_cb, q > 0);
+                mma_commit(S.bar(kBarCB));
+                ++S.issued()[kBarCB];
+            };
+            auto issue_z = [&](int s, int zb) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    mma_f16(tmem + kTmZ + 64u * zb, dadd(dC0, st(s) + kofs(q)), dadd(dH, q * 2048), idesc_z, q > 0);
+                mma_commit(S.bar(kBarZ));
+                ++S.issued()[kBarZ];
+            };
+            auto issue_sy = [&](int s) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    mma_f16(tmem + kTmS, dadd(dBm0, st(s) + q * 2048), dadd(dWX0, wxs(s) + q * 2048), idesc_s, q > 0);
+                mma_commit(S.bar(kBarS));
+                ++S.issued()[kBarS];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    mma_f16_ts(tmem + kTmY, tmem + kTmW + 8u * q, dadd(dX0, st(s) + q * 2048), idesc_y, q > 0);
+                mma_commit(S.bar(kBarY));
+                ++S.issued()[kBarY];
+            };
+            bool ok = mbar_wait_abortable(S.bar(kBarOps), 0, kWaitBudget, abort_flag);
+            tc_fence_after();
+            if (ok) issue_cb(0);
+            ok = ok && mbar_wait_abortable(S.bar(kBarH16), 0, kWaitBudget, abort_flag);
+            tc_fence_after();
+            if (ok) issue_z(0, 0);
             for (int k = kb0; k < kb1 && ok; ++k) {
                 const int i = k - kb0, s = i & 1, s1 = s ^ 1;
                 const uint32_t par = (uint32_t)i & 1u, par1 = (uint32_t)(i + 1) & 1u;
-                const uint32_t tcb = 128u + 128u * s, tcb1 = 128u + 128u * s1;
-                // W.X(k) and the state update once W and w.X are in place
                 ok = mbar_wait_abortable(S.bar(kBarW), par, kWaitBudget, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                {
-                    const uint32_t x_base = smem_u32(S.X(s)), b_base = smem_u32(S.B(s));
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        mma_f16(tmem + tcb, sdesc_sw128(w_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
-                                sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc_y, q > 0);
-                        mma_f16(tmem + tH, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
-                                sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_s, 1u);
-                    }
-                    mma_commit(S.bar(kBarYS));
-                }
+                issue_sy(s);
                 if (k + 1 < kb1) {
-                    // C.B^T of block k+1 as soon as its operands are ready
                     ok = mbar_wait_abortable(S.bar(kBarOps), par1, kWaitBudget, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t c_base = smem_u32(S.C(s1)), b_base = smem_u32(S.B(s1));
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        mma_f16(tmem + tcb1, sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
-                                sdesc_sw128(b_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024), idesc_cb,
-                                q > 0);
-                    // C.H of block k+1 once its fp16 entering state is in HW; one commit for both
-                    ok = mbar_wait_abortable(S.bar(kBarH16), par, kWaitBudget, abort_flag);
+                    issue_cb(s1);
+                    ok = mbar_wait_abortable(S.bar(kBarH16), par1, kWaitBudget, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        mma_f16(tmem + co_tz(s1), sdesc_sw128(c_base + (q >> 2) * kTileBytes + (q & 3) * 32, 16, 1024),
-                                sdesc_sw128(h_base + q * 2048, kTileBytes, 1024), idesc_z, q > 0);
-                    mma_commit(S.bar(kBarCBZ));
+                    issue_z(s1, (int)par1);
                 }
-                // y(k) staged: store it, then refill stage s with block k+2
-                ok = mbar_wait_abortable(S.bar(kBarEpi), par, kWaitBudget, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
+            }
+            if (!ok) *abort_flag = 1;
+        }
+        __syncwarp();
+    } else if (warp == kCoTmaWarp) {
+        // ------------------------------ TMA warp ------------------------------
+        if (lane == 0) {
+            co_load(S, maps, dtg, cumg, 0, kb0, g, h, b);
+            if (kb0 + 1 < kb1) co_load(S, maps, dtg, cumg, 1, kb0 + 1, g, h, b);
+            for (int k = kb0; k < kb1; ++k) {
+                const int i = k - kb0, s = i & 1;
+                if (!mbar_wait_abortable(S.bar(kBarFree), (uint32_t)i & 1u, kWaitBudget, abort_flag)) break;
+                // y(k) sits in block k's C tiles as two 32-column fp32 tiles
                 tma_store_4d(&maps.y, S.C(s), 0, h, k * kBlk, b);
                 tma_store_4d(&maps.y, S.C(s) + kTileBytes, 32, h, k * kBlk, b);
                 tma_store_commit();
                 if (k + 2 < kb1) {
-                    // every MMA of block k has completed (the compute warps waited on
-                    // them) and its epilogue is done: only the y store still reads
-                    // stage s, from its C tiles
-                    co_load_bx(S, maps, dtg, cumg, s, k + 2, g, h, b);
                     tma_store_wait_read();
-                    co_load_c(S, maps, s, k + 2, g, b);
+                    co_load(S, maps, dtg, cumg, s, k + 2, g, h, b);
                 }
             }
             tma_store_wait_all();
-            if (!ok) *abort_flag = 1;
         }
         __syncwarp();
     } else {
         // ------------------------------ compute warps -------------------------
         const int lg = warp & 3;                    // row group: rows 32*lg .. 32*lg+31
         const int row = 32 * lg + lane;             // TMEM lane / tile row of this thread
-        const int cq = warp >> 2;                   // column slice 0..3
+        const int ch = warp >> 2;                   // column half 0..1
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * lg) << 16);
         const float Dh = D[h];
         __half2 amax = __float2half2_rn(0.f);
         bool ok = true;
 
-        // state entering the unit -> TMEM (fp32) and HW (fp16): row `row`, columns 16*cq..
+        // entering state of the unit, row `row`, columns 32*ch..: registers and fp16 copy
+        float hv[32];
         {
             const float *src = states_from_ws ? ws.states + (bh * U + u) * (size_t)kNP
                                               : (init ? init + bh * kNP : nullptr);
-            float v[16];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 f = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kP + cq * 16 + 4 * q)
+            for (int q = 0; q < 8; ++q) {
+                const float4 f = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kP + ch * 32 + 4 * q)
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+                hv[4 * q] = f.x; hv[4 * q + 1] = f.y; hv[4 * q + 2] = f.z; hv[4 * q + 3] = f.w;
             }
-            tmem_st16(lane_addr + tH + cq * 16, v);
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
-                *reinterpret_cast<uint4 *>(S.HW() + sw128_off(row, cq * 2 + q)) = pack8(v + 8 * q, amax);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t o[8];
+                pack16(hv + 16 * hh, o, amax);
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+                    *reinterpret_cast<uint4 *>(S.H16() + sw128_off(row, 4 * ch + 2 * hh + q)) =
+                        make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            }
+            // W above the diagonal sub-blocks stays zero for the whole kernel
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int cq = 2 * ch + t;
+                if (cq > lg) {
+                    uint32_t z[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) z[q] = 0u;
+                    tmem_st16u(lane_addr + kTmW + 16 * cq, z);
+                }
+            }
+            // causal masks of a diagonal sub-block: lane l keeps columns jj <= l;
+            // word q holds jj = 2q (low half) and 2q+1 (high half)
+            if (tid < 128) {
+                const int ml = tid & 31, q4 = tid >> 5;
+                uint32_t mw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int q = 4 * q4 + e;
+                    mw[e] = (2 * q + 1 <= ml ? 0xFFFF0000u : 0u) | (2 * q <= ml ? 0x0000FFFFu : 0u);
+                }
+                S.Mask()[q4 * 32 + ml] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+            }
         }
-        // block kb0: tiles landed -> factors, widened X -> ops_ready
+        co_arrive(S.bar(kBarH16), lane);
+        // block kb0: tiles landed -> factors, widened X and w.X
         ok = mbar_wait_abortable(S.bar(kBarTma0), 0, kWaitBudget, abort_flag);
-        if (ok) {
-            co_factors(S, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
-            co_widen_x(S, 0, tid, amax);
-        }
-        co_signal(S.bar(kBarOps), tid);
+        if (ok) co_factors(S, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
+        named_bar_sync(kCoCompute);                 // factors and masks visible to every compute warp
+        if (ok) co_widen_x(S, 0, tid, amax);
+        co_arrive(S.bar(kBarOps), lane);
 
-        // every compute thread runs every iteration (and so every named barrier);
+        // every compute warp runs every iteration (and so every named barrier);
         // after an abort the waits return at once and the work is skipped
         for (int k = kb0; k < kb1; ++k) {
             const int i = k - kb0, s = i & 1, s1 = s ^ 1;
             const uint32_t par = (uint32_t)i & 1u;
-            const uint32_t tcb = 128u + 128u * s;
             const int t0 = k * kBlk;
             const float *cum = S.cum(s);
-            const float *F = S.F(s);
 
-            // [1] C.B^T(k), C.H(k) done -> W, w.X, state * decay -> w_ready
-            ok = ok && mbar_wait_abortable(S.bar(kBarCBZ), par, kWaitBudget, abort_flag);
+            // [1] C.B^T(k) done -> W(k) (fp16 pairs) into TMEM
+            ok = ok && mbar_wait_abortable(S.bar(kBarCB), par, kWaitBudget, abort_flag);
             ok = __all_sync(0xffffffffu, ok);        // warp-uniform before tcgen05.ld
             tc_fence_after();
             if (ok) {
-                const int c32 = cq;
                 const float ci = cum[row];
-                uint4 out[4];
-                if (c32 < lg) {                          // below the diagonal: factored decay
-                    float v[32];
-                    tmem_ld32(lane_addr + tcb + c32 * 32, v);
-                    const float ui = expf(fminf(ci - cum[32 * lg - 1], 0.f));
-                    const float4 *vf = reinterpret_cast<const float4 *>(F + kBlk * lg + c32 * 32);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 f = vf[q];
-                        v[4 * q] *= f.x * ui;
-                        v[4 * q + 1] *= f.y * ui;
-                        v[4 * q + 2] *= f.z * ui;
-                        v[4 * q + 3] *= f.w * ui;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, amax);
-                } else if (c32 == lg) {                  // diagonal 32x32: causal select first
-                    float v[32];
-                    tmem_ld32(lane_addr + tcb + c32 * 32, v);
-                    if (S.G(s)[lg]) {
-                        const float ui = expf(fminf(ci - cum[32 * lg], 0.f));
-                        const float4 *vf = reinterpret_cast<const float4 *>(F + 4 * kBlk + c32 * 32);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 f = vf[q];
-                            const float fv[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int jj = 4 * q + e;
-                                v[jj] = (jj <= lane) ? v[jj] * (fv[e] * ui) : 0.f;
-                            }
-                        }
-                    } else {
-                        const float *dts = S.dt(s);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int j = c32 * 32 + jj;
-                            v[jj] = (jj <= lane) ? v[jj] * expf(fminf(ci - cum[j], 0.f)) * dts[j] : 0.f;
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) out[q] = pack8(v + 8 * q, amax);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) out[q] = make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(S.W() + (c32 >> 1) * kTileBytes + sw128_off(row, (c32 & 1) * 4 + q)) =
-                        out[q];
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {            // 1024 chunks of w.X
-                    const int c = tid + r * kCoCompute;
-                    const int j = c >> 3, q = c & 7;
-                    float f[8];
-                    f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(j, q)), f);
-                    const float wj = F[j];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] *= wj;
-                    *reinterpret_cast<uint4 *>(S.HW() + sw128_off(j, q)) = pack8(f, amax);
-                }
-                const float decay = expf(fminf(cum[min(kBlk - 1, L - 1 - t0)], 0.f));
-                float hv[16];
-                tmem_ld16(lane_addr + tH + cq * 16, hv);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) hv[q] *= decay;
-                tmem_st16(lane_addr + tH + cq * 16, hv);
+                if (2 * ch <= lg) co_w_slice(S, s, lane_addr, lg, 2 * ch, lane, ci, amax);
+                if (2 * ch + 1 <= lg) co_w_slice(S, s, lane_addr, lg, 2 * ch + 1, lane, ci, amax);
             }
-            co_signal(S.bar(kBarW), tid);
+            co_arrive(S.bar(kBarW), lane);
 
-            // [2] block k+1: tiles landed -> factors, widened X -> ops_ready (overlaps W.X(k))
+            // [2] block k+1: tiles landed -> factors, widened X, w.X (overlaps S(k), Y(k))
             if (k + 1 < kb1) {
                 ok = ok && mbar_wait_abortable(S.bar(kBarTma0 + s1), ((uint32_t)(i + 1) >> 1) & 1u, kWaitBudget,
                                                abort_flag);
-                if (ok) {
-                    co_factors(S, s1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
-                    co_widen_x(S, s1, tid, amax);
-                }
-                co_signal(S.bar(kBarOps), tid);
+                if (ok) co_factors(S, s1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
+                named_bar_sync(kCoCompute);
+                if (ok) co_widen_x(S, s1, tid, amax);
+                co_arrive(S.bar(kBarOps), lane);
             }
 
-            // [3] W.X(k), state update done -> fp16 entering state of block k+1 -> h16_ready
-            ok = __all_sync(0xffffffffu, ok && mbar_wait_abortable(S.bar(kBarYS), par, kWaitBudget, abort_flag));
+            // [3] S(k) done (and Z(k), which read the fp16 copy) -> H_in(k+1)
+            ok = ok && mbar_wait_abortable(S.bar(kBarS), par, kWaitBudget, abort_flag);
+            ok = ok && mbar_wait_abortable(S.bar(kBarZ), par, kWaitBudget, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            float yv[16], zv[16];
             if (ok) {
-                float hv[16];
-                tmem_ld16x3(lane_addr + tH + cq * 16, hv, lane_addr + tcb + cq * 16, yv, lane_addr + co_tz(s) + cq * 16,
-                            zv);
+                float sv[32];
+                tmem_ld32(lane_addr + kTmS + ch * 32, sv);
+                const float a = expf(fminf(cum[min(kBlk - 1, L - 1 - t0)], 0.f));
+                const float2 a2 = make_float2(a, a);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float2 r = __ffma2_rn(a2, make_float2(hv[2 * q], hv[2 * q + 1]),
+                                                make_float2(sv[2 * q], sv[2 * q + 1]));
+                    hv[2 * q] = r.x;
+                    hv[2 * q + 1] = r.y;
+                }
                 if (k + 1 < kb1) {
 #pragma unroll
-                    for (int q = 0; q < 2; ++q)
-                        *reinterpret_cast<uint4 *>(S.HW() + sw128_off(row, 2 * cq + q)) = pack8(hv + 8 * q, amax);
-                } else if (final_state && u == U - 1) {
-                    float *dst = final_state + bh * kNP + (size_t)row * kP + cq * 16;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t o[8];
+                        pack16(hv + 16 * hh, o, amax);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
+                        for (int q = 0; q < 2; ++q)
+                            *reinterpret_cast<uint4 *>(S.H16() + sw128_off(row, 4 * ch + 2 * hh + q)) =
+                                make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                    }
+                } else if (final_state && u == U - 1) {
+                    float *dst = final_state + bh * kNP + (size_t)row * kP + ch * 32;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
                         *reinterpret_cast<float4 *>(dst + 4 * q) =
                             make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
                 }
             }
-            if (k + 1 < kb1) co_signal(S.bar(kBarH16), tid);
+            if (k + 1 < kb1) co_arrive(S.bar(kBarH16), lane);
 
-            // [4] y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging (the C tiles of stage s,
-            //     as two 32-column fp32 tiles) -> epi_done; the control warp stores it
+            // [4] Y(k) done -> y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging in block k's C tiles
+            ok = ok && mbar_wait_abortable(S.bar(kBarY), par, kWaitBudget, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
             if (ok) {
                 const float ei = expf(fminf(cum[row], 0.f));
-                float xs[16];
-                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 2 * cq)), xs);
-                f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 2 * cq + 1)), xs + 8);
+                const float2 e2 = make_float2(ei, ei), d2 = make_float2(Dh, Dh);
+                uint8_t *stg = S.C(s) + ch * kTileBytes;
 #pragma unroll
-                for (int p = 0; p < 16; ++p) yv[p] = fmaf(Dh, xs[p], fmaf(ei, zv[p], yv[p]));
-                uint8_t *stg = S.C(s) + (cq >> 1) * kTileBytes;
+                for (int hh = 0; hh < 2; ++hh) {
+                    float yv[16], zv[16];
+                    tmem_ld16x2(lane_addr + kTmY + ch * 32 + 16 * hh, yv,
+                                lane_addr + kTmZ + 64u * par + ch * 32 + 16 * hh, zv);
+                    float xs[16];
+                    f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 4 * ch + 2 * hh)),
+                                     xs);
+                    f16_chunk_to_f32(
+                        *reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 4 * ch + 2 * hh + 1)), xs + 8);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<float4 *>(stg + sw128_off(row, (cq & 1) * 4 + q)) =
-                        make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
+                    for (int q = 0; q < 8; ++q) {
+                        float2 r = __ffma2_rn(e2, make_float2(zv[2 * q], zv[2 * q + 1]),
+                                              make_float2(yv[2 * q], yv[2 * q + 1]));
+                        r = __ffma2_rn(d2, make_float2(xs[2 * q], xs[2 * q + 1]), r);
+                        yv[2 * q] = r.x;
+                        yv[2 * q + 1] = r.y;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<float4 *>(stg + sw128_off(row, 4 * hh + q)) =
+                            make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
+                }
             }
-            co_signal(S.bar(kBarEpi), tid);
+            co_arrive(S.bar(kBarFree), lane);
         }
-        named_bar_sync(kCoCompute);
         if (__any_sync(0xffffffffu, !in_f16_range(amax)) && lane == 0) flag_status(ws.status, kStatusRange);
     }
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *abort_flag) flag_status(ws.status, kStatusTimeout);
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (tid == 0 && *abort_flag) {
+        // let every copy and MMA already issued finish before the CTA
+        // releases its shared memory and TMEM (bounded waits)
+        for (int q = 0; q <= kBarZ; ++q) {
+            const int cnt = S.issued()[q];
+            if (cnt) mbar_wait(S.bar(q), (uint32_t)((cnt - 1) & 1), kWaitBudget);
+        }
+        flag_status(ws.status, kStatusTimeout);
+    }
+    if (warp == 0) {
+        __syncwarp();
+        tmem_dealloc(tmem, 512);
+    }
 }
 
 }  // namespace
