@@ -481,34 +481,37 @@ tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
 // stall on an issue (a tcgen05.mma holds its issuing thread for about as
 // long as it runs).  Per 128-token block k the compute warps run:
 //   [1] C.B^T(k) done -> W(k) into TMEM (fp16, the A operand of W.X)
-//                                                 -> MMA: S(k) = B^T (w.X(k)), Y(k) = W(k) X(k)
-//   [2] tiles(k+1) landed -> decay factors, X(k+1) widened in place and w.X(k+1)
-//                                                 -> MMA: C.B^T(k+1)
-//   [3] S(k), Z(k) done -> H_in(k+1) = a_k H_in(k) + S(k) in registers, fp16 copy
-//                                                 -> MMA: Z(k+1) = C(k+1) H_in(k+1)
-//   [4] Y(k) done -> y(k) = Y + exp(cum) Z(k) + D x, staged in block k's C tiles
-//                                                 -> TMA: store y(k), then tiles(k+2)
-// so the tensor pipe runs S(k), Y(k), C.B^T(k+1), Z(k+1) back to back while
-// the compute warps form operands.  Compute warp w owns TMEM lanes
-// 32*(w%4).. (its rows) and column half w/4: 64 of the 128 C.B^T columns and
-// 32 of the 64 Y/Z/S/state columns.
+//                                     -> MMA: S(k) = B^T (w.X(k)), Y(k) = W(k) X(k)
+//   [2] x/dt/cum(k+1) landed -> decay factors, X(k+1) widened in place
+//   [3] S(k), Z(k) done -> H_in(k+1) = a_k H_in(k) + S(k) in registers, its
+//       fp16 copy, and w.X(k+1)       -> MMA: Z(k+1) = C(k+1) H_in(k+1)
+//   [4] Y(k) done -> y(k) = Y + exp(cum) Z(k) + D x, staged in block k's B tiles
+//                                     -> TMA: store y(k); x/dt/cum(k+3), C/B(k+2)
+// while the MMA warp issues C.B^T(k+1) as soon as C/B(k+1) have landed.  C
+// and B (fp16 copies) are double-buffered by block parity; x with dt and cum
+// rotates through three slots, so it is fetched more than a block ahead.
+// Compute warp w owns TMEM lanes 32*(w%4).. (its rows) and column half w/4:
+// C.B^T column slices w/4 and w/4+2, and 32 of the 64 Y/Z/S/state columns.
 constexpr int kCoCompute = 256;                                 // 8 compute warps
 constexpr int kCoWarps = kCoCompute / 32;
 constexpr int kCoMmaWarp = kCoWarps, kCoTmaWarp = kCoWarps + 1;
 constexpr int kCoThreads = kCoCompute + 64;                     // + MMA warp + TMA warp
-constexpr uint32_t kCoStage = 5 * kTileBytes + 2 * kBlk * 4;   // C(2) B(2) X(1) tiles, dt, cum
-constexpr uint32_t kCoOffWX = 2 * kCoStage;                     // w.X fp16, one tile per stage
-constexpr uint32_t kCoOffH16 = kCoOffWX + 2 * kTileBytes;       // fp16 entering state [n][p]
-constexpr uint32_t kCoFactors = 640;                            // w[128], v[3][128], vd[128]
-constexpr uint32_t kCoOffF = kCoOffH16 + kTileBytes;            // factors [2][640] floats
+constexpr uint32_t kCoCB = 4 * kTileBytes;                      // C(2 tiles) B(2 tiles) of one block
+constexpr uint32_t kCoXS = kTileBytes + 1024;                   // X tile, dt[128], cum[128]
+constexpr int kCoXSlots = 3;
+constexpr uint32_t kCoOffXS = 2 * kCoCB;                        // x ring
+constexpr uint32_t kCoOffWX = kCoOffXS + kCoXSlots * kCoXS;     // w.X fp16
+constexpr uint32_t kCoOffH16 = kCoOffWX + kTileBytes;           // fp16 entering state [n][p]
+constexpr uint32_t kCoFactors = 320;                            // w[128], v0[32], v1[64], v2[96]
+constexpr uint32_t kCoOffF = kCoOffH16 + kTileBytes;            // factors [2][320] floats
 constexpr uint32_t kCoOffG = kCoOffF + 2 * kCoFactors * 4;      // diagonal fast-path flags [2][4]
 constexpr uint32_t kCoOffMask = kCoOffG + 8 * 4;                // causal masks of the diagonal [4][32 lanes] x 16 B
 constexpr uint32_t kCoOffIss = kCoOffMask + 32 * 16 * 4;        // issue counters (drain after an abort)
 constexpr uint32_t kCoOffBar = kCoOffIss + 16 * 4;              // mbarriers, TMEM slot, abort flag
-constexpr int kCoBars = 10;
+constexpr int kCoBars = 12;
 constexpr size_t kCoSmem = 1024 + kCoOffBar + kCoBars * 8 + 16;
 constexpr float kDiagExpCap = 64.0f;                            // largest exponent on the diagonal fast path
-static_assert(kCoStage % 1024 == 0, "stage tiles must stay 1024-byte aligned");
+static_assert(kCoXS % 1024 == 0 && kCoCB % 1024 == 0, "tiles must stay 1024-byte aligned");
 static_assert(kCoSmem <= 232448, "chunk_out shared memory exceeds the per-CTA limit");
 
 // TMEM columns (512 allocated)
@@ -518,17 +521,22 @@ constexpr uint32_t kTmY = 192;     // W.X fp32, 64 columns
 constexpr uint32_t kTmS = 256;     // B^T.(w.X) fp32, 64 columns
 constexpr uint32_t kTmZ = 320;     // C.H fp32, two buffers of 64 columns (block parity)
 
-enum CoBar { kBarTma0 = 0, kBarTma1 = 1, kBarCB = 2, kBarS = 3, kBarY = 4, kBarZ = 5,   // completion
-             kBarW = 6, kBarOps = 7, kBarH16 = 8, kBarFree = 9 };                       // compute -> issuers
+enum CoBar { kBarTcb0 = 0, kBarTcb1 = 1, kBarTx0 = 2, kBarTx1 = 3, kBarTx2 = 4,       // copies landed
+             kBarCB = 5, kBarS = 6, kBarY = 7, kBarZ = 8,                            // MMAs done
+             kBarW = 9, kBarH16 = 10, kBarFree = 11 };                                // compute -> issuers
+constexpr int kFirstComputeBar = kBarW;
+
+// v_g (pivot m = 32g+31, j <= m) starts at this factor index; w is v_3.
+__host__ __device__ constexpr int voff(int g) { return g == 3 ? 0 : 128 + 16 * g * (g + 1); }
 
 struct CoSmem {
     uint8_t *base;
-    __device__ uint8_t *C(int s) const { return base + s * kCoStage; }
-    __device__ uint8_t *B(int s) const { return base + s * kCoStage + 2 * kTileBytes; }
-    __device__ uint8_t *X(int s) const { return base + s * kCoStage + 4 * kTileBytes; }
-    __device__ float *dt(int s) const { return reinterpret_cast<float *>(base + s * kCoStage + 5 * kTileBytes); }
-    __device__ float *cum(int s) const { return dt(s) + kBlk; }
-    __device__ uint8_t *WX(int s) const { return base + kCoOffWX + s * kTileBytes; }
+    __device__ uint8_t *C(int s) const { return base + s * kCoCB; }
+    __device__ uint8_t *B(int s) const { return base + s * kCoCB + 2 * kTileBytes; }
+    __device__ uint8_t *X(int r) const { return base + kCoOffXS + r * kCoXS; }
+    __device__ float *dt(int r) const { return reinterpret_cast<float *>(X(r) + kTileBytes); }
+    __device__ float *cum(int r) const { return dt(r) + kBlk; }
+    __device__ uint8_t *WX() const { return base + kCoOffWX; }
     __device__ uint8_t *H16() const { return base + kCoOffH16; }
     __device__ float *F(int s) const { return reinterpret_cast<float *>(base + kCoOffF) + s * kCoFactors; }
     __device__ int *G(int s) const { return reinterpret_cast<int *>(base + kCoOffG) + s * 4; }
@@ -543,69 +551,85 @@ struct CoSmem {
 // (smem addresses stay below 2^18, so the 14-bit field never carries).
 __device__ __forceinline__ uint64_t dadd(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
 
-// TMA for block k into stage s: C and B (fp16 copies), X (bf16), dt and cum
-// rows, all completing on the stage's barrier.
-__device__ __forceinline__ void co_load(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
-                                        int s, int k, int g, int h, int b) {
+// TMA: C and B (fp16 copies) of block k into stage s
+__device__ __forceinline__ void co_load_cb(const CoSmem &S, const TcMaps &maps, int s, int k, int g, int b) {
     const int t0 = k * kBlk;
-    uint64_t *bar = S.bar(kBarTma0 + s);
-    mbar_arrive_expect_tx(bar, kCoStage);
+    uint64_t *bar = S.bar(kBarTcb0 + s);
+    mbar_arrive_expect_tx(bar, kCoCB);
     tma_load_4d(S.C(s), &maps.C, bar, 0, g, t0, b);
     tma_load_4d(S.C(s) + kTileBytes, &maps.C, bar, 64, g, t0, b);
     tma_load_4d(S.B(s), &maps.B, bar, 0, g, t0, b);
     tma_load_4d(S.B(s) + kTileBytes, &maps.B, bar, 64, g, t0, b);
-    tma_load_4d(S.X(s), &maps.x, bar, 0, h, t0, b);
-    bulk_load(S.dt(s), dtv + (size_t)t0, kBlk * 4, bar);
-    bulk_load(S.cum(s), cum + (size_t)t0, kBlk * 4, bar);
-    ++S.issued()[kBarTma0 + s];
+    ++S.issued()[kBarTcb0 + s];
 }
 
-// Per-block decay factors (all exponents clamped as stated):
-//   w[j]        = exp(min(cum_last - cum_j, 0)) dt_j               (state update)
-//   v[g-1][j]   = exp(min(cum_m - cum_j, 0)) dt_j, m = 32g-1, j<=m (below the diagonal, row group g)
-//   vd[j]       = exp(min(cum_s0 - cum_j, cap)) dt_j, s0 = 32*(j/32) (diagonal sub-blocks)
-// and flags: the diagonal sub-block of row group g may use vd (its decay is
-// below exp(-cap), so no factor there exceeds exp(cap)).
-__device__ __forceinline__ void co_factors(const CoSmem &S, int s, int last_valid, int tid) {
-    const float *cum = S.cum(s), *dt = S.dt(s);
-    float *F = S.F(s);
+// TMA: X (bf16), dt and cum rows of block k into x slot r
+__device__ __forceinline__ void co_load_x(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
+                                          int r, int k, int h, int b) {
+    const int t0 = k * kBlk;
+    uint64_t *bar = S.bar(kBarTx0 + r);
+    mbar_arrive_expect_tx(bar, kCoXS);
+    tma_load_4d(S.X(r), &maps.x, bar, 0, h, t0, b);
+    bulk_load(S.dt(r), dtv + (size_t)t0, kBlk * 4, bar);
+    bulk_load(S.cum(r), cum + (size_t)t0, kBlk * 4, bar);
+    ++S.issued()[kBarTx0 + r];
+}
+
+// Per-block decay factors into F(f), from the dt/cum of x slot r (all
+// exponents clamped as stated):
+//   v_g[j] = exp(min(cum_m - cum_j, 0)) dt_j,  m = 32g+31, j <= m, g = 0..2
+//   w[j]   = v_3[j] = exp(min(cum_last - cum_j, 0)) dt_j         (state update)
+// Row group g uses v_{g-1} below its diagonal sub-block and v_g on it; the
+// flag says the diagonal may use the factored form (its total decay is
+// below exp(-cap), so no row factor there exceeds exp(cap)).
+__device__ __forceinline__ void co_factors(const CoSmem &S, int r, int f, int last_valid, int tid) {
+    const float *cum = S.cum(r), *dt = S.dt(r);
+    float *F = S.F(f);
     const float clast = cum[last_valid];
     for (int idx = tid; idx < (int)kCoFactors; idx += kCoCompute) {
-        float f = 0.f;
+        float cm;
+        int j;
         if (idx < kBlk) {
-            f = expf(fminf(clast - cum[idx], 0.f)) * dt[idx];
-        } else if (idx < 4 * kBlk) {
-            const int q = idx - kBlk, gm = q >> 7, j = q & (kBlk - 1), m = 32 * (gm + 1) - 1;
-            if (j <= m) f = expf(fminf(cum[m] - cum[j], 0.f)) * dt[j];
+            cm = clast;
+            j = idx;
         } else {
-            const int j = idx - 4 * kBlk;
-            f = expf(fminf(cum[j & ~31] - cum[j], kDiagExpCap)) * dt[j];
+            const int q = idx - kBlk, g = q < 32 ? 0 : (q < 96 ? 1 : 2);
+            j = q - 16 * g * (g + 1);
+            cm = cum[32 * g + 31];
         }
-        F[idx] = f;
+        F[idx] = expf(fminf(cm - cum[j], 0.f)) * dt[j];
     }
-    if (tid < 4) S.G(s)[tid] = (cum[32 * tid] - cum[32 * tid + 31]) <= kDiagExpCap ? 1 : 0;
+    if (tid < 4) S.G(f)[tid] = (cum[32 * tid] - cum[32 * tid + 31]) <= kDiagExpCap ? 1 : 0;
 }
 
-// X tile of stage s: bf16 -> fp16 in place, and w.X (fp16) into WX(s) in the
-// same swizzled layout (four 16-byte chunks per thread; a chunk's row is its
-// offset / 128 whatever the swizzle).
-__device__ __forceinline__ void co_widen_x(const CoSmem &S, int s, int tid, __half2 &amax) {
-    const float *w = S.F(s);
+// X tile of slot r: bf16 -> fp16 in place (four 16-byte chunks per thread).
+__device__ __forceinline__ void co_widen_x(const CoSmem &S, int r, int tid, __half2 &amax) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int c = tid + r * kCoCompute;
-        uint4 *p = reinterpret_cast<uint4 *>(S.X(s) + c * 16);
+    for (int q = 0; q < 4; ++q) {
+        uint4 *p = reinterpret_cast<uint4 *>(S.X(r) + (tid + q * kCoCompute) * 16);
         float f[8];
         bf16_chunk_to_f32(*p, f);
         *p = pack8(f, amax);
+    }
+}
+
+// w.X (fp16) of the widened X tile of slot r into WX, same swizzled layout (a
+// chunk's row is its offset / 128 whatever the swizzle).
+__device__ __forceinline__ void co_form_wx(const CoSmem &S, int r, int f, int tid, __half2 &amax) {
+    const float *w = S.F(f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int c = tid + q * kCoCompute;
+        float x8[8];
+        f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(r) + c * 16), x8);
         const float2 wj = make_float2(w[c >> 3], w[c >> 3]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float2 m = __fmul2_rn(make_float2(f[2 * e], f[2 * e + 1]), wj);
-            f[2 * e] = m.x;
-            f[2 * e + 1] = m.y;
+            const float2 m = __fmul2_rn(make_float2(x8[2 * e], x8[2 * e + 1]), wj);
+            x8[2 * e] = m.x;
+            x8[2 * e + 1] = m.y;
         }
-        *reinterpret_cast<uint4 *>(S.WX(s) + c * 16) = pack8(f, amax);
+        *reinterpret_cast<uint4 *>(S.WX() + c * 16) = pack8(x8, amax);
     }
 }
 
@@ -627,41 +651,42 @@ __device__ __forceinline__ void pack16(const float *v, uint32_t *o, __half2 &ama
     }
 }
 
-// W for one 32-column slice cq <= lg of this thread's row (see co_factors).
-__device__ __forceinline__ void co_w_slice(const CoSmem &S, int s, uint32_t lane_addr, int lg, int cq, int lane,
-                                           float ci, __half2 &amax) {
-    const float *cum = S.cum(s);
-    const float *F = S.F(s);
+// W for one 32-column slice cq <= lg of this thread's row i (see co_factors).
+__device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32_t lane_addr, int lg, int cq,
+                                           int lane, float ci, __half2 &amax) {
+    const float *cum = S.cum(r);
+    const float *F = S.F(f);
     float v[32];
     tmem_ld32(lane_addr + kTmCB + cq * 32, v);
     uint32_t o[16];
-    if (cq < lg) {                                   // below the diagonal: factored decay
+    if (cq < lg) {                                   // below the diagonal: pivot at row 32*lg-1
         const float ui = expf(fminf(ci - cum[32 * lg - 1], 0.f));
         const float2 u2 = make_float2(ui, ui);
-        const float2 *vf = reinterpret_cast<const float2 *>(F + kBlk * lg + cq * 32);
+        const float2 *vf = reinterpret_cast<const float2 *>(F + voff(lg - 1) + cq * 32);
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-            const float2 f = __fmul2_rn(vf[q], u2);
-            const float2 m = __fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), f);
+            const float2 fq = __fmul2_rn(vf[q], u2);
+            const float2 m = __fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), fq);
             v[2 * q] = m.x;
             v[2 * q + 1] = m.y;
         }
         pack16(v, o, amax);
         pack16(v + 16, o + 8, amax);
-    } else {                                         // diagonal 32x32
-        if (S.G(s)[lg]) {
-            const float ud = expf(fminf(ci - cum[32 * lg], 0.f));
+    } else {                                         // diagonal 32x32: pivot at its last row m
+        if (S.G(f)[lg]) {
+            // exp(cum_i - cum_j) = exp(cum_i - cum_m) exp(cum_m - cum_j); the first
+            // factor is >= 1 and at most exp(cap) (flag), the second <= 1
+            const float ud = expf(fminf(ci - cum[32 * lg + 31], kDiagExpCap));
             const float2 u2 = make_float2(ud, ud);
-            const float2 *vf = reinterpret_cast<const float2 *>(F + 4 * kBlk + cq * 32);
+            const float2 *vf = reinterpret_cast<const float2 *>(F + voff(lg) + cq * 32);
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-                const float2 f = __fmul2_rn(vf[q], u2);
-                const float2 m = __fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), f);
+                const float2 m = __fmul2_rn(__fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), vf[q]), u2);
                 v[2 * q] = m.x;
                 v[2 * q + 1] = m.y;
             }
         } else {                                     // steep decay: one exp per element
-            const float *dts = S.dt(s) + cq * 32, *cj = cum + cq * 32;
+            const float *dts = S.dt(r) + cq * 32, *cj = cum + cq * 32;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
                 v[jj] = v[jj] * expf(fminf(ci - cj[jj], 0.f)) * dts[jj];
@@ -707,7 +732,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     }
     if (tid == 0) {
         for (int i = 0; i < kCoBars; ++i) {
-            mbar_init(S.bar(i), i < kBarW ? 1 : kCoWarps);
+            mbar_init(S.bar(i), i < kFirstComputeBar ? 1 : kCoWarps);
             S.issued()[i] = 0;
         }
         *abort_flag = 0;
@@ -725,16 +750,16 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             const uint32_t idesc_z = idesc_f16(128, 64, 0, 1);    // A=C K-major, B=H MN-major
             const uint32_t idesc_y = idesc_f16(128, 64, 0, 1);    // A=W (TMEM) K-major, B=X MN-major
             const uint32_t idesc_s = idesc_f16(128, 64, 1, 1);    // A=B^T MN-major, B=wX MN-major
-            // stage 1's descriptors are stage 0's plus the stage stride (no array:
-            // a dynamically indexed one would live in local memory)
+            // per-stage / per-slot descriptors are the first one's plus a byte offset
+            // (no arrays: a dynamically indexed one would live in local memory)
             const uint64_t dC0 = sdesc_sw128(smem_u32(S.C(0)), 16, 1024);
             const uint64_t dBk0 = sdesc_sw128(smem_u32(S.B(0)), 16, 1024);
             const uint64_t dBm0 = sdesc_sw128(smem_u32(S.B(0)), kTileBytes, 1024);
             const uint64_t dX0 = sdesc_sw128(smem_u32(S.X(0)), kTileBytes, 1024);
-            const uint64_t dWX0 = sdesc_sw128(smem_u32(S.WX(0)), kTileBytes, 1024);
+            const uint64_t dWX = sdesc_sw128(smem_u32(S.WX()), kTileBytes, 1024);
             const uint64_t dH = sdesc_sw128(smem_u32(S.H16()), kTileBytes, 1024);
-            auto st = [](int s) { return (uint32_t)s * kCoStage; };
-            auto wxs = [](int s) { return (uint32_t)s * kTileBytes; };
+            auto st = [](int s) { return (uint32_t)s * kCoCB; };
+            auto xs = [](int r) { return (uint32_t)r * kCoXS; };
             // K-major K-step q of a 128-wide tile: column block q/4, 32 bytes per step inside it
             auto kofs = [](int q) { return (uint32_t)((q >> 2) * kTileBytes + (q & 3) * 32); };
             auto issue_cb = [&](int s) {
@@ -751,19 +776,19 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 mma_commit(S.bar(kBarZ));
                 ++S.issued()[kBarZ];
             };
-            auto issue_sy = [&](int s) {
+            auto issue_sy = [&](int s, int r) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    mma_f16(tmem + kTmS, dadd(dBm0, st(s) + q * 2048), dadd(dWX0, wxs(s) + q * 2048), idesc_s, q > 0);
+                    mma_f16(tmem + kTmS, dadd(dBm0, st(s) + q * 2048), dadd(dWX, q * 2048), idesc_s, q > 0);
                 mma_commit(S.bar(kBarS));
                 ++S.issued()[kBarS];
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    mma_f16_ts(tmem + kTmY, tmem + kTmW + 8u * q, dadd(dX0, st(s) + q * 2048), idesc_y, q > 0);
+                    mma_f16_ts(tmem + kTmY, tmem + kTmW + 8u * q, dadd(dX0, xs(r) + q * 2048), idesc_y, q > 0);
                 mma_commit(S.bar(kBarY));
                 ++S.issued()[kBarY];
             };
-            bool ok = mbar_wait_abortable(S.bar(kBarOps), 0, kWaitBudget, abort_flag);
+            bool ok = mbar_wait_abortable(S.bar(kBarTcb0), 0, kWaitBudget, abort_flag);
             tc_fence_after();
             if (ok) issue_cb(0);
             ok = ok && mbar_wait_abortable(S.bar(kBarH16), 0, kWaitBudget, abort_flag);
@@ -775,9 +800,11 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 ok = mbar_wait_abortable(S.bar(kBarW), par, kWaitBudget, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                issue_sy(s);
+                issue_sy(s, i % kCoXSlots);
                 if (k + 1 < kb1) {
-                    ok = mbar_wait_abortable(S.bar(kBarOps), par1, kWaitBudget, abort_flag);
+                    // C.B^T(k+1) once its tiles have landed (W(k) has read C.B^T(k))
+                    ok = mbar_wait_abortable(S.bar(kBarTcb0 + s1), ((uint32_t)(i + 1) >> 1) & 1u, kWaitBudget,
+                                             abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     issue_cb(s1);
@@ -793,18 +820,19 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     } else if (warp == kCoTmaWarp) {
         // ------------------------------ TMA warp ------------------------------
         if (lane == 0) {
-            co_load(S, maps, dtg, cumg, 0, kb0, g, h, b);
-            if (kb0 + 1 < kb1) co_load(S, maps, dtg, cumg, 1, kb0 + 1, g, h, b);
+            for (int q = 0; q < 2 && kb0 + q < kb1; ++q) co_load_cb(S, maps, q, kb0 + q, g, b);
+            for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q) co_load_x(S, maps, dtg, cumg, q, kb0 + q, h, b);
             for (int k = kb0; k < kb1; ++k) {
                 const int i = k - kb0, s = i & 1;
                 if (!mbar_wait_abortable(S.bar(kBarFree), (uint32_t)i & 1u, kWaitBudget, abort_flag)) break;
-                // y(k) sits in block k's C tiles as two 32-column fp32 tiles
-                tma_store_4d(&maps.y, S.C(s), 0, h, k * kBlk, b);
-                tma_store_4d(&maps.y, S.C(s) + kTileBytes, 32, h, k * kBlk, b);
+                // block k is done with its x slot; its y sits in its B tiles
+                if (k + kCoXSlots < kb1) co_load_x(S, maps, dtg, cumg, i % kCoXSlots, k + kCoXSlots, h, b);
+                tma_store_4d(&maps.y, S.B(s), 0, h, k * kBlk, b);
+                tma_store_4d(&maps.y, S.B(s) + kTileBytes, 32, h, k * kBlk, b);
                 tma_store_commit();
                 if (k + 2 < kb1) {
                     tma_store_wait_read();
-                    co_load(S, maps, dtg, cumg, s, k + 2, g, h, b);
+                    co_load_cb(S, maps, s, k + 2, g, b);
                 }
             }
             tma_store_wait_all();
@@ -827,9 +855,9 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                                               : (init ? init + bh * kNP : nullptr);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float4 f = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kP + ch * 32 + 4 * q)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-                hv[4 * q] = f.x; hv[4 * q + 1] = f.y; hv[4 * q + 2] = f.z; hv[4 * q + 3] = f.w;
+                const float4 f4 = src ? *reinterpret_cast<const float4 *>(src + (size_t)row * kP + ch * 32 + 4 * q)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                hv[4 * q] = f4.x; hv[4 * q + 1] = f4.y; hv[4 * q + 2] = f4.z; hv[4 * q + 3] = f4.w;
             }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -843,7 +871,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             // W above the diagonal sub-blocks stays zero for the whole kernel
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const int cq = 2 * ch + t;
+                const int cq = ch + 2 * t;
                 if (cq > lg) {
                     uint32_t z[16];
 #pragma unroll
@@ -865,20 +893,22 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             }
         }
         co_arrive(S.bar(kBarH16), lane);
-        // block kb0: tiles landed -> factors, widened X and w.X
-        ok = mbar_wait_abortable(S.bar(kBarTma0), 0, kWaitBudget, abort_flag);
-        if (ok) co_factors(S, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
+        // block kb0: x landed -> factors, widened X, w.X
+        ok = mbar_wait_abortable(S.bar(kBarTx0), 0, kWaitBudget, abort_flag);
+        if (ok) co_factors(S, 0, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
         named_bar_sync(kCoCompute);                 // factors and masks visible to every compute warp
         if (ok) co_widen_x(S, 0, tid, amax);
-        co_arrive(S.bar(kBarOps), lane);
+        named_bar_sync(kCoCompute);
+        if (ok) co_form_wx(S, 0, 0, tid, amax);
 
         // every compute warp runs every iteration (and so every named barrier);
         // after an abort the waits return at once and the work is skipped
         for (int k = kb0; k < kb1; ++k) {
-            const int i = k - kb0, s = i & 1, s1 = s ^ 1;
+            const int i = k - kb0, f = i & 1, f1 = f ^ 1;
+            const int r = i % kCoXSlots, r1 = (i + 1) % kCoXSlots;
             const uint32_t par = (uint32_t)i & 1u;
             const int t0 = k * kBlk;
-            const float *cum = S.cum(s);
+            const float *cum = S.cum(r);
 
             // [1] C.B^T(k) done -> W(k) (fp16 pairs) into TMEM
             ok = ok && mbar_wait_abortable(S.bar(kBarCB), par, kWaitBudget, abort_flag);
@@ -886,22 +916,21 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             tc_fence_after();
             if (ok) {
                 const float ci = cum[row];
-                if (2 * ch <= lg) co_w_slice(S, s, lane_addr, lg, 2 * ch, lane, ci, amax);
-                if (2 * ch + 1 <= lg) co_w_slice(S, s, lane_addr, lg, 2 * ch + 1, lane, ci, amax);
+                if (ch <= lg) co_w_slice(S, r, f, lane_addr, lg, ch, lane, ci, amax);
+                if (ch + 2 <= lg) co_w_slice(S, r, f, lane_addr, lg, ch + 2, lane, ci, amax);
             }
             co_arrive(S.bar(kBarW), lane);
 
-            // [2] block k+1: tiles landed -> factors, widened X, w.X (overlaps S(k), Y(k))
+            // [2] block k+1: x landed -> factors, widened X (overlaps S(k), Y(k))
             if (k + 1 < kb1) {
-                ok = ok && mbar_wait_abortable(S.bar(kBarTma0 + s1), ((uint32_t)(i + 1) >> 1) & 1u, kWaitBudget,
-                                               abort_flag);
-                if (ok) co_factors(S, s1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
-                named_bar_sync(kCoCompute);
-                if (ok) co_widen_x(S, s1, tid, amax);
-                co_arrive(S.bar(kBarOps), lane);
+                ok = ok && mbar_wait_abortable(S.bar(kBarTx0 + r1), ((uint32_t)(i + 1) / kCoXSlots) & 1u,
+                                               kWaitBudget, abort_flag);
+                if (ok) co_factors(S, r1, f1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
+                if (ok) co_widen_x(S, r1, tid, amax);
+                named_bar_sync(kCoCompute);          // factors and widened X of block k+1 visible
             }
 
-            // [3] S(k) done (and Z(k), which read the fp16 copy) -> H_in(k+1)
+            // [3] S(k) done (and Z(k), which read the fp16 copy) -> H_in(k+1), w.X(k+1)
             ok = ok && mbar_wait_abortable(S.bar(kBarS), par, kWaitBudget, abort_flag);
             ok = ok && mbar_wait_abortable(S.bar(kBarZ), par, kWaitBudget, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
@@ -913,10 +942,10 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 const float2 a2 = make_float2(a, a);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
-                    const float2 r = __ffma2_rn(a2, make_float2(hv[2 * q], hv[2 * q + 1]),
-                                                make_float2(sv[2 * q], sv[2 * q + 1]));
-                    hv[2 * q] = r.x;
-                    hv[2 * q + 1] = r.y;
+                    const float2 rr = __ffma2_rn(a2, make_float2(hv[2 * q], hv[2 * q + 1]),
+                                                 make_float2(sv[2 * q], sv[2 * q + 1]));
+                    hv[2 * q] = rr.x;
+                    hv[2 * q + 1] = rr.y;
                 }
                 if (k + 1 < kb1) {
 #pragma unroll
@@ -928,6 +957,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                             *reinterpret_cast<uint4 *>(S.H16() + sw128_off(row, 4 * ch + 2 * hh + q)) =
                                 make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
                     }
+                    co_form_wx(S, r1, f1, tid, amax);
                 } else if (final_state && u == U - 1) {
                     float *dst = final_state + bh * kNP + (size_t)row * kP + ch * 32;
 #pragma unroll
@@ -938,31 +968,31 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             }
             if (k + 1 < kb1) co_arrive(S.bar(kBarH16), lane);
 
-            // [4] Y(k) done -> y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging in block k's C tiles
+            // [4] Y(k) done -> y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging in block k's B tiles
             ok = ok && mbar_wait_abortable(S.bar(kBarY), par, kWaitBudget, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
             if (ok) {
                 const float ei = expf(fminf(cum[row], 0.f));
                 const float2 e2 = make_float2(ei, ei), d2 = make_float2(Dh, Dh);
-                uint8_t *stg = S.C(s) + ch * kTileBytes;
+                uint8_t *stg = S.B(i & 1) + ch * kTileBytes;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float yv[16], zv[16];
                     tmem_ld16x2(lane_addr + kTmY + ch * 32 + 16 * hh, yv,
                                 lane_addr + kTmZ + 64u * par + ch * 32 + 16 * hh, zv);
-                    float xs[16];
-                    f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 4 * ch + 2 * hh)),
-                                     xs);
+                    float xv[16];
+                    f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(r) + sw128_off(row, 4 * ch + 2 * hh)),
+                                     xv);
                     f16_chunk_to_f32(
-                        *reinterpret_cast<const uint4 *>(S.X(s) + sw128_off(row, 4 * ch + 2 * hh + 1)), xs + 8);
+                        *reinterpret_cast<const uint4 *>(S.X(r) + sw128_off(row, 4 * ch + 2 * hh + 1)), xv + 8);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        float2 r = __ffma2_rn(e2, make_float2(zv[2 * q], zv[2 * q + 1]),
-                                              make_float2(yv[2 * q], yv[2 * q + 1]));
-                        r = __ffma2_rn(d2, make_float2(xs[2 * q], xs[2 * q + 1]), r);
-                        yv[2 * q] = r.x;
-                        yv[2 * q + 1] = r.y;
+                        float2 rr = __ffma2_rn(e2, make_float2(zv[2 * q], zv[2 * q + 1]),
+                                               make_float2(yv[2 * q], yv[2 * q + 1]));
+                        rr = __ffma2_rn(d2, make_float2(xv[2 * q], xv[2 * q + 1]), rr);
+                        yv[2 * q] = rr.x;
+                        yv[2 * q + 1] = rr.y;
                     }
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
@@ -979,7 +1009,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     if (tid == 0 && *abort_flag) {
         // let every copy and MMA already issued finish before the CTA
         // releases its shared memory and TMEM (bounded waits)
-        for (int q = 0; q <= kBarZ; ++q) {
+        for (int q = 0; q < kFirstComputeBar; ++q) {
             const int cnt = S.issued()[q];
             if (cnt) mbar_wait(S.bar(q), (uint32_t)((cnt - 1) & 1), kWaitBudget);
         }
