@@ -206,36 +206,40 @@ __device__ __forceinline__ void f16_chunk_to_f32(uint4 v, float *f) {
 }
 
 // ---------------------------------------------------------------------------
-// prep: grid (nblk, ceil(H/32) + G, b), 256 threads.  y-slices below
-// ceil(H/32) do dt/cum for 32 heads; the rest convert B and C of one group.
+// prep: grid (nblk, ceil(H/8) + 4 G, b), 256 threads.  y-slices below
+// ceil(H/8) do dt/cum for 8 heads of one 128-token block; the rest convert a
+// 32-row quarter of the block's B and C of one group.  Small slices keep many
+// CTAs in flight: every thread issues its few loads before any arithmetic.
+constexpr int kPrepHeads = 8;
+
 __global__ void __launch_bounds__(256)
 prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias, const float *__restrict__ A,
             const __nv_bfloat16 *__restrict__ Bm, const __nv_bfloat16 *__restrict__ Cm, TcWs ws, int L, int H,
             int G, int nblk, float lo, float hi) {
-    __shared__ float s_dt[kBlk][33];
-    __shared__ float s_da[kBlk][33];
+    __shared__ float s_dt[kPrepHeads][kBlk + 4];
+    __shared__ float s_da[kPrepHeads][kBlk + 4];
     const int blk = blockIdx.x, b = blockIdx.z;
-    const int nhy = (H + 31) / 32;
+    const int nhy = (H + kPrepHeads - 1) / kPrepHeads;
     if ((int)blockIdx.y >= nhy) {
-        const int g = blockIdx.y - nhy;
-        const int t0 = blk * kBlk;
+        const int g = (blockIdx.y - nhy) >> 2, quarter = (blockIdx.y - nhy) & 3;
+        const int t0 = blk * kBlk + 32 * quarter;
         const size_t Lp = (size_t)nblk * kBlk;
         __half2 amax = __float2half2_rn(0.f);
-        // all 16 loads of a thread in flight before any conversion
-        uint4 v[16];
+        // 2 tensors x 32 rows x 16 chunks of 8: four chunks per thread, all loads first
+        uint4 v[4];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
+        for (int r = 0; r < 4; ++r) {
             const int c = threadIdx.x + 256 * r;
-            const int which = c >> 11, row = (c >> 4) & (kBlk - 1), kk = c & 15;
+            const int which = c >> 9, row = (c >> 4) & 31, kk = c & 15;
             const int t = t0 + row;
             const __nv_bfloat16 *src = which ? Cm : Bm;
             v[r] = make_uint4(0u, 0u, 0u, 0u);
             if (t < L) v[r] = __ldg(reinterpret_cast<const uint4 *>(src + (((size_t)b * L + t) * G + g) * kN + kk * 8));
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
+        for (int r = 0; r < 4; ++r) {
             const int c = threadIdx.x + 256 * r;
-            const int which = c >> 11, row = (c >> 4) & (kBlk - 1), kk = c & 15;
+            const int which = c >> 9, row = (c >> 4) & 31, kk = c & 15;
             const int t = t0 + row;
             __half *dst = which ? ws.Ch : ws.Bh;
             float f[8];
@@ -245,39 +249,37 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
         if (!in_f16_range(amax)) flag_status(ws.status, kStatusRange);
         return;
     }
-    const int h0 = blockIdx.y * 32;
-    const int nh = min(32, H - h0);
+    const int h0 = blockIdx.y * kPrepHeads;
+    const int nh = min(kPrepHeads, H - h0);
     {
-        // thread -> head hh = tid % 32 (fixed), tokens tid / 32 + 8 r: all 16
-        // loads in flight before the softplus
-        const int hh = threadIdx.x & 31;
+        // thread -> head hh = tid % 8, tokens tid / 8 + 32 r: all 4 loads in flight first
+        const int hh = threadIdx.x & (kPrepHeads - 1);
         const bool hv = hh < nh;
         const float bias = hv ? dt_bias[h0 + hh] : 0.f, Ah = hv ? A[h0 + hh] : 0.f;
-        float raw[16];
+        float raw[4];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int tok = (threadIdx.x >> 5) + 8 * r;
-            const int t = blk * kBlk + tok;
+        for (int r = 0; r < 4; ++r) {
+            const int t = blk * kBlk + (threadIdx.x >> 3) + 32 * r;
             raw[r] = (hv && t < L) ? dt_raw[((size_t)b * L + t) * H + h0 + hh] : 0.f;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int tok = (threadIdx.x >> 5) + 8 * r;
+        for (int r = 0; r < 4; ++r) {
+            const int tok = (threadIdx.x >> 3) + 32 * r;
             const int t = blk * kBlk + tok;
             float d = 0.f;
             if (hv && t < L) d = dt_of(raw[r], bias, lo, hi);
-            s_dt[tok][hh] = d;
-            s_da[tok][hh] = d * Ah;
+            s_dt[hh][tok] = d;
+            s_da[hh][tok] = d * Ah;
         }
     }
     if (blk == 0 && b == 0 && threadIdx.x < nh && A[h0 + threadIdx.x] > 0.f)
         flag_status(ws.status, kStatusPrecondition);
     __syncthreads();
+    // warp w: inclusive cumsum of dA over the block for head w (four tokens per lane, fixed order)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int hh = warp; hh < nh; hh += 8) {
-        const float v0 = s_da[4 * lane][hh], v1 = s_da[4 * lane + 1][hh];
-        const float v2 = s_da[4 * lane + 2][hh], v3 = s_da[4 * lane + 3][hh];
-        const float c0 = v0, c1 = c0 + v1, c2 = c1 + v2, c3 = c2 + v3;
+    if (warp < nh) {
+        const float4 da = *reinterpret_cast<const float4 *>(&s_da[warp][4 * lane]);
+        const float c0 = da.x, c1 = c0 + da.y, c2 = c1 + da.z, c3 = c2 + da.w;
         float incl = c3;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -285,10 +287,9 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
             if (lane >= o) incl += u;
         }
         const float ex = incl - c3;
-        const size_t base = ((size_t)b * H + h0 + hh) * (size_t)nblk * kBlk + (size_t)blk * kBlk + 4 * lane;
+        const size_t base = ((size_t)b * H + h0 + warp) * (size_t)nblk * kBlk + (size_t)blk * kBlk + 4 * lane;
         *reinterpret_cast<float4 *>(ws.cum + base) = make_float4(ex + c0, ex + c1, ex + c2, ex + c3);
-        *reinterpret_cast<float4 *>(ws.dt + base) =
-            make_float4(s_dt[4 * lane][hh], s_dt[4 * lane + 1][hh], s_dt[4 * lane + 2][hh], s_dt[4 * lane + 3][hh]);
+        *reinterpret_cast<float4 *>(ws.dt + base) = *reinterpret_cast<const float4 *>(&s_dt[warp][4 * lane]);
     }
 }
 
@@ -1028,7 +1029,7 @@ bool tc_supported(const ScanDims &d, int bf16) {
     if (d.Q != 64 && d.Q != 128 && d.Q != 256) return false;
     if (d.H > 65535 || d.b > 65535 || d.L > 0x7fffffffll - kBlk) return false;
     const TcPlan p = make_plan(d);
-    return p.U <= 65535 && (d.H + 31) / 32 + d.G <= 65535;
+    return p.U <= 65535 && (d.H + kPrepHeads - 1) / kPrepHeads + 4 * d.G <= 65535;
 }
 
 size_t tc_workspace_bytes(const ScanDims &d) { return ws_bytes(d, make_plan(d)); }
@@ -1052,7 +1053,7 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     }
     {
         TraceScope tr(s, kTrTcDtPrep);
-        const unsigned ny = (unsigned)((d.H + 31) / 32 + d.G);
+        const unsigned ny = (unsigned)((d.H + kPrepHeads - 1) / kPrepHeads + 4 * d.G);
         prep_kernel<<<dim3((unsigned)p.nblk, ny, (unsigned)d.b), 256, 0, s>>>(
             a.dt_raw, a.dt_bias, a.A, static_cast<const __nv_bfloat16 *>(a.B), static_cast<const __nv_bfloat16 *>(a.C),
             ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, a.dt_lo, a.dt_hi);
