@@ -218,6 +218,7 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
             int G, int nblk, float lo, float hi) {
     __shared__ float s_dt[kPrepHeads][kBlk + 4];
     __shared__ float s_da[kPrepHeads][kBlk + 4];
+    pdl_launch_dependents();                     // the next kernel waits for this one's writes itself
     const int blk = blockIdx.x, b = blockIdx.z;
     const int nhy = (H + kPrepHeads - 1) / kPrepHeads;
     if ((int)blockIdx.y >= nhy) {
@@ -339,6 +340,8 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
+    pdl_launch_dependents();
+    pdl_wait_prerequisites();                    // dt, cum and the fp16 B come from prep
 
     if (warp == kUsCompute / 32) {
         // ------------------------------ control warp --------------------------
@@ -443,6 +446,8 @@ constexpr int kSpBatch = 8;
 
 __global__ void __launch_bounds__(256)
 tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
+    pdl_launch_dependents();
+    pdl_wait_prerequisites();                    // the unit states come from unit_state
     const int e4 = blockIdx.x * 256 + threadIdx.x;
     const size_t bh = (size_t)blockIdx.z * H + blockIdx.y;
     float4 hs = init ? reinterpret_cast<const float4 *>(init + bh * kNP)[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -743,6 +748,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *S.tslot();
+    pdl_wait_prerequisites();                    // prep (and the unit passes) wrote what follows reads
 
     if (warp == kCoMmaWarp) {
         // ------------------------------ MMA warp ------------------------------
@@ -1053,31 +1059,50 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     }
     {
         TraceScope tr(s, kTrTcDtPrep);
+        // a plain launch: it overwrites the workspace the previous call's kernels read
         const unsigned ny = (unsigned)((d.H + kPrepHeads - 1) / kPrepHeads + 4 * d.G);
         prep_kernel<<<dim3((unsigned)p.nblk, ny, (unsigned)d.b), 256, 0, s>>>(
             a.dt_raw, a.dt_bias, a.A, static_cast<const __nv_bfloat16 *>(a.B), static_cast<const __nv_bfloat16 *>(a.C),
             ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, a.dt_lo, a.dt_hi);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the kernels after prep may start their prologue while their predecessor
+    // finishes; each waits (griddepcontrol.wait) before reading its outputs
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    auto cfg = [&](dim3 grid, unsigned threads, size_t smem) {
+        cudaLaunchConfig_t c = {};
+        c.gridDim = grid;
+        c.blockDim = dim3(threads);
+        c.dynamicSmemBytes = smem;
+        c.stream = s;
+        c.attrs = pdl;
+        c.numAttrs = 1;
+        return c;
+    };
     if (p.U > 1) {
         {
             TraceScope tr(s, kTrTcUnitState);
-            unit_state_kernel<<<dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kUsThreads, kUsSmem, s>>>(
-                maps, ws, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu);
+            const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kUsThreads, kUsSmem);
+            if ((e = cudaLaunchKernelEx(&c, unit_state_kernel, maps, ws, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U,
+                                        (int)p.bpu)) != cudaSuccess)
+                return e;
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
         {
             TraceScope tr(s, kTrTcStatePass);
-            tc_state_pass_kernel<<<dim3(kNP / 4 / 256, (unsigned)d.H, (unsigned)d.b), 256, 0, s>>>(
-                ws, a.init_state, (int)d.H, (int)p.U);
+            const cudaLaunchConfig_t c = cfg(dim3(kNP / 4 / 256, (unsigned)d.H, (unsigned)d.b), 256, 0);
+            if ((e = cudaLaunchKernelEx(&c, tc_state_pass_kernel, ws, a.init_state, (int)d.H, (int)p.U)) != cudaSuccess)
+                return e;
         }
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
         TraceScope tr(s, kTrTcChunkOut);
-        chunk_out_kernel<<<dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem, s>>>(
-            maps, a.D, a.init_state, a.final_state, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U,
-            (int)p.bpu, p.U > 1 ? 1 : 0);
+        const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem);
+        if ((e = cudaLaunchKernelEx(&c, chunk_out_kernel, maps, a.D, a.init_state, a.final_state, ws, (int)d.L,
+                                    (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0)) !=
+            cudaSuccess)
+            return e;
     }
     return cudaGetLastError();
 }

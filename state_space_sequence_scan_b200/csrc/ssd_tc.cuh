@@ -359,6 +359,14 @@ __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
+// ---- programmatic dependent launch (the kernel after this one in the stream
+// may start its prologue before this one ends; see the launches in ssd_scan_tc.cu)
+// Let the next kernel in the stream begin launching.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Wait until every kernel this one depends on has completed and its writes
+// are visible (a no-op when the kernel was launched without the attribute).
+__device__ __forceinline__ void pdl_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- fp16 packing helpers
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
