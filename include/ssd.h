@@ -57,7 +57,10 @@ typedef enum ssd_status {
     SSD_ERR_CUDA = 5,           /* a CUDA call failed; see ssd_last_cuda_error() */
     SSD_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait gave up */
     SSD_ERR_PRECONDITION = 7    /* the GPU saw A > 0 (the log decay must be non-positive), or on the
-                                   tensor path an operand outside the fp16 range (|v| > 65504) */
+                                   tensor path an operand outside the fp16 range (|v| > 65504).  The
+                                   tensor path detects the latter as a non-finite y or final state
+                                   (an fp16 overflow always reaches one of them), so non-finite
+                                   inputs report it too */
 } ssd_status;
 
 typedef enum ssd_dtype {

@@ -612,13 +612,19 @@ __device__ __forceinline__ void co_factors(const CoSmem &S, int r, int f, int la
 }
 
 // X tile of slot r: bf16 -> fp16 in place (four 16-byte chunks per thread).
-__device__ __forceinline__ void co_widen_x(const CoSmem &S, int r, int tid, __half2 &amax) {
+//
+// chunk_out tracks no fp16 range per operand: a value beyond +-65504 in any
+// fp16 operand it forms (X, W, w.X, the entering state) rounds to inf, and
+// every such operand reaches y or the final state through a product and a
+// sum, where inf stays inf or turns NaN (inf * 0).  One finiteness check on
+// y and the final state (co_nonfinite) therefore reports it, off the W path.
+__device__ __forceinline__ void co_widen_x(const CoSmem &S, int r, int tid) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         uint4 *p = reinterpret_cast<uint4 *>(S.X(r) + (tid + q * kCoCompute) * 16);
         float f[8];
         bf16_chunk_to_f32(*p, f);
-        *p = pack8(f, amax);
+        *p = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
     }
 }
 
@@ -627,7 +633,7 @@ __device__ __forceinline__ void co_widen_x(const CoSmem &S, int r, int tid, __ha
 // products: w_j is rounded to fp16 once (w_j <= dt_j; one below the fp16
 // normal range only adds an absolute error under 3e-8 |x|), and no element
 // goes through fp32.
-__device__ __forceinline__ void co_form_wx(const CoSmem &S, int r, int f, int tid, __half2 &amax) {
+__device__ __forceinline__ void co_form_wx(const CoSmem &S, int r, int f, int tid) {
     const float *w = S.F(f);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -639,7 +645,6 @@ __device__ __forceinline__ void co_form_wx(const CoSmem &S, int r, int f, int ti
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const __half2 m = __hmul2(*reinterpret_cast<const __half2 *>(&xi[e]), wj);
-            amax = __hmax2(amax, __habs2(m));
             o[e] = *reinterpret_cast<const uint32_t *>(&m);
         }
         *reinterpret_cast<uint4 *>(S.WX() + c * 16) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -656,17 +661,22 @@ __device__ __forceinline__ void co_arrive(uint64_t *bar, int lane) {
 }
 
 // 16 floats -> 8 fp16 pairs
-__device__ __forceinline__ void pack16(const float *v, uint32_t *o, __half2 &amax) {
+__device__ __forceinline__ void pack16(const float *v, uint32_t *o) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        o[q] = pack_h2(v[2 * q], v[2 * q + 1]);
-        amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&o[q])));
-    }
+    for (int q = 0; q < 8; ++q) o[q] = pack_h2(v[2 * q], v[2 * q + 1]);
+}
+
+// Accumulates v*0 over 32 floats: the sum stays 0 unless a value is inf or NaN.
+__device__ __forceinline__ void co_nonfinite(const float *v, int n, float2 &acc) {
+    const float2 z = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+        if (2 * q < n) acc = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), z, acc);
 }
 
 // W for one 32-column slice cq <= lg of this thread's row i (see co_factors).
 __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32_t lane_addr, int lg, int cq,
-                                           int lane, float ci, __half2 &amax) {
+                                           int lane, float ci) {
     const float *cum = S.cum(r);
     const float *F = S.F(f);
     float v[32];
@@ -675,28 +685,34 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
     if (cq < lg) {                                   // below the diagonal: pivot at row 32*lg-1
         const float ui = expf(fminf(ci - cum[32 * lg - 1], 0.f));
         const float2 u2 = make_float2(ui, ui);
-        const float2 *vf = reinterpret_cast<const float2 *>(F + voff(lg - 1) + cq * 32);
+        const float4 *vf = reinterpret_cast<const float4 *>(F + voff(lg - 1) + cq * 32);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const float2 fq = __fmul2_rn(vf[q], u2);
-            const float2 m = __fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), fq);
-            v[2 * q] = m.x;
-            v[2 * q + 1] = m.y;
+        for (int q = 0; q < 8; ++q) {
+            const float4 f4 = vf[q];
+            const float2 m0 = __fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), __fmul2_rn(make_float2(f4.x, f4.y), u2));
+            const float2 m1 =
+                __fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), __fmul2_rn(make_float2(f4.z, f4.w), u2));
+            o[2 * q] = pack_h2(m0.x, m0.y);
+            o[2 * q + 1] = pack_h2(m1.x, m1.y);
         }
-        pack16(v, o, amax);
-        pack16(v + 16, o + 8, amax);
     } else {                                         // diagonal 32x32: pivot at its last row m
         if (S.G(f)[lg]) {
             // exp(cum_i - cum_j) = exp(cum_i - cum_m) exp(cum_m - cum_j); the first
             // factor is >= 1 and at most exp(cap) (flag), the second <= 1
             const float ud = expf(fminf(ci - cum[32 * lg + 31], kDiagExpCap));
             const float2 u2 = make_float2(ud, ud);
-            const float2 *vf = reinterpret_cast<const float2 *>(F + voff(lg) + cq * 32);
+            const float4 *vf = reinterpret_cast<const float4 *>(F + voff(lg) + cq * 32);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float2 m = __fmul2_rn(__fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), vf[q]), u2);
-                v[2 * q] = m.x;
-                v[2 * q + 1] = m.y;
+            for (int q = 0; q < 8; ++q) {
+                const float4 f4 = vf[q];
+                const float2 m0 =
+                    __fmul2_rn(__fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), make_float2(f4.x, f4.y)), u2);
+                const float2 m1 =
+                    __fmul2_rn(__fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), make_float2(f4.z, f4.w)), u2);
+                v[4 * q] = m0.x;
+                v[4 * q + 1] = m0.y;
+                v[4 * q + 2] = m1.x;
+                v[4 * q + 3] = m1.y;
             }
         } else {                                     // steep decay: one exp per element
             const float *dts = S.dt(r) + cq * 32, *cj = cum + cq * 32;
@@ -706,7 +722,7 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
                 asm volatile("" ::: "memory");       // one element at a time: keeps the loads from piling up
             }
         }
-        // causal select on the packed pairs (j <= i kept), before the range check
+        // causal select on the packed pairs (j <= i kept)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
             const uint4 m4 = S.Mask()[q4 * 32 + lane];
@@ -715,7 +731,6 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
             for (int e = 0; e < 4; ++e) {
                 const int q = 4 * q4 + e;
                 o[q] = pack_h2(v[2 * q], v[2 * q + 1]) & mw[e];
-                amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&o[q])));
             }
         }
     }
@@ -860,7 +875,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         const int ch = warp >> 2;                   // column half 0..1
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * lg) << 16);
         const float Dh = D[h];
-        __half2 amax = __float2half2_rn(0.f);
+        float2 nonfinite = make_float2(0.f, 0.f);  // stays 0 unless y or the final state is inf or NaN
         bool ok = true;
 
         // entering state of the unit, row `row`, columns 32*ch..: registers and fp16 copy
@@ -877,7 +892,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t o[8];
-                pack16(hv + 16 * hh, o, amax);
+                pack16(hv + 16 * hh, o);
 #pragma unroll
                 for (int q = 0; q < 2; ++q)
                     *reinterpret_cast<uint4 *>(S.H16() + sw128_off(row, 4 * ch + 2 * hh + q)) =
@@ -912,9 +927,9 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         ok = mbar_wait_abortable(S.bar(kBarTx0), 0, kWaitBudget, abort_flag);
         if (ok) co_factors(S, 0, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
         named_bar_sync(kCoCompute);                 // factors and masks visible to every compute warp
-        if (ok) co_widen_x(S, 0, tid, amax);
+        if (ok) co_widen_x(S, 0, tid);
         named_bar_sync(kCoCompute);
-        if (ok) co_form_wx(S, 0, 0, tid, amax);
+        if (ok) co_form_wx(S, 0, 0, tid);
 
         // every compute warp runs every iteration (and so every named barrier);
         // after an abort the waits return at once and the work is skipped
@@ -931,8 +946,8 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             tc_fence_after();
             if (ok) {
                 const float ci = cum[row];
-                if (ch <= lg) co_w_slice(S, r, f, lane_addr, lg, ch, lane, ci, amax);
-                if (ch + 2 <= lg) co_w_slice(S, r, f, lane_addr, lg, ch + 2, lane, ci, amax);
+                if (ch <= lg) co_w_slice(S, r, f, lane_addr, lg, ch, lane, ci);
+                if (ch + 2 <= lg) co_w_slice(S, r, f, lane_addr, lg, ch + 2, lane, ci);
             }
             co_arrive(S.bar(kBarW), lane);
 
@@ -941,7 +956,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 ok = ok && mbar_wait_abortable(S.bar(kBarTx0 + r1), ((uint32_t)(i + 1) / kCoXSlots) & 1u,
                                                kWaitBudget, abort_flag);
                 if (ok) co_factors(S, r1, f1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
-                if (ok) co_widen_x(S, r1, tid, amax);
+                if (ok) co_widen_x(S, r1, tid);
                 named_bar_sync(kCoCompute);          // factors and widened X of block k+1 visible
             }
 
@@ -966,19 +981,20 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         uint32_t o[8];
-                        pack16(hv + 16 * hh, o, amax);
+                        pack16(hv + 16 * hh, o);
 #pragma unroll
                         for (int q = 0; q < 2; ++q)
                             *reinterpret_cast<uint4 *>(S.H16() + sw128_off(row, 4 * ch + 2 * hh + q)) =
                                 make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
                     }
-                    co_form_wx(S, r1, f1, tid, amax);
+                    co_form_wx(S, r1, f1, tid);
                 } else if (final_state && u == U - 1) {
                     float *dst = final_state + bh * kNP + (size_t)row * kP + ch * 32;
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
                         *reinterpret_cast<float4 *>(dst + 4 * q) =
                             make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+                    co_nonfinite(hv, 32, nonfinite);
                 }
             }
             if (k + 1 < kb1) co_arrive(S.bar(kBarH16), lane);
@@ -1009,6 +1025,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                         yv[2 * q] = rr.x;
                         yv[2 * q + 1] = rr.y;
                     }
+                    co_nonfinite(yv, 16, nonfinite);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         *reinterpret_cast<float4 *>(stg + sw128_off(row, 4 * hh + q)) =
@@ -1017,7 +1034,9 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             }
             co_arrive(S.bar(kBarFree0 + f), lane);
         }
-        if (__any_sync(0xffffffffu, !in_f16_range(amax)) && lane == 0) flag_status(ws.status, kStatusRange);
+        // an fp16 operand out of range (see co_widen_x) or a non-finite input
+        if (__any_sync(0xffffffffu, !(nonfinite.x == 0.f && nonfinite.y == 0.f)) && lane == 0)
+            flag_status(ws.status, kStatusRange);
     }
     tc_fence_before();
     __syncthreads();
