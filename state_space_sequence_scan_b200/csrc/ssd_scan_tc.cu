@@ -487,10 +487,12 @@ tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
 // stall on an issue (a tcgen05.mma holds its issuing thread for about as
 // long as it runs).  Per 128-token block k the compute warps run:
 //   [1] C.B^T(k) done -> W(k) into TMEM (fp16, the A operand of W.X)
-//                                     -> MMA: S(k) = B^T (w.X(k)), Y(k) = W(k) X(k)
+//                                     -> MMA: Y(k) = W(k) X(k), then C.B^T(k+1)
 //   [2] x/dt/cum(k+1) landed -> decay factors, X(k+1) widened in place
 //   [3] S(k), Z(k) done -> H_in(k+1) = a_k H_in(k) + S(k) in registers, its
-//       fp16 copy, and w.X(k+1)       -> MMA: Z(k+1) = C(k+1) H_in(k+1)
+//       fp16 copy, and w.X(k+1)       -> MMA: Z(k+1) = C(k+1) H_in(k+1) and
+//                                        S(k+1) = B^T (w.X(k+1))
+// S(k+1) needs no W, so it runs a whole block before [3] of k+1 reads it.
 //   [4] Y(k) done -> y(k) = Y + exp(cum) Z(k) + D x, staged in block k's B tiles
 //                                     -> TMA: store y(k); x/dt/cum(k+3), C/B(k+2)
 // while the MMA warp issues C.B^T(k+1) as soon as C/B(k+1) have landed.  C
@@ -660,6 +662,14 @@ __device__ __forceinline__ void co_arrive(uint64_t *bar, int lane) {
     if (lane == 0) mbar_arrive(bar);
 }
 
+// The same for TMEM writes only (tcgen05.st, already waited for): no
+// generic-to-async proxy fence is needed for them.
+__device__ __forceinline__ void co_arrive_tmem(uint64_t *bar, int lane) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
 // 16 floats -> 8 fp16 pairs
 __device__ __forceinline__ void pack16(const float *v, uint32_t *o) {
 #pragma unroll
@@ -805,31 +815,37 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 mma_commit(S.bar(kBarZ));
                 ++S.issued()[kBarZ];
             };
-            auto issue_sy = [&](int s, int r) {
+            auto issue_s = [&](int s) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     mma_f16(tmem + kTmS, dadd(dBm0, st(s) + q * 2048), dadd(dWX, q * 2048), idesc_s, q > 0);
                 mma_commit(S.bar(kBarS));
                 ++S.issued()[kBarS];
+            };
+            auto issue_y = [&](int r) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     mma_f16_ts(tmem + kTmY, tmem + kTmW + 8u * q, dadd(dX0, xs(r) + q * 2048), idesc_y, q > 0);
                 mma_commit(S.bar(kBarY));
                 ++S.issued()[kBarY];
             };
+            // "fp16 state ready" also means w.X of that block is formed
             bool ok = mbar_wait_abortable(S.bar(kBarTcb0), 0, kWaitBudget, abort_flag);
             tc_fence_after();
             if (ok) issue_cb(0);
             ok = ok && mbar_wait_abortable(S.bar(kBarH16), 0, kWaitBudget, abort_flag);
             tc_fence_after();
-            if (ok) issue_z(0, 0);
+            if (ok) {
+                issue_z(0, 0);
+                issue_s(0);
+            }
             for (int k = kb0; k < kb1 && ok; ++k) {
-                const int i = k - kb0, s = i & 1, s1 = s ^ 1;
+                const int i = k - kb0, s1 = (i & 1) ^ 1;
                 const uint32_t par = (uint32_t)i & 1u, par1 = (uint32_t)(i + 1) & 1u;
                 ok = mbar_wait_abortable(S.bar(kBarW), par, kWaitBudget, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                issue_sy(s, i % kCoXSlots);
+                issue_y(i % kCoXSlots);
                 if (k + 1 < kb1) {
                     // C.B^T(k+1) once its tiles have landed (W(k) has read C.B^T(k))
                     ok = mbar_wait_abortable(S.bar(kBarTcb0 + s1), ((uint32_t)(i + 1) >> 1) & 1u, kWaitBudget,
@@ -837,10 +853,13 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                     if (!ok) break;
                     tc_fence_after();
                     issue_cb(s1);
+                    // Z(k+1), S(k+1) once the fp16 state and w.X of k+1 are formed (S(k)
+                    // and Z(k) have been read by then)
                     ok = mbar_wait_abortable(S.bar(kBarH16), par1, kWaitBudget, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     issue_z(s1, (int)par1);
+                    issue_s(s1);
                 }
             }
             if (!ok) *abort_flag = 1;
@@ -922,14 +941,14 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 S.Mask()[q4 * 32 + ml] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
             }
         }
-        co_arrive(S.bar(kBarH16), lane);
-        // block kb0: x landed -> factors, widened X, w.X
+        // block kb0: x landed -> factors, widened X, w.X; then "state ready"
         ok = mbar_wait_abortable(S.bar(kBarTx0), 0, kWaitBudget, abort_flag);
         if (ok) co_factors(S, 0, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
         named_bar_sync(kCoCompute);                 // factors and masks visible to every compute warp
         if (ok) co_widen_x(S, 0, tid);
         named_bar_sync(kCoCompute);
         if (ok) co_form_wx(S, 0, 0, tid);
+        co_arrive(S.bar(kBarH16), lane);
 
         // every compute warp runs every iteration (and so every named barrier);
         // after an abort the waits return at once and the work is skipped
@@ -949,7 +968,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 if (ch <= lg) co_w_slice(S, r, f, lane_addr, lg, ch, lane, ci);
                 if (ch + 2 <= lg) co_w_slice(S, r, f, lane_addr, lg, ch + 2, lane, ci);
             }
-            co_arrive(S.bar(kBarW), lane);
+            co_arrive_tmem(S.bar(kBarW), lane);
 
             // [2] block k+1: x landed -> factors, widened X (overlaps S(k), Y(k))
             if (k + 1 < kb1) {
