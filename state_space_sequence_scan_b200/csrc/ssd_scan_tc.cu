@@ -519,6 +519,7 @@ constexpr uint32_t kCoOffBar = kCoOffIss + 16 * 4;              // mbarriers, TM
 constexpr int kCoBars = 13;
 constexpr size_t kCoSmem = 1024 + kCoOffBar + kCoBars * 8 + 16;
 constexpr float kDiagExpCap = 64.0f;                            // largest exponent on the diagonal fast path
+constexpr double kL2Bytes = 126e6;                              // B200 L2
 static_assert(kCoXS % 1024 == 0 && kCoCB % 1024 == 0, "tiles must stay 1024-byte aligned");
 static_assert(kCoSmem <= 232448, "chunk_out shared memory exceeds the per-CTA limit");
 
@@ -572,6 +573,17 @@ __device__ __forceinline__ void co_load_cb(const CoSmem &S, const TcMaps &maps, 
     tma_load_4d(S.B(s), &maps.B, bar, 0, g, t0, b);
     tma_load_4d(S.B(s) + kTileBytes, &maps.B, bar, 64, g, t0, b);
     ++S.issued()[kBarTcb0 + s];
+}
+
+// TMA: C and B (fp16 copies) of block k into L2 a block ahead of their load
+// into shared memory (the heads of a group read them at about the same time,
+// so the first request would otherwise wait for DRAM with the rest behind it)
+__device__ __forceinline__ void co_prefetch_cb(const TcMaps &maps, int k, int g, int b) {
+    const int t0 = k * kBlk;
+    tma_prefetch_4d(&maps.C, 0, g, t0, b);
+    tma_prefetch_4d(&maps.C, 64, g, t0, b);
+    tma_prefetch_4d(&maps.B, 0, g, t0, b);
+    tma_prefetch_4d(&maps.B, 64, g, t0, b);
 }
 
 // TMA: X (bf16), dt and cum rows of block k into x slot r
@@ -750,7 +762,7 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
 __global__ void __launch_bounds__(kCoThreads, 1)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
                  const float *__restrict__ init, float *__restrict__ final_state, TcWs ws,
-                 int L, int H, int G, int nblk, int U, int bpu, int states_from_ws) {
+                 int L, int H, int G, int nblk, int U, int bpu, int states_from_ws, int prefetch_cb) {
     extern __shared__ uint8_t smem_raw[];
     CoSmem S;
     S.base = align1024(smem_raw);
@@ -870,12 +882,14 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         if (lane == 0) {
             for (int q = 0; q < 2 && kb0 + q < kb1; ++q) co_load_cb(S, maps, q, kb0 + q, g, b);
             for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q) co_load_x(S, maps, dtg, cumg, q, kb0 + q, h, b);
+            if (prefetch_cb && kb0 + 2 < kb1) co_prefetch_cb(maps, kb0 + 2, g, b);
             for (int k = kb0; k < kb1; ++k) {
                 const int i = k - kb0, s = i & 1;
                 if (!mbar_wait_abortable(S.bar(kBarFree0 + s), ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag))
                     break;
                 // block k is done with its x slot; its y sits in its B tiles
                 if (k + kCoXSlots < kb1) co_load_x(S, maps, dtg, cumg, i % kCoXSlots, k + kCoXSlots, h, b);
+                if (prefetch_cb && k + 3 < kb1) co_prefetch_cb(maps, k + 3, g, b);
                 tma_store_4d(&maps.y, S.B(s), 0, h, k * kBlk, b);
                 tma_store_4d(&maps.y, S.B(s) + kTileBytes, 32, h, k * kBlk, b);
                 tma_store_commit();
@@ -1144,10 +1158,14 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     }
     {
         TraceScope tr(s, kTrTcChunkOut);
+        // C/B prefetch into L2 only pays when the call streams more x and y than
+        // L2 holds: otherwise prep's fp16 copies are still there when read.
+        const double streamed = (double)d.b * d.L * d.H * d.P * (2.0 + 4.0);
+        const int prefetch_cb = streamed > kL2Bytes ? 1 : 0;
         const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem);
         if ((e = cudaLaunchKernelEx(&c, chunk_out_kernel, maps, a.D, a.init_state, a.final_state, ws, (int)d.L,
-                                    (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0)) !=
-            cudaSuccess)
+                                    (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0,
+                                    prefetch_cb)) != cudaSuccess)
             return e;
     }
     return cudaGetLastError();
