@@ -586,28 +586,16 @@ __device__ __forceinline__ void co_prefetch_cb(const TcMaps &maps, int k, int g,
     tma_prefetch_4d(&maps.B, 64, g, t0, b);
 }
 
-// TMA: X (bf16) of block k into x slot r; the slot's barrier expects the dt
-// and cum rows too (co_load_dtcum)
-__device__ __forceinline__ void co_load_xtile(const CoSmem &S, const TcMaps &maps, int r, int k, int h, int b) {
-    uint64_t *bar = S.bar(kBarTx0 + r);
-    mbar_arrive_expect_tx(bar, kCoXS);
-    tma_load_4d(S.X(r), &maps.x, bar, 0, h, k * kBlk, b);
-    ++S.issued()[kBarTx0 + r];
-}
-
-// TMA: dt and cum rows of block k (written by prep) into x slot r
-__device__ __forceinline__ void co_load_dtcum(const CoSmem &S, const float *dtv, const float *cum, int r, int k) {
-    const int t0 = k * kBlk;
-    uint64_t *bar = S.bar(kBarTx0 + r);
-    bulk_load(S.dt(r), dtv + (size_t)t0, kBlk * 4, bar);
-    bulk_load(S.cum(r), cum + (size_t)t0, kBlk * 4, bar);
-}
-
 // TMA: X (bf16), dt and cum rows of block k into x slot r
 __device__ __forceinline__ void co_load_x(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
                                           int r, int k, int h, int b) {
-    co_load_xtile(S, maps, r, k, h, b);
-    co_load_dtcum(S, dtv, cum, r, k);
+    const int t0 = k * kBlk;
+    uint64_t *bar = S.bar(kBarTx0 + r);
+    mbar_arrive_expect_tx(bar, kCoXS);
+    tma_load_4d(S.X(r), &maps.x, bar, 0, h, t0, b);
+    bulk_load(S.dt(r), dtv + (size_t)t0, kBlk * 4, bar);
+    bulk_load(S.cum(r), cum + (size_t)t0, kBlk * 4, bar);
+    ++S.issued()[kBarTx0 + r];
 }
 
 // Per-block decay factors into F(f), from the dt/cum of x slot r (all
@@ -804,9 +792,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *S.tslot();
-    // prep (and the unit passes) write what this kernel reads: each thread that
-    // reads it waits for them first.  The MMA warp reads only shared memory and
-    // TMEM; the TMA warp puts the first x tiles (the caller's) in flight before.
+    pdl_wait_prerequisites();                    // prep (and the unit passes) wrote what follows reads
 
     if (warp == kCoMmaWarp) {
         // ------------------------------ MMA warp ------------------------------
@@ -894,10 +880,8 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     } else if (warp == kCoTmaWarp) {
         // ------------------------------ TMA warp ------------------------------
         if (lane == 0) {
-            for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q) co_load_xtile(S, maps, q, kb0 + q, h, b);
-            pdl_wait_prerequisites();
             for (int q = 0; q < 2 && kb0 + q < kb1; ++q) co_load_cb(S, maps, q, kb0 + q, g, b);
-            for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q) co_load_dtcum(S, dtg, cumg, q, kb0 + q);
+            for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q) co_load_x(S, maps, dtg, cumg, q, kb0 + q, h, b);
             if (prefetch_cb && kb0 + 2 < kb1) co_prefetch_cb(maps, kb0 + 2, g, b);
             for (int k = kb0; k < kb1; ++k) {
                 const int i = k - kb0, s = i & 1;
@@ -927,7 +911,6 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         float2 nonfinite = make_float2(0.f, 0.f);  // stays 0 unless y or the final state is inf or NaN
         bool ok = true;
 
-        pdl_wait_prerequisites();
         // entering state of the unit, row `row`, columns 32*ch..: registers and fp16 copy
         float hv[32];
         {
