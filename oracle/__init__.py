@@ -7,6 +7,7 @@ from .ssd_oracle import (  # noqa: F401
     build_oracle,
     oracle_library_path,
     scan,
+    scan_states,
     softplus,
     step,
 )

@@ -21,6 +21,10 @@
  * The decode step (nnterp guide "Mamba-2", section "The state between
  * steps") is the same loop body for one token with the state updated in
  * place.
+ * The chunk-boundary states (same guide, "The state after every token"):
+ *   states[b, c, h] = S after token min((c+1) Q, L) - 1, for c < ceil(L / Q),
+ *   so the last one is final_state and Q = 1 gives the state after every
+ *   token.
  *
  * Readings where the pages are silent: softplus in its exact stable form;
  * the clamp is applied after the softplus; groups are contiguous blocks of
@@ -31,6 +35,7 @@
  * Layouts (row-major, contiguous):
  *   x [b,L,H,P]  dt_raw [b,L,H]  dt_bias [H]  A [H]  B,C [b,L,G,N]  D [H]
  *   init_state [b,H,N,P] (may be NULL)   y [b,L,H,P]  final_state [b,H,N,P]
+ *   chunk_states [b, ceil(L/Q), H, N, P] (may be NULL)
  *
  * Parity: pinned by tests/test_oracle.py (closed form, invariants, special
  * cases, hand-computed golden example).
@@ -60,7 +65,9 @@ double ssd_oracle_softplus(double z) { return sp_exact(z); }
 typedef struct {
     const float *x, *dt_raw, *dt_bias, *A, *B, *C, *D, *init_state;
     double *y, *final_state;
+    double *chunk_states;     /* [b, nc, H, N, P] or NULL */
     int64_t b, L, H, P, N, G;
+    int64_t Q, nc;            /* chunk size and count for chunk_states */
     double dt_lo, dt_hi;
     int64_t next;             /* next chain to claim */
     pthread_mutex_t lock;
@@ -114,6 +121,12 @@ static int run_chain(scan_job *J, int64_t bi, int64_t h, double *S, double *yacc
             for (p = 0; p < P; ++p) yacc[p] += c * Sn[p];
         }
         for (p = 0; p < P; ++p) yr[p] = yacc[p] + Dh * (double)xr[p];
+
+        /* the state after the last token of a chunk */
+        if (J->chunk_states && ((t + 1) % J->Q == 0 || t == L - 1)) {
+            double *sc = J->chunk_states + ((bi * J->nc + t / J->Q) * H + h) * N * P;
+            memcpy(sc, S, sizeof(double) * (size_t)(N * P));
+        }
     }
 
     if (J->final_state) {
@@ -168,26 +181,42 @@ static int run_threads(void *(*fn)(void *), void *job, int nthreads)
     return 0;
 }
 
-/* Whole-sequence recurrence.  Returns 0, or -1 on bad dimensions, -2 when out
- * of memory.  nthreads <= 0 uses every online core. */
-int ssd_oracle_scan(const float *x, const float *dt_raw, const float *dt_bias,
-                    const float *A, const float *B, const float *C, const float *D,
-                    const float *init_state, double *y, double *final_state,
-                    int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
-                    double dt_lo, double dt_hi, int nthreads)
+/* Whole-sequence recurrence, also recording the state after every chunk of Q
+ * tokens into chunk_states when that is not NULL.  Returns 0, or -1 on bad
+ * dimensions, -2 when out of memory.  nthreads <= 0 uses every online core. */
+int ssd_oracle_scan_states(const float *x, const float *dt_raw, const float *dt_bias,
+                           const float *A, const float *B, const float *C, const float *D,
+                           const float *init_state, double *y, double *final_state,
+                           double *chunk_states, int64_t b, int64_t L, int64_t H, int64_t P,
+                           int64_t N, int64_t G, int64_t Q, double dt_lo, double dt_hi, int nthreads)
 {
     scan_job J;
     if (b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0) return -1;
+    if (chunk_states && Q < 1) return -1;
     if (b == 0) return 0;
     memset(&J, 0, sizeof J);
     J.x = x; J.dt_raw = dt_raw; J.dt_bias = dt_bias; J.A = A; J.B = B; J.C = C; J.D = D;
     J.init_state = init_state; J.y = y; J.final_state = final_state;
+    J.chunk_states = chunk_states;
+    J.Q = Q > 0 ? Q : 1;
+    J.nc = (L + J.Q - 1) / J.Q;
     J.b = b; J.L = L; J.H = H; J.P = P; J.N = N; J.G = G;
     J.dt_lo = dt_lo; J.dt_hi = dt_hi;
     pthread_mutex_init(&J.lock, NULL);
     run_threads(scan_worker, &J, pick_threads(nthreads, b * H));
     pthread_mutex_destroy(&J.lock);
     return J.status;
+}
+
+/* Whole-sequence recurrence: y and final_state only. */
+int ssd_oracle_scan(const float *x, const float *dt_raw, const float *dt_bias,
+                    const float *A, const float *B, const float *C, const float *D,
+                    const float *init_state, double *y, double *final_state,
+                    int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G,
+                    double dt_lo, double dt_hi, int nthreads)
+{
+    return ssd_oracle_scan_states(x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, NULL,
+                                  b, L, H, P, N, G, 1, dt_lo, dt_hi, nthreads);
 }
 
 typedef struct {

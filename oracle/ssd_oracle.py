@@ -51,6 +51,9 @@ def _load():
         lib.ssd_oracle_scan.restype = ctypes.c_int
         lib.ssd_oracle_scan.argtypes = [f32p] * 8 + [f64p, f64p] + [i64] * 6 + [
             ctypes.c_double, ctypes.c_double, ctypes.c_int]
+        lib.ssd_oracle_scan_states.restype = ctypes.c_int
+        lib.ssd_oracle_scan_states.argtypes = [f32p] * 8 + [f64p, f64p, f64p] + [i64] * 7 + [
+            ctypes.c_double, ctypes.c_double, ctypes.c_int]
         lib.ssd_oracle_step.restype = ctypes.c_int
         lib.ssd_oracle_step.argtypes = [f32p] * 7 + [f64p, f64p] + [i64] * 5 + [
             ctypes.c_double, ctypes.c_double, ctypes.c_int]
@@ -111,6 +114,43 @@ def scan(x, dt_raw, dt_bias, A, B, C, D, init_state=None,
     if rc != 0:
         raise RuntimeError("ssd_oracle_scan failed with code %d" % rc)
     return y, fs
+
+
+def scan_states(x, dt_raw, dt_bias, A, B, C, D, chunk_size: int, init_state=None,
+                dt_limit: Tuple[float, float] = (0.0, float("inf")),
+                nthreads: int = 0) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """As scan(), also returning the chunk-boundary states (nnterp guide
+    "Mamba-2", "The state after every token"): states [b, ceil(L/Q), H, N, P]
+    float64, states[:, c] the state after token min((c+1) Q, L) - 1, so
+    states[:, -1] is final_state and Q = 1 gives the state after every token.
+    """
+    x, dt_raw, dt_bias, A, B, C, D = (_f32(v) for v in (x, dt_raw, dt_bias, A, B, C, D))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    Q = int(chunk_size)
+    if Q < 1:
+        raise ValueError("oracle.scan_states: chunk_size must be >= 1")
+    if dt_raw.shape != (b, L, H) or B.shape != (b, L, G, N) or C.shape != B.shape:
+        raise ValueError("oracle.scan_states: inconsistent shapes")
+    if dt_bias.shape != (H,) or A.shape != (H,) or D.shape != (H,) or H % G:
+        raise ValueError("oracle.scan_states: bad per-head parameter shapes or H % G != 0")
+    s0 = None
+    if init_state is not None:
+        s0 = _f32(init_state)
+        if s0.shape != (b, H, N, P):
+            raise ValueError("oracle.scan_states: init_state must be [b,H,N,P]")
+    nc = (L + Q - 1) // Q
+    y = np.empty((b, L, H, P), dtype=np.float64)
+    fs = np.empty((b, H, N, P), dtype=np.float64)
+    states = np.empty((b, nc, H, N, P), dtype=np.float64)
+    rc = _load().ssd_oracle_scan_states(
+        _p32(x), _p32(dt_raw), _p32(dt_bias), _p32(A), _p32(B), _p32(C), _p32(D),
+        _p32(s0) if s0 is not None else ctypes.POINTER(ctypes.c_float)(),
+        _p64(y), _p64(fs), _p64(states), b, L, H, P, N, G, Q,
+        float(dt_limit[0]), float(dt_limit[1]), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("ssd_oracle_scan_states failed with code %d" % rc)
+    return y, fs, states
 
 
 def step(x, dt_raw, dt_bias, A, B, C, D, state: np.ndarray,

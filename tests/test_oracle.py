@@ -339,6 +339,87 @@ def test_golden_shapes_of_the_130m_layer():
     assert list(y.shape) == g["y"] and list(fs.shape) == g["state"]
 
 
+def _closed_form_states(case, lo=0.0, hi=INF):
+    """Brute force: the state after every token, S_t = exp(sum_{r<=t} la_r) H0
+    + sum_{s<=t} exp(sum_{s<r<=t} la_r) dt_s B_s x_s^T, explicit loops."""
+    x = case["x"].astype(np.float64)
+    B = case["B"].astype(np.float64)
+    A = case["A"].astype(np.float64)
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dt = _dt(case, lo, hi)
+    H0 = (np.zeros((b, H, N, P)) if case["init_state"] is None
+          else case["init_state"].astype(np.float64))
+    out = np.zeros((b, L, H, N, P))
+    for bi in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            la = dt[bi, :, h] * A[h]
+            for t in range(L):
+                st = math.exp(la[: t + 1].sum()) * H0[bi, h]
+                for s in range(t + 1):
+                    st = st + math.exp(la[s + 1: t + 1].sum()) * dt[bi, s, h] * np.outer(B[bi, s, g], x[bi, s, h])
+                out[bi, t, h] = st
+    return out
+
+
+@pytest.mark.parametrize("seed,init", [(40, True), (41, False)])
+def test_states_after_every_token_equal_closed_form(seed, init):
+    """Chunk size 1: every token is a chunk boundary (nnterp guide, "The
+    state after every token"), so states[:, t] is the state after token t."""
+    case = _rand_case(seed, b=2, L=9, H=4, P=3, N=2, G=2, init=init)
+    y, fs, st = oracle.scan_states(chunk_size=1, **case)
+    ref = _closed_form_states(case)
+    assert st.shape == ref.shape
+    assert _rel(st, ref) < 1e-12
+    y0, fs0 = oracle.scan(**case)
+    assert np.array_equal(y, y0) and np.array_equal(fs, fs0)
+
+
+@pytest.mark.parametrize("Q", [2, 3, 5, 23, 64])
+def test_chunk_states_are_the_per_token_states_at_boundaries(Q):
+    """states[:, c] is the state after token min((c+1) Q, L) - 1, the last one
+    is final_state (the guide prints states[:, -1] == final as True)."""
+    case = _rand_case(42, b=2, L=23, init=True)
+    _, fs, st = oracle.scan_states(chunk_size=Q, **case)
+    _, _, per_tok = oracle.scan_states(chunk_size=1, **case)
+    L = case["x"].shape[1]
+    nc = (L + Q - 1) // Q
+    assert st.shape[1] == nc
+    for c in range(nc):
+        assert np.array_equal(st[:, c], per_tok[:, min((c + 1) * Q, L) - 1])
+    assert np.array_equal(st[:, -1], fs)
+
+
+def test_skip_token_holds_the_state():
+    """The guide's check: with betas (dt) of token 3 set to 0, the state after
+    token 3 equals the state after token 2 exactly."""
+    case = _rand_case(43, b=1, L=10, init=False)
+    case["dt_raw"][:, 3, :] = -1.0e4                   # softplus underflows to exactly 0
+    _, _, held = oracle.scan_states(chunk_size=1, **case)
+    assert np.array_equal(held[:, 3], held[:, 2])
+    assert not np.array_equal(held[:, 4], held[:, 3])
+
+
+def test_golden_states_shape_of_the_130m_layer():
+    """Shape of the per-token states the nnterp guide prints for mamba2-130m
+    on a 10-token prompt, and its states[:, -1] == final."""
+    with open(os.path.join(GOLDEN, "nnterp_mamba2_130m_shapes.json")) as f:
+        g = json.load(f)
+    b, L = g["batch"], g["seq"]
+    H, P, N, G = g["heads"], g["head_dim"], g["state_dim"], g["groups"]
+    rng = np.random.default_rng(1)
+    case = dict(x=rng.standard_normal((b, L, H, P)).astype(np.float32),
+                dt_raw=rng.standard_normal((b, L, H)).astype(np.float32),
+                dt_bias=np.zeros(H, np.float32), A=-np.ones(H, np.float32),
+                B=rng.standard_normal((b, L, G, N)).astype(np.float32),
+                C=rng.standard_normal((b, L, G, N)).astype(np.float32),
+                D=np.ones(H, np.float32), init_state=None)
+    _, fs, st = oracle.scan_states(chunk_size=1, **case)
+    assert list(st.shape) == g["states_per_token"]
+    assert np.array_equal(st[:, -1], fs)
+
+
 def test_bad_shapes_raise():
     case = _rand_case(18)
     bad = dict(case)
