@@ -44,7 +44,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # algorithmic work (bytes every implementation must move, flops of the causal
 # chunked form with C.B^T counted once per group)
 
-def scan_bytes(cfg) -> float:
+def states_bytes(cfg) -> float:
+    """The chunk-boundary states [b, nc, H, N, P] fp32 (--chunk-states)."""
+    nc = math.ceil(cfg.seqlen / cfg.chunk_size)
+    return float(cfg.batch * nc * cfg.nheads * cfg.state_dim * cfg.head_dim * 4)
+
+
+def scan_bytes(cfg, states=False) -> float:
     b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
     e = 4 if cfg.dtype == "f32" else 2
     tok = b * L
@@ -52,7 +58,7 @@ def scan_bytes(cfg) -> float:
     byt += tok * H * P * 4                                      # y (fp32)
     byt += b * H * N * P * 4 * (2 if cfg.init == "normal" else 1)  # init (if any) + final state
     byt += 3 * H * 4
-    return float(byt)
+    return float(byt) + (states_bytes(cfg) if states else 0.0)
 
 
 def scan_flops(cfg) -> float:
@@ -208,21 +214,28 @@ def bench_scan(cfg, args, ws, rank, local):
     from state_space_sequence_scan_b200 import ssd
     dev = torch.device("cuda", local)
     inp = make_scan_inputs(cfg, seed=cfg.seed + 1000 * rank)
-    one = scan_bytes(cfg)
+    one = scan_bytes(cfg, args.chunk_states)
     nsets = max(1, min(8, math.ceil(3 * L2_BYTES / one)))
     sets = _dev_sets(inp, nsets, dev)
     b, L, H, P, N, G, Q = (cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups,
                            cfg.chunk_size)
-    outs = [(torch.empty(b, L, H, P, device=dev), torch.empty(b, H, N, P, device=dev)) for _ in range(nsets)]
+    nc = math.ceil(L / Q)
+    outs = [(torch.empty(b, L, H, P, device=dev), torch.empty(b, H, N, P, device=dev),
+             torch.empty(b, nc, H, N, P, device=dev) if args.chunk_states else None) for _ in range(nsets)]
     wsz = ssd.workspace_size(b, L, H, P, N, G, Q, sets[0]["x"].dtype, args.path)
     work = ssd.alloc_workspace(wsz, dev)
 
     def step(k):
         s = sets[k % nsets]
-        y, fs = outs[k % nsets]
-        ssd.chunk_scan_fwd(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"],
-                           init_state=s["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
-                           final_state=fs)
+        y, fs, cs = outs[k % nsets]
+        if cs is None:
+            ssd.chunk_scan_fwd(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"],
+                               init_state=s["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
+                               final_state=fs)
+        else:
+            ssd.chunk_scan_fwd_states(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"],
+                                      init_state=s["init_state"], chunk_size=Q, path=args.path, workspace=work,
+                                      y=y, final_state=fs, chunk_states=cs)
 
     for k in range(args.warmup):
         step(k)
@@ -282,7 +295,8 @@ def capture_steps(step, steps):
 
 def e2e_scan(inp, cfg, args, dev, work):
     """Same metric through the public call with host buffers: pinned host
-    inputs copied in, the scan, y and final_state copied back, every step."""
+    inputs copied in, the scan, y and final_state (and with --chunk-states the
+    chunk-boundary states) copied back, every step."""
     from state_space_sequence_scan_b200 import ssd
     host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
     d = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in inp.items()}
@@ -291,17 +305,26 @@ def e2e_scan(inp, cfg, args, dev, work):
     fs = torch.empty(b, H, N, P, device=dev)
     y_h = torch.empty(b, L, H, P).pin_memory()
     fs_h = torch.empty(b, H, N, P).pin_memory()
+    nc = math.ceil(L / Q)
+    cs = torch.empty(b, nc, H, N, P, device=dev) if args.chunk_states else None
+    cs_h = torch.empty(b, nc, H, N, P).pin_memory() if args.chunk_states else None
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = y_h.numel() * 4 + fs_h.numel() * 4
+    d2h = y_h.numel() * 4 + fs_h.numel() * 4 + (cs_h.numel() * 4 if cs_h is not None else 0)
     steps = max(3, min(args.steps, 20))
 
     def one():
         for k, v in host.items():
             if v is not None:
                 d[k].copy_(v, non_blocking=True)
-        ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
-                           init_state=d["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
-                           final_state=fs)
+        if cs is None:
+            ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                               init_state=d["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
+                               final_state=fs)
+        else:
+            ssd.chunk_scan_fwd_states(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                                      init_state=d["init_state"], chunk_size=Q, path=args.path, workspace=work,
+                                      y=y, final_state=fs, chunk_states=cs)
+            cs_h.copy_(cs, non_blocking=True)
         y_h.copy_(y, non_blocking=True)
         fs_h.copy_(fs, non_blocking=True)
 
@@ -389,19 +412,19 @@ def dominant(trace):
 
 
 # algorithmic bytes each traced kernel must move (per launch), as fractions of the call
-def kernel_bytes(cfg, name) -> float:
+def kernel_bytes(cfg, name, states=False) -> float:
     b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
     e = 4 if cfg.dtype == "f32" else 2
     tok = b * L
     x, bc, dt, y = tok * H * P * e, tok * G * N * e, tok * H * 4, tok * H * P * 4
     st = b * H * N * P * 4
     if name.endswith("chunk_out"):
-        return float(x + 2 * bc + y)
+        return float(x + 2 * bc + y) + (states_bytes(cfg) if states and name.startswith("tc_") else 0.0)
     if name.endswith("chunk_state") or name.endswith("unit_state"):
         return float(x + bc + dt)
     if name.endswith("state_pass"):
         return float(st * (2 if cfg.init == "normal" else 1))
-    return scan_bytes(cfg)
+    return scan_bytes(cfg, states)
 
 
 def cpu_baseline_scan(cfg, budget_s=12.0):
@@ -498,7 +521,7 @@ def pick(name):
     raise SystemExit("unknown workload %s (scan: %s; decode: %s)" % (name, list(SCAN_CONFIGS), list(STEP_CONFIGS)))
 
 
-def workload_config(cfg, is_step, nsets=None):
+def workload_config(cfg, is_step, nsets=None, states=False):
     if is_step:
         c = {"workload": cfg.name, "batch": cfg.batch, "heads": cfg.nheads, "head_dim": cfg.head_dim,
              "state_dim": cfg.state_dim, "groups": cfg.ngroups, "state_dtype": "f32", "in_dtype": cfg.dtype,
@@ -510,8 +533,11 @@ def workload_config(cfg, is_step, nsets=None):
              "chunk_size": cfg.chunk_size, "in_dtype": cfg.dtype, "y_dtype": "f32",
              "init_state": cfg.init != "zero"}
         if nsets is not None:
-            c["l2"] = ("rotating %d input/output sets (%.0f MB > 2x L2)" % (nsets, nsets * scan_bytes(cfg) / 1e6)
-                       if nsets > 1 else "inputs %.0f MB > L2" % (scan_bytes(cfg) / 1e6))
+            one = scan_bytes(cfg, states)
+            c["l2"] = ("rotating %d input/output sets (%.0f MB > 2x L2)" % (nsets, nsets * one / 1e6)
+                       if nsets > 1 else "inputs %.0f MB > L2" % (one / 1e6))
+        if states:
+            c["chunk_states"] = "[b, %d, H, N, P] f32 written every step" % math.ceil(cfg.seqlen / cfg.chunk_size)
     return c
 
 
@@ -525,6 +551,8 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-decode", action="store_true", help="skip the decode figure on the scan line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--chunk-states", action="store_true",
+                    help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -575,7 +603,7 @@ def finish(cfg, is_step, r, args, ws, rank, peaks, peak_kind, sub=False):
     else:
         value = ws * r["tokens"] / (ms_step * 1e-3) / 1e6
         unit = "Mtokens/s"
-        kb = kernel_bytes(cfg, name) if name else r["bytes"]
+        kb = kernel_bytes(cfg, name, args.chunk_states) if name else r["bytes"]
         dtype = "f32" if cfg.dtype == "f32" else "bf16-in/f32"
         e2e_val = ws * r["tokens"] / (r["e2e"]["ms_per_step"] * 1e-3) / 1e6
     achieved = kb / (avg * 1e-3) / 1e9 if avg > 0 else None
@@ -597,7 +625,8 @@ def finish(cfg, is_step, r, args, ws, rank, peaks, peak_kind, sub=False):
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded; shapes/distributions of the workload)",
-            "config": workload_config(cfg, is_step, r.get("nsets")), "roofline": roof, "clocks": r["clocks"],
+            "config": workload_config(cfg, is_step, r.get("nsets"), (not is_step) and args.chunk_states),
+            "roofline": roof, "clocks": r["clocks"],
             "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": r["e2e"]["h2d"],
                     "d2h_bytes_per_step": r["e2e"]["d2h"]},
             "gpu_launches": r["launches"]}

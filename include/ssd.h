@@ -113,6 +113,30 @@ SSD_API ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const 
                               float dt_lo, float dt_hi, int in_dtype, int path,
                               void *workspace, size_t workspace_bytes, void *stream);
 
+/* ssd_chunk_scan_fwd that also writes the chunk-boundary states (nnterp
+ * guide "Mamba-2", section "The state after every token": the chunk scan
+ * holds the state at every chunk boundary, and with chunk_size 1 every token
+ * is one).
+ *   chunk_states  [batch, nchunks, nheads, state_dim, head_dim] float32 out,
+ *                 nchunks = ceil(seqlen / chunk_size).  Chunk c holds the
+ *                 state after token min((c+1) chunk_size, seqlen) - 1, so the
+ *                 last one equals final_state.  16-byte aligned; must not
+ *                 overlap the inputs, y, final_state or the workspace.  NULL
+ *                 makes the call ssd_chunk_scan_fwd.
+ * Every other argument is as for ssd_chunk_scan_fwd, the workspace sized by
+ * ssd_chunk_scan_workspace_size for the same path.  The tensor-core path
+ * holds the state only at the ends of its 128-token blocks: when the call
+ * resolves to it (SSD_PATH_TENSOR, or SSD_PATH_AUTO on a shape it takes), a
+ * chunk_size that is not a multiple of 128 returns SSD_ERR_UNSUPPORTED before
+ * anything is enqueued.  SSD_PATH_SIMT takes any chunk size. */
+SSD_API ssd_status ssd_chunk_scan_fwd_states(const void *x, const float *dt_raw, const float *dt_bias,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const float *init_state, float *y, float *final_state,
+                                     float *chunk_states, int64_t batch, int64_t seqlen, int64_t nheads,
+                                     int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                                     int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype, int path,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
 /* One decode token (nnterp guide "Mamba-2", section "The state between
  * steps": the update writes the new state into the cache and returns only y;
  * there is no sequence axis).

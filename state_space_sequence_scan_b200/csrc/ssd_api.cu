@@ -116,13 +116,14 @@ ssd_status ssd_chunk_scan_workspace_size(int64_t batch, int64_t seqlen, int64_t 
     return SSD_OK;
 }
 
-ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const float *dt_bias,
-                              const float *A, const void *B, const void *C, const float *D,
-                              const float *init_state, float *y, float *final_state,
-                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
-                              int64_t state_dim, int64_t ngroups, int64_t chunk_size,
-                              float dt_lo, float dt_hi, int in_dtype, int path,
-                              void *workspace, size_t workspace_bytes, void *stream) {
+namespace {
+
+// The forward scan, with or without the chunk-boundary states.
+ssd_status scan_fwd(const void *x, const float *dt_raw, const float *dt_bias, const float *A, const void *B,
+                    const void *C, const float *D, const float *init_state, float *y, float *final_state,
+                    float *chunk_states, int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                    int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi,
+                    int in_dtype, int path, void *workspace, size_t workspace_bytes, void *stream) {
     ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size,
                                     in_dtype, path);
     if (st != SSD_OK) return st;
@@ -131,11 +132,14 @@ ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const float *d
     const bool has_tokens = batch > 0 && seqlen > 0;
     if (has_tokens && (!x || !dt_raw || !B || !C || !y)) return SSD_ERR_INVALID_ARG;
     if ((x && !aligned16(x)) || (B && !aligned16(B)) || (C && !aligned16(C)) || (y && !aligned16(y)) ||
-        (init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
+        (init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)) ||
+        (chunk_states && !aligned16(chunk_states)))
         return SSD_ERR_ALIGNMENT;
     const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
     int chosen = 0;
     if ((st = resolve_path(d, in_dtype, path, &chosen)) != SSD_OK) return st;
+    // the tensor path has the state at its 128-token block ends only
+    if (chunk_states && chosen == SSD_PATH_TENSOR && chunk_size % 128 != 0) return SSD_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < path_ws(d, chosen)) return SSD_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
 
@@ -156,11 +160,37 @@ ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const float *d
 
     ssd::ScanArgs a;
     a.x = x; a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.B = B; a.C = C; a.D = D;
-    a.init_state = init_state; a.y = y; a.final_state = final_state;
+    a.init_state = init_state; a.y = y; a.final_state = final_state; a.chunk_states = chunk_states;
     a.dt_lo = dt_lo; a.dt_hi = dt_hi; a.bf16 = in_dtype == SSD_BF16;
     e = chosen == SSD_PATH_TENSOR ? ssd::tc_scan(a, d, workspace, s) : ssd::simt_scan(a, d, workspace, s);
     if (e != cudaSuccess) return cuda_fail(e);
     return SSD_OK;
+}
+
+}  // namespace
+
+ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const float *dt_bias,
+                              const float *A, const void *B, const void *C, const float *D,
+                              const float *init_state, float *y, float *final_state,
+                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                              int64_t state_dim, int64_t ngroups, int64_t chunk_size,
+                              float dt_lo, float dt_hi, int in_dtype, int path,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, nullptr, batch, seqlen, nheads,
+                    head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
+                    workspace_bytes, stream);
+}
+
+ssd_status ssd_chunk_scan_fwd_states(const void *x, const float *dt_raw, const float *dt_bias,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const float *init_state, float *y, float *final_state,
+                                     float *chunk_states, int64_t batch, int64_t seqlen, int64_t nheads,
+                                     int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                                     int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype, int path,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, chunk_states, batch, seqlen,
+                    nheads, head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
+                    workspace_bytes, stream);
 }
 
 ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_bias, const float *A,

@@ -18,6 +18,7 @@ struct ScanArgs {
     const void *B, *C;
     const float *D, *init_state;
     float *y, *final_state;
+    float *chunk_states = nullptr;  // [b, nc, H, N, P] or null: the state after every chunk
     float dt_lo, dt_hi;
     int bf16;                      // 1: x/B/C are bfloat16, 0: float32
 };

@@ -136,10 +136,12 @@ chunk_state_kernel(const T *__restrict__ x, const float *__restrict__ dt_raw,
 
 __global__ void __launch_bounds__(kThreads)
 state_pass_kernel(SimtWs ws, const float *__restrict__ init, float *__restrict__ final_state,
-                  int H, int NP, int nc) {
+                  float *__restrict__ chunk_states, int H, int NP, int nc) {
     const int e = blockIdx.x * kThreads + threadIdx.x;
     if (e >= NP) return;
     const size_t bh = (size_t)blockIdx.z * H + blockIdx.y;
+    // state after chunk c at chunk_states[b, c, h, e]: chunk c's stride is H * NP
+    float *out = chunk_states ? chunk_states + ((size_t)blockIdx.z * nc * H + blockIdx.y) * NP + e : nullptr;
     float hs = init ? init[bh * NP + e] : 0.f;
     float *S = ws.states + bh * nc * (size_t)NP + e;
     const float *ell = ws.ell + bh * nc;
@@ -149,6 +151,7 @@ state_pass_kernel(SimtWs ws, const float *__restrict__ init, float *__restrict__
         if (c + 1 < nc) nxt = S[(size_t)(c + 1) * NP];
         S[(size_t)c * NP] = hs;                         // state entering chunk c
         hs = fmaf(expf(fminf(ell[c], 0.f)), hs, s);
+        if (out) out[(size_t)c * H * NP] = hs;          // state after chunk c
     }
     if (final_state) final_state[bh * NP + e] = hs;
 }
@@ -306,7 +309,8 @@ cudaError_t run(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s)
     const dim3 g2((unsigned)((NP + kThreads - 1) / kThreads), (unsigned)d.H, (unsigned)d.b);
     {
         TraceScope tr(s, kTrSimtStatePass);
-        state_pass_kernel<<<g2, kThreads, 0, s>>>(ws, a.init_state, a.final_state, (int)d.H, NP, (int)d.nc);
+        state_pass_kernel<<<g2, kThreads, 0, s>>>(ws, a.init_state, a.final_state, a.chunk_states, (int)d.H, NP,
+                                                  (int)d.nc);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int tiles = (int)((d.Q + TI - 1) / TI);

@@ -762,7 +762,8 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
 __global__ void __launch_bounds__(kCoThreads, 1)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
                  const float *__restrict__ init, float *__restrict__ final_state, TcWs ws,
-                 int L, int H, int G, int nblk, int U, int bpu, int states_from_ws, int prefetch_cb) {
+                 int L, int H, int G, int nblk, int U, int bpu, int states_from_ws, int prefetch_cb,
+                 float *__restrict__ chunk_states, int bpc, int nc) {
     extern __shared__ uint8_t smem_raw[];
     CoSmem S;
     S.base = align1024(smem_raw);
@@ -1029,6 +1030,15 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                             make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
                     co_nonfinite(hv, 32, nonfinite);
                 }
+                // block k ends chunk k / bpc (the last block ends the last chunk)
+                if (chunk_states && ((k + 1) % bpc == 0 || k == nblk - 1)) {
+                    float *dst =
+                        chunk_states + (((size_t)b * nc + k / bpc) * H + h) * kNP + (size_t)row * kP + ch * 32;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4 *>(dst + 4 * q) =
+                            make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+                }
             }
             if (k + 1 < kb1) co_arrive(S.bar(kBarH16), lane);
 
@@ -1163,9 +1173,11 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         const double streamed = (double)d.b * d.L * d.H * d.P * (2.0 + 4.0);
         const int prefetch_cb = streamed > kL2Bytes ? 1 : 0;
         const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem);
+        // the caller checked that chunk_states come with chunk_size a multiple of kBlk
+        const int bpc = (int)(d.Q / kBlk) > 0 ? (int)(d.Q / kBlk) : 1;
         if ((e = cudaLaunchKernelEx(&c, chunk_out_kernel, maps, a.D, a.init_state, a.final_state, ws, (int)d.L,
                                     (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0,
-                                    prefetch_cb)) != cudaSuccess)
+                                    prefetch_cb, a.chunk_states, bpc, (int)d.nc)) != cudaSuccess)
             return e;
     }
     return cudaGetLastError();

@@ -27,7 +27,7 @@ STATUS_NAMES = {
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 
-EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_step",
+EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_states", "ssd_step",
             "ssd_read_device_status", "ssd_status_string", "ssd_last_cuda_error", "ssd_version",
             "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count")
 
@@ -56,6 +56,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_chunk_scan_workspace_size.argtypes = [i64] * 7 + [i32, i32, ctypes.POINTER(sz)]
     lib.ssd_chunk_scan_fwd.restype = i32
     lib.ssd_chunk_scan_fwd.argtypes = [vp] * 10 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
+    lib.ssd_chunk_scan_fwd_states.restype = i32
+    lib.ssd_chunk_scan_fwd_states.argtypes = [vp] * 11 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
     lib.ssd_step.restype = i32
     lib.ssd_step.argtypes = [vp] * 9 + [i64] * 5 + [f32, f32, i32, vp]
     lib.ssd_read_device_status.restype = i32
@@ -165,6 +167,62 @@ def chunk_scan_fwd(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check("ssd_chunk_scan_fwd", st)
     return y, final_state
+
+
+def chunk_scan_fwd_states(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor, A: torch.Tensor,
+                          B: torch.Tensor, C: torch.Tensor, D: torch.Tensor,
+                          init_state: Optional[torch.Tensor] = None, chunk_size: int = 256,
+                          dt_limit: Tuple[float, float] = (0.0, math.inf), path: str = "auto",
+                          workspace: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                          final_state: Optional[torch.Tensor] = None,
+                          chunk_states: Optional[torch.Tensor] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """chunk_scan_fwd that also returns the chunk-boundary states
+    [b, ceil(L/chunk_size), H, N, P] f32 (ssd_chunk_scan_fwd_states): chunk c
+    holds the state after token min((c+1) chunk_size, L) - 1.  Under
+    path="auto" a chunk size that is not a multiple of 128 runs on the SIMT
+    path, the one that has the state at any token."""
+    lib = load_library()
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    _need_cuda("x", x)
+    if x.dtype not in DTYPES:
+        raise ValueError("x/B/C must be float32 or bfloat16")
+    _need_cuda("B", B, x.dtype, (b, L, G, N))
+    _need_cuda("C", C, x.dtype, (b, L, G, N))
+    _need_cuda("dt_raw", dt_raw, torch.float32, (b, L, H))
+    for nm, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need_cuda(nm, t, torch.float32, (H,))
+    if init_state is not None:
+        _need_cuda("init_state", init_state, torch.float32, (b, H, N, P))
+    if path == "auto" and int(chunk_size) % 128 != 0:
+        path = "simt"
+    nc = (L + int(chunk_size) - 1) // int(chunk_size)
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
+    else:
+        _need_cuda("y", y, torch.float32, (b, L, H, P))
+    if final_state is None:
+        final_state = torch.empty((b, H, N, P), dtype=torch.float32, device=dev)
+    else:
+        _need_cuda("final_state", final_state, torch.float32, (b, H, N, P))
+    if chunk_states is None:
+        chunk_states = torch.empty((b, nc, H, N, P), dtype=torch.float32, device=dev)
+    else:
+        _need_cuda("chunk_states", chunk_states, torch.float32, (b, nc, H, N, P))
+    need = workspace_size(b, L, H, P, N, G, chunk_size, x.dtype, path)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    st = lib.ssd_chunk_scan_fwd_states(
+        _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+        _ptr(y), _ptr(final_state), _ptr(chunk_states), b, L, H, P, N, G, int(chunk_size),
+        float(dt_limit[0]), float(dt_limit[1]), DTYPES[x.dtype], PATHS[path],
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _check("ssd_chunk_scan_fwd_states", st)
+    return y, final_state, chunk_states
 
 
 def read_device_status(workspace: torch.Tensor) -> int:

@@ -97,6 +97,34 @@ def test_forward_rejects_bad_arguments_on_host(lib):
     assert _fwd(lib, **ok, path=2, dtype=0) == 2              # tensor path needs bf16
 
 
+def _fwd_states(lib, **kw):
+    a = dict(x=None, dt_raw=None, dt_bias=None, A=None, B=None, C=None, D=None, init=None, y=None, fs=None,
+             cs=None, b=1, L=8, H=2, P=16, N=16, G=1, Q=4, lo=0.0, hi=math.inf, dtype=0, path=0, ws=None, wsb=0,
+             stream=None)
+    a.update(kw)
+    return lib.ssd_chunk_scan_fwd_states(a["x"], a["dt_raw"], a["dt_bias"], a["A"], a["B"], a["C"], a["D"],
+                                         a["init"], a["y"], a["fs"], a["cs"], a["b"], a["L"], a["H"], a["P"],
+                                         a["N"], a["G"], a["Q"], a["lo"], a["hi"], a["dtype"], a["path"], a["ws"],
+                                         a["wsb"], a["stream"])
+
+
+def test_forward_states_rejects_bad_arguments_on_host(lib):
+    """The chunk-states entry point checks as the plain one does, plus: the
+    states pointer's alignment, and that a call resolving to the tensor path
+    has a chunk size that is a multiple of its 128-token blocks."""
+    fake = 0x10000
+    ok = dict(x=fake, dt_raw=fake, dt_bias=fake, A=fake, B=fake, C=fake, D=fake, y=fake, fs=fake, cs=fake)
+    assert _fwd_states(lib) == 1
+    assert _fwd_states(lib, **dict(ok, cs=fake + 4)) == 3                  # misaligned states
+    assert _fwd_states(lib, **ok) == 4                                     # no workspace (SIMT, any Q)
+    tc = dict(ok, dtype=1, H=2, P=64, N=128, G=1, L=512)
+    for path in (0, 2):                                                    # auto resolves to the tensor path
+        assert _fwd_states(lib, **tc, Q=64, path=path) == 2                # no 64-token boundary there
+        assert _fwd_states(lib, **tc, Q=128, path=path) == 4               # fine, then no workspace
+        assert _fwd_states(lib, **dict(tc, cs=None), Q=64, path=path) == 4  # no states: as the plain call
+    assert _fwd_states(lib, **tc, Q=64, path=1) == 4                       # SIMT takes it
+
+
 def test_step_rejects_bad_arguments_on_host(lib):
     fake = 0x10000
     f = lambda **kw: lib.ssd_step(*([kw.get("p", fake)] * 9), kw.get("b", 2), kw.get("H", 4), kw.get("P", 16),
