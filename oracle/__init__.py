@@ -5,6 +5,8 @@ benchmark's CPU-baseline leg, never by the CUDA path.  See ``ssd_oracle.py``.
 """
 from .ssd_oracle import (  # noqa: F401
     build_oracle,
+    conv1d_silu,
+    gated_rmsnorm,
     oracle_library_path,
     scan,
     scan_states,

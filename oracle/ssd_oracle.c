@@ -284,3 +284,60 @@ int ssd_oracle_step(const float *x, const float *dt_raw, const float *dt_bias,
     pthread_mutex_destroy(&J.lock);
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * The steps either side of the scan in a Mamba-2 layer (the nnterp guide's y
+ * is taken "before the gated norm and out_proj"; the state-spaces/mamba
+ * issue names causal_conv1d_fn applied before the chunk scan).  Readings
+ * where the pages give no numbers: the conv is causal and depthwise over the
+ * channels that become x, B and C, width K, with a bias and SiLU, starting
+ * from zeros; the gate is y * silu(z) and the norm an RMS norm over groups of
+ * `group` channels, times a per-channel weight.
+ *
+ * conv1d_silu:  in [b, L, Cd] (Cd channels), w [Cd, K], bias [Cd] ->
+ *   out[b,t,c] = silu(bias[c] + sum_{k<K} w[c,k] in[b, t-(K-1)+k, c]),
+ *   in[b, t<0, c] = 0.
+ * gated_rmsnorm: y, z [T, D], weight [D], groups of `group` channels ->
+ *   v = y * silu(z);  out = v / sqrt(mean_group(v^2) + eps) * weight.
+ * silu(u) = u / (1 + exp(-u)).
+ */
+static double silu_d(double u) { return u / (1.0 + exp(-u)); }
+
+int ssd_oracle_conv1d_silu(const float *in, const float *w, const float *bias, double *out,
+                           int64_t b, int64_t L, int64_t Cd, int64_t K)
+{
+    int64_t bi, t, c, k;
+    if (b < 0 || L < 0 || Cd <= 0 || K <= 0) return -1;
+    for (bi = 0; bi < b; ++bi)
+        for (t = 0; t < L; ++t)
+            for (c = 0; c < Cd; ++c) {
+                double acc = (double)bias[c];
+                for (k = 0; k < K; ++k) {
+                    const int64_t s = t - (K - 1) + k;
+                    if (s >= 0) acc += (double)w[c * K + k] * (double)in[(bi * L + s) * Cd + c];
+                }
+                out[(bi * L + t) * Cd + c] = silu_d(acc);
+            }
+    return 0;
+}
+
+int ssd_oracle_gated_rmsnorm(const float *y, const float *z, const float *weight, double *out,
+                             int64_t T, int64_t D, int64_t group, double eps)
+{
+    int64_t t, g0, j;
+    if (T < 0 || D <= 0 || group <= 0 || D % group != 0 || eps < 0) return -1;
+    for (t = 0; t < T; ++t)
+        for (g0 = 0; g0 < D; g0 += group) {
+            double ss = 0.0, r;
+            for (j = g0; j < g0 + group; ++j) {
+                const double v = (double)y[t * D + j] * silu_d((double)z[t * D + j]);
+                ss += v * v;
+            }
+            r = 1.0 / sqrt(ss / (double)group + eps);
+            for (j = g0; j < g0 + group; ++j) {
+                const double v = (double)y[t * D + j] * silu_d((double)z[t * D + j]);
+                out[t * D + j] = v * r * (double)weight[j];
+            }
+        }
+    return 0;
+}

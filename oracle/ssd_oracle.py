@@ -54,6 +54,10 @@ def _load():
         lib.ssd_oracle_scan_states.restype = ctypes.c_int
         lib.ssd_oracle_scan_states.argtypes = [f32p] * 8 + [f64p, f64p, f64p] + [i64] * 7 + [
             ctypes.c_double, ctypes.c_double, ctypes.c_int]
+        lib.ssd_oracle_conv1d_silu.restype = ctypes.c_int
+        lib.ssd_oracle_conv1d_silu.argtypes = [f32p] * 3 + [f64p] + [i64] * 4
+        lib.ssd_oracle_gated_rmsnorm.restype = ctypes.c_int
+        lib.ssd_oracle_gated_rmsnorm.argtypes = [f32p] * 3 + [f64p] + [i64] * 3 + [ctypes.c_double]
         lib.ssd_oracle_step.restype = ctypes.c_int
         lib.ssd_oracle_step.argtypes = [f32p] * 7 + [f64p, f64p] + [i64] * 5 + [
             ctypes.c_double, ctypes.c_double, ctypes.c_int]
@@ -151,6 +155,37 @@ def scan_states(x, dt_raw, dt_bias, A, B, C, D, chunk_size: int, init_state=None
     if rc != 0:
         raise RuntimeError("ssd_oracle_scan_states failed with code %d" % rc)
     return y, fs, states
+
+
+def conv1d_silu(xbc, weight, bias) -> np.ndarray:
+    """Causal depthwise conv of width K over channels, plus bias, then SiLU,
+    from zeros (the conv before the scan, read as in ssd_oracle.c).
+    xbc [b, L, Cd], weight [Cd, K], bias [Cd] -> [b, L, Cd] float64."""
+    xbc, weight, bias = _f32(xbc), _f32(weight), _f32(bias)
+    b, L, Cd = xbc.shape
+    if weight.ndim != 2 or weight.shape[0] != Cd or bias.shape != (Cd,):
+        raise ValueError("oracle.conv1d_silu: weight must be [Cd, K] and bias [Cd]")
+    out = np.empty((b, L, Cd), dtype=np.float64)
+    rc = _load().ssd_oracle_conv1d_silu(_p32(xbc), _p32(weight), _p32(bias), _p64(out), b, L, Cd,
+                                        weight.shape[1])
+    if rc != 0:
+        raise RuntimeError("ssd_oracle_conv1d_silu failed with code %d" % rc)
+    return out
+
+
+def gated_rmsnorm(y, z, weight, group: int, eps: float) -> np.ndarray:
+    """v = y * silu(z); out = v / sqrt(mean over each group of `group`
+    channels of v^2 + eps) * weight.  y, z [..., D], weight [D]."""
+    y, z, weight = _f32(y), _f32(z), _f32(weight)
+    D = y.shape[-1]
+    if z.shape != y.shape or weight.shape != (D,):
+        raise ValueError("oracle.gated_rmsnorm: z must match y and weight be [D]")
+    T = y.size // D
+    out = np.empty(y.shape, dtype=np.float64)
+    rc = _load().ssd_oracle_gated_rmsnorm(_p32(y), _p32(z), _p32(weight), _p64(out), T, D, int(group), float(eps))
+    if rc != 0:
+        raise RuntimeError("ssd_oracle_gated_rmsnorm failed with code %d" % rc)
+    return out
 
 
 def step(x, dt_raw, dt_bias, A, B, C, D, state: np.ndarray,
