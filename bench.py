@@ -81,8 +81,8 @@ def step_bytes(cfg) -> float:
 # sha256 at capture time: once that file changes the number no longer
 # describes the kernel and the bench reports null.
 NCU_TRAFFIC = {
-    ("c1_130m", "tc_chunk_out"): (35.405568e6, "state_space_sequence_scan_b200/csrc/ssd_scan_tc.cu",
-                                  "c17a52433f6b9010", "profiles/tc_chunk_out_c1_130m.md"),
+    ("c1_130m", "tc_chunk_out"): (35.664896e6, "state_space_sequence_scan_b200/csrc/ssd_scan_tc.cu",
+                                  "522d59fac3fd38eb", "profiles/tc_chunk_out_c1_130m.md"),
     ("c4_decode", "decode_step"): (1291.7568e6, "state_space_sequence_scan_b200/csrc/ssd_step.cu",
                                    "a5f3c2cec738b994", "profiles/decode_step_c4_decode.md"),
 }
@@ -412,6 +412,82 @@ def dominant(trace):
 
 
 # algorithmic bytes each traced kernel must move (per launch), as fractions of the call
+def bench_stage(cfg, args, local, peaks, peak_kind):
+    """--stage conv1d | gated_norm: one of the steps either side of the scan,
+    alone, on the workload's shapes (conv: x|B|C channels of width 4 from
+    bf16 inputs; norm: y f32 and z bf16 over groups of H*P/G channels).  HBM
+    bytes: conv reads xbc and writes x, B, C; the norm reads y and z and
+    writes out (weights are negligible).  Timed like the scan: inputs rotated
+    past L2, K steps in one CUDA graph, CUDA events on the launching stream."""
+    from state_space_sequence_scan_b200 import ssd
+    dev = torch.device("cuda", local)
+    b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
+    gen = torch.Generator().manual_seed(cfg.seed + 77)
+    if args.stage == "conv1d":
+        Cd, K = H * P + 2 * G * N, 4
+        one = 2.0 * b * L * Cd * 2
+        nsets = max(1, min(8, math.ceil(3 * L2_BYTES / one)))
+        w = (torch.randn(Cd, K, generator=gen) / 2).to(dev)
+        bias = (0.1 * torch.randn(Cd, generator=gen)).to(dev)
+        sets = [torch.randn(b, L, Cd, generator=gen).to(torch.bfloat16).to(dev) for _ in range(nsets)]
+        outs = [(torch.empty(b, L, H, P, dtype=torch.bfloat16, device=dev),
+                 torch.empty(b, L, G, N, dtype=torch.bfloat16, device=dev),
+                 torch.empty(b, L, G, N, dtype=torch.bfloat16, device=dev)) for _ in range(nsets)]
+        lib = ssd.load_library()
+
+        def step(k):
+            x, B, C = outs[k % nsets]
+            st = lib.ssd_conv1d_silu_split(sets[k % nsets].data_ptr(), w.data_ptr(), bias.data_ptr(), x.data_ptr(),
+                                           B.data_ptr(), C.data_ptr(), b, L, H, P, G, N, K, 1,
+                                           torch.cuda.current_stream(dev).cuda_stream)
+            if st != 0:
+                raise RuntimeError("ssd_conv1d_silu_split: %d" % st)
+        kname = "conv1d_silu"
+    else:
+        D, grp = H * P, H * P // G
+        one = float(b * L * D * (4 + 2 + 4))
+        nsets = max(1, min(8, math.ceil(3 * L2_BYTES / one)))
+        wt = (torch.rand(D, generator=gen) + 0.5).to(dev)
+        sets = [(torch.randn(b * L, D, generator=gen).to(dev),
+                 torch.randn(b * L, D, generator=gen).to(torch.bfloat16).to(dev)) for _ in range(nsets)]
+        outs = [torch.empty(b * L, D, device=dev) for _ in range(nsets)]
+        lib = ssd.load_library()
+
+        def step(k):
+            y, z = sets[k % nsets]
+            st = lib.ssd_gated_rmsnorm(y.data_ptr(), z.data_ptr(), wt.data_ptr(), outs[k % nsets].data_ptr(), b * L, D,
+                                       grp, 1e-5, 1, torch.cuda.current_stream(dev).cuda_stream)
+            if st != 0:
+                raise RuntimeError("ssd_gated_rmsnorm: %d" % st)
+        kname = "gated_rmsnorm"
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    graph = capture_steps(step, args.steps)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = one / (ms * 1e-3) / 1e9
+    return {"stage": args.stage, "metric": "%s HBM GB/s" % args.stage, "value": gbs, "unit": "GB/s",
+            "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16-in",
+            "config": {"workload": cfg.name, "batch": b, "seqlen": L, "heads": H, "head_dim": P, "groups": G,
+                       "state_dim": N, "l2": "rotating %d sets" % nsets},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "kernel_bytes": one, "traffic": None,
+                         "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind},
+            "clocks": clk}
+
+
 def kernel_bytes(cfg, name, states=False) -> float:
     b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
     e = 4 if cfg.dtype == "f32" else 2
@@ -553,6 +629,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--chunk-states", action="store_true",
                     help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
+    ap.add_argument("--stage", default="scan", choices=["scan", "conv1d", "gated_norm"],
+                    help="time one of the steps either side of the scan instead (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -567,6 +645,10 @@ def main():
         ssd.load_library()
         peaks, peak_kind = load_peaks()
         cfg, is_step = pick(args.workload)
+        if args.stage != "scan" and not is_step:
+            if rank == 0:
+                print(json.dumps(bench_stage(cfg, args, local, peaks, peak_kind)), flush=True)
+            return
         if is_step:
             r = bench_step(cfg, args, ws, rank, local)
         else:

@@ -181,6 +181,38 @@ SSD_API ssd_status ssd_chunk_scan_fwd_noalloc(const void *x, const float *dt_raw
                                       int64_t state_dim, int64_t ngroups, int64_t chunk_size,
                                       float dt_lo, float dt_hi, int in_dtype, int path, void *stream);
 
+/* The causal depthwise conv1d that runs before the scan in a Mamba-2 layer
+ * (state-spaces/mamba issue on the training and inference paths:
+ * causal_conv1d_fn, then the chunk scan), in the split arrangement: it
+ * writes the scan's x, B and C directly.  For every channel c of
+ *   xbc [batch, seqlen, Cd],  Cd = nheads*head_dim + 2*ngroups*state_dim
+ *   (channels in the order x | B | C, the same dtype as the outputs),
+ *   out[t, c] = silu(bias[c] + sum_{k<K} weight[c, k] * xbc[t - (K-1) + k, c]),
+ *   xbc[t < 0] = 0 (a fresh sequence),  silu(u) = u / (1 + exp(-u)),
+ * and out is split into x [batch, seqlen, nheads, head_dim] and
+ * B, C [batch, seqlen, ngroups, state_dim].
+ *   weight [Cd, K] and bias [Cd] float32; K = kernel_width, 1..4.
+ *   in_dtype  ssd_dtype of xbc, x, B, C.
+ * nheads*head_dim and ngroups*state_dim must be multiples of 8; xbc, x, B
+ * and C 16-byte aligned and not overlapping.  Queued on `stream`. */
+SSD_API ssd_status ssd_conv1d_silu_split(const void *xbc, const float *weight, const float *bias, void *x,
+                                 void *B, void *C, int64_t batch, int64_t seqlen, int64_t nheads,
+                                 int64_t head_dim, int64_t ngroups, int64_t state_dim,
+                                 int64_t kernel_width, int in_dtype, void *stream);
+
+/* The gated RMS norm that takes y after the scan (nnterp guide "Mamba-2",
+ * table "The values": y is taken before the gated norm and out_proj):
+ *   v = y * silu(z),  out = v / sqrt(mean_{group}(v^2) + eps) * weight
+ * over each group of group_size consecutive channels of a token.
+ *   y [tokens, dim] float32 (the scan's y viewed as [b*L, H*P]),
+ *   z [tokens, dim] of z_dtype, weight [dim] float32, out [tokens, dim]
+ *   float32.  dim a multiple of group_size, group_size a multiple of 4;
+ *   y, weight and out 16-byte aligned, z 8-byte aligned; eps >= 0.
+ * Queued on `stream`. */
+SSD_API ssd_status ssd_gated_rmsnorm(const float *y, const void *z, const float *weight, float *out,
+                             int64_t tokens, int64_t dim, int64_t group_size, float eps, int z_dtype,
+                             void *stream);
+
 /* Waits for `stream`, then reads the device status word that the last
  * ssd_chunk_scan_fwd on this workspace left: SSD_OK, SSD_ERR_PRECONDITION or
  * SSD_ERR_DEVICE_TIMEOUT.  `workspace` is a device pointer. */

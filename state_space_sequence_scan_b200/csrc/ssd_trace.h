@@ -14,7 +14,9 @@ enum TraceKernel {
     kTrTcStatePass = 5,
     kTrTcChunkOut = 6,
     kTrTcDtPrep = 7,
-    kKernelCount = 8,
+    kTrConv1d = 8,
+    kTrGatedNorm = 9,
+    kKernelCount = 10,
 };
 
 bool trace_on();

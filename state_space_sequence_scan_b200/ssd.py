@@ -29,7 +29,8 @@ PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 
 EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_states", "ssd_step",
             "ssd_read_device_status", "ssd_status_string", "ssd_last_cuda_error", "ssd_version",
-            "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count")
+            "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count",
+            "ssd_conv1d_silu_split", "ssd_gated_rmsnorm")
 
 _lib = None
 
@@ -76,6 +77,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_trace_kernel_name.argtypes = [i32]
     lib.ssd_trace_kernel_count.restype = i32
     lib.ssd_trace_kernel_count.argtypes = []
+    lib.ssd_conv1d_silu_split.restype = i32
+    lib.ssd_conv1d_silu_split.argtypes = [vp] * 6 + [i64] * 7 + [i32, vp]
+    lib.ssd_gated_rmsnorm.restype = i32
+    lib.ssd_gated_rmsnorm.argtypes = [vp] * 4 + [i64] * 3 + [f32, i32, vp]
     _lib = lib
     return lib
 
@@ -223,6 +228,50 @@ def chunk_scan_fwd_states(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check("ssd_chunk_scan_fwd_states", st)
     return y, final_state, chunk_states
+
+
+def conv1d_silu_split(xbc: torch.Tensor, weight: torch.Tensor, bias: torch.Tensor, nheads: int, head_dim: int,
+                      ngroups: int, state_dim: int) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Causal depthwise conv1d + SiLU over xbc [b, L, H*P + 2*G*N] (channels
+    x | B | C), split into the scan's x [b,L,H,P], B and C [b,L,G,N] (same
+    dtype as xbc).  weight [Cd, K] f32, bias [Cd] f32 (ssd_conv1d_silu_split)."""
+    lib = load_library()
+    if xbc.dim() != 3 or weight.dim() != 2:
+        raise ValueError("xbc must be [b, L, Cd] and weight [Cd, K]")
+    b, L, Cd = xbc.shape
+    if Cd != nheads * head_dim + 2 * ngroups * state_dim:
+        raise ValueError("xbc has %d channels, not H*P + 2*G*N" % Cd)
+    _need_cuda("xbc", xbc)
+    if xbc.dtype not in DTYPES:
+        raise ValueError("xbc must be float32 or bfloat16")
+    _need_cuda("weight", weight, torch.float32, (Cd, weight.shape[1]))
+    _need_cuda("bias", bias, torch.float32, (Cd,))
+    dev = xbc.device
+    x = torch.empty((b, L, nheads, head_dim), dtype=xbc.dtype, device=dev)
+    B = torch.empty((b, L, ngroups, state_dim), dtype=xbc.dtype, device=dev)
+    C = torch.empty_like(B)
+    st = lib.ssd_conv1d_silu_split(_ptr(xbc), _ptr(weight), _ptr(bias), _ptr(x), _ptr(B), _ptr(C), b, L, nheads,
+                                   head_dim, ngroups, state_dim, weight.shape[1], DTYPES[xbc.dtype], _stream(dev))
+    _check("ssd_conv1d_silu_split", st)
+    return x, B, C
+
+
+def gated_rmsnorm(y: torch.Tensor, z: torch.Tensor, weight: torch.Tensor, group_size: int,
+                  eps: float = 1e-5) -> torch.Tensor:
+    """out = rmsnorm_over_groups(y * silu(z)) * weight, f32 (ssd_gated_rmsnorm).
+    y f32 [..., D], z [..., D] f32 or bf16, weight [D] f32."""
+    lib = load_library()
+    D = y.shape[-1]
+    _need_cuda("y", y, torch.float32)
+    _need_cuda("z", z, None, tuple(y.shape))
+    if z.dtype not in DTYPES:
+        raise ValueError("z must be float32 or bfloat16")
+    _need_cuda("weight", weight, torch.float32, (D,))
+    out = torch.empty(y.shape, dtype=torch.float32, device=y.device)
+    st = lib.ssd_gated_rmsnorm(_ptr(y), _ptr(z), _ptr(weight), _ptr(out), y.numel() // D, D, int(group_size),
+                               float(eps), DTYPES[z.dtype], _stream(y.device))
+    _check("ssd_gated_rmsnorm", st)
+    return out
 
 
 def read_device_status(workspace: torch.Tensor) -> int:

@@ -125,6 +125,32 @@ def test_forward_states_rejects_bad_arguments_on_host(lib):
     assert _fwd_states(lib, **tc, Q=64, path=1) == 4                       # SIMT takes it
 
 
+def test_front_back_reject_bad_arguments_on_host(lib):
+    """The conv1d and gated-norm entry points check sizes, dtypes and
+    alignment before anything is queued."""
+    fake = 0x10000
+    conv = lambda **kw: lib.ssd_conv1d_silu_split(*([kw.get("p", fake)] * 3), *([kw.get("o", fake)] * 3),
+                                                  kw.get("b", 2), kw.get("L", 40), kw.get("H", 4), kw.get("P", 16),
+                                                  kw.get("G", 2), kw.get("N", 16), kw.get("K", 4),
+                                                  kw.get("dtype", 1), None)
+    assert conv(b=0) == 0 and conv(L=0) == 0          # nothing to do
+    assert conv(H=0) == 1
+    assert conv(K=5) == 2 and conv(K=0) == 2           # widths 1..4
+    assert conv(P=5) == 2                              # H*P = 20, not a multiple of 8
+    assert conv(dtype=7) == 2
+    assert conv(p=None) == 1
+    assert conv(o=fake + 8) == 3                       # misaligned outputs
+    norm = lambda **kw: lib.ssd_gated_rmsnorm(kw.get("y", fake), kw.get("z", fake), fake, kw.get("out", fake),
+                                              kw.get("T", 10), kw.get("D", 64), kw.get("g", 16), kw.get("eps", 1e-5),
+                                              kw.get("dtype", 1), None)
+    assert norm(T=0) == 0
+    assert norm(g=24) == 1                             # 64 % 24
+    assert norm(g=6, D=60) == 2                        # group not a multiple of 4
+    assert norm(eps=-1.0) == 1 and norm(eps=float("nan")) == 1
+    assert norm(y=None) == 1
+    assert norm(out=fake + 4) == 3 and norm(z=fake + 2) == 3
+
+
 def test_step_rejects_bad_arguments_on_host(lib):
     fake = 0x10000
     f = lambda **kw: lib.ssd_step(*([kw.get("p", fake)] * 9), kw.get("b", 2), kw.get("H", 4), kw.get("P", 16),
