@@ -10,6 +10,7 @@ from .ssd_oracle import (  # noqa: F401
     oracle_library_path,
     scan,
     scan_states,
+    scan_varlen,
     softplus,
     step,
 )

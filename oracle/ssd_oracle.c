@@ -21,6 +21,10 @@
  * The decode step (nnterp guide "Mamba-2", section "The state between
  * steps") is the same loop body for one token with the state updated in
  * place.
+ * Packed sequences (the "Mamba2" knowledge page notes sample packing for
+ * Mamba2): with seq_idx [b, L] given, a token whose seq_idx differs from the
+ * previous token's starts a new document, and the state is set to zero
+ * before its update; the first document of a row starts from init_state.
  * The chunk-boundary states (same guide, "The state after every token"):
  *   states[b, c, h] = S after token min((c+1) Q, L) - 1, for c < ceil(L / Q),
  *   so the last one is final_state and Q = 1 gives the state after every
@@ -66,6 +70,7 @@ typedef struct {
     const float *x, *dt_raw, *dt_bias, *A, *B, *C, *D, *init_state;
     double *y, *final_state;
     double *chunk_states;     /* [b, nc, H, N, P] or NULL */
+    const int32_t *seq_idx;   /* [b, L] or NULL: document ids of packed rows */
     int64_t b, L, H, P, N, G;
     int64_t Q, nc;            /* chunk size and count for chunk_states */
     double dt_lo, dt_hi;
@@ -100,6 +105,8 @@ static int run_chain(scan_job *J, int64_t bi, int64_t h, double *S, double *yacc
 
     for (t = 0; t < L; ++t) {
         const double z = (double)J->dt_raw[(bi * L + t) * H + h] + bias;
+        if (J->seq_idx && t > 0 && J->seq_idx[bi * L + t] != J->seq_idx[bi * L + t - 1])
+            memset(S, 0, sizeof(double) * (size_t)(N * P));      /* a new document */
         const double dt = clamp_dt(sp_exact(z), J->dt_lo, J->dt_hi);
         const double a = exp(dt * A);
         const float *xr = J->x + ((bi * L + t) * H + h) * P;
@@ -184,11 +191,12 @@ static int run_threads(void *(*fn)(void *), void *job, int nthreads)
 /* Whole-sequence recurrence, also recording the state after every chunk of Q
  * tokens into chunk_states when that is not NULL.  Returns 0, or -1 on bad
  * dimensions, -2 when out of memory.  nthreads <= 0 uses every online core. */
-int ssd_oracle_scan_states(const float *x, const float *dt_raw, const float *dt_bias,
+int ssd_oracle_scan_varlen(const float *x, const float *dt_raw, const float *dt_bias,
                            const float *A, const float *B, const float *C, const float *D,
-                           const float *init_state, double *y, double *final_state,
-                           double *chunk_states, int64_t b, int64_t L, int64_t H, int64_t P,
-                           int64_t N, int64_t G, int64_t Q, double dt_lo, double dt_hi, int nthreads)
+                           const float *init_state, const int32_t *seq_idx, double *y,
+                           double *final_state, double *chunk_states, int64_t b, int64_t L, int64_t H,
+                           int64_t P, int64_t N, int64_t G, int64_t Q, double dt_lo, double dt_hi,
+                           int nthreads)
 {
     scan_job J;
     if (b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0) return -1;
@@ -198,6 +206,7 @@ int ssd_oracle_scan_states(const float *x, const float *dt_raw, const float *dt_
     J.x = x; J.dt_raw = dt_raw; J.dt_bias = dt_bias; J.A = A; J.B = B; J.C = C; J.D = D;
     J.init_state = init_state; J.y = y; J.final_state = final_state;
     J.chunk_states = chunk_states;
+    J.seq_idx = seq_idx;
     J.Q = Q > 0 ? Q : 1;
     J.nc = (L + J.Q - 1) / J.Q;
     J.b = b; J.L = L; J.H = H; J.P = P; J.N = N; J.G = G;
@@ -206,6 +215,17 @@ int ssd_oracle_scan_states(const float *x, const float *dt_raw, const float *dt_
     run_threads(scan_worker, &J, pick_threads(nthreads, b * H));
     pthread_mutex_destroy(&J.lock);
     return J.status;
+}
+
+/* Whole-sequence recurrence with the chunk-boundary states, no packing. */
+int ssd_oracle_scan_states(const float *x, const float *dt_raw, const float *dt_bias,
+                           const float *A, const float *B, const float *C, const float *D,
+                           const float *init_state, double *y, double *final_state,
+                           double *chunk_states, int64_t b, int64_t L, int64_t H, int64_t P,
+                           int64_t N, int64_t G, int64_t Q, double dt_lo, double dt_hi, int nthreads)
+{
+    return ssd_oracle_scan_varlen(x, dt_raw, dt_bias, A, B, C, D, init_state, NULL, y, final_state,
+                                  chunk_states, b, L, H, P, N, G, Q, dt_lo, dt_hi, nthreads);
 }
 
 /* Whole-sequence recurrence: y and final_state only. */

@@ -54,6 +54,10 @@ def _load():
         lib.ssd_oracle_scan_states.restype = ctypes.c_int
         lib.ssd_oracle_scan_states.argtypes = [f32p] * 8 + [f64p, f64p, f64p] + [i64] * 7 + [
             ctypes.c_double, ctypes.c_double, ctypes.c_int]
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.ssd_oracle_scan_varlen.restype = ctypes.c_int
+        lib.ssd_oracle_scan_varlen.argtypes = [f32p] * 8 + [i32p, f64p, f64p, f64p] + [i64] * 7 + [
+            ctypes.c_double, ctypes.c_double, ctypes.c_int]
         lib.ssd_oracle_conv1d_silu.restype = ctypes.c_int
         lib.ssd_oracle_conv1d_silu.argtypes = [f32p] * 3 + [f64p] + [i64] * 4
         lib.ssd_oracle_gated_rmsnorm.restype = ctypes.c_int
@@ -154,6 +158,39 @@ def scan_states(x, dt_raw, dt_bias, A, B, C, D, chunk_size: int, init_state=None
         float(dt_limit[0]), float(dt_limit[1]), int(nthreads))
     if rc != 0:
         raise RuntimeError("ssd_oracle_scan_states failed with code %d" % rc)
+    return y, fs, states
+
+
+def scan_varlen(x, dt_raw, dt_bias, A, B, C, D, seq_idx, chunk_size: int = 1, init_state=None,
+                dt_limit: Tuple[float, float] = (0.0, float("inf")),
+                nthreads: int = 0) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Packed rows: seq_idx [b, L] int32 document ids; the state is zeroed
+    before the first token of every document but a row's first (which starts
+    from init_state).  Returns (y, final_state, chunk states) as scan_states."""
+    x, dt_raw, dt_bias, A, B, C, D = (_f32(v) for v in (x, dt_raw, dt_bias, A, B, C, D))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    Q = int(chunk_size)
+    si = np.ascontiguousarray(np.asarray(seq_idx, dtype=np.int32))
+    if si.shape != (b, L):
+        raise ValueError("oracle.scan_varlen: seq_idx must be [b, L]")
+    if Q < 1 or dt_raw.shape != (b, L, H) or B.shape != (b, L, G, N) or C.shape != B.shape:
+        raise ValueError("oracle.scan_varlen: inconsistent shapes")
+    s0 = None
+    if init_state is not None:
+        s0 = _f32(init_state)
+    nc = (L + Q - 1) // Q
+    y = np.empty((b, L, H, P), dtype=np.float64)
+    fs = np.empty((b, H, N, P), dtype=np.float64)
+    states = np.empty((b, nc, H, N, P), dtype=np.float64)
+    rc = _load().ssd_oracle_scan_varlen(
+        _p32(x), _p32(dt_raw), _p32(dt_bias), _p32(A), _p32(B), _p32(C), _p32(D),
+        _p32(s0) if s0 is not None else ctypes.POINTER(ctypes.c_float)(),
+        si.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+        _p64(y), _p64(fs), _p64(states), b, L, H, P, N, G, Q,
+        float(dt_limit[0]), float(dt_limit[1]), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("ssd_oracle_scan_varlen failed with code %d" % rc)
     return y, fs, states
 
 

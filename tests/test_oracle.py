@@ -429,3 +429,55 @@ def test_bad_shapes_raise():
     odd = _rand_case(19, H=3, G=2)
     with pytest.raises(ValueError):
         oracle.scan(**odd)
+
+
+def _docs(rng, L, min_len=1, max_len=9):
+    """Random document lengths covering L (some of length 1)."""
+    lens = []
+    while sum(lens) < L:
+        lens.append(int(rng.integers(min_len, max_len + 1)))
+    lens[-1] -= sum(lens) - L
+    if lens[-1] == 0:
+        lens.pop()
+    return lens
+
+
+@pytest.mark.parametrize("seed", [60, 61])
+def test_packed_row_equals_separate_documents(seed):
+    """Packing (the "Mamba2" knowledge page: sample packing for Mamba2): a row
+    of documents gives, token for token, what each document gives alone from
+    a zero state (the first from init_state), and its final state is the last
+    document's.  Exactly: the reset writes the same zeros a fresh run starts
+    from."""
+    rng = np.random.default_rng(seed)
+    case = _rand_case(seed, b=2, L=31, H=4, P=3, N=2, G=2, init=True)
+    b, L = 2, 31
+    seq = np.zeros((b, L), np.int32)
+    bounds = []
+    for bi in range(b):
+        lens = _docs(rng, L)
+        pos = 0
+        for d, ln in enumerate(lens):
+            seq[bi, pos:pos + ln] = 10 * d + bi                # ids need only differ from the neighbour's
+            pos += ln
+        bounds.append(lens)
+    y, fs, st = oracle.scan_varlen(seq_idx=seq, chunk_size=4, **case)
+    for bi in range(b):
+        pos = 0
+        for d, ln in enumerate(bounds[bi]):
+            one = {k: (v[bi:bi + 1, pos:pos + ln] if k in ("x", "dt_raw", "B", "C") else v)
+                   for k, v in case.items()}
+            one["init_state"] = case["init_state"][bi:bi + 1] if d == 0 else None
+            yd, fd = oracle.scan(**one)
+            assert np.array_equal(y[bi:bi + 1, pos:pos + ln], yd)
+            pos += ln
+        assert np.array_equal(fs[bi:bi + 1], fd)
+    assert np.array_equal(st[:, -1], fs)
+
+
+def test_one_document_is_the_plain_scan():
+    case = _rand_case(62, b=2, L=19, init=True)
+    seq = np.full((2, 19), 7, np.int32)
+    y, fs, st = oracle.scan_varlen(seq_idx=seq, chunk_size=5, **case)
+    y0, fs0, st0 = oracle.scan_states(chunk_size=5, **case)
+    assert np.array_equal(y, y0) and np.array_equal(fs, fs0) and np.array_equal(st, st0)
