@@ -222,13 +222,26 @@ def bench_scan(cfg, args, ws, rank, local):
     nc = math.ceil(L / Q)
     outs = [(torch.empty(b, L, H, P, device=dev), torch.empty(b, H, N, P, device=dev),
              torch.empty(b, nc, H, N, P, device=dev) if args.chunk_states else None) for _ in range(nsets)]
-    wsz = ssd.workspace_size(b, L, H, P, N, G, Q, sets[0]["x"].dtype, args.path)
+    wsz = ssd.workspace_size(b, L, H, P, N, G, Q, sets[0]["x"].dtype, "simt" if args.packed else args.path)
     work = ssd.alloc_workspace(wsz, dev)
+    seqs = None
+    if args.packed:
+        # documents of about 512 tokens (seeded lengths), the same ids for every set
+        import numpy as np
+        rng = np.random.default_rng(cfg.seed + 5)
+        ids = np.zeros((b, L), np.int32)
+        for bi in range(b):
+            cuts = np.sort(rng.integers(1, L, size=max(1, L // 512)))
+            ids[bi] = np.searchsorted(cuts, np.arange(L), side="right")
+        seqs = torch.from_numpy(ids).to(dev)
 
     def step(k):
         s = sets[k % nsets]
         y, fs, cs = outs[k % nsets]
-        if cs is None:
+        if seqs is not None:
+            ssd.chunk_scan_fwd_varlen(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"], seqs,
+                                      init_state=s["init_state"], chunk_size=Q, workspace=work)
+        elif cs is None:
             ssd.chunk_scan_fwd(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"],
                                init_state=s["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
                                final_state=fs)
@@ -597,7 +610,7 @@ def pick(name):
     raise SystemExit("unknown workload %s (scan: %s; decode: %s)" % (name, list(SCAN_CONFIGS), list(STEP_CONFIGS)))
 
 
-def workload_config(cfg, is_step, nsets=None, states=False):
+def workload_config(cfg, is_step, nsets=None, states=False, packed=False):
     if is_step:
         c = {"workload": cfg.name, "batch": cfg.batch, "heads": cfg.nheads, "head_dim": cfg.head_dim,
              "state_dim": cfg.state_dim, "groups": cfg.ngroups, "state_dtype": "f32", "in_dtype": cfg.dtype,
@@ -614,6 +627,8 @@ def workload_config(cfg, is_step, nsets=None, states=False):
                        if nsets > 1 else "inputs %.0f MB > L2" % (one / 1e6))
         if states:
             c["chunk_states"] = "[b, %d, H, N, P] f32 written every step" % math.ceil(cfg.seqlen / cfg.chunk_size)
+        if packed:
+            c["packed"] = "documents of about 512 tokens per row (seq_idx), SIMT path; e2e leg unpacked"
     return c
 
 
@@ -629,6 +644,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--chunk-states", action="store_true",
                     help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
+    ap.add_argument("--packed", action="store_true",
+                    help="rows packed with documents of about 512 tokens (seq_idx; the SIMT path)")
     ap.add_argument("--stage", default="scan", choices=["scan", "conv1d", "gated_norm"],
                     help="time one of the steps either side of the scan instead (one GPU)")
     args = ap.parse_args()
@@ -707,7 +724,8 @@ def finish(cfg, is_step, r, args, ws, rank, peaks, peak_kind, sub=False):
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": dtype, "data": "synthetic (seeded; shapes/distributions of the workload)",
-            "config": workload_config(cfg, is_step, r.get("nsets"), (not is_step) and args.chunk_states),
+            "config": workload_config(cfg, is_step, r.get("nsets"), (not is_step) and args.chunk_states,
+                                      (not is_step) and args.packed),
             "roofline": roof, "clocks": r["clocks"],
             "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": r["e2e"]["h2d"],
                     "d2h_bytes_per_step": r["e2e"]["d2h"]},

@@ -181,6 +181,29 @@ SSD_API ssd_status ssd_chunk_scan_fwd_noalloc(const void *x, const float *dt_raw
                                       int64_t state_dim, int64_t ngroups, int64_t chunk_size,
                                       float dt_lo, float dt_hi, int in_dtype, int path, void *stream);
 
+/* ssd_chunk_scan_fwd_states over packed rows (the "Mamba2" knowledge page:
+ * sample packing for Mamba2).
+ *   seq_idx  [batch, seqlen] int32, 4-byte aligned: a document id per token.
+ *            A token whose id differs from the previous token's starts a new
+ *            document: the state is zero before its update, so no token
+ *            reads across a document start.  The first document of a row
+ *            starts from init_state (NULL: zeros).  final_state is the state
+ *            after the row's last token (its last document's) and
+ *            chunk_states (may be NULL) as for ssd_chunk_scan_fwd_states.
+ *            NULL makes the call ssd_chunk_scan_fwd_states.
+ * With seq_idx, the scan runs on the SIMT path: SSD_PATH_AUTO resolves to
+ * it (size the workspace with ssd_chunk_scan_workspace_size(...,
+ * SSD_PATH_SIMT, ...)) and SSD_PATH_TENSOR returns SSD_ERR_UNSUPPORTED
+ * before anything is enqueued.  Every other argument as for
+ * ssd_chunk_scan_fwd_states. */
+SSD_API ssd_status ssd_chunk_scan_fwd_varlen(const void *x, const float *dt_raw, const float *dt_bias,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const float *init_state, const int32_t *seq_idx, float *y,
+                                     float *final_state, float *chunk_states, int64_t batch, int64_t seqlen,
+                                     int64_t nheads, int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                                     int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype, int path,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
 /* The causal depthwise conv1d that runs before the scan in a Mamba-2 layer
  * (state-spaces/mamba issue on the training and inference paths:
  * causal_conv1d_fn, then the chunk scan), in the split arrangement: it

@@ -118,12 +118,12 @@ ssd_status ssd_chunk_scan_workspace_size(int64_t batch, int64_t seqlen, int64_t 
 
 namespace {
 
-// The forward scan, with or without the chunk-boundary states.
+// The forward scan, with or without the chunk-boundary states and packed rows.
 ssd_status scan_fwd(const void *x, const float *dt_raw, const float *dt_bias, const float *A, const void *B,
-                    const void *C, const float *D, const float *init_state, float *y, float *final_state,
-                    float *chunk_states, int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
-                    int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi,
-                    int in_dtype, int path, void *workspace, size_t workspace_bytes, void *stream) {
+                    const void *C, const float *D, const float *init_state, const int32_t *seq_idx, float *y,
+                    float *final_state, float *chunk_states, int64_t batch, int64_t seqlen, int64_t nheads,
+                    int64_t head_dim, int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo,
+                    float dt_hi, int in_dtype, int path, void *workspace, size_t workspace_bytes, void *stream) {
     ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size,
                                     in_dtype, path);
     if (st != SSD_OK) return st;
@@ -136,8 +136,11 @@ ssd_status scan_fwd(const void *x, const float *dt_raw, const float *dt_bias, co
         (chunk_states && !aligned16(chunk_states)))
         return SSD_ERR_ALIGNMENT;
     const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
+    // packed rows run on the SIMT path only
+    if (seq_idx && path == SSD_PATH_TENSOR) return SSD_ERR_UNSUPPORTED;
+    if (seq_idx && (reinterpret_cast<uintptr_t>(seq_idx) & 3u)) return SSD_ERR_ALIGNMENT;
     int chosen = 0;
-    if ((st = resolve_path(d, in_dtype, path, &chosen)) != SSD_OK) return st;
+    if ((st = resolve_path(d, in_dtype, seq_idx ? SSD_PATH_SIMT : path, &chosen)) != SSD_OK) return st;
     // the tensor path has the state at its 128-token block ends only
     if (chunk_states && chosen == SSD_PATH_TENSOR && chunk_size % 128 != 0) return SSD_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < path_ws(d, chosen)) return SSD_ERR_WORKSPACE;
@@ -161,6 +164,7 @@ ssd_status scan_fwd(const void *x, const float *dt_raw, const float *dt_bias, co
     ssd::ScanArgs a;
     a.x = x; a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.B = B; a.C = C; a.D = D;
     a.init_state = init_state; a.y = y; a.final_state = final_state; a.chunk_states = chunk_states;
+    a.seq_idx = seq_idx;
     a.dt_lo = dt_lo; a.dt_hi = dt_hi; a.bf16 = in_dtype == SSD_BF16;
     e = chosen == SSD_PATH_TENSOR ? ssd::tc_scan(a, d, workspace, s) : ssd::simt_scan(a, d, workspace, s);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -176,8 +180,8 @@ ssd_status ssd_chunk_scan_fwd(const void *x, const float *dt_raw, const float *d
                               int64_t state_dim, int64_t ngroups, int64_t chunk_size,
                               float dt_lo, float dt_hi, int in_dtype, int path,
                               void *workspace, size_t workspace_bytes, void *stream) {
-    return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, nullptr, batch, seqlen, nheads,
-                    head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
+    return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, nullptr, y, final_state, nullptr, batch, seqlen,
+                    nheads, head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
                     workspace_bytes, stream);
 }
 
@@ -188,8 +192,20 @@ ssd_status ssd_chunk_scan_fwd_states(const void *x, const float *dt_raw, const f
                                      int64_t head_dim, int64_t state_dim, int64_t ngroups,
                                      int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype, int path,
                                      void *workspace, size_t workspace_bytes, void *stream) {
-    return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, y, final_state, chunk_states, batch, seqlen,
-                    nheads, head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
+    return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, nullptr, y, final_state, chunk_states, batch,
+                    seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
+                    workspace_bytes, stream);
+}
+
+ssd_status ssd_chunk_scan_fwd_varlen(const void *x, const float *dt_raw, const float *dt_bias,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const float *init_state, const int32_t *seq_idx, float *y,
+                                     float *final_state, float *chunk_states, int64_t batch, int64_t seqlen,
+                                     int64_t nheads, int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                                     int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype, int path,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, seq_idx, y, final_state, chunk_states, batch,
+                    seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
                     workspace_bytes, stream);
 }
 

@@ -19,6 +19,7 @@ struct ScanArgs {
     const float *D, *init_state;
     float *y, *final_state;
     float *chunk_states = nullptr;  // [b, nc, H, N, P] or null: the state after every chunk
+    const int32_t *seq_idx = nullptr;  // [b, L] document ids of packed rows, or null (SIMT path)
     float dt_lo, dt_hi;
     int bf16;                      // 1: x/B/C are bfloat16, 0: float32
 };

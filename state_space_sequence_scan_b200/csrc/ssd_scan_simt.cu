@@ -19,6 +19,13 @@
 // Every exponent is taken on min(cum_i - cum_j, 0) after the j <= i select,
 // so no exp() can overflow (the NaN class reported for an SM90 chunk-scan
 // kernel on the "Mamba2" knowledge page).
+//
+// Packed rows (seq_idx given): doc_i counts the document starts (a token
+// whose id differs from the previous token's) from the chunk's first token
+// through i, a block sum-scan of 0/1 flags.  A pair (j, i) contributes only
+// when doc_j == doc_i, the entering state only when doc_i == 0, the chunk
+// state only its last document's tokens, and a chunk holding a start passes
+// no decayed state on (log decay -inf).
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
 #include "ssd_trace.h"
@@ -53,16 +60,22 @@ SimtWs carve(const ScanDims &d, void *ws) {
     return w;
 }
 
+// 1 when token t of row b starts a document of a packed row
+__device__ __forceinline__ float doc_start(const int32_t *seq_idx, size_t b, int L, int t) {
+    return (t > 0 && seq_idx[b * L + t] != seq_idx[b * L + t - 1]) ? 1.f : 0.f;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 chunk_state_kernel(const T *__restrict__ x, const float *__restrict__ dt_raw,
                    const float *__restrict__ dt_bias, const float *__restrict__ A,
-                   const T *__restrict__ Bm, SimtWs ws, int L, int H, int P, int N, int G,
-                   int Q, int nc, float lo, float hi) {
+                   const T *__restrict__ Bm, const int32_t *__restrict__ seq_idx, SimtWs ws, int L, int H,
+                   int P, int N, int G, int Q, int nc, float lo, float hi) {
     extern __shared__ float sm[];
     float *s_dt = sm;                 // Q
     float *s_cum = s_dt + Q;          // Q
-    float *s_B = s_cum + Q;           // kTK * N
+    float *s_doc = s_cum + Q;         // Q (packed rows only)
+    float *s_B = s_doc + Q;           // kTK * N
     float *s_X = s_B + kTK * N;       // kTK * P
     __shared__ float wtot[32];
 
@@ -74,7 +87,7 @@ chunk_state_kernel(const T *__restrict__ x, const float *__restrict__ dt_raw,
     const size_t bh = (size_t)b * H + h;
     if (threadIdx.x == 0 && Ah > 0.f) flag_status(ws.status, kStatusPrecondition);
 
-    float carry = 0.f;
+    float carry = 0.f, dcarry = 0.f;
     for (int base = 0; base < q; base += kThreads) {
         const int i = base + threadIdx.x;
         float d = 0.f, da = 0.f;
@@ -91,10 +104,18 @@ chunk_state_kernel(const T *__restrict__ x, const float *__restrict__ dt_raw,
             ws.cum[bh * L + t0 + i] = s;
         }
         carry += tot;
+        if (seq_idx) {                                // uniform over the block
+            float dtot;
+            const float dc = block_inclusive_scan(i < q ? doc_start(seq_idx, b, L, t0 + i) : 0.f, wtot, dtot);
+            if (i < q) s_doc[i] = dc + dcarry;
+            dcarry += dtot;
+        }
     }
     __syncthreads();
     const float clast = s_cum[q - 1];
-    if (threadIdx.x == 0) ws.ell[bh * nc + c] = clast;
+    const float dlast = seq_idx ? s_doc[q - 1] : 0.f;
+    // a chunk that holds a document start passes no decayed state on
+    if (threadIdx.x == 0) ws.ell[bh * nc + c] = dlast > 0.f ? -INFINITY : clast;
 
     // S[n, p] = sum_k w_k B[k, n] x[k, p]; thread owns column p, rows n0 + RN*r.
     const int p = threadIdx.x % P, n0 = threadIdx.x / P, RN = kThreads / P;
@@ -112,7 +133,9 @@ chunk_state_kernel(const T *__restrict__ x, const float *__restrict__ dt_raw,
         }
         for (int e = threadIdx.x; e < kk * P; e += kThreads) {
             const int k = e / P, pp = e - k * P;
-            const float w = expf(fminf(clast - s_cum[k0 + k], 0.f)) * s_dt[k0 + k];
+            // only the chunk's last document writes into the state it passes on
+            const bool live = !seq_idx || s_doc[k0 + k] == dlast;
+            const float w = live ? expf(fminf(clast - s_cum[k0 + k], 0.f)) * s_dt[k0 + k] : 0.f;
             s_X[k * P + pp] = w * to_f(x[(((size_t)b * L + t0 + k0 + k) * H + h) * P + pp]);
         }
         __syncthreads();
@@ -159,11 +182,13 @@ state_pass_kernel(SimtWs ws, const float *__restrict__ init, float *__restrict__
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 chunk_out_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restrict__ Cm,
-                 const float *__restrict__ D, SimtWs ws, float *__restrict__ y, int L, int H,
-                 int P, int N, int G, int Q, int nc, int TI) {
+                 const float *__restrict__ D, const int32_t *__restrict__ seq_idx, SimtWs ws,
+                 float *__restrict__ y, int L, int H, int P, int N, int G, int Q, int nc, int TI) {
     extern __shared__ float sm[];
+    __shared__ float wtot[32];
     const int NB = N + 1;                       // padded B row
-    float *s_C = sm;                            // TI * N
+    float *s_doc = sm;                          // Q (packed rows only)
+    float *s_C = s_doc + Q;                     // TI * N
     float *s_cumi = s_C + TI * N;               // TI
     float *s_Bj = s_cumi + TI;                  // kTJ * NB
     float *s_xj = s_Bj + kTJ * NB;              // kTJ * P
@@ -189,6 +214,20 @@ chunk_out_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__r
 #pragma unroll
     for (int r = 0; r < kMaxAcc; ++r) acc[r] = 0.f;
 
+    // document counters of the chunk's tokens through the tile's last row
+    const int jend = i0 + ti;
+    if (seq_idx) {                              // uniform over the block
+        float dcarry = 0.f;
+        for (int base = 0; base < jend; base += kThreads) {
+            const int i = base + threadIdx.x;
+            float dtot;
+            const float dc = block_inclusive_scan(i < jend ? doc_start(seq_idx, b, L, t0 + i) : 0.f, wtot, dtot);
+            if (i < jend) s_doc[i] = dc + dcarry;
+            dcarry += dtot;
+        }
+        __syncthreads();
+    }
+
     for (int e = threadIdx.x; e < TI * N; e += kThreads) {
         const int ii = e / N, n = e - ii * N;
         s_C[e] = ii < ti ? to_f(Cm[(((size_t)b * L + t0 + i0 + ii) * G + g) * N + n]) : 0.f;
@@ -212,12 +251,15 @@ chunk_out_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__r
             }
         }
     }
+    // the entering state reaches row i only if no document starts in the chunk up to i
 #pragma unroll
-    for (int r = 0; r < kMaxAcc; ++r)
-        if (r < nacc && ib + r * RI < TI) acc[r] *= expf(fminf(s_cumi[ib + r * RI], 0.f));
+    for (int r = 0; r < kMaxAcc; ++r) {
+        const int ii = ib + r * RI;
+        if (r < nacc && ii < TI)
+            acc[r] *= (!seq_idx || ii >= ti || s_doc[i0 + ii] == 0.f) ? expf(fminf(s_cumi[ii], 0.f)) : 0.f;
+    }
 
     // intra-chunk part: j from the chunk start through the tile's last row
-    const int jend = i0 + ti;
     for (int j0 = 0; j0 < jend; j0 += kTJ) {
         const int tj = min(kTJ, jend - j0);
         __syncthreads();
@@ -238,7 +280,8 @@ chunk_out_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__r
             const int ii = e / kTJ, jj = e - ii * kTJ;
             const int gi = i0 + ii, gj = j0 + jj;
             float v = 0.f;
-            if (ii < ti && jj < tj && gj <= gi) {          // causal select before any exp()
+            // causal select (and, on packed rows, same document) before any exp()
+            if (ii < ti && jj < tj && gj <= gi && (!seq_idx || s_doc[gj] == s_doc[gi])) {
                 const float *cr = s_C + ii * N;
                 const float *br = s_Bj + jj * NB;
                 float dot = 0.f;
@@ -277,11 +320,11 @@ int pick_ti(const ScanDims &d) {
 }
 
 size_t state_smem(const ScanDims &d) {
-    return sizeof(float) * (2 * (size_t)d.Q + (size_t)kTK * d.N + (size_t)kTK * d.P);
+    return sizeof(float) * (3 * (size_t)d.Q + (size_t)kTK * d.N + (size_t)kTK * d.P);
 }
 
 size_t out_smem(const ScanDims &d, int TI) {
-    return sizeof(float) * ((size_t)TI * d.N + TI + (size_t)kTJ * (d.N + 1) + (size_t)kTJ * d.P +
+    return sizeof(float) * ((size_t)d.Q + (size_t)TI * d.N + TI + (size_t)kTJ * (d.N + 1) + (size_t)kTJ * d.P +
                             2 * kTJ + (size_t)TI * (kTJ + 1) + (size_t)kTKH * d.P);
 }
 
@@ -301,8 +344,8 @@ cudaError_t run(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s)
     {
         TraceScope tr(s, kTrSimtChunkState);
         chunk_state_kernel<T><<<g1, kThreads, sm1, s>>>(
-            (const T *)a.x, a.dt_raw, a.dt_bias, a.A, (const T *)a.B, ws, (int)d.L, (int)d.H, (int)d.P,
-            (int)d.N, (int)d.G, (int)d.Q, (int)d.nc, a.dt_lo, a.dt_hi);
+            (const T *)a.x, a.dt_raw, a.dt_bias, a.A, (const T *)a.B, a.seq_idx, ws, (int)d.L, (int)d.H,
+            (int)d.P, (int)d.N, (int)d.G, (int)d.Q, (int)d.nc, a.dt_lo, a.dt_hi);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int NP = (int)(d.N * d.P);
@@ -318,8 +361,8 @@ cudaError_t run(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s)
     {
         TraceScope tr(s, kTrSimtChunkOut);
         chunk_out_kernel<T><<<g3, kThreads, sm3, s>>>(
-            (const T *)a.x, (const T *)a.B, (const T *)a.C, a.D, ws, a.y, (int)d.L, (int)d.H, (int)d.P,
-            (int)d.N, (int)d.G, (int)d.Q, (int)d.nc, TI);
+            (const T *)a.x, (const T *)a.B, (const T *)a.C, a.D, a.seq_idx, ws, a.y, (int)d.L, (int)d.H,
+            (int)d.P, (int)d.N, (int)d.G, (int)d.Q, (int)d.nc, TI);
     }
     return cudaGetLastError();
 }

@@ -30,7 +30,7 @@ PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_states", "ssd_step",
             "ssd_read_device_status", "ssd_status_string", "ssd_last_cuda_error", "ssd_version",
             "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count",
-            "ssd_conv1d_silu_split", "ssd_gated_rmsnorm")
+            "ssd_conv1d_silu_split", "ssd_gated_rmsnorm", "ssd_chunk_scan_fwd_varlen")
 
 _lib = None
 
@@ -57,6 +57,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_chunk_scan_workspace_size.argtypes = [i64] * 7 + [i32, i32, ctypes.POINTER(sz)]
     lib.ssd_chunk_scan_fwd.restype = i32
     lib.ssd_chunk_scan_fwd.argtypes = [vp] * 10 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
+    lib.ssd_chunk_scan_fwd_varlen.restype = i32
+    lib.ssd_chunk_scan_fwd_varlen.argtypes = [vp] * 12 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
     lib.ssd_chunk_scan_fwd_states.restype = i32
     lib.ssd_chunk_scan_fwd_states.argtypes = [vp] * 11 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
     lib.ssd_step.restype = i32
@@ -228,6 +230,48 @@ def chunk_scan_fwd_states(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check("ssd_chunk_scan_fwd_states", st)
     return y, final_state, chunk_states
+
+
+def chunk_scan_fwd_varlen(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor, A: torch.Tensor,
+                          B: torch.Tensor, C: torch.Tensor, D: torch.Tensor, seq_idx: torch.Tensor,
+                          init_state: Optional[torch.Tensor] = None, chunk_size: int = 256,
+                          dt_limit: Tuple[float, float] = (0.0, math.inf),
+                          workspace: Optional[torch.Tensor] = None, want_chunk_states: bool = False
+                          ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """Packed rows (ssd_chunk_scan_fwd_varlen): seq_idx [b, L] int32 document
+    ids; the state restarts from zero at every document start (a row's first
+    document from init_state).  Runs on the SIMT path.  Returns (y, final
+    state, chunk-boundary states or None)."""
+    lib = load_library()
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    _need_cuda("x", x)
+    if x.dtype not in DTYPES:
+        raise ValueError("x/B/C must be float32 or bfloat16")
+    _need_cuda("B", B, x.dtype, (b, L, G, N))
+    _need_cuda("C", C, x.dtype, (b, L, G, N))
+    _need_cuda("dt_raw", dt_raw, torch.float32, (b, L, H))
+    _need_cuda("seq_idx", seq_idx, torch.int32, (b, L))
+    for nm, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need_cuda(nm, t, torch.float32, (H,))
+    if init_state is not None:
+        _need_cuda("init_state", init_state, torch.float32, (b, H, N, P))
+    Q = int(chunk_size)
+    y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
+    fs = torch.empty((b, H, N, P), dtype=torch.float32, device=dev)
+    cs = torch.empty((b, (L + Q - 1) // Q, H, N, P), dtype=torch.float32, device=dev) if want_chunk_states else None
+    need = workspace_size(b, L, H, P, N, G, Q, x.dtype, "simt")
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    st = lib.ssd_chunk_scan_fwd_varlen(
+        _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(seq_idx),
+        _ptr(y), _ptr(fs), _ptr(cs), b, L, H, P, N, G, Q, float(dt_limit[0]), float(dt_limit[1]),
+        DTYPES[x.dtype], PATHS["auto"], _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _check("ssd_chunk_scan_fwd_varlen", st)
+    return y, fs, cs
 
 
 def conv1d_silu_split(xbc: torch.Tensor, weight: torch.Tensor, bias: torch.Tensor, nheads: int, head_dim: int,
