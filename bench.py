@@ -222,7 +222,7 @@ def bench_scan(cfg, args, ws, rank, local):
     nc = math.ceil(L / Q)
     outs = [(torch.empty(b, L, H, P, device=dev), torch.empty(b, H, N, P, device=dev),
              torch.empty(b, nc, H, N, P, device=dev) if args.chunk_states else None) for _ in range(nsets)]
-    wsz = ssd.workspace_size(b, L, H, P, N, G, Q, sets[0]["x"].dtype, "simt" if args.packed else args.path)
+    wsz = ssd.workspace_size(b, L, H, P, N, G, Q, sets[0]["x"].dtype, args.path)
     work = ssd.alloc_workspace(wsz, dev)
     seqs = None
     if args.packed:
@@ -240,7 +240,7 @@ def bench_scan(cfg, args, ws, rank, local):
         y, fs, cs = outs[k % nsets]
         if seqs is not None:
             ssd.chunk_scan_fwd_varlen(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"], seqs,
-                                      init_state=s["init_state"], chunk_size=Q, workspace=work)
+                                      init_state=s["init_state"], chunk_size=Q, path=args.path, workspace=work)
         elif cs is None:
             ssd.chunk_scan_fwd(s["x"], s["dt_raw"], s["dt_bias"], s["A"], s["B"], s["C"], s["D"],
                                init_state=s["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
@@ -628,7 +628,7 @@ def workload_config(cfg, is_step, nsets=None, states=False, packed=False):
         if states:
             c["chunk_states"] = "[b, %d, H, N, P] f32 written every step" % math.ceil(cfg.seqlen / cfg.chunk_size)
         if packed:
-            c["packed"] = "documents of about 512 tokens per row (seq_idx), SIMT path; e2e leg unpacked"
+            c["packed"] = "documents of about 512 tokens per row (seq_idx); e2e leg unpacked"
     return c
 
 
@@ -645,7 +645,7 @@ def main():
     ap.add_argument("--chunk-states", action="store_true",
                     help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
     ap.add_argument("--packed", action="store_true",
-                    help="rows packed with documents of about 512 tokens (seq_idx; the SIMT path)")
+                    help="rows packed with documents of about 512 tokens (seq_idx)")
     ap.add_argument("--stage", default="scan", choices=["scan", "conv1d", "gated_norm"],
                     help="time one of the steps either side of the scan instead (one GPU)")
     args = ap.parse_args()

@@ -191,10 +191,8 @@ SSD_API ssd_status ssd_chunk_scan_fwd_noalloc(const void *x, const float *dt_raw
  *            after the row's last token (its last document's) and
  *            chunk_states (may be NULL) as for ssd_chunk_scan_fwd_states.
  *            NULL makes the call ssd_chunk_scan_fwd_states.
- * With seq_idx, the scan runs on the SIMT path: SSD_PATH_AUTO resolves to
- * it (size the workspace with ssd_chunk_scan_workspace_size(...,
- * SSD_PATH_SIMT, ...)) and SSD_PATH_TENSOR returns SSD_ERR_UNSUPPORTED
- * before anything is enqueued.  Every other argument as for
+ * Both paths take packed rows and resolve as for ssd_chunk_scan_fwd (the
+ * workspace is sized the same way).  Every other argument as for
  * ssd_chunk_scan_fwd_states. */
 SSD_API ssd_status ssd_chunk_scan_fwd_varlen(const void *x, const float *dt_raw, const float *dt_bias,
                                      const float *A, const void *B, const void *C, const float *D,

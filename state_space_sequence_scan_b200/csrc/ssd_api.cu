@@ -136,11 +136,9 @@ ssd_status scan_fwd(const void *x, const float *dt_raw, const float *dt_bias, co
         (chunk_states && !aligned16(chunk_states)))
         return SSD_ERR_ALIGNMENT;
     const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
-    // packed rows run on the SIMT path only
-    if (seq_idx && path == SSD_PATH_TENSOR) return SSD_ERR_UNSUPPORTED;
     if (seq_idx && (reinterpret_cast<uintptr_t>(seq_idx) & 3u)) return SSD_ERR_ALIGNMENT;
     int chosen = 0;
-    if ((st = resolve_path(d, in_dtype, seq_idx ? SSD_PATH_SIMT : path, &chosen)) != SSD_OK) return st;
+    if ((st = resolve_path(d, in_dtype, path, &chosen)) != SSD_OK) return st;
     // the tensor path has the state at its 128-token block ends only
     if (chunk_states && chosen == SSD_PATH_TENSOR && chunk_size % 128 != 0) return SSD_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < path_ws(d, chosen)) return SSD_ERR_WORKSPACE;

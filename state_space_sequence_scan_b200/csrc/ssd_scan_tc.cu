@@ -81,6 +81,8 @@ struct TcWs {
     float *states;   // [b, H, U, N, P]
     __half *Bh;      // [b, nblk*128, G, N]  fp16 copy of B, zero rows past L
     __half *Ch;      // [b, nblk*128, G, N]  fp16 copy of C
+    int *rs;         // [b, nblk*128] packed rows: the last document start at or before
+                     // each token within its 128-token block (block offset), -1 if none
 };
 
 struct TcPlan {
@@ -140,14 +142,16 @@ TcWs carve(const ScanDims &d, const TcPlan &p, void *ws) {
     w.ell = reinterpret_cast<float *>(c + off); off += align256((size_t)d.b * d.H * p.U * sizeof(float));
     w.states = reinterpret_cast<float *>(c + off); off += align256((size_t)d.b * d.H * p.U * kNP * sizeof(float));
     w.Bh = reinterpret_cast<__half *>(c + off); off += align256(bc_bytes(d, p));
-    w.Ch = reinterpret_cast<__half *>(c + off);
+    w.Ch = reinterpret_cast<__half *>(c + off); off += align256(bc_bytes(d, p));
+    w.rs = reinterpret_cast<int *>(c + off);
     return w;
 }
 
 size_t ws_bytes(const ScanDims &d, const TcPlan &p) {
     const size_t tok = (size_t)d.b * d.H * p.nblk * kBlk * sizeof(float);
     return kStatusBytes + 2 * align256(tok) + align256((size_t)d.b * d.H * p.U * sizeof(float)) +
-           align256((size_t)d.b * d.H * p.U * kNP * sizeof(float)) + 2 * align256(bc_bytes(d, p));
+           align256((size_t)d.b * d.H * p.U * kNP * sizeof(float)) + 2 * align256(bc_bytes(d, p)) +
+           align256((size_t)d.b * p.nblk * kBlk * sizeof(int));
 }
 
 // Tensor maps (4-D, innermost first) with 128-token boxes: x bf16 [b,L,H,P]
@@ -214,8 +218,8 @@ constexpr int kPrepHeads = 8;
 
 __global__ void __launch_bounds__(256)
 prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias, const float *__restrict__ A,
-            const __nv_bfloat16 *__restrict__ Bm, const __nv_bfloat16 *__restrict__ Cm, TcWs ws, int L, int H,
-            int G, int nblk, float lo, float hi) {
+            const __nv_bfloat16 *__restrict__ Bm, const __nv_bfloat16 *__restrict__ Cm,
+            const int32_t *__restrict__ seq_idx, TcWs ws, int L, int H, int G, int nblk, float lo, float hi) {
     __shared__ float s_dt[kPrepHeads][kBlk + 4];
     __shared__ float s_da[kPrepHeads][kBlk + 4];
     pdl_launch_dependents();                     // the next kernel waits for this one's writes itself
@@ -292,6 +296,28 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
         *reinterpret_cast<float4 *>(ws.cum + base) = make_float4(ex + c0, ex + c1, ex + c2, ex + c3);
         *reinterpret_cast<float4 *>(ws.dt + base) = *reinterpret_cast<const float4 *>(&s_dt[warp][4 * lane]);
     }
+    // packed rows: the first head slice also records, for each token of the
+    // block, the last document start at or before it (an inclusive max-scan
+    // of the start positions; a start is a token whose id differs from the
+    // previous token's, tokens past L start nothing)
+    if (seq_idx && blockIdx.y == 0) {
+        __shared__ int s_wmax[4];
+        const int t = blk * kBlk + threadIdx.x;
+        int v = -1;
+        if (threadIdx.x < kBlk && t > 0 && t < L && seq_idx[(size_t)b * L + t] != seq_idx[(size_t)b * L + t - 1])
+            v = threadIdx.x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v = max(v, u);
+        }
+        if (lane == 31 && warp < 4) s_wmax[warp] = v;
+        __syncthreads();
+        if (threadIdx.x < kBlk) {
+            for (int w2 = 0; w2 < warp; ++w2) v = max(v, s_wmax[w2]);
+            ws.rs[(size_t)b * nblk * kBlk + (size_t)blk * kBlk + threadIdx.x] = v;
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -308,7 +334,8 @@ constexpr uint32_t kUsOffBar = kUsOffW + 2 * kBlk * 4;         // tma[2], mma[2]
 constexpr size_t kUsSmem = 1024 + kUsOffBar + 6 * 8 + 16;
 
 __global__ void __launch_bounds__(kUsThreads, 2)
-unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, int nblk, int U, int bpu) {
+unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, int nblk, int U, int bpu,
+                  int packed) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     // per stage: [0,1] TMA landed, [2,3] MMAs done, [4,5] X converted.  One barrier of
@@ -381,11 +408,21 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
         // ------------------------------ compute warps -------------------------
         __half2 amax = __float2half2_rn(0.f);
         bool ok = true;
-        // the unit's log decay after the current block (sum of later block totals)
+        // the unit's log decay after the current block (sum of later block totals);
+        // packed rows: how many later blocks of the unit hold a document start
+        const int *rsb = ws.rs + (size_t)b * nblk * kBlk;
         float suffix = 0.f;
+        int later = 0;
         if (tid < kBlk)
-            for (int k = kb0 + 1; k < kb1; ++k) suffix += cumg[(size_t)k * kBlk + kBlk - 1];
-        if (tid == 0) ws.ell[bh * U + u] = suffix + cumg[(size_t)kb0 * kBlk + kBlk - 1];
+            for (int k = kb0 + 1; k < kb1; ++k) {
+                suffix += cumg[(size_t)k * kBlk + kBlk - 1];
+                if (packed) later += rsb[(size_t)k * kBlk + kBlk - 1] >= 0;
+            }
+        if (tid == 0) {
+            const bool starts = packed && (later > 0 || rsb[(size_t)kb0 * kBlk + kBlk - 1] >= 0);
+            // a unit that holds a document start passes no decayed state on
+            ws.ell[bh * U + u] = starts ? -INFINITY : suffix + cumg[(size_t)kb0 * kBlk + kBlk - 1];
+        }
         for (int i = 0; i < nk; ++i) {
             const int s = i & 1;
             uint8_t *st = stage(s);
@@ -393,8 +430,15 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
             const float *cum = dt + kBlk;
             float *w = reinterpret_cast<float *>(sm + kUsOffW) + s * kBlk;
             ok = ok && mbar_wait_abortable(bar + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
-            if (ok && tid < kBlk) w[tid] = expf(fminf(cum[kBlk - 1] - cum[tid] + suffix, 0.f)) * dt[tid];
-            if (tid < kBlk && kb0 + i + 1 < kb1) suffix -= cumg[(size_t)(kb0 + i + 1) * kBlk + kBlk - 1];
+            if (ok && tid < kBlk) {
+                // packed rows: only the unit's last document writes into its state
+                const bool cut = packed && (later > 0 || tid < rsb[(size_t)(kb0 + i) * kBlk + kBlk - 1]);
+                w[tid] = cut ? 0.f : expf(fminf(cum[kBlk - 1] - cum[tid] + suffix, 0.f)) * dt[tid];
+            }
+            if (tid < kBlk && kb0 + i + 1 < kb1) {
+                suffix -= cumg[(size_t)(kb0 + i + 1) * kBlk + kBlk - 1];
+                if (packed) later -= rsb[(size_t)(kb0 + i + 1) * kBlk + kBlk - 1] >= 0;
+            }
             named_bar_sync(kUsCompute);                 // w[] visible
             if (ok) {
                 uint8_t *sx = st + 2 * kTileBytes;      // X (bf16) -> w.X (fp16); row = offset / 128
@@ -646,14 +690,15 @@ __device__ __forceinline__ void co_widen_x(const CoSmem &S, int r, int tid) {
 // chunk's row is its offset / 128 whatever the swizzle).  Packed fp16
 // products: w_j is rounded to fp16 once (w_j <= dt_j; one below the fp16
 // normal range only adds an absolute error under 3e-8 |x|), and no element
-// goes through fp32.
-__device__ __forceinline__ void co_form_wx(const CoSmem &S, int r, int f, int tid) {
+// goes through fp32.  Packed rows: tokens before the block's last document
+// start (rs_last; -1 for none) write nothing into the state the block passes on.
+__device__ __forceinline__ void co_form_wx(const CoSmem &S, int r, int f, int tid, int rs_last) {
     const float *w = S.F(f);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int c = tid + q * kCoCompute;
         const uint4 xv = *reinterpret_cast<const uint4 *>(S.X(r) + c * 16);
-        const __half2 wj = __float2half2_rn(w[c >> 3]);
+        const __half2 wj = __float2half2_rn((c >> 3) >= rs_last ? w[c >> 3] : 0.f);
         const uint32_t xi[4] = {xv.x, xv.y, xv.z, xv.w};
         uint32_t o[4];
 #pragma unroll
@@ -697,8 +742,10 @@ __device__ __forceinline__ void co_nonfinite(const float *v, int n, float2 &acc)
 }
 
 // W for one 32-column slice cq <= lg of this thread's row i (see co_factors).
+// Packed rows: rs_i is the last document start at or before row i in the
+// block (-1 for none); columns before it drop out of the row.
 __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32_t lane_addr, int lg, int cq,
-                                           int lane, float ci) {
+                                           int lane, float ci, int rs_i) {
     const float *cum = S.cum(r);
     const float *F = S.F(f);
     float v[32];
@@ -756,9 +803,18 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
             }
         }
     }
+    const int j0 = 32 * cq;
+    if (rs_i > j0) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            o[q] &= (j0 + 2 * q >= rs_i ? 0x0000FFFFu : 0u) | (j0 + 2 * q + 1 >= rs_i ? 0xFFFF0000u : 0u);
+    }
     tmem_st16u(lane_addr + kTmW + 16 * cq, o);
 }
 
+// kPacked: packed rows (the document starts of ws.rs mask W, the C.H term,
+// w.X and the block decay); the unpacked instantiation carries none of it.
+template <bool kPacked>
 __global__ void __launch_bounds__(kCoThreads, 1)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
                  const float *__restrict__ init, float *__restrict__ final_state, TcWs ws,
@@ -962,7 +1018,9 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         named_bar_sync(kCoCompute);                 // factors and masks visible to every compute warp
         if (ok) co_widen_x(S, 0, tid);
         named_bar_sync(kCoCompute);
-        if (ok) co_form_wx(S, 0, 0, tid);
+        // packed rows: document starts of each block (ws.rs, written by prep)
+        const int *rsb = ws.rs + (size_t)b * nblk * kBlk;
+        if (ok) co_form_wx(S, 0, 0, tid, kPacked ? rsb[(size_t)kb0 * kBlk + kBlk - 1] : -1);
         co_arrive(S.bar(kBarH16), lane);
 
         // every compute warp runs every iteration (and so every named barrier);
@@ -973,6 +1031,9 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             const uint32_t par = (uint32_t)i & 1u;
             const int t0 = k * kBlk;
             const float *cum = S.cum(r);
+            const int rs_row = kPacked ? rsb[(size_t)t0 + row] : -1;
+            const int rs_last = kPacked ? rsb[(size_t)t0 + kBlk - 1] : -1;
+            const int rs_last1 = (kPacked && k + 1 < kb1) ? rsb[(size_t)t0 + 2 * kBlk - 1] : -1;
 
             // [1] C.B^T(k) done -> W(k) (fp16 pairs) into TMEM
             ok = ok && mbar_wait_abortable(S.bar(kBarCB), par, kWaitBudget, abort_flag);
@@ -980,8 +1041,8 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             tc_fence_after();
             if (ok) {
                 const float ci = cum[row];
-                if (ch <= lg) co_w_slice(S, r, f, lane_addr, lg, ch, lane, ci);
-                if (ch + 2 <= lg) co_w_slice(S, r, f, lane_addr, lg, ch + 2, lane, ci);
+                if (ch <= lg) co_w_slice(S, r, f, lane_addr, lg, ch, lane, ci, rs_row);
+                if (ch + 2 <= lg) co_w_slice(S, r, f, lane_addr, lg, ch + 2, lane, ci, rs_row);
             }
             co_arrive_tmem(S.bar(kBarW), lane);
 
@@ -1002,7 +1063,8 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             if (ok) {
                 float sv[32];
                 tmem_ld32(lane_addr + kTmS + ch * 32, sv);
-                const float a = expf(fminf(cum[min(kBlk - 1, L - 1 - t0)], 0.f));
+                // a block that holds a document start passes no decayed state on
+                const float a = rs_last >= 0 ? 0.f : expf(fminf(cum[min(kBlk - 1, L - 1 - t0)], 0.f));
                 const float2 a2 = make_float2(a, a);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
@@ -1021,7 +1083,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                             *reinterpret_cast<uint4 *>(S.H16() + sw128_off(row, 4 * ch + 2 * hh + q)) =
                                 make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
                     }
-                    co_form_wx(S, r1, f1, tid);
+                    co_form_wx(S, r1, f1, tid, rs_last1);
                 } else if (final_state && u == U - 1) {
                     float *dst = final_state + bh * kNP + (size_t)row * kP + ch * 32;
 #pragma unroll
@@ -1047,7 +1109,8 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
             if (ok) {
-                const float ei = expf(fminf(cum[row], 0.f));
+                // the entering state reaches a row only before the block's first document start
+                const float ei = rs_row >= 0 ? 0.f : expf(fminf(cum[row], 0.f));
                 const float2 e2 = make_float2(ei, ei), d2 = make_float2(Dh, Dh);
                 uint8_t *stg = S.B(i & 1) + ch * kTileBytes;
 #pragma unroll
@@ -1122,7 +1185,10 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         if ((e = cudaFuncSetAttribute(unit_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kUsSmem)) != cudaSuccess)
             return e;
-        if ((e = cudaFuncSetAttribute(chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(chunk_out_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kCoSmem)) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(chunk_out_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kCoSmem)) != cudaSuccess)
             return e;
         attr_done = true;
@@ -1133,7 +1199,7 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         const unsigned ny = (unsigned)((d.H + kPrepHeads - 1) / kPrepHeads + 4 * d.G);
         prep_kernel<<<dim3((unsigned)p.nblk, ny, (unsigned)d.b), 256, 0, s>>>(
             a.dt_raw, a.dt_bias, a.A, static_cast<const __nv_bfloat16 *>(a.B), static_cast<const __nv_bfloat16 *>(a.C),
-            ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, a.dt_lo, a.dt_hi);
+            a.seq_idx, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, a.dt_lo, a.dt_hi);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // the kernels after prep may start their prologue while their predecessor
@@ -1156,7 +1222,7 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
             TraceScope tr(s, kTrTcUnitState);
             const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kUsThreads, kUsSmem);
             if ((e = cudaLaunchKernelEx(&c, unit_state_kernel, maps, ws, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U,
-                                        (int)p.bpu)) != cudaSuccess)
+                                        (int)p.bpu, a.seq_idx ? 1 : 0)) != cudaSuccess)
                 return e;
         }
         {
@@ -1175,9 +1241,10 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem);
         // the caller checked that chunk_states come with chunk_size a multiple of kBlk
         const int bpc = (int)(d.Q / kBlk) > 0 ? (int)(d.Q / kBlk) : 1;
-        if ((e = cudaLaunchKernelEx(&c, chunk_out_kernel, maps, a.D, a.init_state, a.final_state, ws, (int)d.L,
-                                    (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0,
-                                    prefetch_cb, a.chunk_states, bpc, (int)d.nc)) != cudaSuccess)
+        if ((e = cudaLaunchKernelEx(&c, a.seq_idx ? chunk_out_kernel<true> : chunk_out_kernel<false>, maps, a.D,
+                                    a.init_state, a.final_state, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk,
+                                    (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0, prefetch_cb, a.chunk_states, bpc,
+                                    (int)d.nc)) != cudaSuccess)
             return e;
     }
     return cudaGetLastError();

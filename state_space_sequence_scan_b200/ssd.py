@@ -235,13 +235,14 @@ def chunk_scan_fwd_states(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.
 def chunk_scan_fwd_varlen(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor, A: torch.Tensor,
                           B: torch.Tensor, C: torch.Tensor, D: torch.Tensor, seq_idx: torch.Tensor,
                           init_state: Optional[torch.Tensor] = None, chunk_size: int = 256,
-                          dt_limit: Tuple[float, float] = (0.0, math.inf),
+                          dt_limit: Tuple[float, float] = (0.0, math.inf), path: str = "auto",
                           workspace: Optional[torch.Tensor] = None, want_chunk_states: bool = False
                           ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     """Packed rows (ssd_chunk_scan_fwd_varlen): seq_idx [b, L] int32 document
     ids; the state restarts from zero at every document start (a row's first
-    document from init_state).  Runs on the SIMT path.  Returns (y, final
-    state, chunk-boundary states or None)."""
+    document from init_state).  Returns (y, final state, chunk-boundary
+    states or None); with the states, path="auto" and a chunk size that is
+    not a multiple of 128 runs on the SIMT path."""
     lib = load_library()
     if x.dim() != 4 or B.dim() != 4:
         raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
@@ -263,13 +264,15 @@ def chunk_scan_fwd_varlen(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.
     y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
     fs = torch.empty((b, H, N, P), dtype=torch.float32, device=dev)
     cs = torch.empty((b, (L + Q - 1) // Q, H, N, P), dtype=torch.float32, device=dev) if want_chunk_states else None
-    need = workspace_size(b, L, H, P, N, G, Q, x.dtype, "simt")
+    if want_chunk_states and path == "auto" and Q % 128 != 0:
+        path = "simt"
+    need = workspace_size(b, L, H, P, N, G, Q, x.dtype, path)
     if workspace is None:
         workspace = alloc_workspace(need, dev)
     st = lib.ssd_chunk_scan_fwd_varlen(
         _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(seq_idx),
         _ptr(y), _ptr(fs), _ptr(cs), b, L, H, P, N, G, Q, float(dt_limit[0]), float(dt_limit[1]),
-        DTYPES[x.dtype], PATHS["auto"], _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+        DTYPES[x.dtype], PATHS[path], _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check("ssd_chunk_scan_fwd_varlen", st)
     return y, fs, cs
 

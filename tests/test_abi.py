@@ -126,16 +126,15 @@ def test_forward_states_rejects_bad_arguments_on_host(lib):
 
 
 def test_forward_varlen_rejects_bad_arguments_on_host(lib):
-    """Packed rows: refused on the tensor path, seq_idx 4-byte aligned, and
-    auto resolves to SIMT (then no workspace here)."""
+    """Packed rows: seq_idx 4-byte aligned; both paths take them (then no
+    workspace here)."""
     fake = 0x10000
     f = lambda **kw: lib.ssd_chunk_scan_fwd_varlen(
         *([fake] * 8), kw.get("si", fake), fake, fake, None, 1, 512, 2, 64, 128, 1, kw.get("Q", 128), 0.0, math.inf,
         1, kw.get("path", 0), None, 0, None)
-    assert f(path=2) == 2                              # the tensor path takes no seq_idx
     assert f(si=fake + 2) == 3                         # misaligned ids
-    assert f() == 4 and f(Q=64) == 4                   # auto -> SIMT, then no workspace
-    assert f(path=1) == 4
+    for path in (0, 1, 2):
+        assert f(path=path) == 4 and f(Q=64, path=path) == 4
 
 
 def test_front_back_reject_bad_arguments_on_host(lib):
