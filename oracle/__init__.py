@@ -9,6 +9,7 @@ from .ssd_oracle import (  # noqa: F401
     gated_rmsnorm,
     oracle_library_path,
     scan,
+    scan_bwd,
     scan_states,
     scan_varlen,
     softplus,

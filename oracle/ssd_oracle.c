@@ -361,3 +361,195 @@ int ssd_oracle_gated_rmsnorm(const float *y, const float *z, const float *weight
         }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Backward of the scan: reverse mode of the token-by-token recurrence.  The
+ * pages say only that the backward pass of the usual mamba kernels is not
+ * deterministic (HF transformers issue "mamba2 mixer different outputs",
+ * reply on the backward pass); the gradients themselves are the plain
+ * derivatives of the recurrence above.  For an upstream gradient dy of y and
+ * dfinal of final_state, with G = dLoss/dS_t running backwards from
+ * G = dfinal (zeros when NULL):
+ *   G      += C_t dy_t^T                        (y_t reads S_t)
+ *   dC_t    = S_t dy_t
+ *   dx_t    = dt_t G^T B_t + D dy_t
+ *   dB_t    = dt_t G x_t
+ *   ddt_t   = B_t^T G x_t + A a_t <G, S_{t-1}>  (a_t = exp(dt_t A))
+ *   dA     += dt_t a_t <G, S_{t-1}>,   dD += dy_t . x_t
+ *   dz_t    = ddt_t softplus'(z_t) [dt_lo <= softplus(z_t) <= dt_hi]
+ *   G       = a_t G                             (S_t = a_t S_{t-1} + ...)
+ * and dinit = G after token 0.  dz_t is the gradient of dt_raw[t] and, summed
+ * over tokens, of dt_bias.  Per head: dB_h/dC_h [b,L,H,N] (the caller sums the
+ * heads of each group), dA_h/ddt_bias_h/dD_h [b,H] (the caller sums over b).
+ * The states S_t are recomputed forward from checkpoints every kSeg tokens,
+ * which changes no arithmetic (the same products in the same order).
+ */
+#define kSeg 64
+
+typedef struct {
+    const float *x, *dt_raw, *dt_bias, *A, *B, *C, *D, *init_state, *dy, *dfinal;
+    double *dx, *ddt_raw, *dB_h, *dC_h, *dA_h, *ddt_bias_h, *dD_h, *dinit;
+    int64_t b, L, H, P, N, G;
+    double dt_lo, dt_hi;
+    int64_t next;
+    pthread_mutex_t lock;
+    int status;
+} bwd_job;
+
+static double sigmoid_exact(double z)
+{
+    /* d softplus / dz, in a form that never overflows */
+    return z >= 0.0 ? 1.0 / (1.0 + exp(-z)) : exp(z) / (1.0 + exp(z));
+}
+
+/* forward update of S by token t of chain (bi, h) */
+static void fwd_token(const bwd_job *J, int64_t bi, int64_t h, int64_t t, double *S, double *dt_out,
+                      double *a_out)
+{
+    const int64_t L = J->L, H = J->H, P = J->P, N = J->N, G = J->G, g = h / (H / G);
+    const double z = (double)J->dt_raw[(bi * L + t) * H + h] + (double)J->dt_bias[h];
+    const double dt = clamp_dt(sp_exact(z), J->dt_lo, J->dt_hi);
+    const double a = exp(dt * (double)J->A[h]);
+    const float *xr = J->x + ((bi * L + t) * H + h) * P;
+    const float *Br = J->B + ((bi * L + t) * G + g) * N;
+    int64_t n, p;
+    for (n = 0; n < N; ++n) {
+        const double w = dt * (double)Br[n];
+        for (p = 0; p < P; ++p) S[n * P + p] = a * S[n * P + p] + w * (double)xr[p];
+    }
+    *dt_out = dt;
+    *a_out = a;
+}
+
+static void bwd_chain(bwd_job *J, int64_t bi, int64_t h, double *ck, double *seg, double *Gm)
+{
+    const int64_t L = J->L, H = J->H, P = J->P, N = J->N, G = J->G, g = h / (H / G);
+    const int64_t NP = N * P, nseg = (L + kSeg - 1) / kSeg;
+    const double A = J->A[h], Dh = J->D[h];
+    double dA = 0.0, dbias = 0.0, dD = 0.0, dt, a;
+    int64_t s, t, n, p, i;
+
+    /* checkpoints: ck[s] = the state before token s*kSeg */
+    if (J->init_state) {
+        for (i = 0; i < NP; ++i) ck[i] = (double)J->init_state[(bi * H + h) * NP + i];
+    } else {
+        memset(ck, 0, sizeof(double) * (size_t)NP);
+    }
+    for (s = 0; s + 1 < nseg; ++s) {
+        memcpy(ck + (s + 1) * NP, ck + s * NP, sizeof(double) * (size_t)NP);
+        for (t = s * kSeg; t < (s + 1) * kSeg; ++t) fwd_token(J, bi, h, t, ck + (s + 1) * NP, &dt, &a);
+    }
+
+    if (J->dfinal) {
+        for (i = 0; i < NP; ++i) Gm[i] = (double)J->dfinal[(bi * H + h) * NP + i];
+    } else {
+        memset(Gm, 0, sizeof(double) * (size_t)NP);
+    }
+    for (s = nseg - 1; s >= 0; --s) {
+        const int64_t t0 = s * kSeg, t1 = (t0 + kSeg < L) ? t0 + kSeg : L;
+        /* seg[k] = S after token t0 + k - 1 (seg[0] = the checkpoint) */
+        double dts[kSeg], as[kSeg];
+        memcpy(seg, ck + s * NP, sizeof(double) * (size_t)NP);
+        for (t = t0; t < t1; ++t) {
+            memcpy(seg + (t - t0 + 1) * NP, seg + (t - t0) * NP, sizeof(double) * (size_t)NP);
+            fwd_token(J, bi, h, t, seg + (t - t0 + 1) * NP, &dts[t - t0], &as[t - t0]);
+        }
+        for (t = t1 - 1; t >= t0; --t) {
+            const double *Scur = seg + (t - t0 + 1) * NP, *Sprev = seg + (t - t0) * NP;
+            const double dtt = dts[t - t0], at = as[t - t0];
+            const float *xr = J->x + ((bi * L + t) * H + h) * P;
+            const float *Br = J->B + ((bi * L + t) * G + g) * N;
+            const float *Cr = J->C + ((bi * L + t) * G + g) * N;
+            const float *dyr = J->dy + ((bi * L + t) * H + h) * P;
+            double *dxr = J->dx + ((bi * L + t) * H + h) * P;
+            double *dBr = J->dB_h + ((bi * L + t) * H + h) * N;
+            double *dCr = J->dC_h + ((bi * L + t) * H + h) * N;
+            const double z = (double)J->dt_raw[(bi * L + t) * H + h] + (double)J->dt_bias[h];
+            const double sp = sp_exact(z);
+            double bgx = 0.0, gs = 0.0, dz;
+
+            for (n = 0; n < N; ++n)
+                for (p = 0; p < P; ++p) Gm[n * P + p] += (double)Cr[n] * (double)dyr[p];
+            for (n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (p = 0; p < P; ++p) acc += Scur[n * P + p] * (double)dyr[p];
+                dCr[n] = acc;
+            }
+            for (p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (n = 0; n < N; ++n) acc += Gm[n * P + p] * (double)Br[n];
+                dxr[p] = dtt * acc + Dh * (double)dyr[p];
+            }
+            for (n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (p = 0; p < P; ++p) acc += Gm[n * P + p] * (double)xr[p];
+                dBr[n] = dtt * acc;
+                bgx += (double)Br[n] * acc;
+            }
+            for (i = 0; i < NP; ++i) gs += Gm[i] * Sprev[i];
+            for (p = 0; p < P; ++p) dD += (double)dyr[p] * (double)xr[p];
+            dA += dtt * at * gs;
+            dz = (bgx + A * at * gs) * ((sp >= J->dt_lo && sp <= J->dt_hi) ? sigmoid_exact(z) : 0.0);
+            J->ddt_raw[(bi * L + t) * H + h] = dz;
+            dbias += dz;
+            for (i = 0; i < NP; ++i) Gm[i] *= at;
+        }
+    }
+    memcpy(J->dinit + (bi * H + h) * NP, Gm, sizeof(double) * (size_t)NP);
+    J->dA_h[bi * H + h] = dA;
+    J->ddt_bias_h[bi * H + h] = dbias;
+    J->dD_h[bi * H + h] = dD;
+}
+
+static void *bwd_worker(void *arg)
+{
+    bwd_job *J = (bwd_job *)arg;
+    const int64_t NP = J->N * J->P, nseg = (J->L + kSeg - 1) / kSeg;
+    double *ck = (double *)malloc(sizeof(double) * (size_t)(NP * (nseg > 0 ? nseg : 1)));
+    double *seg = (double *)malloc(sizeof(double) * (size_t)(NP * (kSeg + 1)));
+    double *Gm = (double *)malloc(sizeof(double) * (size_t)NP);
+    int64_t c;
+    if (!ck || !seg || !Gm) {
+        J->status = -2;
+    } else {
+        for (;;) {
+            pthread_mutex_lock(&J->lock);
+            c = J->next++;
+            pthread_mutex_unlock(&J->lock);
+            if (c >= J->b * J->H) break;
+            bwd_chain(J, c / J->H, c % J->H, ck, seg, Gm);
+        }
+    }
+    free(ck);
+    free(seg);
+    free(Gm);
+    return NULL;
+}
+
+/* Gradients of <dy, y> + <dfinal, final_state> for the whole-sequence scan
+ * (no packing).  dy [b,L,H,P] and dfinal [b,H,N,P] (may be NULL) are float32
+ * as given to the GPU; outputs are double: dx [b,L,H,P], ddt_raw [b,L,H],
+ * dB_h, dC_h [b,L,H,N] (per head), dA_h, ddt_bias_h, dD_h [b,H] (per chain),
+ * dinit [b,H,N,P].  Returns 0, -1 on bad dimensions, -2 when out of memory. */
+int ssd_oracle_scan_bwd(const float *x, const float *dt_raw, const float *dt_bias, const float *A,
+                        const float *B, const float *C, const float *D, const float *init_state,
+                        const float *dy, const float *dfinal, double *dx, double *ddt_raw, double *dB_h,
+                        double *dC_h, double *dA_h, double *ddt_bias_h, double *dD_h, double *dinit,
+                        int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, double dt_lo,
+                        double dt_hi, int nthreads)
+{
+    bwd_job J;
+    if (b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0) return -1;
+    if (b == 0) return 0;
+    memset(&J, 0, sizeof J);
+    J.x = x; J.dt_raw = dt_raw; J.dt_bias = dt_bias; J.A = A; J.B = B; J.C = C; J.D = D;
+    J.init_state = init_state; J.dy = dy; J.dfinal = dfinal;
+    J.dx = dx; J.ddt_raw = ddt_raw; J.dB_h = dB_h; J.dC_h = dC_h;
+    J.dA_h = dA_h; J.ddt_bias_h = ddt_bias_h; J.dD_h = dD_h; J.dinit = dinit;
+    J.b = b; J.L = L; J.H = H; J.P = P; J.N = N; J.G = G;
+    J.dt_lo = dt_lo; J.dt_hi = dt_hi;
+    pthread_mutex_init(&J.lock, NULL);
+    run_threads(bwd_worker, &J, pick_threads(nthreads, b * H));
+    pthread_mutex_destroy(&J.lock);
+    return J.status;
+}

@@ -65,6 +65,9 @@ def _load():
         lib.ssd_oracle_step.restype = ctypes.c_int
         lib.ssd_oracle_step.argtypes = [f32p] * 7 + [f64p, f64p] + [i64] * 5 + [
             ctypes.c_double, ctypes.c_double, ctypes.c_int]
+        lib.ssd_oracle_scan_bwd.restype = ctypes.c_int
+        lib.ssd_oracle_scan_bwd.argtypes = [f32p] * 10 + [f64p] * 8 + [i64] * 6 + [
+            ctypes.c_double, ctypes.c_double, ctypes.c_int]
         lib.ssd_oracle_softplus.restype = ctypes.c_double
         lib.ssd_oracle_softplus.argtypes = [ctypes.c_double]
         _lib = lib
@@ -192,6 +195,50 @@ def scan_varlen(x, dt_raw, dt_bias, A, B, C, D, seq_idx, chunk_size: int = 1, in
     if rc != 0:
         raise RuntimeError("ssd_oracle_scan_varlen failed with code %d" % rc)
     return y, fs, states
+
+
+def scan_bwd(x, dt_raw, dt_bias, A, B, C, D, dy, dfinal=None, init_state=None,
+             dt_limit: Tuple[float, float] = (0.0, float("inf")), nthreads: int = 0) -> dict:
+    """Gradients of <dy, y> + <dfinal, final_state> for scan() (reverse mode
+    of the recurrence; see ssd_oracle.c).  dy [b,L,H,P], dfinal [b,H,N,P] or
+    None (zeros).  Returns float64 arrays keyed by input: x, dt_raw [b,L,H],
+    dt_bias, A, D [H], B, C [b,L,G,N] (the heads of each group summed),
+    init_state [b,H,N,P] (always, also when init_state is None)."""
+    x, dt_raw, dt_bias, A, B, C, D, dy = (_f32(v) for v in (x, dt_raw, dt_bias, A, B, C, D, dy))
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if dt_raw.shape != (b, L, H) or B.shape != (b, L, G, N) or C.shape != B.shape or dy.shape != x.shape:
+        raise ValueError("oracle.scan_bwd: inconsistent shapes")
+    if dt_bias.shape != (H,) or A.shape != (H,) or D.shape != (H,) or H % G:
+        raise ValueError("oracle.scan_bwd: bad per-head parameter shapes or H % G != 0")
+    null = ctypes.POINTER(ctypes.c_float)()
+    s0 = _f32(init_state) if init_state is not None else None
+    df = _f32(dfinal) if dfinal is not None else None
+    for nm, v in (("init_state", s0), ("dfinal", df)):
+        if v is not None and v.shape != (b, H, N, P):
+            raise ValueError("oracle.scan_bwd: %s must be [b,H,N,P]" % nm)
+    out = {
+        "x": np.zeros((b, L, H, P)), "dt_raw": np.zeros((b, L, H)),
+        "B_h": np.zeros((b, L, H, N)), "C_h": np.zeros((b, L, H, N)),
+        "A_h": np.zeros((b, H)), "dt_bias_h": np.zeros((b, H)), "D_h": np.zeros((b, H)),
+        "init_state": np.zeros((b, H, N, P)),
+    }
+    rc = _load().ssd_oracle_scan_bwd(
+        _p32(x), _p32(dt_raw), _p32(dt_bias), _p32(A), _p32(B), _p32(C), _p32(D),
+        _p32(s0) if s0 is not None else null, _p32(dy), _p32(df) if df is not None else null,
+        _p64(out["x"]), _p64(out["dt_raw"]), _p64(out["B_h"]), _p64(out["C_h"]), _p64(out["A_h"]),
+        _p64(out["dt_bias_h"]), _p64(out["D_h"]), _p64(out["init_state"]), b, L, H, P, N, G,
+        float(dt_limit[0]), float(dt_limit[1]), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("ssd_oracle_scan_bwd failed with code %d" % rc)
+    hpg = H // G
+    return {
+        "x": out["x"], "dt_raw": out["dt_raw"],
+        "B": out["B_h"].reshape(b, L, G, hpg, N).sum(axis=3),
+        "C": out["C_h"].reshape(b, L, G, hpg, N).sum(axis=3),
+        "A": out["A_h"].sum(axis=0), "dt_bias": out["dt_bias_h"].sum(axis=0), "D": out["D_h"].sum(axis=0),
+        "init_state": out["init_state"],
+    }
 
 
 def conv1d_silu(xbc, weight, bias) -> np.ndarray:

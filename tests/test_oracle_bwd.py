@@ -1,0 +1,142 @@
+"""Pins for the backward oracle (oracle.scan_bwd), CPU only.
+
+The gradients are checked against things other than the backward code
+itself:
+  * directional finite differences of the forward oracle (itself pinned by
+    test_oracle.py), with the exact float32 perturbation that reached it;
+  * closed forms: dD = sum dy.x; with dy = 0 the seed dfinal reaches the
+    initial state and every token through products of decays only;
+  * the group sum: G = 1 equals G = H with B, C replicated and the per-head
+    gradients of B, C added.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+NAMES = ["x", "dt_raw", "dt_bias", "A", "B", "C", "D", "init_state"]
+
+
+def make(b, L, H, P, N, G, seed, A_scale=1.0):
+    rng = np.random.default_rng(seed)
+    f = np.float32
+    inp = {
+        "x": rng.standard_normal((b, L, H, P)).astype(f),
+        "dt_raw": rng.standard_normal((b, L, H)).astype(f),
+        "dt_bias": rng.uniform(-3, 0, H).astype(f),
+        "A": (-A_scale * np.exp(rng.uniform(0, np.log(16), H))).astype(f),
+        "B": rng.standard_normal((b, L, G, N)).astype(f),
+        "C": rng.standard_normal((b, L, G, N)).astype(f),
+        "D": rng.normal(1, 0.1, H).astype(f),
+        "init_state": rng.normal(0, 0.1, (b, H, N, P)).astype(f),
+    }
+    dy = rng.standard_normal((b, L, H, P)).astype(f)
+    dfinal = rng.standard_normal((b, H, N, P)).astype(f)
+    return inp, dy, dfinal
+
+
+def loss(inp, dy, dfinal, limit):
+    y, fs = oracle.scan(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"],
+                        init_state=inp["init_state"], dt_limit=limit)
+    return float(np.sum(y * dy.astype(np.float64)) + np.sum(fs * dfinal.astype(np.float64)))
+
+
+def grads(inp, dy, dfinal, limit):
+    return oracle.scan_bwd(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"], dy,
+                           dfinal=dfinal, init_state=inp["init_state"], dt_limit=limit)
+
+
+@pytest.mark.parametrize("limit", [(0.0, float("inf")), (0.02, 0.3)])
+@pytest.mark.parametrize("name", NAMES)
+def test_directional_finite_difference(name, limit):
+    # 70 tokens: the oracle's recompute checkpoints (64 tokens) are crossed
+    inp, dy, dfinal = make(2, 70, 4, 3, 5, 2, seed=11)
+    g = grads(inp, dy, dfinal, limit)
+    rng = np.random.default_rng(100 + NAMES.index(name))
+    v = rng.standard_normal(inp[name].shape)
+    # x, B, C, D and init_state enter linearly (no truncation error); dt and A
+    # through exponentials, where the step sets the third-order term
+    eps = 1e-3 if name in ("x", "B", "C", "D", "init_state") else 1e-4
+    base = inp[name].astype(np.float64)
+    plus, minus = dict(inp), dict(inp)
+    plus[name] = (base + eps * v).astype(np.float32)
+    minus[name] = (base - eps * v).astype(np.float32)
+    # the perturbation that really reached the float32 inputs
+    delta = plus[name].astype(np.float64) - minus[name].astype(np.float64)
+    fd = loss(plus, dy, dfinal, limit) - loss(minus, dy, dfinal, limit)
+    pred = float(np.sum(g[name] * delta))
+    assert abs(fd - pred) <= 1e-6 * max(abs(pred), 1e-3 * float(np.sum(np.abs(g[name] * delta)))), (fd, pred)
+
+
+def test_clamped_tokens_pass_no_gradient_to_dt_raw():
+    inp, dy, dfinal = make(1, 30, 2, 3, 4, 1, seed=12)
+    lo, hi = 0.05, 0.2
+    g = grads(inp, dy, dfinal, (lo, hi))
+    z = inp["dt_raw"].astype(np.float64) + inp["dt_bias"].astype(np.float64)
+    sp = np.logaddexp(0.0, z)
+    out = (sp < lo) | (sp > hi)
+    assert out.any() and (~out).any()
+    assert np.all(g["dt_raw"][out] == 0.0)
+    assert np.all(g["dt_raw"][~out] != 0.0)
+
+
+def test_dD_is_the_sum_of_dy_x():
+    inp, dy, dfinal = make(2, 40, 3, 4, 5, 3, seed=13)
+    g = grads(inp, dy, dfinal, (0.0, float("inf")))
+    ref = np.einsum("blhp,blhp->h", dy.astype(np.float64), inp["x"].astype(np.float64))
+    np.testing.assert_allclose(g["D"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_final_state_seed_reaches_back_through_the_decays():
+    """dy = 0: the loss is <dfinal, S_L> with S_L = (prod a) S_0 +
+    sum_t dt_t (prod_{r>t} a_r) B_t x_t^T, so dinit = (prod a) dfinal,
+    dx_t = dt_t (prod_{r>t} a_r) dfinal^T B_t, dB_t = the same with x_t, dC = 0."""
+    b, L, H, P, N, G = 2, 9, 2, 3, 4, 2
+    inp, _, dfinal = make(b, L, H, P, N, G, seed=14)
+    dy = np.zeros((b, L, H, P), np.float32)
+    g = grads(inp, dy, dfinal, (0.0, float("inf")))
+    z = inp["dt_raw"].astype(np.float64) + inp["dt_bias"].astype(np.float64)
+    dt = np.logaddexp(0.0, z)
+    a = np.exp(dt * inp["A"].astype(np.float64))             # [b, L, H]
+    after = np.ones_like(a)                                  # prod_{r>t} a_r
+    for t in range(L - 2, -1, -1):
+        after[:, t] = after[:, t + 1] * a[:, t + 1]
+    df = dfinal.astype(np.float64)
+    np.testing.assert_allclose(g["init_state"], np.prod(a, axis=1)[:, :, None, None] * df, rtol=1e-12, atol=1e-14)
+    Bh = np.repeat(inp["B"].astype(np.float64), H // G, axis=2)   # [b, L, H, N]
+    xh = inp["x"].astype(np.float64)
+    dx = (dt * after)[..., None] * np.einsum("bhnp,blhn->blhp", df, Bh)
+    np.testing.assert_allclose(g["x"], dx, rtol=1e-11, atol=1e-14)
+    dBh = (dt * after)[..., None] * np.einsum("bhnp,blhp->blhn", df, xh)
+    np.testing.assert_allclose(g["B"], dBh.reshape(b, L, G, H // G, N).sum(3), rtol=1e-11, atol=1e-14)
+    assert np.all(g["C"] == 0.0)
+
+
+def test_group_gradients_are_sums_over_the_heads_of_the_group():
+    b, L, H, P, N = 1, 20, 4, 3, 5
+    inp, dy, dfinal = make(b, L, H, P, N, 1, seed=15)
+    g1 = grads(inp, dy, dfinal, (0.0, float("inf")))
+    rep = dict(inp)
+    rep["B"] = np.repeat(inp["B"], H, axis=2)
+    rep["C"] = np.repeat(inp["C"], H, axis=2)
+    gh = grads(rep, dy, dfinal, (0.0, float("inf")))
+    np.testing.assert_allclose(g1["B"][:, :, 0], gh["B"].sum(axis=2), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(g1["C"][:, :, 0], gh["C"].sum(axis=2), rtol=1e-12, atol=1e-13)
+    for k in ("x", "dt_raw", "A", "dt_bias", "D", "init_state"):
+        np.testing.assert_allclose(g1[k], gh[k], rtol=1e-12, atol=1e-13)
+
+
+def test_a_planted_sign_error_is_caught():
+    """The finite-difference pin sees a flipped term: negate the A-direction
+    gradient's decay part and the check fails."""
+    inp, dy, dfinal = make(1, 20, 2, 3, 4, 1, seed=16)
+    g = grads(inp, dy, dfinal, (0.0, float("inf")))
+    v = np.ones(2)
+    eps = 1e-3
+    plus, minus = dict(inp), dict(inp)
+    plus["A"] = (inp["A"] + eps * v).astype(np.float32)
+    minus["A"] = (inp["A"] - eps * v).astype(np.float32)
+    delta = plus["A"].astype(np.float64) - minus["A"].astype(np.float64)
+    fd = loss(plus, dy, dfinal, (0.0, float("inf"))) - loss(minus, dy, dfinal, (0.0, float("inf")))
+    assert abs(fd - float(np.sum(g["A"] * delta))) <= 1e-6 * abs(fd)
+    assert abs(fd - float(np.sum(-g["A"] * delta))) > 1e-2 * abs(fd)
