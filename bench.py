@@ -501,6 +501,145 @@ def bench_stage(cfg, args, local, peaks, peak_kind):
             "clocks": clk}
 
 
+# fp32 FMA throughput of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 flop x
+# 1965 MHz (the clocks.max.sm of these B200s) = 74.45 TFLOP/s.
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
+
+
+def bwd_flops(cfg):
+    """Algorithmic FLOPs of the backward per call, causal triangles counted
+    once: (whole call, the bwd_cols kernel's share).  Per (batch, chunk of q
+    tokens): C.B^T once per group, G q(q+1) N; per head the dy.x^T pairs and
+    the dx pairs, 2 q(q+1) P; the dB and dC pairs, 2 q(q+1) N; and ten
+    q N P products (the forward's chunk state, the reverse pass's, the G_c
+    terms of dx and dB, the H_in term of dC)."""
+    b, L, H, P, N, G, Q = (cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups,
+                           cfg.chunk_size)
+    tot = cols = 0.0
+    for c in range((L + Q - 1) // Q):
+        q = min(Q, L - c * Q)
+        T = q * (q + 1)
+        tot += G * T * N + H * (2 * T * P + 2 * T * N + 10 * q * N * P)
+        cols += G * T * N + H * (2 * T * P + T * N + 4 * q * N * P)
+    return b * tot, b * cols
+
+
+def bench_backward(cfg, args, local, peaks, peak_kind):
+    """--stage backward: the deterministic backward (ssd_chunk_scan_bwd) on
+    the workload's shapes, inputs and upstream gradients rotated past L2, K
+    calls in one CUDA graph, CUDA events on the launching stream; then the
+    same K calls eagerly with the library's per-kernel event brackets for
+    the kernel shares.  The path runs on CUDA cores in fp32, so the roofline
+    is the fp32 ALU peak (FP32_ALU_TFLOPS); the HBM time of its algorithmic
+    bytes is reported beside it."""
+    from state_space_sequence_scan_b200 import ssd
+    from state_space_sequence_scan_b200.inputs import make_grad_inputs
+    dev = torch.device("cuda", local)
+    b, L, H, P, N, G, Q = (cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups,
+                           cfg.chunk_size)
+    e = 4 if cfg.dtype == "f32" else 2
+    tok, st = b * L, b * H * N * P * 4
+    nbytes = float(tok * (H * P * e + 2 * G * N * e + H * 4)          # x, B, C, dt_raw
+                   + tok * H * P * 4 + st * (2 if cfg.init == "normal" else 1)   # dy, dfinal, init
+                   + tok * (H * P * 4 + H * 4 + 2 * G * N * 4) + st)   # dx, ddt_raw, dB, dC, dinit
+    nsets = max(1, min(4, math.ceil(3 * L2_BYTES / nbytes)))
+    sets, outs = [], []
+    for k in range(nsets):
+        inp = make_scan_inputs(cfg, seed=cfg.seed + 31 * k)
+        gr = make_grad_inputs(cfg, seed=cfg.seed + 31 * k)
+        sets.append(({kk: (v.to(dev) if v is not None else None) for kk, v in inp.items()},
+                     gr["dy"].to(dev), gr["dfinal"].to(dev)))
+        outs.append({"x": torch.empty(b, L, H, P, device=dev), "dt_raw": torch.empty(b, L, H, device=dev),
+                     "dt_bias": torch.empty(H, device=dev), "A": torch.empty(H, device=dev),
+                     "B": torch.empty(b, L, G, N, device=dev), "C": torch.empty(b, L, G, N, device=dev),
+                     "D": torch.empty(H, device=dev), "init_state": torch.empty(b, H, N, P, device=dev)})
+    work = ssd.alloc_workspace(ssd.bwd_workspace_size(b, L, H, P, N, G, Q, sets[0][0]["x"].dtype), dev)
+
+    def step(k):
+        d, dy, df = sets[k % nsets]
+        ssd.chunk_scan_bwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], dy,
+                           dfinal_state=df, init_state=d["init_state"], chunk_size=Q, workspace=work,
+                           out=outs[k % nsets])
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    if ssd.read_device_status(work) != 0:
+        raise RuntimeError("device status %d after warm-up" % ssd.read_device_status(work))
+    graph = capture_steps(step, args.steps)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    del graph
+    ssd.trace_enable(min(8192, 16 * args.steps + 16))
+    for k in range(args.steps):
+        step(k)
+    torch.cuda.synchronize()
+    trace = ssd.trace_read()
+    ssd.trace_enable(0)
+    tot_ms = sum(v[1] for v in trace.values())
+    flops, cols_flops = bwd_flops(cfg)
+    cols_ms = trace["bwd_cols"][1] / max(trace["bwd_cols"][0], 1)
+    ach = cols_flops / (cols_ms * 1e-3) / 1e12
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    mtok = tok / (ms * 1e-3) / 1e6
+    out = {"stage": "backward", "metric": "SSD chunked-scan backward Mtokens/s", "value": mtok,
+           "unit": "Mtokens/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+           "higher_is_better": True, "dtype": "%s-in/f32" % cfg.dtype, "data": "synthetic (seeded)",
+           "config": {"workload": cfg.name, "batch": b, "seqlen": L, "heads": H, "head_dim": P, "state_dim": N,
+                      "groups": G, "chunk_size": Q, "in_dtype": cfg.dtype, "grads": "f32",
+                      "init_state": cfg.init == "normal", "l2": "rotating %d input/gradient sets" % nsets},
+           "roofline": {"bound": "alu", "kernel": "bwd_cols", "achieved": ach, "peak": FP32_ALU_TFLOPS,
+                        "unit": "TFLOP/s", "frac": ach / FP32_ALU_TFLOPS, "traffic": None,
+                        "kernel_ms_avg": cols_ms, "kernel_flops": cols_flops,
+                        "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz",
+                        "shares": {k: round(v[1] / max(tot_ms, 1e-12), 4) for k, v in trace.items()},
+                        "path": {"algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+                                 "alu_ms": flops / (FP32_ALU_TFLOPS * 1e12) * 1e3,
+                                 "hbm_ms": nbytes / (hbm * 1e9) * 1e3,
+                                 "frac": flops / (FP32_ALU_TFLOPS * 1e12) * 1e3 / ms}},
+           "clocks": clk, "gpu_launches": int(sum(v[0] for v in trace.values()))}
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_bwd(cfg)
+    return out
+
+
+def cpu_baseline_bwd(cfg):
+    """The oracle's backward on a bounded sample: every head of batch 0 over
+    the full sequence (one thread per head), token-heads scaled to tokens."""
+    import oracle
+    from state_space_sequence_scan_b200.inputs import make_grad_inputs
+    inp = make_scan_inputs(cfg)
+    gr = make_grad_inputs(cfg)
+    hs = cfg.nheads
+    hpg = cfg.nheads // cfg.ngroups
+    sub = {k: v for k, v in inp.items()}
+    sub["x"] = inp["x"][:1, :, :hs]
+    sub["dt_raw"] = inp["dt_raw"][:1, :, :hs]
+    for k in ("dt_bias", "A", "D"):
+        sub[k] = inp[k][:hs]
+    gsel = [h // hpg for h in range(hs)]
+    sub["B"] = inp["B"][:1][:, :, gsel]
+    sub["C"] = inp["C"][:1][:, :, gsel]
+    sub["init_state"] = None if inp["init_state"] is None else inp["init_state"][:1, :hs]
+    t0 = time.perf_counter()
+    oracle.scan_bwd(sub["x"], sub["dt_raw"], sub["dt_bias"], sub["A"], sub["B"], sub["C"], sub["D"],
+                    gr["dy"][:1, :, :hs], dfinal=gr["dfinal"][:1, :hs], init_state=sub["init_state"])
+    sec = time.perf_counter() - t0
+    return {"value": cfg.seqlen * hs / cfg.nheads / sec / 1e6, "unit": "Mtokens/s", "cores": min(hs, os.cpu_count()),
+            "kind": "oracle", "sample": "%d heads of batch 0 (each its own group), full seqlen %d (%.1f s); "
+                                        "tokens counted as token-heads / heads" % (hs, cfg.seqlen, sec)}
+
+
 def kernel_bytes(cfg, name, states=False) -> float:
     b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
     e = 4 if cfg.dtype == "f32" else 2
@@ -646,7 +785,7 @@ def main():
                     help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
     ap.add_argument("--packed", action="store_true",
                     help="rows packed with documents of about 512 tokens (seq_idx)")
-    ap.add_argument("--stage", default="scan", choices=["scan", "conv1d", "gated_norm"],
+    ap.add_argument("--stage", default="scan", choices=["scan", "conv1d", "gated_norm", "backward"],
                     help="time one of the steps either side of the scan instead (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -664,7 +803,8 @@ def main():
         cfg, is_step = pick(args.workload)
         if args.stage != "scan" and not is_step:
             if rank == 0:
-                print(json.dumps(bench_stage(cfg, args, local, peaks, peak_kind)), flush=True)
+                fn = bench_backward if args.stage == "backward" else bench_stage
+                print(json.dumps(fn(cfg, args, local, peaks, peak_kind)), flush=True)
             return
         if is_step:
             r = bench_step(cfg, args, ws, rank, local)

@@ -234,6 +234,48 @@ SSD_API ssd_status ssd_gated_rmsnorm(const float *y, const void *z, const float 
                              int64_t tokens, int64_t dim, int64_t group_size, float eps, int z_dtype,
                              void *stream);
 
+/* Bytes of device workspace ssd_chunk_scan_bwd needs for these sizes.  Host
+ * only.  SSD_ERR_UNSUPPORTED for sizes the backward does not take. */
+SSD_API ssd_status ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads,
+                                             int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                                             int64_t chunk_size, int in_dtype, size_t *bytes);
+
+/* Backward of the chunked scan, deterministic (the HF transformers issue
+ * "mamba2 mixer different outputs" notes that the backward pass of the usual
+ * mamba kernels is not; this one has no atomics and sums in a fixed order, so
+ * repeated calls on the same inputs give the same bits).
+ *
+ * Given the forward's inputs (as for ssd_chunk_scan_fwd, no packed rows) and
+ * the gradients dy of y and dfinal_state of final_state, writes the gradient
+ * of <dy, y> + <dfinal_state, final_state> with respect to every input:
+ *   dy           [batch, seqlen, nheads, head_dim] float32 in
+ *   dfinal_state [batch, nheads, state_dim, head_dim] float32 in, NULL = zeros
+ *   dx           [batch, seqlen, nheads, head_dim] float32 out
+ *   ddt_raw      [batch, seqlen, nheads] float32 out (4-byte aligned), zero
+ *                where the time-step limit clamps softplus(dt_raw + dt_bias)
+ *                strictly outside [dt_lo, dt_hi]
+ *   ddt_bias, dA, dD  [nheads] float32 out
+ *   dB, dC       [batch, seqlen, ngroups, state_dim] float32 out (the heads of
+ *                a group summed)
+ *   dinit_state  [batch, nheads, state_dim, head_dim] float32 out, or NULL
+ *                when not wanted (written also when init_state is NULL)
+ * Gradients are float32 whatever in_dtype is.  The states the gradients need
+ * are recomputed from the inputs inside the call; nothing from a forward call
+ * is reused.  The work runs on CUDA cores in fp32 in chunks of chunk_size
+ * tokens (any chunk_size >= 1); head_dim must be 8, 16, 32 or 64 and
+ * state_dim a multiple of 8 up to 128, else SSD_ERR_UNSUPPORTED.  16-byte
+ * alignment as for the forward; outputs must not overlap the inputs or each
+ * other; the workspace is at least ssd_chunk_scan_bwd_workspace_size() bytes,
+ * 256-byte aligned, its status word read by ssd_read_device_status()
+ * (SSD_ERR_PRECONDITION for A > 0). */
+SSD_API ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
+                              const void *B, const void *C, const float *D, const float *init_state,
+                              const float *dy, const float *dfinal_state, float *dx, float *ddt_raw,
+                              float *ddt_bias, float *dA, float *dB, float *dC, float *dD, float *dinit_state,
+                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                              int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi,
+                              int in_dtype, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Waits for `stream`, then reads the device status word that the last
  * ssd_chunk_scan_fwd on this workspace left: SSD_OK, SSD_ERR_PRECONDITION or
  * SSD_ERR_DEVICE_TIMEOUT.  `workspace` is a device pointer. */

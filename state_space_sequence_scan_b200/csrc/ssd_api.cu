@@ -207,6 +207,72 @@ ssd_status ssd_chunk_scan_fwd_varlen(const void *x, const float *dt_raw, const f
                     workspace_bytes, stream);
 }
 
+ssd_status ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                                             int64_t state_dim, int64_t ngroups, int64_t chunk_size, int in_dtype,
+                                             size_t *bytes) {
+    if (!bytes) return SSD_ERR_INVALID_ARG;
+    ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, in_dtype,
+                                    SSD_PATH_SIMT);
+    if (st != SSD_OK) return st;
+    const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
+    if (!ssd::bwd_supported(d)) return SSD_ERR_UNSUPPORTED;
+    *bytes = ssd::bwd_workspace_bytes(d);
+    return SSD_OK;
+}
+
+ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
+                              const void *B, const void *C, const float *D, const float *init_state,
+                              const float *dy, const float *dfinal_state, float *dx, float *ddt_raw,
+                              float *ddt_bias, float *dA, float *dB, float *dC, float *dD, float *dinit_state,
+                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim, int64_t state_dim,
+                              int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, in_dtype,
+                                    SSD_PATH_SIMT);
+    if (st != SSD_OK) return st;
+    if (!limits_ok(dt_lo, dt_hi)) return SSD_ERR_INVALID_ARG;
+    if (!dt_bias || !A || !D || !ddt_bias || !dA || !dD) return SSD_ERR_INVALID_ARG;
+    const bool has_tokens = batch > 0 && seqlen > 0;
+    if (has_tokens && (!x || !dt_raw || !B || !C || !dy || !dx || !ddt_raw || !dB || !dC))
+        return SSD_ERR_INVALID_ARG;
+    const void *al[] = {x, B, C, init_state, dy, dfinal_state, dx, dB, dC, dinit_state};
+    for (const void *p : al)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(dt_raw) | reinterpret_cast<uintptr_t>(ddt_raw)) & 3u) return SSD_ERR_ALIGNMENT;
+    const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
+    if (!ssd::bwd_supported(d)) return SSD_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < ssd::bwd_workspace_bytes(d)) return SSD_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, ssd::kStatusBytes, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!has_tokens) {
+        // no tokens: the per-head sums are zero and the seed passes to the initial state as it is
+        const size_t hb = (size_t)nheads * sizeof(float);
+        if ((e = cudaMemsetAsync(dA, 0, hb, s)) != cudaSuccess || (e = cudaMemsetAsync(dD, 0, hb, s)) != cudaSuccess ||
+            (e = cudaMemsetAsync(ddt_bias, 0, hb, s)) != cudaSuccess)
+            return cuda_fail(e);
+        if (dinit_state && batch > 0) {
+            const size_t sb = (size_t)batch * nheads * state_dim * head_dim * sizeof(float);
+            e = dfinal_state ? cudaMemcpyAsync(dinit_state, dfinal_state, sb, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(dinit_state, 0, sb, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return SSD_OK;
+    }
+    ssd::BwdArgs a;
+    a.f.x = x; a.f.dt_raw = dt_raw; a.f.dt_bias = dt_bias; a.f.A = A; a.f.B = B; a.f.C = C; a.f.D = D;
+    a.f.init_state = init_state; a.f.y = nullptr; a.f.final_state = nullptr;
+    a.f.dt_lo = dt_lo; a.f.dt_hi = dt_hi; a.f.bf16 = in_dtype == SSD_BF16;
+    a.dy = dy; a.dfinal = dfinal_state;
+    a.dx = dx; a.ddt_raw = ddt_raw; a.ddt_bias = ddt_bias; a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD;
+    a.dinit = dinit_state;
+    e = ssd::bwd_scan(a, d, workspace, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return SSD_OK;
+}
+
 ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
                     const void *B, const void *C, const float *D, float *state, float *y,
                     int64_t batch, int64_t nheads, int64_t head_dim, int64_t state_dim,

@@ -42,9 +42,31 @@ int record_cuda_error(cudaError_t e);
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // ---- SIMT fp32 path (any chunk size) --------------------------------------
+// Its workspace after the status region (every region 256-byte aligned).
+struct SimtWs {
+    unsigned *status;
+    float *dtv;     // [b, H, L]  dt
+    float *cum;     // [b, H, L]  within-chunk inclusive cumsum of dt * A
+    float *ell;     // [b, H, nc] chunk log decay (cum at the chunk's last token)
+    float *states;  // [b, H, nc, N, P]  after the state pass: the state entering each chunk
+};
+SimtWs simt_carve(const ScanDims &d, void *workspace);
 bool simt_supported(const ScanDims &d);
 size_t simt_workspace_bytes(const ScanDims &d);
 cudaError_t simt_scan(const ScanArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
+// The first two launches of simt_scan alone (no y): fills dtv, cum, ell and
+// the entering states; writes final_state / chunk_states when not null.
+cudaError_t simt_scan_states(const ScanArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
+
+// ---- backward of the scan (SIMT fp32, deterministic) -----------------------
+struct BwdArgs {
+    ScanArgs f;                    // the forward's inputs (y, final_state, chunk_states unused)
+    const float *dy, *dfinal;      // [b,L,H,P], [b,H,N,P] or null
+    float *dx, *ddt_raw, *ddt_bias, *dA, *dB, *dC, *dD, *dinit;
+};
+bool bwd_supported(const ScanDims &d);
+size_t bwd_workspace_bytes(const ScanDims &d);
+cudaError_t bwd_scan(const BwdArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
 
 // ---- tcgen05 tensor-core path -----------------------------------------------
 bool tc_supported(const ScanDims &d, int bf16);

@@ -39,15 +39,9 @@ constexpr int kTJ = 32;      // j tokens per tile in chunk_out
 constexpr int kTKH = 32;     // state rows per smem tile in chunk_out
 constexpr int kMaxAcc = 32;  // accumulators per thread
 
-struct SimtWs {
-    unsigned *status;
-    float *dtv;     // [b, H, L]
-    float *cum;     // [b, H, L]
-    float *ell;     // [b, H, nc]   chunk log decay (cum at the chunk's last token)
-    float *states;  // [b, H, nc, N, P]
-};
+}  // namespace
 
-SimtWs carve(const ScanDims &d, void *ws) {
+SimtWs simt_carve(const ScanDims &d, void *ws) {
     char *p = static_cast<char *>(ws);
     SimtWs w;
     w.status = reinterpret_cast<unsigned *>(p);
@@ -59,6 +53,8 @@ SimtWs carve(const ScanDims &d, void *ws) {
     w.states = reinterpret_cast<float *>(p + off);
     return w;
 }
+
+namespace {
 
 // 1 when token t of row b starts a document of a packed row
 __device__ __forceinline__ float doc_start(const int32_t *seq_idx, size_t b, int L, int t) {
@@ -328,17 +324,14 @@ size_t out_smem(const ScanDims &d, int TI) {
                             2 * kTJ + (size_t)TI * (kTJ + 1) + (size_t)kTKH * d.P);
 }
 
+// Launches 1 and 2: dt, cum, the chunk log decays and the state entering
+// every chunk (ws.states), plus final_state / chunk_states when asked for.
 template <typename T>
-cudaError_t run(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) {
-    SimtWs ws = carve(d, wsp);
-    const int TI = pick_ti(d);
-    const size_t sm1 = state_smem(d), sm3 = out_smem(d, TI);
+cudaError_t run_states(const ScanArgs &a, const ScanDims &d, const SimtWs &ws, cudaStream_t s) {
+    const size_t sm1 = state_smem(d);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(chunk_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)sm1)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(chunk_out_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)sm3)) != cudaSuccess)
         return e;
     const dim3 g1((unsigned)d.nc, (unsigned)d.H, (unsigned)d.b);
     {
@@ -355,7 +348,19 @@ cudaError_t run(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s)
         state_pass_kernel<<<g2, kThreads, 0, s>>>(ws, a.init_state, a.final_state, a.chunk_states, (int)d.H, NP,
                                                   (int)d.nc);
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t run(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) {
+    SimtWs ws = simt_carve(d, wsp);
+    const int TI = pick_ti(d);
+    const size_t sm3 = out_smem(d, TI);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(chunk_out_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sm3)) != cudaSuccess)
+        return e;
+    if ((e = run_states<T>(a, d, ws, s)) != cudaSuccess) return e;
     const int tiles = (int)((d.Q + TI - 1) / TI);
     const dim3 g3((unsigned)(d.nc * tiles), (unsigned)d.H, (unsigned)d.b);
     {
@@ -385,6 +390,11 @@ size_t simt_workspace_bytes(const ScanDims &d) {
 
 cudaError_t simt_scan(const ScanArgs &a, const ScanDims &d, void *ws, cudaStream_t s) {
     return a.bf16 ? run<__nv_bfloat16>(a, d, ws, s) : run<float>(a, d, ws, s);
+}
+
+cudaError_t simt_scan_states(const ScanArgs &a, const ScanDims &d, void *ws, cudaStream_t s) {
+    const SimtWs w = simt_carve(d, ws);
+    return a.bf16 ? run_states<__nv_bfloat16>(a, d, w, s) : run_states<float>(a, d, w, s);
 }
 
 }  // namespace ssd

@@ -16,7 +16,13 @@ enum TraceKernel {
     kTrTcDtPrep = 7,
     kTrConv1d = 8,
     kTrGatedNorm = 9,
-    kKernelCount = 10,
+    kTrBwdDstate = 10,
+    kTrBwdDpass = 11,
+    kTrBwdCols = 12,
+    kTrBwdRows = 13,
+    kTrBwdFinalize = 14,
+    kTrBwdReduce = 15,
+    kKernelCount = 16,
 };
 
 bool trace_on();

@@ -145,3 +145,13 @@ def make_step_inputs(cfg: StepConfig, steps: Optional[int] = None,
     C = torch.randn(T, b, G, N, generator=g, dtype=torch.float32).to(sd)
     dt_raw = torch.randn(T, b, H, generator=g, dtype=torch.float32)
     return dict(x=x, dt_raw=dt_raw, dt_bias=dt_bias, A=A, B=B, C=C, D=D, state=state)
+
+
+def make_grad_inputs(cfg: ScanConfig, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Host fp32 upstream gradients for a backward call: dy [b,L,H,P] and
+    dfinal [b,H,N,P], both N(0, 1)."""
+    g = _gen((cfg.seed if seed is None else seed) + 7919)
+    b, L, H, P, N = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim
+    dy = torch.randn(b, L, H, P, generator=g, dtype=torch.float32)
+    dfinal = torch.randn(b, H, N, P, generator=g, dtype=torch.float32)
+    return dict(dy=dy, dfinal=dfinal)

@@ -30,7 +30,8 @@ PATHS = {"auto": 0, "simt": 1, "tensor": 2}
 EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_chunk_scan_fwd_states", "ssd_step",
             "ssd_read_device_status", "ssd_status_string", "ssd_last_cuda_error", "ssd_version",
             "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count",
-            "ssd_conv1d_silu_split", "ssd_gated_rmsnorm", "ssd_chunk_scan_fwd_varlen")
+            "ssd_conv1d_silu_split", "ssd_gated_rmsnorm", "ssd_chunk_scan_fwd_varlen",
+            "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd")
 
 _lib = None
 
@@ -61,6 +62,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_chunk_scan_fwd_varlen.argtypes = [vp] * 12 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
     lib.ssd_chunk_scan_fwd_states.restype = i32
     lib.ssd_chunk_scan_fwd_states.argtypes = [vp] * 11 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
+    lib.ssd_chunk_scan_bwd_workspace_size.restype = i32
+    lib.ssd_chunk_scan_bwd_workspace_size.argtypes = [i64] * 7 + [i32, ctypes.POINTER(sz)]
+    lib.ssd_chunk_scan_bwd.restype = i32
+    lib.ssd_chunk_scan_bwd.argtypes = [vp] * 18 + [i64] * 7 + [f32, f32, i32, vp, sz, vp]
     lib.ssd_step.restype = i32
     lib.ssd_step.argtypes = [vp] * 9 + [i64] * 5 + [f32, f32, i32, vp]
     lib.ssd_read_device_status.restype = i32
@@ -230,6 +235,70 @@ def chunk_scan_fwd_states(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check("ssd_chunk_scan_fwd_states", st)
     return y, final_state, chunk_states
+
+
+def bwd_workspace_size(b: int, L: int, H: int, P: int, N: int, G: int, Q: int, in_dtype=torch.bfloat16) -> int:
+    """Bytes of workspace ssd_chunk_scan_bwd needs for these sizes."""
+    lib = load_library()
+    out = ctypes.c_size_t(0)
+    _check("ssd_chunk_scan_bwd_workspace_size",
+           lib.ssd_chunk_scan_bwd_workspace_size(b, L, H, P, N, G, Q, DTYPES[in_dtype], ctypes.byref(out)))
+    return int(out.value)
+
+
+def chunk_scan_bwd(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor, A: torch.Tensor,
+                   B: torch.Tensor, C: torch.Tensor, D: torch.Tensor, dy: torch.Tensor,
+                   dfinal_state: Optional[torch.Tensor] = None, init_state: Optional[torch.Tensor] = None,
+                   chunk_size: int = 256, dt_limit: Tuple[float, float] = (0.0, math.inf),
+                   workspace: Optional[torch.Tensor] = None, want_dinit: bool = True,
+                   out: Optional[dict] = None) -> dict:
+    """Deterministic backward of chunk_scan_fwd (ssd_chunk_scan_bwd): the
+    gradients of <dy, y> + <dfinal_state, final_state> with respect to every
+    input, float32, keyed by input name ("x", "dt_raw", "dt_bias", "A", "B",
+    "C", "D", "init_state"; the last None unless want_dinit).  `out` may hold
+    preallocated outputs under the same keys."""
+    lib = load_library()
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    _need_cuda("x", x)
+    if x.dtype not in DTYPES:
+        raise ValueError("x/B/C must be float32 or bfloat16")
+    _need_cuda("B", B, x.dtype, (b, L, G, N))
+    _need_cuda("C", C, x.dtype, (b, L, G, N))
+    _need_cuda("dt_raw", dt_raw, torch.float32, (b, L, H))
+    _need_cuda("dy", dy, torch.float32, (b, L, H, P))
+    for nm, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need_cuda(nm, t, torch.float32, (H,))
+    for nm, t in (("init_state", init_state), ("dfinal_state", dfinal_state)):
+        if t is not None:
+            _need_cuda(nm, t, torch.float32, (b, H, N, P))
+    f = torch.float32
+    shapes = {"x": (b, L, H, P), "dt_raw": (b, L, H), "dt_bias": (H,), "A": (H,), "B": (b, L, G, N),
+              "C": (b, L, G, N), "D": (H,), "init_state": (b, H, N, P)}
+    g = dict(out or {})
+    for k, shp in shapes.items():
+        if k == "init_state" and not want_dinit:
+            g[k] = None
+            continue
+        if g.get(k) is None:
+            g[k] = torch.empty(shp, dtype=f, device=dev)
+        else:
+            _need_cuda("out[%s]" % k, g[k], f, shp)
+    Q = int(chunk_size)
+    need = bwd_workspace_size(b, L, H, P, N, G, Q, x.dtype)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    st = lib.ssd_chunk_scan_bwd(
+        _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(dy),
+        _ptr(dfinal_state), _ptr(g["x"]), _ptr(g["dt_raw"]), _ptr(g["dt_bias"]), _ptr(g["A"]), _ptr(g["B"]),
+        _ptr(g["C"]), _ptr(g["D"]), _ptr(g["init_state"]), b, L, H, P, N, G, Q, float(dt_limit[0]),
+        float(dt_limit[1]), DTYPES[x.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(dev))
+    _check("ssd_chunk_scan_bwd", st)
+    return g
 
 
 def chunk_scan_fwd_varlen(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor, A: torch.Tensor,

@@ -137,6 +137,33 @@ def test_forward_varlen_rejects_bad_arguments_on_host(lib):
         assert f(path=path) == 4 and f(Q=64, path=path) == 4
 
 
+def _bwd(lib, **kw):
+    fake = 0x10000
+    a = dict(ptrs=[fake] * 18, b=1, L=64, H=2, P=16, N=16, G=1, Q=16, lo=0.0, hi=math.inf, dtype=0, ws=None, wsb=0)
+    a.update(kw)
+    return lib.ssd_chunk_scan_bwd(*a["ptrs"], a["b"], a["L"], a["H"], a["P"], a["N"], a["G"], a["Q"], a["lo"],
+                                  a["hi"], a["dtype"], a["ws"], a["wsb"], None)
+
+
+def test_backward_rejects_bad_arguments_on_host(lib):
+    """The backward checks its sizes, pointers and workspace before anything
+    is enqueued: head_dim 8/16/32/64, state_dim a multiple of 8 up to 128."""
+    fake = 0x10000
+    sz = ctypes.c_size_t(0)
+    assert lib.ssd_chunk_scan_bwd_workspace_size(1, 64, 2, 16, 16, 1, 16, 0, ctypes.byref(sz)) == 0 and sz.value > 0
+    for P, N, want in ((48, 16, 2), (16, 136, 2), (16, 12, 2), (128, 16, 2), (64, 128, 0), (8, 8, 0)):
+        assert lib.ssd_chunk_scan_bwd_workspace_size(1, 64, 2, P, N, 1, 16, 0, ctypes.byref(sz)) == want, (P, N)
+    assert lib.ssd_chunk_scan_bwd_workspace_size(1, 64, 3, 16, 16, 2, 16, 0, ctypes.byref(sz)) == 1   # H % G
+    assert _bwd(lib) == 4                                                  # no workspace
+    assert _bwd(lib, ptrs=[fake] * 8 + [None] + [fake] * 9) == 1          # dy missing
+    assert _bwd(lib, ptrs=[fake] * 10 + [fake + 4] + [fake] * 7) == 3     # dx misaligned
+    assert _bwd(lib, ptrs=[fake] * 11 + [fake + 2] + [fake] * 6) == 3     # ddt_raw misaligned
+    assert _bwd(lib, P=48) == 2
+    assert _bwd(lib, lo=0.5, hi=0.1) == 1
+    assert _bwd(lib, ws=fake, wsb=16) == 4
+    assert _bwd(lib, ws=fake + 16, wsb=1 << 30) == 3
+
+
 def test_front_back_reject_bad_arguments_on_host(lib):
     """The conv1d and gated-norm entry points check sizes, dtypes and
     alignment before anything is queued."""
