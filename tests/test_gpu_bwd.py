@@ -5,9 +5,14 @@ finite differences in test_oracle_bwd.py).
 Bars, per gradient tensor, with bf16 or fp32 inputs alike (both sides read
 the same values, bf16 widening to fp32 exactly, and the GPU computes in fp32
 throughout):
-  * relative L2 error <= 1e-5;
   * max|gpu - oracle| / RMS(oracle) <= 2e-4 on the small layers (up to about
-    1M elements per tensor), <= 1e-3 on the full-size 130m layer.
+    1M elements per tensor), <= 1e-3 on the full-size 130m layer;
+  * relative L2 error <= 1e-5 for the per-element gradients (x, dt_raw, B, C,
+    init_state).  The per-head gradients dA, d(dt_bias), dD are sums over all
+    of a head's tokens whose terms cancel: their fp32 error scales with the
+    sum of the terms' sizes, not with the result (the chunked form in fp32 on
+    the CPU already gives dA a 1.5e-5 relative error on a 200-token, 2-head
+    layer whose dA is [-0.45, 0.96]), so they carry the max bar only.
 Derived from the arithmetic: the chunked form evaluated in fp32 on the CPU
 lands at 1e-6 to 2.3e-5 max/RMS on 300-600-token rows (Q = 64, 256).  The
 maximum over a tensor grows with its size: on the full-size layer's dx (12.6M
@@ -55,10 +60,14 @@ def oracle_bwd(inp, grads, dt_limit=(0.0, math.inf), with_dfinal=True):
                            init_state=inp["init_state"], dt_limit=dt_limit)
 
 
+PER_ELEMENT = ("x", "dt_raw", "B", "C", "init_state")
+
+
 def check_all(got, ref, what, tol=TOL_BWD):
     for k in KEYS:
         _, l2 = compare(got[k], ref[k], tol, "%s: d%s" % (what, k))
-        assert l2 <= TOL_BWD_L2, "%s: d%s: relative L2 %.3e > %.0e" % (what, k, l2, TOL_BWD_L2)
+        if k in PER_ELEMENT:
+            assert l2 <= TOL_BWD_L2, "%s: d%s: relative L2 %.3e > %.0e" % (what, k, l2, TOL_BWD_L2)
 
 
 CASES = [
