@@ -83,3 +83,81 @@ def test_unmutated_copy_passes(tmp_path):
     y, fs = _scan_with(so, case)
     y_ref, fs_ref = _closed_form(case)
     assert max(_rel(y, y_ref), _rel(fs, fs_ref)) < 1e-12
+
+
+# ---- the backward oracle: each planted mistake must fail the finite-difference pin
+BWD_MUTANTS = {
+    "bwd_drop_D": ("dxr[p] = dtt * acc + Dh * (double)dyr[p];", "dxr[p] = dtt * acc;"),
+    "bwd_no_decay_carry": ("for (i = 0; i < NP; ++i) Gm[i] *= at;", "for (i = 0; i < NP; ++i) Gm[i] *= 1.0;"),
+    "bwd_dA_no_dt": ("dA += dtt * at * gs;", "dA += at * gs;"),
+    "bwd_ddt_no_A": ("dz = (bgx + A * at * gs)", "dz = (bgx + at * gs)"),
+    "bwd_dC_previous_state": ("acc += Scur[n * P + p] * (double)dyr[p];", "acc += Sprev[n * P + p] * (double)dyr[p];"),
+    "bwd_sigmoid_sign": ("? sigmoid_exact(z) : 0.0);", "? sigmoid_exact(-z) : 0.0);"),
+    "bwd_dB_no_dt": ("dBr[n] = dtt * acc;", "dBr[n] = acc;"),
+    "bwd_seed_ignored": ("for (i = 0; i < NP; ++i) Gm[i] = (double)J->dfinal[(bi * H + h) * NP + i];",
+                         "for (i = 0; i < NP; ++i) Gm[i] = 0.0 * J->dfinal[(bi * H + h) * NP + i];"),
+}
+
+
+def _bwd_with(lib_path, inp, dy, dfinal):
+    lib = ctypes.CDLL(lib_path)
+    f32p = ctypes.POINTER(ctypes.c_float)
+    f64p = ctypes.POINTER(ctypes.c_double)
+    lib.ssd_oracle_scan_bwd.restype = ctypes.c_int
+    lib.ssd_oracle_scan_bwd.argtypes = [f32p] * 10 + [f64p] * 8 + [ctypes.c_int64] * 6 + [
+        ctypes.c_double, ctypes.c_double, ctypes.c_int]
+    b, L, H, P = inp["x"].shape
+    G, N = inp["B"].shape[2:]
+    o = {"x": np.zeros((b, L, H, P)), "dt_raw": np.zeros((b, L, H)), "B_h": np.zeros((b, L, H, N)),
+         "C_h": np.zeros((b, L, H, N)), "A_h": np.zeros((b, H)), "dt_bias_h": np.zeros((b, H)),
+         "D_h": np.zeros((b, H)), "init_state": np.zeros((b, H, N, P))}
+    p32 = lambda a: np.ascontiguousarray(a, np.float32).ctypes.data_as(f32p)
+    keep = [np.ascontiguousarray(inp[k], np.float32) for k in ("x", "dt_raw", "dt_bias", "A", "B", "C", "D",
+                                                              "init_state")]
+    keep += [np.ascontiguousarray(dy, np.float32), np.ascontiguousarray(dfinal, np.float32)]
+    rc = lib.ssd_oracle_scan_bwd(*[a.ctypes.data_as(f32p) for a in keep],
+                                 *[o[k].ctypes.data_as(f64p) for k in ("x", "dt_raw", "B_h", "C_h", "A_h",
+                                                                       "dt_bias_h", "D_h", "init_state")],
+                                 b, L, H, P, N, G, 0.0, float("inf"), 1)
+    assert rc == 0
+    hpg = H // G
+    return {"x": o["x"], "dt_raw": o["dt_raw"], "B": o["B_h"].reshape(b, L, G, hpg, N).sum(3),
+            "C": o["C_h"].reshape(b, L, G, hpg, N).sum(3), "A": o["A_h"].sum(0), "dt_bias": o["dt_bias_h"].sum(0),
+            "D": o["D_h"].sum(0), "init_state": o["init_state"]}
+
+
+def _fd_misses(g, inp, dy, dfinal):
+    """Names whose directional finite difference (of the pinned forward
+    oracle) disagrees with g."""
+    from test_oracle_bwd import NAMES, loss
+    bad = []
+    lim = (0.0, float("inf"))
+    for name in NAMES:
+        v = np.random.default_rng(200 + NAMES.index(name)).standard_normal(inp[name].shape)
+        eps = 1e-3 if name in ("x", "B", "C", "D", "init_state") else 1e-4
+        base = inp[name].astype(np.float64)
+        plus, minus = dict(inp), dict(inp)
+        plus[name] = (base + eps * v).astype(np.float32)
+        minus[name] = (base - eps * v).astype(np.float32)
+        delta = plus[name].astype(np.float64) - minus[name].astype(np.float64)
+        fd = loss(plus, dy, dfinal, lim) - loss(minus, dy, dfinal, lim)
+        pred = float(np.sum(g[name] * delta))
+        if abs(fd - pred) > 1e-6 * max(abs(pred), 1e-3 * float(np.sum(np.abs(g[name] * delta)))):
+            bad.append(name)
+    return bad
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_backward_pin_rejects_planted_mistake(tmp_path, name):
+    from test_oracle_bwd import make
+    old, new = BWD_MUTANTS[name]
+    so = _build(tmp_path, name, old, new)
+    inp, dy, dfinal = make(1, 70, 4, 3, 5, 2, seed=31)
+    assert _fd_misses(_bwd_with(so, inp, dy, dfinal), inp, dy, dfinal), "planted mistake went unnoticed"
+
+
+def test_backward_unmutated_copy_passes(tmp_path):
+    from test_oracle_bwd import make
+    so = _build(tmp_path, "bwd_clean", "#define kSeg 64", "#define kSeg 64")
+    inp, dy, dfinal = make(1, 70, 4, 3, 5, 2, seed=31)
+    assert _fd_misses(_bwd_with(so, inp, dy, dfinal), inp, dy, dfinal) == []
