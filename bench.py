@@ -781,6 +781,8 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-decode", action="store_true", help="skip the decode figure on the scan line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="leave the backward (ssd_chunk_scan_bwd) line out of the default scan run")
     ap.add_argument("--chunk-states", action="store_true",
                     help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
     ap.add_argument("--packed", action="store_true",
@@ -817,6 +819,8 @@ def main():
             dline = finish(dcfg, True, dr, args, ws, rank, peaks, peak_kind, sub=True)
             if out is not None:
                 out["decode"] = dline
+        if not is_step and ws == 1 and not args.no_backward and out is not None:
+            out["backward"] = bench_backward(cfg, args, local, peaks, peak_kind)
         if rank == 0 and out is not None:
             if ws == 1 and not args.no_cpu_baseline:
                 cb = cpu_baseline_step(cfg) if is_step else cpu_baseline_scan(cfg)
