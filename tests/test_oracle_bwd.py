@@ -140,3 +140,48 @@ def test_a_planted_sign_error_is_caught():
     fd = loss(plus, dy, dfinal, (0.0, float("inf"))) - loss(minus, dy, dfinal, (0.0, float("inf")))
     assert abs(fd - float(np.sum(g["A"] * delta))) <= 1e-6 * abs(fd)
     assert abs(fd - float(np.sum(-g["A"] * delta))) > 1e-2 * abs(fd)
+
+
+def test_split_and_carry_backward():
+    """Backward over [T1, L) from dfinal gives the gradient of the state at T1;
+    used as the seed of the backward over [0, T1) (which starts from
+    init_state), the pieces equal the whole-sequence gradients (per-head sums
+    added over the two segments)."""
+    b, L, H, P, N, G, T1 = 2, 50, 4, 3, 5, 2, 23
+    inp, dy, dfinal = make(b, L, H, P, N, G, seed=17)
+    lim = (0.0, float("inf"))
+    whole = grads(inp, dy, dfinal, lim)
+    # the state at T1 from the forward oracle over the first segment
+    first = {k: (v[:, :T1] if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
+    _, s1 = oracle.scan(first["x"], first["dt_raw"], first["dt_bias"], first["A"], first["B"], first["C"],
+                        first["D"], init_state=inp["init_state"], dt_limit=lim)
+    second = {k: (v[:, T1:] if k in ("x", "dt_raw", "B", "C") else v) for k, v in inp.items()}
+    second["init_state"] = s1.astype(np.float32)
+    g2 = grads(second, dy[:, T1:], dfinal, lim)
+    # the carried state is float32-rounded for the second segment: compare the
+    # first segment with its own seed, exactly as the chain rule composes
+    g1 = grads(first, dy[:, :T1], g2["init_state"].astype(np.float32), lim)
+    np.testing.assert_allclose(np.concatenate([g1["x"], g2["x"]], axis=1), whole["x"], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(np.concatenate([g1["B"], g2["B"]], axis=1), whole["B"], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(np.concatenate([g1["C"], g2["C"]], axis=1), whole["C"], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(np.concatenate([g1["dt_raw"], g2["dt_raw"]], axis=1), whole["dt_raw"], rtol=1e-5,
+                               atol=1e-6)
+    for k in ("A", "D", "dt_bias"):
+        np.testing.assert_allclose(g1[k] + g2[k], whole[k], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(g1["init_state"], whole["init_state"], rtol=1e-5, atol=1e-6)
+
+
+def test_gradients_are_linear_in_the_seeds():
+    inp, dy1, df1 = make(1, 30, 2, 3, 4, 1, seed=18)
+    _, dy2, df2 = make(1, 30, 2, 3, 4, 1, seed=19)
+    lim = (0.0, float("inf"))
+    # seeds on a 1/64 grid: 0.5 a + 2 b is then exact in float32
+    dy1, dy2, df1, df2 = (np.round(v * 64) / 64 for v in (dy1, dy2, df1, df2))
+    dy1, dy2, df1, df2 = (v.astype(np.float32) for v in (dy1, dy2, df1, df2))
+    g1 = grads(inp, dy1, df1, lim)
+    g2 = grads(inp, dy2, df2, lim)
+    dy12, df12 = 0.5 * dy1 + 2.0 * dy2, 0.5 * df1 + 2.0 * df2
+    assert np.array_equal(dy12.astype(np.float64), 0.5 * dy1.astype(np.float64) + 2.0 * dy2.astype(np.float64))
+    g12 = grads(inp, dy12, df12, lim)
+    for k in NAMES:
+        np.testing.assert_allclose(g12[k], 0.5 * g1[k] + 2.0 * g2[k], rtol=1e-11, atol=1e-12)
