@@ -379,7 +379,9 @@ int ssd_oracle_gated_rmsnorm(const float *y, const float *z, const float *weight
  *   dz_t    = ddt_t softplus'(z_t) [dt_lo <= softplus(z_t) <= dt_hi]
  *   G       = a_t G                             (S_t = a_t S_{t-1} + ...)
  * and dinit = G after token 0.  dz_t is the gradient of dt_raw[t] and, summed
- * over tokens, of dt_bias.  Per head: dB_h/dC_h [b,L,H,N] (the caller sums the
+ * over tokens, of dt_bias.  Packed rows (seq_idx given): at a document start
+ * the state is zeroed before the update, so S_{t-1} reads as zero there (no
+ * decay term) and no gradient passes to earlier tokens (G = 0 after it).  Per head: dB_h/dC_h [b,L,H,N] (the caller sums the
  * heads of each group), dA_h/ddt_bias_h/dD_h [b,H] (the caller sums over b).
  * The states S_t are recomputed forward from checkpoints every kSeg tokens,
  * which changes no arithmetic (the same products in the same order).
@@ -388,6 +390,7 @@ int ssd_oracle_gated_rmsnorm(const float *y, const float *z, const float *weight
 
 typedef struct {
     const float *x, *dt_raw, *dt_bias, *A, *B, *C, *D, *init_state, *dy, *dfinal;
+    const int32_t *seq_idx;   /* [b, L] or NULL */
     double *dx, *ddt_raw, *dB_h, *dC_h, *dA_h, *ddt_bias_h, *dD_h, *dinit;
     int64_t b, L, H, P, N, G;
     double dt_lo, dt_hi;
@@ -402,6 +405,12 @@ static double sigmoid_exact(double z)
     return z >= 0.0 ? 1.0 / (1.0 + exp(-z)) : exp(z) / (1.0 + exp(z));
 }
 
+/* 1 when token t of row bi starts a document of a packed row */
+static int doc_start(const bwd_job *J, int64_t bi, int64_t t)
+{
+    return J->seq_idx && t > 0 && J->seq_idx[bi * J->L + t] != J->seq_idx[bi * J->L + t - 1];
+}
+
 /* forward update of S by token t of chain (bi, h) */
 static void fwd_token(const bwd_job *J, int64_t bi, int64_t h, int64_t t, double *S, double *dt_out,
                       double *a_out)
@@ -413,6 +422,7 @@ static void fwd_token(const bwd_job *J, int64_t bi, int64_t h, int64_t t, double
     const float *xr = J->x + ((bi * L + t) * H + h) * P;
     const float *Br = J->B + ((bi * L + t) * G + g) * N;
     int64_t n, p;
+    if (doc_start(J, bi, t)) memset(S, 0, sizeof(double) * (size_t)(N * P));    /* a new document */
     for (n = 0; n < N; ++n) {
         const double w = dt * (double)Br[n];
         for (p = 0; p < P; ++p) S[n * P + p] = a * S[n * P + p] + w * (double)xr[p];
@@ -456,6 +466,7 @@ static void bwd_chain(bwd_job *J, int64_t bi, int64_t h, double *ck, double *seg
         }
         for (t = t1 - 1; t >= t0; --t) {
             const double *Scur = seg + (t - t0 + 1) * NP, *Sprev = seg + (t - t0) * NP;
+            const int start = doc_start(J, bi, t);
             const double dtt = dts[t - t0], at = as[t - t0];
             const float *xr = J->x + ((bi * L + t) * H + h) * P;
             const float *Br = J->B + ((bi * L + t) * G + g) * N;
@@ -486,13 +497,14 @@ static void bwd_chain(bwd_job *J, int64_t bi, int64_t h, double *ck, double *seg
                 dBr[n] = dtt * acc;
                 bgx += (double)Br[n] * acc;
             }
-            for (i = 0; i < NP; ++i) gs += Gm[i] * Sprev[i];
+            if (!start)
+                for (i = 0; i < NP; ++i) gs += Gm[i] * Sprev[i];
             for (p = 0; p < P; ++p) dD += (double)dyr[p] * (double)xr[p];
             dA += dtt * at * gs;
             dz = (bgx + A * at * gs) * ((sp >= J->dt_lo && sp <= J->dt_hi) ? sigmoid_exact(z) : 0.0);
             J->ddt_raw[(bi * L + t) * H + h] = dz;
             dbias += dz;
-            for (i = 0; i < NP; ++i) Gm[i] *= at;
+            for (i = 0; i < NP; ++i) Gm[i] = start ? 0.0 : Gm[i] * at;
         }
     }
     memcpy(J->dinit + (bi * H + h) * NP, Gm, sizeof(double) * (size_t)NP);
@@ -526,24 +538,24 @@ static void *bwd_worker(void *arg)
     return NULL;
 }
 
-/* Gradients of <dy, y> + <dfinal, final_state> for the whole-sequence scan
- * (no packing).  dy [b,L,H,P] and dfinal [b,H,N,P] (may be NULL) are float32
+/* Gradients of <dy, y> + <dfinal, final_state> for the whole-sequence scan,
+ * over packed rows when seq_idx [b, L] (document ids) is not NULL.  dy [b,L,H,P] and dfinal [b,H,N,P] (may be NULL) are float32
  * as given to the GPU; outputs are double: dx [b,L,H,P], ddt_raw [b,L,H],
  * dB_h, dC_h [b,L,H,N] (per head), dA_h, ddt_bias_h, dD_h [b,H] (per chain),
  * dinit [b,H,N,P].  Returns 0, -1 on bad dimensions, -2 when out of memory. */
-int ssd_oracle_scan_bwd(const float *x, const float *dt_raw, const float *dt_bias, const float *A,
-                        const float *B, const float *C, const float *D, const float *init_state,
-                        const float *dy, const float *dfinal, double *dx, double *ddt_raw, double *dB_h,
-                        double *dC_h, double *dA_h, double *ddt_bias_h, double *dD_h, double *dinit,
-                        int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, double dt_lo,
-                        double dt_hi, int nthreads)
+int ssd_oracle_scan_bwd_varlen(const float *x, const float *dt_raw, const float *dt_bias, const float *A,
+                               const float *B, const float *C, const float *D, const float *init_state,
+                               const int32_t *seq_idx, const float *dy, const float *dfinal, double *dx,
+                               double *ddt_raw, double *dB_h, double *dC_h, double *dA_h, double *ddt_bias_h,
+                               double *dD_h, double *dinit, int64_t b, int64_t L, int64_t H, int64_t P, int64_t N,
+                               int64_t G, double dt_lo, double dt_hi, int nthreads)
 {
     bwd_job J;
     if (b < 0 || L < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0) return -1;
     if (b == 0) return 0;
     memset(&J, 0, sizeof J);
     J.x = x; J.dt_raw = dt_raw; J.dt_bias = dt_bias; J.A = A; J.B = B; J.C = C; J.D = D;
-    J.init_state = init_state; J.dy = dy; J.dfinal = dfinal;
+    J.init_state = init_state; J.dy = dy; J.dfinal = dfinal; J.seq_idx = seq_idx;
     J.dx = dx; J.ddt_raw = ddt_raw; J.dB_h = dB_h; J.dC_h = dC_h;
     J.dA_h = dA_h; J.ddt_bias_h = ddt_bias_h; J.dD_h = dD_h; J.dinit = dinit;
     J.b = b; J.L = L; J.H = H; J.P = P; J.N = N; J.G = G;
@@ -552,4 +564,17 @@ int ssd_oracle_scan_bwd(const float *x, const float *dt_raw, const float *dt_bia
     run_threads(bwd_worker, &J, pick_threads(nthreads, b * H));
     pthread_mutex_destroy(&J.lock);
     return J.status;
+}
+
+/* ssd_oracle_scan_bwd_varlen without packing. */
+int ssd_oracle_scan_bwd(const float *x, const float *dt_raw, const float *dt_bias, const float *A,
+                        const float *B, const float *C, const float *D, const float *init_state,
+                        const float *dy, const float *dfinal, double *dx, double *ddt_raw, double *dB_h,
+                        double *dC_h, double *dA_h, double *ddt_bias_h, double *dD_h, double *dinit,
+                        int64_t b, int64_t L, int64_t H, int64_t P, int64_t N, int64_t G, double dt_lo,
+                        double dt_hi, int nthreads)
+{
+    return ssd_oracle_scan_bwd_varlen(x, dt_raw, dt_bias, A, B, C, D, init_state, NULL, dy, dfinal, dx, ddt_raw,
+                                      dB_h, dC_h, dA_h, ddt_bias_h, dD_h, dinit, b, L, H, P, N, G, dt_lo, dt_hi,
+                                      nthreads);
 }

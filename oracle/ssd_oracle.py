@@ -68,6 +68,9 @@ def _load():
         lib.ssd_oracle_scan_bwd.restype = ctypes.c_int
         lib.ssd_oracle_scan_bwd.argtypes = [f32p] * 10 + [f64p] * 8 + [i64] * 6 + [
             ctypes.c_double, ctypes.c_double, ctypes.c_int]
+        lib.ssd_oracle_scan_bwd_varlen.restype = ctypes.c_int
+        lib.ssd_oracle_scan_bwd_varlen.argtypes = [f32p] * 8 + [i32p] + [f32p] * 2 + [f64p] * 8 + [i64] * 6 + [
+            ctypes.c_double, ctypes.c_double, ctypes.c_int]
         lib.ssd_oracle_softplus.restype = ctypes.c_double
         lib.ssd_oracle_softplus.argtypes = [ctypes.c_double]
         _lib = lib
@@ -198,9 +201,10 @@ def scan_varlen(x, dt_raw, dt_bias, A, B, C, D, seq_idx, chunk_size: int = 1, in
 
 
 def scan_bwd(x, dt_raw, dt_bias, A, B, C, D, dy, dfinal=None, init_state=None,
-             dt_limit: Tuple[float, float] = (0.0, float("inf")), nthreads: int = 0) -> dict:
-    """Gradients of <dy, y> + <dfinal, final_state> for scan() (reverse mode
-    of the recurrence; see ssd_oracle.c).  dy [b,L,H,P], dfinal [b,H,N,P] or
+             dt_limit: Tuple[float, float] = (0.0, float("inf")), nthreads: int = 0, seq_idx=None) -> dict:
+    """Gradients of <dy, y> + <dfinal, final_state> for scan(), or for
+    scan_varlen() when seq_idx [b, L] is given (reverse mode of the
+    recurrence; see ssd_oracle.c).  dy [b,L,H,P], dfinal [b,H,N,P] or
     None (zeros).  Returns float64 arrays keyed by input: x, dt_raw [b,L,H],
     dt_bias, A, D [H], B, C [b,L,G,N] (the heads of each group summed),
     init_state [b,H,N,P] (always, also when init_state is None)."""
@@ -223,9 +227,16 @@ def scan_bwd(x, dt_raw, dt_bias, A, B, C, D, dy, dfinal=None, init_state=None,
         "A_h": np.zeros((b, H)), "dt_bias_h": np.zeros((b, H)), "D_h": np.zeros((b, H)),
         "init_state": np.zeros((b, H, N, P)),
     }
-    rc = _load().ssd_oracle_scan_bwd(
+    si = None
+    if seq_idx is not None:
+        si = np.ascontiguousarray(np.asarray(seq_idx, dtype=np.int32))
+        if si.shape != (b, L):
+            raise ValueError("oracle.scan_bwd: seq_idx must be [b, L]")
+    rc = _load().ssd_oracle_scan_bwd_varlen(
         _p32(x), _p32(dt_raw), _p32(dt_bias), _p32(A), _p32(B), _p32(C), _p32(D),
-        _p32(s0) if s0 is not None else null, _p32(dy), _p32(df) if df is not None else null,
+        _p32(s0) if s0 is not None else null,
+        si.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if si is not None else ctypes.POINTER(ctypes.c_int32)(),
+        _p32(dy), _p32(df) if df is not None else null,
         _p64(out["x"]), _p64(out["dt_raw"]), _p64(out["B_h"]), _p64(out["C_h"]), _p64(out["A_h"]),
         _p64(out["dt_bias_h"]), _p64(out["D_h"]), _p64(out["init_state"]), b, L, H, P, N, G,
         float(dt_limit[0]), float(dt_limit[1]), int(nthreads))

@@ -185,3 +185,87 @@ def test_gradients_are_linear_in_the_seeds():
     g12 = grads(inp, dy12, df12, lim)
     for k in NAMES:
         np.testing.assert_allclose(g12[k], 0.5 * g1[k] + 2.0 * g2[k], rtol=1e-11, atol=1e-12)
+
+
+# ---- packed rows: seq_idx document ids, the state zeroed at every start
+
+def packed_ids(b, L, seed):
+    rng = np.random.default_rng(seed)
+    ids = np.zeros((b, L), np.int32)
+    for bi in range(b):
+        cuts = np.sort(rng.choice(np.arange(1, L), size=4, replace=False))
+        cuts[1] = cuts[0] + 1                 # a one-token document
+        ids[bi] = np.searchsorted(cuts, np.arange(L), side="right")
+    return ids
+
+
+def loss_varlen(inp, dy, dfinal, ids):
+    y, fs, _ = oracle.scan_varlen(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                  ids, init_state=inp["init_state"])
+    return float(np.sum(y * dy.astype(np.float64)) + np.sum(fs * dfinal.astype(np.float64)))
+
+
+def grads_varlen(inp, dy, dfinal, ids):
+    return oracle.scan_bwd(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"], dy,
+                           dfinal=dfinal, init_state=inp["init_state"], seq_idx=ids)
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_packed_directional_finite_difference(name):
+    inp, dy, dfinal = make(2, 60, 4, 3, 5, 2, seed=41)
+    ids = packed_ids(2, 60, seed=42)
+    g = grads_varlen(inp, dy, dfinal, ids)
+    v = np.random.default_rng(300 + NAMES.index(name)).standard_normal(inp[name].shape)
+    eps = 1e-3 if name in ("x", "B", "C", "D", "init_state") else 1e-4
+    base = inp[name].astype(np.float64)
+    plus, minus = dict(inp), dict(inp)
+    plus[name] = (base + eps * v).astype(np.float32)
+    minus[name] = (base - eps * v).astype(np.float32)
+    delta = plus[name].astype(np.float64) - minus[name].astype(np.float64)
+    fd = loss_varlen(plus, dy, dfinal, ids) - loss_varlen(minus, dy, dfinal, ids)
+    pred = float(np.sum(g[name] * delta))
+    assert abs(fd - pred) <= 1e-6 * max(abs(pred), 1e-3 * float(np.sum(np.abs(g[name] * delta)))), (fd, pred)
+
+
+def separate_documents(inp, dy, dfinal, ids):
+    """The packed row's gradients assembled from each document's own
+    backward: the first document starts from init_state, the others from
+    zeros; only the last one's final state is the row's (dfinal seeds it)."""
+    b, L, H, P = inp["x"].shape
+    out = {"x": np.zeros((b, L, H, P)), "dt_raw": np.zeros((b, L, H)), "B": np.zeros(inp["B"].shape),
+           "C": np.zeros(inp["C"].shape), "A": np.zeros(H), "dt_bias": np.zeros(H), "D": np.zeros(H),
+           "init_state": np.zeros(inp["init_state"].shape)}
+    for bi in range(b):
+        starts = [0] + [t for t in range(1, L) if ids[bi, t] != ids[bi, t - 1]] + [L]
+        for k in range(len(starts) - 1):
+            t0, t1 = starts[k], starts[k + 1]
+            doc = {n: (inp[n][bi:bi + 1, t0:t1] if n in ("x", "dt_raw", "B", "C") else inp[n])
+                   for n in ("x", "dt_raw", "B", "C", "dt_bias", "A", "D")}
+            s0 = inp["init_state"][bi:bi + 1] if k == 0 else None
+            seed = dfinal[bi:bi + 1] if t1 == L else np.zeros_like(dfinal[bi:bi + 1])
+            g = oracle.scan_bwd(doc["x"], doc["dt_raw"], doc["dt_bias"], doc["A"], doc["B"], doc["C"], doc["D"],
+                                dy[bi:bi + 1, t0:t1], dfinal=seed, init_state=s0)
+            for n in ("x", "dt_raw", "B", "C"):
+                out[n][bi, t0:t1] = g[n][0]
+            for n in ("A", "dt_bias", "D"):
+                out[n] += g[n]
+            if k == 0:
+                out["init_state"][bi] = g["init_state"][0]
+    return out
+
+
+def test_packed_row_gradients_are_its_documents_gradients():
+    inp, dy, dfinal = make(2, 60, 4, 3, 5, 2, seed=43)
+    ids = packed_ids(2, 60, seed=44)
+    g = grads_varlen(inp, dy, dfinal, ids)
+    ref = separate_documents(inp, dy, dfinal, ids)
+    for n in NAMES:
+        np.testing.assert_allclose(g[n], ref[n], rtol=1e-12, atol=1e-13, err_msg=n)
+
+
+def test_one_document_is_the_plain_backward():
+    inp, dy, dfinal = make(1, 40, 2, 3, 4, 1, seed=45)
+    g = grads_varlen(inp, dy, dfinal, np.full((1, 40), 7, np.int32))
+    ref = grads(inp, dy, dfinal, (0.0, float("inf")))
+    for n in NAMES:
+        assert np.array_equal(g[n], ref[n]), n

@@ -88,7 +88,7 @@ def test_unmutated_copy_passes(tmp_path):
 # ---- the backward oracle: each planted mistake must fail the finite-difference pin
 BWD_MUTANTS = {
     "bwd_drop_D": ("dxr[p] = dtt * acc + Dh * (double)dyr[p];", "dxr[p] = dtt * acc;"),
-    "bwd_no_decay_carry": ("for (i = 0; i < NP; ++i) Gm[i] *= at;", "for (i = 0; i < NP; ++i) Gm[i] *= 1.0;"),
+    "bwd_no_decay_carry": ("Gm[i] = start ? 0.0 : Gm[i] * at;", "Gm[i] = start ? 0.0 : Gm[i] * 1.0;"),
     "bwd_dA_no_dt": ("dA += dtt * at * gs;", "dA += at * gs;"),
     "bwd_ddt_no_A": ("dz = (bgx + A * at * gs)", "dz = (bgx + at * gs)"),
     "bwd_dC_previous_state": ("acc += Scur[n * P + p] * (double)dyr[p];", "acc += Sprev[n * P + p] * (double)dyr[p];"),
@@ -161,3 +161,31 @@ def test_backward_unmutated_copy_passes(tmp_path):
     so = _build(tmp_path, "bwd_clean", "#define kSeg 64", "#define kSeg 64")
     inp, dy, dfinal = make(1, 70, 4, 3, 5, 2, seed=31)
     assert _fd_misses(_bwd_with(so, inp, dy, dfinal), inp, dy, dfinal) == []
+
+
+PACKED_BWD_MUTANTS = {
+    "bwd_gradient_crosses_start": ("Gm[i] = start ? 0.0 : Gm[i] * at;", "Gm[i] = Gm[i] * at;"),
+    "bwd_decay_term_at_start": ("            if (!start)\n                for (i = 0; i < NP; ++i) gs",
+                                "            if (1)\n                for (i = 0; i < NP; ++i) gs"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PACKED_BWD_MUTANTS))
+def test_packed_backward_pin_rejects_planted_mistake(tmp_path, name, monkeypatch):
+    """The separate-documents pin sees a backward that lets a gradient or a
+    decay term cross a document start."""
+    import oracle
+    from oracle import ssd_oracle
+    from test_oracle_bwd import make, packed_ids, separate_documents
+    old, new = PACKED_BWD_MUTANTS[name]
+    so = _build(tmp_path, name, old, new)
+    inp, dy, dfinal = make(2, 60, 4, 3, 5, 2, seed=43)
+    ids = packed_ids(2, 60, seed=44)
+    ref = separate_documents(inp, dy, dfinal, ids)       # the clean oracle's per-document runs
+    monkeypatch.setattr(ssd_oracle, "_lib", None)
+    monkeypatch.setattr(ssd_oracle, "build_oracle", lambda force=False: so)
+    g = oracle.scan_bwd(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"], dy,
+                        dfinal=dfinal, init_state=inp["init_state"], seq_idx=ids)
+    monkeypatch.setattr(ssd_oracle, "_lib", None)
+    worst = max(float(np.max(np.abs(g[n] - ref[n])) / (np.sqrt(np.mean(ref[n] ** 2)) + 1e-300)) for n in ref)
+    assert worst > 1e-6, "planted mistake went unnoticed"
