@@ -211,3 +211,18 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         ssd.chunk_scan_fwd(x, torch.zeros(1, 4, 2), torch.zeros(2), torch.zeros(2), torch.zeros(1, 4, 1, 16),
                            torch.zeros(1, 4, 1, 16), torch.zeros(2), chunk_size=4)
+
+
+def test_backward_workspace_holds_per_head_buffers_only_when_groups_are_shared(lib):
+    """With G < H the pair kernels write per-head dB, dC ([b, L, H, N] f32
+    each) that a last launch sums per group; with G = H they write dB, dC
+    directly and the workspace has no room for them."""
+    sz = ctypes.c_size_t(0)
+
+    def ws(G):
+        assert lib.ssd_chunk_scan_bwd_workspace_size(2, 300, 4, 64, 128, G, 64, 1, ctypes.byref(sz)) == 0
+        return sz.value
+
+    per_head = 2 * 2 * 300 * 4 * 128 * 4
+    assert ws(2) - ws(4) >= per_head
+    assert ws(1) == ws(2)
