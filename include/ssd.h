@@ -301,7 +301,8 @@ SSD_API ssd_status ssd_trace_read(int kernel, int *launches, double *total_ms);
 SSD_API const char *ssd_trace_kernel_name(int kernel);
 SSD_API int ssd_trace_kernel_count(void);
 
-/* ABI version: (major << 16) | minor. */
+/* ABI version: (major << 16) | minor.  1.1 added the chunk-state, packed-row,
+ * conv/norm and backward entry points to the 1.0 scan and step. */
 SSD_API int ssd_version(void);
 
 #ifdef __cplusplus

@@ -83,7 +83,7 @@ size_t path_ws(const ssd::ScanDims &d, int chosen) {
 
 extern "C" {
 
-int ssd_version(void) { return (1 << 16) | 0; }
+int ssd_version(void) { return (1 << 16) | 1; }
 
 int ssd_last_cuda_error(void) { return g_last_cuda_error; }
 
