@@ -1,7 +1,13 @@
 #!/usr/bin/env python
 """Throughput of the B200 SSD scan (and decode step) on synthetic workloads.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--also A,B] [--impl ours|reference]
+
+The headline line is the largest single-GPU scan workload (c3_long: one
+65536-token row, 80 heads in 8 groups, carried initial state); the other scan
+workloads (c1_130m, c2_2p7b) are timed in the same run and nested under
+"configs" with the same keys, the decode step under "decode" and the
+backward under "backward".
 
 A "step" is one chunked forward scan (every stage of the hot path: dt
 preparation, chunk cumsum, intra-chunk C.B^T, chunk states, state passing,
@@ -76,31 +82,33 @@ def step_bytes(cfg) -> float:
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# dominant kernel, from one ncu capture each (summaries in profiles/).  Each
-# entry names the source file of the kernel and the first 16 hex digits of its
-# sha256 at capture time: once that file changes the number no longer
-# describes the kernel and the bench reports null.
+# dominant kernel, from one ncu capture each.  Each entry names the source file
+# of the kernel and the first 16 hex digits of its sha256 at capture time: once
+# that file changes the number no longer describes the kernel and the bench
+# reports null.
 NCU_TRAFFIC = {
     ("c1_130m", "tc_chunk_out"): (35.329792e6, "state_space_sequence_scan_b200/csrc/ssd_scan_tc.cu",
-                                  "a0afdb27d5acb42a", "profiles/tc_chunk_out_c1_130m.md"),
+                                  "a0afdb27d5acb42a"),
     ("c4_decode", "decode_step"): (1291.7568e6, "state_space_sequence_scan_b200/csrc/ssd_step.cu",
-                                   "a5f3c2cec738b994", "profiles/decode_step_c4_decode.md"),
+                                   "a5f3c2cec738b994"),
 }
 
 
 def measured_traffic(workload, kernel):
-    """(bytes per launch, summary file) if the capture still describes the kernel, else (None, None)."""
+    """(bytes per launch, description) if the capture still describes the kernel, else (None, None)."""
     import hashlib
     e = NCU_TRAFFIC.get((workload, kernel))
     if e is None:
         return None, None
-    nbytes, src, digest, summary = e
+    nbytes, src, digest = e
     try:
         with open(os.path.join(ROOT, src), "rb") as f:
             cur = hashlib.sha256(f.read()).hexdigest()[:16]
     except OSError:
         return None, None
-    return (nbytes, summary) if cur == digest else (None, None)
+    if cur != digest:
+        return None, None
+    return nbytes, "ncu capture of %s on %s (source sha256 %s)" % (kernel, workload, digest)
 
 
 def load_peaks():
@@ -782,12 +790,18 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c1_130m")
+    ap.add_argument("--workload", default="c3_long",
+                    help="the headline workload (default: the largest single-GPU scan, c3_long)")
+    ap.add_argument("--also", default="c1_130m,c2_2p7b",
+                    help="comma-separated scan workloads timed in the same run and nested in the line "
+                         "under 'configs' ('none' for none)")
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
     ap.add_argument("--no-decode", action="store_true", help="skip the decode figure on the scan line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="leave the backward (ssd_chunk_scan_bwd) line out of the default scan run")
+    ap.add_argument("--backward-workload", default="c1_130m",
+                    help="the workload of the nested backward line")
     ap.add_argument("--chunk-states", action="store_true",
                     help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
     ap.add_argument("--packed", action="store_true",
@@ -818,6 +832,27 @@ def main():
         else:
             r = bench_scan(cfg, args, ws, rank, local)
         out = finish(cfg, is_step, r, args, ws, rank, peaks, peak_kind)
+        del r
+        torch.cuda.empty_cache()
+        if not is_step:
+            # the other scan workloads, each a full record nested under "configs"
+            extra = [w for w in args.also.split(",") if w and w != "none" and w != cfg.name]
+            nested = {}
+            for wname in extra:
+                wcfg, wstep = pick(wname)
+                if wstep:
+                    continue
+                wr = bench_scan(wcfg, args, ws, rank, local)
+                line = finish(wcfg, False, wr, args, ws, rank, peaks, peak_kind, sub=True)
+                del wr
+                torch.cuda.empty_cache()
+                if line is not None:
+                    if ws == 1 and not args.no_cpu_baseline:
+                        cb = cpu_baseline_scan(wcfg, budget_s=5.0)
+                        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+                    nested[wname] = line
+            if out is not None and nested:
+                out["configs"] = nested
         if not is_step and not args.no_decode:
             dcfg = STEP_CONFIGS["c4_decode"]
             dr = bench_step(dcfg, args, ws, rank, local)
@@ -825,7 +860,8 @@ def main():
             if out is not None:
                 out["decode"] = dline
         if not is_step and ws == 1 and not args.no_backward and out is not None:
-            out["backward"] = bench_backward(cfg, args, local, peaks, peak_kind)
+            bcfg, _ = pick(args.backward_workload)
+            out["backward"] = bench_backward(bcfg, args, local, peaks, peak_kind)
         if rank == 0 and out is not None:
             if ws == 1 and not args.no_cpu_baseline:
                 cb = cpu_baseline_step(cfg) if is_step else cpu_baseline_scan(cfg)

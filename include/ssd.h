@@ -166,7 +166,10 @@ SSD_API ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_
  *   - It never calls cudaMalloc, cudaFree or any allocating routine.
  *   - The first call on each device looks the array's device address up
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept per device index and
+ *     holds for the device's primary context, the one the CUDA runtime and
+ *     PyTorch use: after cudaDeviceReset, or from a context made current
+ *     through the driver API, it no longer names the array.
  *   - Every call shares the one array and it keeps the last call's contents
  *     (each call clears the part that must start at zero).  Calls whose work
  *     overlaps on the GPU -- two streams, or two host threads -- race on it;

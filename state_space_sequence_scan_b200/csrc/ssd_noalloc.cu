@@ -8,7 +8,9 @@
 // Every GPU that loads this library holds it until the process exits.  In
 // host code its name is only a host-side stand-in, not a device address: the
 // device address is looked up once per device with cudaGetSymbolAddress and
-// that pointer is what the kernels receive.
+// that pointer is what the kernels receive.  The cached address belongs to the
+// device's primary context (the runtime's); a cudaDeviceReset or a context
+// made current through the driver API invalidates it.
 #include <mutex>
 
 #include "../../include/ssd.h"
