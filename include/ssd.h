@@ -304,8 +304,19 @@ SSD_API ssd_status ssd_trace_read(int kernel, int *launches, double *total_ms);
 SSD_API const char *ssd_trace_kernel_name(int kernel);
 SSD_API int ssd_trace_kernel_count(void);
 
+/* TEST ONLY: makes the device-side timeout path run, without any fault.
+ * kind 1: from the next tensor-path scan call on, the chunk-output kernel
+ * never requests its first C and B tiles, and every bounded
+ * wait gives up after about 2^21 clock cycles instead of 2^32.  The call
+ * then completes, the CTAs drain the copies and MMAs they issued, release
+ * their tensor memory and return, and ssd_read_device_status() reports
+ * SSD_ERR_DEVICE_TIMEOUT; the outputs are undefined.  kind 0 restores
+ * normal operation.  Not for production use; affects every host thread. */
+SSD_API ssd_status ssd_set_test_fault(int kind);
+
 /* ABI version: (major << 16) | minor.  1.1 added the chunk-state, packed-row,
- * conv/norm and backward entry points to the 1.0 scan and step. */
+ * conv/norm and backward entry points to the 1.0 scan and step; 1.2 the test
+ * hook ssd_set_test_fault. */
 SSD_API int ssd_version(void);
 
 #ifdef __cplusplus

@@ -83,7 +83,13 @@ size_t path_ws(const ssd::ScanDims &d, int chosen) {
 
 extern "C" {
 
-int ssd_version(void) { return (1 << 16) | 1; }
+int ssd_version(void) { return (1 << 16) | 2; }
+
+ssd_status ssd_set_test_fault(int kind) {
+    if (kind != 0 && kind != 1) return SSD_ERR_INVALID_ARG;
+    ssd::tc_set_test_fault(kind);
+    return SSD_OK;
+}
 
 int ssd_last_cuda_error(void) { return g_last_cuda_error; }
 

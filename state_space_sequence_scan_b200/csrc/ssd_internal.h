@@ -72,6 +72,11 @@ cudaError_t bwd_scan(const BwdArgs &a, const ScanDims &d, void *workspace, cudaS
 bool tc_supported(const ScanDims &d, int bf16);
 size_t tc_workspace_bytes(const ScanDims &d);
 cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
+// Test hook for the device-side timeout path (ssd_set_test_fault): 0 = off;
+// 1 = the tensor-path chunk-output kernel never requests its first C and B
+// tiles and its waits give up after about a millisecond.
+void tc_set_test_fault(int kind);
+int tc_test_fault();
 
 // ---- decode step ------------------------------------------------------------
 bool step_supported(int64_t P, int64_t N);

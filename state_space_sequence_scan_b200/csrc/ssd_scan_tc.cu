@@ -1,11 +1,15 @@
 // Chunked SSD forward scan on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // Scope: bf16 x/B/C, state_dim N = 128, head_dim P = 64, fp32 dt/A/D/state,
-// fp32 y.  Every contraction runs as a kind::f16 MMA with fp16 operands and
-// fp32 accumulation in TMEM.  bf16 -> fp16 is exact for inputs within fp16
-// range; the decay-weighted operands are formed in fp16, whose 11-bit
-// significand the 2e-2 bar needs (bf16's 8 bits are not enough).  Tiles
-// arrive by TMA already in the 128-byte-swizzled operand layout.
+// fp32 y.  Every contraction runs as a kind::f16 MMA with fp32 accumulation
+// in TMEM.  C.B^T, the state terms B^T (w x) and C H take fp16 operands
+// (bf16 -> fp16 is exact for inputs within fp16 range; the decay-weighted
+// w x and the carried state need fp16's 11-bit significand, bf16's 8 bits
+// are not enough).  W.X takes the x tile as the TMA delivers it (bf16) and
+// the decay-weighted W as a bf16 high/low pair (two MMAs, about 16
+// significant bits): y is heavy-tailed and its largest elements are single
+// W.X terms, whose fp16 rounding alone exceeds the 2e-2 bar.  Tiles arrive by
+// TMA already in the 128-byte-swizzled operand layout.
 //
 // The sequence of every (batch, head) is cut into 128-token blocks (the MMA
 // M extent) and the blocks into `units` of consecutive blocks.  Four
@@ -44,6 +48,8 @@
 // both factors <= 1, so W there costs two multiplies instead of an exp.
 #include <stdint.h>
 
+#include <atomic>
+
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
 #include "ssd_tc.cuh"
@@ -60,6 +66,7 @@ constexpr int kN = 128;                         // state_dim
 constexpr int kP = 64;                          // head_dim
 constexpr int kNP = kN * kP;
 constexpr long long kWaitBudget = 1ll << 32;    // clock cycles before a wait gives up (~2 s)
+constexpr long long kTestWaitBudget = 1ll << 21;  // the same under the test fault (~1 ms)
 constexpr float kF16Max = 65504.0f;
 constexpr int kSMs = 148;                       // B200 streaming multiprocessors
 // Relative cost of the unit decomposition, in chunk_out block-times (one
@@ -71,6 +78,7 @@ constexpr double kUnitStateRel = 0.35;
 constexpr double kStatePassRel = 5.0;
 constexpr double kCtaStartRel = 2.0;
 constexpr int64_t kMaxUnits = 4096;
+constexpr int kMaxAttrDevices = 64;
 constexpr uint32_t kTileBytes = 16384;          // one 128-row x 128-byte swizzled tile
 
 struct TcWs {
@@ -202,11 +210,6 @@ __device__ __forceinline__ bool in_f16_range(__half2 hmax) {
 __device__ __forceinline__ void bf16_chunk_to_f32(uint4 v, float *f) {
     f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
     f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
-}
-
-__device__ __forceinline__ void f16_chunk_to_f32(uint4 v, float *f) {
-    const float2 a0 = unpack_h2(v.x), a1 = unpack_h2(v.y), a2 = unpack_h2(v.z), a3 = unpack_h2(v.w);
-    f[0] = a0.x; f[1] = a0.y; f[2] = a1.x; f[3] = a1.y; f[4] = a2.x; f[5] = a2.y; f[6] = a3.x; f[7] = a3.y;
 }
 
 // ---------------------------------------------------------------------------
@@ -530,9 +533,10 @@ tc_state_pass_kernel(TcWs ws, const float *__restrict__ init, int H, int U) {
 // every bulk copy; both only wait on mbarriers, so the compute warps never
 // stall on an issue (a tcgen05.mma holds its issuing thread for about as
 // long as it runs).  Per 128-token block k the compute warps run:
-//   [1] C.B^T(k) done -> W(k) into TMEM (fp16, the A operand of W.X)
-//                                     -> MMA: Y(k) = W(k) X(k), then C.B^T(k+1)
-//   [2] x/dt/cum(k+1) landed -> decay factors, X(k+1) widened in place
+//   [1] C.B^T(k) done -> W(k) into TMEM (bf16 high and low parts, the A
+//       operands of W.X)              -> MMA: Y(k) = W_hi(k) X(k) + W_lo(k) X(k),
+//                                        then C.B^T(k+1)
+//   [2] x/dt/cum(k+1) landed -> decay factors of block k+1
 //   [3] S(k), Z(k) done -> H_in(k+1) = a_k H_in(k) + S(k) in registers, its
 //       fp16 copy, and w.X(k+1)       -> MMA: Z(k+1) = C(k+1) H_in(k+1) and
 //                                        S(k+1) = B^T (w.X(k+1))
@@ -569,10 +573,11 @@ static_assert(kCoSmem <= 232448, "chunk_out shared memory exceeds the per-CTA li
 
 // TMEM columns (512 allocated)
 constexpr uint32_t kTmCB = 0;      // C.B^T fp32, 128 columns
-constexpr uint32_t kTmW = 128;     // W fp16 pairs, 64 columns
+constexpr uint32_t kTmW = 128;     // W bf16 pairs, the high part (W truncated to bf16), 64 columns
 constexpr uint32_t kTmY = 192;     // W.X fp32, 64 columns
 constexpr uint32_t kTmS = 256;     // B^T.(w.X) fp32, 64 columns
 constexpr uint32_t kTmZ = 320;     // C.H fp32, two buffers of 64 columns (block parity)
+constexpr uint32_t kTmWlo = 448;   // W bf16 pairs, the low part (W - high, rounded), 64 columns
 
 // "Block done" has one barrier per C/B stage: block k+2 cannot finish before
 // the TMA warp has seen block k finish and loaded k+2's tiles, so that waiter
@@ -669,42 +674,32 @@ __device__ __forceinline__ void co_factors(const CoSmem &S, int r, int f, int la
     if (tid < 4) S.G(f)[tid] = (cum[32 * tid] - cum[32 * tid + 31]) <= kDiagExpCap ? 1 : 0;
 }
 
-// X tile of slot r: bf16 -> fp16 in place (four 16-byte chunks per thread).
+// w.X (fp16) of the X tile of slot r (bf16, as the TMA delivered it) into
+// WX, same swizzled layout (a chunk's row is its offset / 128 whatever the
+// swizzle): products in fp32, rounded to fp16 once.  Packed rows: tokens
+// before the block's last document start (rs_last; -1 for none) write nothing
+// into the state the block passes on.
 //
-// chunk_out tracks no fp16 range per operand: a value beyond +-65504 in any
-// fp16 operand it forms (X, W, w.X, the entering state) rounds to inf, and
-// every such operand reaches y or the final state through a product and a
-// sum, where inf stays inf or turns NaN (inf * 0).  One finiteness check on
-// y and the final state (co_nonfinite) therefore reports it, off the W path.
-__device__ __forceinline__ void co_widen_x(const CoSmem &S, int r, int tid) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 *p = reinterpret_cast<uint4 *>(S.X(r) + (tid + q * kCoCompute) * 16);
-        float f[8];
-        bf16_chunk_to_f32(*p, f);
-        *p = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
-    }
-}
-
-// w.X (fp16) of the widened X tile of slot r into WX, same swizzled layout (a
-// chunk's row is its offset / 128 whatever the swizzle).  Packed fp16
-// products: w_j is rounded to fp16 once (w_j <= dt_j; one below the fp16
-// normal range only adds an absolute error under 3e-8 |x|), and no element
-// goes through fp32.  Packed rows: tokens before the block's last document
-// start (rs_last; -1 for none) write nothing into the state the block passes on.
+// chunk_out tracks no fp16 range per operand: a value beyond +-65504 in an
+// fp16 operand it forms (w.X, the entering state) rounds to inf, and each
+// reaches y or the final state through a product and a sum, where inf stays
+// inf or turns NaN (inf * 0).  One finiteness check on y and the final state
+// (co_nonfinite) therefore reports it, off the W path.  W itself is carried
+// in bf16 (hi/lo), which cannot overflow.
 __device__ __forceinline__ void co_form_wx(const CoSmem &S, int r, int f, int tid, int rs_last) {
     const float *w = S.F(f);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int c = tid + q * kCoCompute;
-        const uint4 xv = *reinterpret_cast<const uint4 *>(S.X(r) + c * 16);
-        const __half2 wj = __float2half2_rn((c >> 3) >= rs_last ? w[c >> 3] : 0.f);
-        const uint32_t xi[4] = {xv.x, xv.y, xv.z, xv.w};
+        float xv[8];
+        bf16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(r) + c * 16), xv);
+        const float wj = (c >> 3) >= rs_last ? w[c >> 3] : 0.f;
+        const float2 w2 = make_float2(wj, wj);
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const __half2 m = __hmul2(*reinterpret_cast<const __half2 *>(&xi[e]), wj);
-            o[e] = *reinterpret_cast<const uint32_t *>(&m);
+            const float2 m = __fmul2_rn(make_float2(xv[2 * e], xv[2 * e + 1]), w2);
+            o[e] = pack_h2(m.x, m.y);
         }
         *reinterpret_cast<uint4 *>(S.WX() + c * 16) = make_uint4(o[0], o[1], o[2], o[3]);
     }
@@ -741,7 +736,12 @@ __device__ __forceinline__ void co_nonfinite(const float *v, int n, float2 &acc)
         if (2 * q < n) acc = __ffma2_rn(make_float2(v[2 * q], v[2 * q + 1]), z, acc);
 }
 
-// W for one 32-column slice cq <= lg of this thread's row i (see co_factors).
+// W for one 32-column slice cq <= lg of this thread's row i (see co_factors),
+// stored as two bf16 pairs per column: the high part (W truncated to bf16)
+// and the low part (the rest, rounded to bf16).  Y = W_hi X + W_lo X then
+// carries W to about 16 significant bits: y is heavy-tailed (single W.X
+// terms of 50 to 60 times the output RMS), and the 11 bits of an fp16 W
+// leave those terms' rounding above the 2e-2 RMS bar.
 // Packed rows: rs_i is the last document start at or before row i in the
 // block (-1 for none); columns before it drop out of the row.
 __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32_t lane_addr, int lg, int cq,
@@ -750,7 +750,7 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
     const float *F = S.F(f);
     float v[32];
     tmem_ld32(lane_addr + kTmCB + cq * 32, v);
-    uint32_t o[16];
+    uint32_t oh[16], ol[16];                         // W as bf16 pairs: high part, low part
     if (cq < lg) {                                   // below the diagonal: pivot at row 32*lg-1
         const float ui = expf(fminf(ci - cum[32 * lg - 1], 0.f));
         const float2 u2 = make_float2(ui, ui);
@@ -761,8 +761,8 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
             const float2 m0 = __fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), __fmul2_rn(make_float2(f4.x, f4.y), u2));
             const float2 m1 =
                 __fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), __fmul2_rn(make_float2(f4.z, f4.w), u2));
-            o[2 * q] = pack_h2(m0.x, m0.y);
-            o[2 * q + 1] = pack_h2(m1.x, m1.y);
+            split_bf16x2(m0.x, m0.y, oh[2 * q], ol[2 * q]);
+            split_bf16x2(m1.x, m1.y, oh[2 * q + 1], ol[2 * q + 1]);
         }
     } else {                                         // diagonal 32x32: pivot at its last row m
         if (S.G(f)[lg]) {
@@ -791,7 +791,7 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
                 asm volatile("" ::: "memory");       // one element at a time: keeps the loads from piling up
             }
         }
-        // causal select on the packed pairs (j <= i kept)
+        // causal select on the packed pairs (j <= i kept), both parts
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
             const uint4 m4 = S.Mask()[q4 * 32 + lane];
@@ -799,17 +799,24 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int q = 4 * q4 + e;
-                o[q] = pack_h2(v[2 * q], v[2 * q + 1]) & mw[e];
+                split_bf16x2(v[2 * q], v[2 * q + 1], oh[q], ol[q]);
+                oh[q] &= mw[e];
+                ol[q] &= mw[e];
             }
         }
     }
     const int j0 = 32 * cq;
     if (rs_i > j0) {
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-            o[q] &= (j0 + 2 * q >= rs_i ? 0x0000FFFFu : 0u) | (j0 + 2 * q + 1 >= rs_i ? 0xFFFF0000u : 0u);
+        for (int q = 0; q < 16; ++q) {
+            const uint32_t keep =
+                (j0 + 2 * q >= rs_i ? 0x0000FFFFu : 0u) | (j0 + 2 * q + 1 >= rs_i ? 0xFFFF0000u : 0u);
+            oh[q] &= keep;
+            ol[q] &= keep;
+        }
     }
-    tmem_st16u(lane_addr + kTmW + 16 * cq, o);
+    tmem_st16u(lane_addr + kTmW + 16 * cq, oh);
+    tmem_st16u(lane_addr + kTmWlo + 16 * cq, ol);
 }
 
 // kPacked: packed rows (the document starts of ws.rs mask W, the C.H term,
@@ -819,7 +826,7 @@ __global__ void __launch_bounds__(kCoThreads, 1)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
                  const float *__restrict__ init, float *__restrict__ final_state, TcWs ws,
                  int L, int H, int G, int nblk, int U, int bpu, int states_from_ws, int prefetch_cb,
-                 float *__restrict__ chunk_states, int bpc, int nc) {
+                 float *__restrict__ chunk_states, int bpc, int nc, long long wait_budget, int test_fault) {
     extern __shared__ uint8_t smem_raw[];
     CoSmem S;
     S.base = align1024(smem_raw);
@@ -856,7 +863,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         if (lane == 0) {
             const uint32_t idesc_cb = idesc_f16(128, 128, 0, 0);  // A=C K-major, B=B K-major
             const uint32_t idesc_z = idesc_f16(128, 64, 0, 1);    // A=C K-major, B=H MN-major
-            const uint32_t idesc_y = idesc_f16(128, 64, 0, 1);    // A=W (TMEM) K-major, B=X MN-major
+            const uint32_t idesc_y = idesc_bf16(128, 64, 0, 1);   // A=W hi/lo (TMEM) bf16, B=X (bf16) MN-major
             const uint32_t idesc_s = idesc_f16(128, 64, 1, 1);    // A=B^T MN-major, B=wX MN-major
             // per-stage / per-slot descriptors are the first one's plus a byte offset
             // (no arrays: a dynamically indexed one would live in local memory)
@@ -895,14 +902,17 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     mma_f16_ts(tmem + kTmY, tmem + kTmW + 8u * q, dadd(dX0, xs(r) + q * 2048), idesc_y, q > 0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    mma_f16_ts(tmem + kTmY, tmem + kTmWlo + 8u * q, dadd(dX0, xs(r) + q * 2048), idesc_y, 1u);
                 mma_commit(S.bar(kBarY));
                 ++S.issued()[kBarY];
             };
             // "fp16 state ready" also means w.X of that block is formed
-            bool ok = mbar_wait_abortable(S.bar(kBarTcb0), 0, kWaitBudget, abort_flag);
+            bool ok = mbar_wait_abortable(S.bar(kBarTcb0), 0, wait_budget, abort_flag);
             tc_fence_after();
             if (ok) issue_cb(0);
-            ok = ok && mbar_wait_abortable(S.bar(kBarH16), 0, kWaitBudget, abort_flag);
+            ok = ok && mbar_wait_abortable(S.bar(kBarH16), 0, wait_budget, abort_flag);
             tc_fence_after();
             if (ok) {
                 issue_z(0, 0);
@@ -911,20 +921,20 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             for (int k = kb0; k < kb1 && ok; ++k) {
                 const int i = k - kb0, s1 = (i & 1) ^ 1;
                 const uint32_t par = (uint32_t)i & 1u, par1 = (uint32_t)(i + 1) & 1u;
-                ok = mbar_wait_abortable(S.bar(kBarW), par, kWaitBudget, abort_flag);
+                ok = mbar_wait_abortable(S.bar(kBarW), par, wait_budget, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 issue_y(i % kCoXSlots);
                 if (k + 1 < kb1) {
                     // C.B^T(k+1) once its tiles have landed (W(k) has read C.B^T(k))
-                    ok = mbar_wait_abortable(S.bar(kBarTcb0 + s1), ((uint32_t)(i + 1) >> 1) & 1u, kWaitBudget,
+                    ok = mbar_wait_abortable(S.bar(kBarTcb0 + s1), ((uint32_t)(i + 1) >> 1) & 1u, wait_budget,
                                              abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     issue_cb(s1);
                     // Z(k+1), S(k+1) once the fp16 state and w.X of k+1 are formed (S(k)
                     // and Z(k) have been read by then)
-                    ok = mbar_wait_abortable(S.bar(kBarH16), par1, kWaitBudget, abort_flag);
+                    ok = mbar_wait_abortable(S.bar(kBarH16), par1, wait_budget, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     issue_z(s1, (int)par1);
@@ -937,12 +947,15 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
     } else if (warp == kCoTmaWarp) {
         // ------------------------------ TMA warp ------------------------------
         if (lane == 0) {
-            for (int q = 0; q < 2 && kb0 + q < kb1; ++q) co_load_cb(S, maps, q, kb0 + q, g, b);
+            // test_fault 1: the first C/B stage is never requested, so every wait
+            // that depends on it runs out of budget (the timeout path)
+            for (int q = 0; q < 2 && kb0 + q < kb1; ++q)
+                if (q > 0 || test_fault != 1) co_load_cb(S, maps, q, kb0 + q, g, b);
             for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q) co_load_x(S, maps, dtg, cumg, q, kb0 + q, h, b);
             if (prefetch_cb && kb0 + 2 < kb1) co_prefetch_cb(maps, kb0 + 2, g, b);
             for (int k = kb0; k < kb1; ++k) {
                 const int i = k - kb0, s = i & 1;
-                if (!mbar_wait_abortable(S.bar(kBarFree0 + s), ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag))
+                if (!mbar_wait_abortable(S.bar(kBarFree0 + s), ((uint32_t)i >> 1) & 1u, wait_budget, abort_flag))
                     break;
                 // block k is done with its x slot; its y sits in its B tiles
                 if (k + kCoXSlots < kb1) co_load_x(S, maps, dtg, cumg, i % kCoXSlots, k + kCoXSlots, h, b);
@@ -997,6 +1010,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
 #pragma unroll
                     for (int q = 0; q < 16; ++q) z[q] = 0u;
                     tmem_st16u(lane_addr + kTmW + 16 * cq, z);
+                    tmem_st16u(lane_addr + kTmWlo + 16 * cq, z);
                 }
             }
             // causal masks of a diagonal sub-block: lane l keeps columns jj <= l;
@@ -1012,12 +1026,10 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 S.Mask()[q4 * 32 + ml] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
             }
         }
-        // block kb0: x landed -> factors, widened X, w.X; then "state ready"
-        ok = mbar_wait_abortable(S.bar(kBarTx0), 0, kWaitBudget, abort_flag);
+        // block kb0: x landed -> factors, w.X; then "state ready"
+        ok = mbar_wait_abortable(S.bar(kBarTx0), 0, wait_budget, abort_flag);
         if (ok) co_factors(S, 0, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
         named_bar_sync(kCoCompute);                 // factors and masks visible to every compute warp
-        if (ok) co_widen_x(S, 0, tid);
-        named_bar_sync(kCoCompute);
         // packed rows: document starts of each block (ws.rs, written by prep)
         const int *rsb = ws.rs + (size_t)b * nblk * kBlk;
         if (ok) co_form_wx(S, 0, 0, tid, kPacked ? rsb[(size_t)kb0 * kBlk + kBlk - 1] : -1);
@@ -1036,7 +1048,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             const int rs_last1 = (kPacked && k + 1 < kb1) ? rsb[(size_t)t0 + 2 * kBlk - 1] : -1;
 
             // [1] C.B^T(k) done -> W(k) (fp16 pairs) into TMEM
-            ok = ok && mbar_wait_abortable(S.bar(kBarCB), par, kWaitBudget, abort_flag);
+            ok = ok && mbar_wait_abortable(S.bar(kBarCB), par, wait_budget, abort_flag);
             ok = __all_sync(0xffffffffu, ok);        // warp-uniform before tcgen05.ld
             tc_fence_after();
             if (ok) {
@@ -1046,18 +1058,17 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             }
             co_arrive_tmem(S.bar(kBarW), lane);
 
-            // [2] block k+1: x landed -> factors, widened X (overlaps S(k), Y(k))
+            // [2] block k+1: x landed -> factors (overlaps S(k), Y(k))
             if (k + 1 < kb1) {
                 ok = ok && mbar_wait_abortable(S.bar(kBarTx0 + r1), ((uint32_t)(i + 1) / kCoXSlots) & 1u,
-                                               kWaitBudget, abort_flag);
+                                               wait_budget, abort_flag);
                 if (ok) co_factors(S, r1, f1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
-                if (ok) co_widen_x(S, r1, tid);
-                named_bar_sync(kCoCompute);          // factors and widened X of block k+1 visible
+                named_bar_sync(kCoCompute);          // factors of block k+1 visible
             }
 
             // [3] S(k) done (and Z(k), which read the fp16 copy) -> H_in(k+1), w.X(k+1)
-            ok = ok && mbar_wait_abortable(S.bar(kBarS), par, kWaitBudget, abort_flag);
-            ok = ok && mbar_wait_abortable(S.bar(kBarZ), par, kWaitBudget, abort_flag);
+            ok = ok && mbar_wait_abortable(S.bar(kBarS), par, wait_budget, abort_flag);
+            ok = ok && mbar_wait_abortable(S.bar(kBarZ), par, wait_budget, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
             if (ok) {
@@ -1105,7 +1116,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             if (k + 1 < kb1) co_arrive(S.bar(kBarH16), lane);
 
             // [4] Y(k) done -> y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging in block k's B tiles
-            ok = ok && mbar_wait_abortable(S.bar(kBarY), par, kWaitBudget, abort_flag);
+            ok = ok && mbar_wait_abortable(S.bar(kBarY), par, wait_budget, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
             if (ok) {
@@ -1119,9 +1130,9 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                     tmem_ld16x2(lane_addr + kTmY + ch * 32 + 16 * hh, yv,
                                 lane_addr + kTmZ + 64u * par + ch * 32 + 16 * hh, zv);
                     float xv[16];
-                    f16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(r) + sw128_off(row, 4 * ch + 2 * hh)),
-                                     xv);
-                    f16_chunk_to_f32(
+                    bf16_chunk_to_f32(*reinterpret_cast<const uint4 *>(S.X(r) + sw128_off(row, 4 * ch + 2 * hh)),
+                                      xv);
+                    bf16_chunk_to_f32(
                         *reinterpret_cast<const uint4 *>(S.X(r) + sw128_off(row, 4 * ch + 2 * hh + 1)), xv + 8);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
@@ -1140,7 +1151,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             }
             co_arrive(S.bar(kBarFree0 + f), lane);
         }
-        // an fp16 operand out of range (see co_widen_x) or a non-finite input
+        // an fp16 operand out of range (see co_form_wx) or a non-finite input
         if (__any_sync(0xffffffffu, !(nonfinite.x == 0.f && nonfinite.y == 0.f)) && lane == 0)
             flag_status(ws.status, kStatusRange);
     }
@@ -1151,7 +1162,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
         // releases its shared memory and TMEM (bounded waits)
         for (int q = 0; q < kFirstComputeBar; ++q) {
             const int cnt = S.issued()[q];
-            if (cnt) mbar_wait(S.bar(q), (uint32_t)((cnt - 1) & 1), kWaitBudget);
+            if (cnt) mbar_wait(S.bar(q), (uint32_t)((cnt - 1) & 1), wait_budget);
         }
         flag_status(ws.status, kStatusTimeout);
     }
@@ -1162,6 +1173,13 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
 }
 
 }  // namespace
+
+namespace {
+std::atomic<int> g_test_fault{0};
+}  // namespace
+
+void tc_set_test_fault(int kind) { g_test_fault.store(kind); }
+int tc_test_fault() { return g_test_fault.load(); }
 
 bool tc_supported(const ScanDims &d, int bf16) {
     if (!bf16 || d.N != kN || d.P != kP) return false;
@@ -1180,8 +1198,12 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     TcMaps maps;
     if (!make_maps(a, d, p, ws, &maps)) return cudaErrorInvalidValue;
     cudaError_t e;
-    static bool attr_done = false;
-    if (!attr_done) {
+    // the shared-memory limits are set once per device
+    static bool attr_done[kMaxAttrDevices] = {};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxAttrDevices) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
         if ((e = cudaFuncSetAttribute(unit_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kUsSmem)) != cudaSuccess)
             return e;
@@ -1191,7 +1213,7 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         if ((e = cudaFuncSetAttribute(chunk_out_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kCoSmem)) != cudaSuccess)
             return e;
-        attr_done = true;
+        attr_done[dev] = true;
     }
     {
         TraceScope tr(s, kTrTcDtPrep);
@@ -1238,13 +1260,14 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         // L2 holds: otherwise prep's fp16 copies are still there when read.
         const double streamed = (double)d.b * d.L * d.H * d.P * (2.0 + 4.0);
         const int prefetch_cb = streamed > kL2Bytes ? 1 : 0;
+        const int fault = tc_test_fault();
         const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem);
         // the caller checked that chunk_states come with chunk_size a multiple of kBlk
         const int bpc = (int)(d.Q / kBlk) > 0 ? (int)(d.Q / kBlk) : 1;
         if ((e = cudaLaunchKernelEx(&c, a.seq_idx ? chunk_out_kernel<true> : chunk_out_kernel<false>, maps, a.D,
                                     a.init_state, a.final_state, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk,
                                     (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0, prefetch_cb, a.chunk_states, bpc,
-                                    (int)d.nc)) != cudaSuccess)
+                                    (int)d.nc, fault ? kTestWaitBudget : kWaitBudget, fault)) != cudaSuccess)
             return e;
     }
     return cudaGetLastError();

@@ -11,6 +11,7 @@
 // M or N); the descriptor says which.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -40,6 +41,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, i
            | (0u << 7) | (0u << 10)                 // A, B format: f16
            | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16)
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---- instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
+    return idesc_f16(M, N, a_mn_major, b_mn_major) | (1u << 7) | (1u << 10);
 }
 
 // ---- mbarrier
@@ -407,6 +413,17 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2(uint32_t u) {
     const float lo = __uint_as_float(u << 16);
     const float hi = __uint_as_float(u & 0xFFFF0000u);
     return pack_h2(lo, hi);
+}
+
+// Two fp32 values as a bf16 hi/lo pair each: hi = the bf16 truncation of
+// the value, lo = the rest rounded to bf16, so hi + lo carries about 16
+// significant bits.  Returns the packed hi pair and the packed lo pair.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+    hi = __byte_perm(ua, ub, 0x7632);                     // high halves: the truncated bf16 pair
+    const float ra = a - __uint_as_float(ua & 0xFFFF0000u), rb = b - __uint_as_float(ub & 0xFFFF0000u);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(ra, rb);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }

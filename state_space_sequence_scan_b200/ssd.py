@@ -84,12 +84,21 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_trace_kernel_name.argtypes = [i32]
     lib.ssd_trace_kernel_count.restype = i32
     lib.ssd_trace_kernel_count.argtypes = []
+    lib.ssd_set_test_fault.restype = i32
+    lib.ssd_set_test_fault.argtypes = [i32]
     lib.ssd_conv1d_silu_split.restype = i32
     lib.ssd_conv1d_silu_split.argtypes = [vp] * 6 + [i64] * 7 + [i32, vp]
     lib.ssd_gated_rmsnorm.restype = i32
     lib.ssd_gated_rmsnorm.argtypes = [vp] * 4 + [i64] * 3 + [f32, i32, vp]
     _lib = lib
     return lib
+
+
+def set_test_fault(kind: int) -> None:
+    """TEST ONLY (ssd_set_test_fault): kind 1 makes the tensor-path scan's
+    waits run out (the first C and B tiles are never requested) so the device-side
+    timeout path runs; kind 0 restores normal operation."""
+    _check("ssd_set_test_fault", load_library().ssd_set_test_fault(int(kind)))
 
 
 def _check(fn: str, st: int):

@@ -67,3 +67,57 @@ def sample_chains(inp, chains):
                    init_state=None if inp["init_state"] is None else inp["init_state"][bi:bi + 1, h:h + 1])
         out.append(sub)
     return out
+
+
+def stack_chains(inp, chains):
+    """The (b, h) chains of a scan input as the heads of one batch row, each
+    head its own group (its chain's B and C): one oracle call threads over all
+    of them.  Pure indexing."""
+    H = inp["x"].shape[2]
+    G = inp["B"].shape[2]
+    bs = [bi for bi, _ in chains]
+    hs = [h for _, h in chains]
+    gs = [h // (H // G) for h in hs]
+    out = dict(x=torch.stack([inp["x"][bi, :, h] for bi, h in chains], 1)[None],
+               dt_raw=torch.stack([inp["dt_raw"][bi, :, h] for bi, h in chains], 1)[None],
+               B=torch.stack([inp["B"][bi, :, g] for bi, g in zip(bs, gs)], 1)[None],
+               C=torch.stack([inp["C"][bi, :, g] for bi, g in zip(bs, gs)], 1)[None],
+               dt_bias=inp["dt_bias"][hs], A=inp["A"][hs], D=inp["D"][hs])
+    out["init_state"] = None if inp["init_state"] is None else torch.stack(
+        [inp["init_state"][bi, h] for bi, h in chains], 0)[None]
+    return {k: (v.contiguous() if isinstance(v, torch.Tensor) else v) for k, v in out.items()}
+
+
+class StreamingCompare:
+    """max|gpu - oracle| / RMS(oracle) over a tensor checked in pieces: the
+    largest error and the sum of squares are accumulated, the bar applied to
+    the whole."""
+
+    def __init__(self, tol, what):
+        self.tol, self.what = tol, what
+        self.maxerr, self.sumsq, self.n = 0.0, 0.0, 0
+
+    def add(self, got, ref):
+        got = np.asarray(got, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        assert got.shape == ref.shape, (got.shape, ref.shape)
+        assert np.isfinite(got).all(), "%s: non-finite output" % self.what
+        self.maxerr = max(self.maxerr, float(np.max(np.abs(got - ref))) if got.size else 0.0)
+        self.sumsq += float(np.sum(ref * ref))
+        self.n += ref.size
+
+    def check(self):
+        rms = math.sqrt(self.sumsq / max(self.n, 1))
+        rel = self.maxerr / rms if rms > 0 else self.maxerr
+        assert rel <= self.tol, "%s: max|err|/RMS = %.3e > %.1e" % (self.what, rel, self.tol)
+        return rel
+
+
+def spread_chains(batch, heads, per_batch, stride=13):
+    """per_batch heads of every batch row, spread over all heads and over the
+    head positions inside a group (row bi starts at a different offset)."""
+    out = []
+    for bi in range(batch):
+        for j in range(per_batch):
+            out.append((bi, (bi * stride + j * max(1, heads // per_batch) + j) % heads))
+    return sorted(set(out))

@@ -37,6 +37,13 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(ssd.EXPORTED) <= set(names)
 
 
+def test_test_fault_hook_validates_its_argument(lib):
+    """The timeout-path test hook takes 0 (off) or 1 only; host-side, no GPU."""
+    assert lib.ssd_set_test_fault(7) == 1
+    assert lib.ssd_set_test_fault(-1) == 1
+    assert lib.ssd_set_test_fault(0) == 0
+
+
 def test_version_and_status_strings(lib):
     assert lib.ssd_version() >> 16 == 1
     for code in range(8):

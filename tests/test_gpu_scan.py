@@ -13,7 +13,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import TOL_BF16, TOL_F32, compare, path_supported, run_scan, sample_chains, tol_for
+from gpu_helpers import (TOL_BF16, TOL_F32, StreamingCompare, compare, path_supported, run_scan, sample_chains,
+                         spread_chains, stack_chains, to_dev, tol_for)
 from state_space_sequence_scan_b200 import ssd
 from state_space_sequence_scan_b200.inputs import SCAN_CONFIGS, ScanConfig, make_scan_inputs
 
@@ -81,22 +82,76 @@ def test_c1_130m_full(path):
 
 
 @pytest.mark.parametrize("path", BF16_PATHS)
-@pytest.mark.parametrize("name,chains", [
-    ("c2_2p7b", [(0, 0), (3, 41), (7, 79), (5, 17)]),
-    ("c3_long", [(0, 0), (0, 37), (0, 79)]),
-])
-def test_full_size_sampled_chains(name, chains, path):
-    """The kernels run on the whole workload (the launch the benchmark times);
-    the oracle evaluates the sampled chains alone."""
-    cfg = SCAN_CONFIGS[name]
+def test_c2_full_size_64_chains(path):
+    """The 2.7B-shaped layer, whole (the launch the benchmark times), against
+    the oracle on 64 chains spread over all 8 batch rows, over the heads and
+    over every head position inside the group; the bar over all of them."""
+    cfg = SCAN_CONFIGS["c2_2p7b"]
     inp = make_scan_inputs(cfg)
     y, fs = run_scan(inp, cfg.chunk_size, path=path)
     assert np.isfinite(y).all() and np.isfinite(fs).all()
-    H, G = cfg.nheads, cfg.ngroups
-    for (bi, h), sub in zip(chains, sample_chains(inp, chains)):
-        yr, fr = _oracle(sub)
-        compare(y[bi:bi + 1, :, h:h + 1], yr, TOL_BF16, "%s chain %s y" % (name, (bi, h)))
-        compare(fs[bi:bi + 1, h:h + 1], fr, TOL_BF16, "%s chain %s final_state" % (name, (bi, h)))
+    chains = spread_chains(cfg.batch, cfg.nheads, 8)
+    assert len(chains) == 64
+    yr, fr = _oracle(stack_chains(inp, chains))
+    cy, cf = StreamingCompare(TOL_BF16, "c2 y"), StreamingCompare(TOL_BF16, "c2 final_state")
+    for j, (bi, h) in enumerate(chains):
+        cy.add(y[bi, :, h], yr[0, :, j])
+        cf.add(fs[bi, h], fr[0, j])
+    cy.check()
+    cf.check()
+
+
+def test_c3_full_size_every_chain():
+    """The long-context layer (one 65536-token row, 80 heads in 8 groups, 11
+    units of 47 blocks each on the tensor path), every (batch, head) chain
+    against the oracle, 16 chains per oracle call; the bar over the whole
+    y and final_state."""
+    cfg = SCAN_CONFIGS["c3_long"]
+    inp = make_scan_inputs(cfg)
+    d = to_dev(inp)
+    b, L, H, P = d["x"].shape
+    G, N = d["B"].shape[2], d["B"].shape[3]
+    ws = ssd.alloc_workspace(ssd.workspace_size(b, L, H, P, N, G, cfg.chunk_size, d["x"].dtype, "tensor"), "cuda")
+    y, fs = ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                               init_state=d["init_state"], chunk_size=cfg.chunk_size, path="tensor", workspace=ws)
+    assert ssd.read_device_status(ws) == 0
+    y = y.cpu().numpy()
+    fs = fs.cpu().numpy()
+    del d, ws
+    cy, cf = StreamingCompare(TOL_BF16, "c3 y"), StreamingCompare(TOL_BF16, "c3 final_state")
+    for h0 in range(0, H, 16):
+        chains = [(0, h) for h in range(h0, min(H, h0 + 16))]
+        yr, fr = _oracle(stack_chains(inp, chains))
+        for j, (bi, h) in enumerate(chains):
+            cy.add(y[bi, :, h], yr[0, :, j])
+            cf.add(fs[bi, h], fr[0, j])
+    cy.check()
+    cf.check()
+
+
+def test_diag_sub_blocks_straddle_the_exp_cap():
+    """Per-token log decays of about -2 make the 31-step decay across a
+    diagonal 32x32 sub-block straddle the cap (64) of the factored form:
+    inside one 128-token block some sub-blocks take the factored path and
+    some the one-exp-per-element path.  A = -1 and dt_raw chosen so that
+    dt (the softplus of dt_raw + dt_bias) is 1.9 .. 2.3."""
+    cfg = ScanConfig("cap", 2, 700, 4, 64, 128, 2, 128, "bf16", "ones", "normal", seed=71)
+    inp = make_scan_inputs(cfg)
+    g = torch.Generator().manual_seed(71)
+    dt = 1.9 + 0.4 * torch.rand(cfg.batch, cfg.seqlen, cfg.nheads, generator=g, dtype=torch.float64)
+    inp["A"][:] = -1.0
+    inp["dt_bias"][:] = 0.0
+    inp["dt_raw"] = (dt + torch.log(-torch.expm1(-dt))).float()       # softplus^-1(dt)
+    # the decays really straddle the cap inside blocks (the kernel's flag test in fp32)
+    da = -dt.float()
+    cum = torch.cumsum(da.view(cfg.batch, -1, cfg.nheads), 1)
+    spans = []
+    for t0 in range(0, cfg.seqlen - 31, 32):
+        spans.append((cum[:, t0] - cum[:, t0 + 31]).flatten())
+    spans = torch.cat(spans)
+    assert (spans <= 64).any() and (spans > 64).any()
+    _check(inp, 128, "tensor", what="exp cap")
+    _check(inp, 128, "simt", what="exp cap")
 
 
 def test_chunk_size_invariance_fp32():
@@ -238,12 +293,30 @@ def test_tensor_path_units():
 
 
 def test_tensor_path_range_guard():
-    """An input outside the fp16 operand range is reported, not silently wrong."""
+    """An fp16 operand the tensor path forms out of range is reported, never
+    silently wrong.  x itself enters W.X as bf16 (no range limit there); the
+    operands formed in fp16 are w.x (for the state) and the carried state.
+    x = 1e30 at one token overflows them: the call reports
+    SSD_ERR_PRECONDITION.  x = 1e6 at one token is either computed within
+    the bar or reported."""
     cfg = ScanConfig("range", 1, 256, 2, 64, 128, 1, 128, "bf16", "ones", "zero", seed=41)
     inp = make_scan_inputs(cfg)
-    inp["x"][0, 10, 0, 3] = 1.0e6
-    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     ws = ssd.alloc_workspace(ssd.workspace_size(1, 256, 2, 64, 128, 1, 128, torch.bfloat16, "tensor"), "cuda")
-    ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], chunk_size=128,
-                       path="tensor", workspace=ws)
-    assert ssd.read_device_status(ws) == 7
+    for big in (1.0e30, 1.0e6):
+        case = dict(inp)
+        case["x"] = inp["x"].clone()
+        case["x"][0, 10, 0, 3] = big
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in case.items()}
+        y, fs = ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                                   chunk_size=128, path="tensor", workspace=ws)
+        st = ssd.read_device_status(ws)
+        if big > 1e20:
+            assert st == 7
+            continue
+        assert st in (0, 7)
+        if st == 0:
+            yr, fr = _oracle(case)
+            compare(y.cpu().double().numpy(), yr, TOL_BF16, "x = 1e6 y")
+            compare(fs.cpu().double().numpy(), fr, TOL_BF16, "x = 1e6 final_state")
+
+

@@ -20,7 +20,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import TOL_BF16, compare, path_supported, run_scan, sample_chains, to_dev, tol_for
+from gpu_helpers import (TOL_BF16, compare, path_supported, run_scan, sample_chains, spread_chains, stack_chains,
+                         to_dev, tol_for)
 from state_space_sequence_scan_b200 import ssd
 from state_space_sequence_scan_b200.inputs import SCAN_CONFIGS, ScanConfig, make_scan_inputs
 
@@ -104,20 +105,22 @@ def test_tensor_path_needs_whole_blocks():
     assert e.value.status == 2
 
 
-@pytest.mark.parametrize("name,chains", [
-    ("c2_2p7b", [(0, 0), (6, 55)]),
-    ("c3_long", [(0, 0), (0, 63)]),                          # units of 47 blocks: the split path
-])
-def test_full_size_sampled_chain_states(name, chains):
-    """The whole workload on the tensor path with the states; the oracle
-    evaluates the sampled chains alone."""
+@pytest.mark.parametrize("name", ["c2_2p7b", "c3_long"])
+def test_full_size_sampled_chain_states(name):
+    """The whole workload on the tensor path with the states (c3: units of 47
+    blocks, the split path); the oracle evaluates sampled chains together:
+    64 spread over all batch rows and heads of c2, every fifth head of c3."""
     cfg = SCAN_CONFIGS[name]
     inp = make_scan_inputs(cfg)
     Q = cfg.chunk_size
     y, fs, cs = run_states(inp, Q, "tensor")
     assert np.isfinite(cs).all()
     assert np.array_equal(cs[:, -1], fs)
-    for (bi, h), sub in zip(chains, sample_chains(inp, chains)):
-        _, fr, sr = oracle_states(sub, Q)
-        compare_states(cs[bi:bi + 1, :, h:h + 1], sr, TOL_BF16, "%s chain %s chunk states" % (name, (bi, h)))
-        compare(fs[bi:bi + 1, h:h + 1], fr, TOL_BF16, "%s chain %s final_state" % (name, (bi, h)))
+    chains = spread_chains(cfg.batch, cfg.nheads, 8) if cfg.batch > 1 else [(0, h) for h in range(0, cfg.nheads, 5)]
+    for c0 in range(0, len(chains), 16):
+        part = chains[c0:c0 + 16]
+        _, fr, sr = oracle_states(stack_chains(inp, part), Q)
+        for j, (bi, h) in enumerate(part):
+            compare_states(cs[bi:bi + 1, :, h:h + 1], sr[:, :, j:j + 1], TOL_BF16,
+                           "%s chain %s chunk states" % (name, (bi, h)))
+            compare(fs[bi:bi + 1, h:h + 1], fr[:, j:j + 1], TOL_BF16, "%s chain %s final_state" % (name, (bi, h)))
