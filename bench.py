@@ -87,8 +87,10 @@ def step_bytes(cfg) -> float:
 # that file changes the number no longer describes the kernel and the bench
 # reports null.
 NCU_TRAFFIC = {
-    ("c1_130m", "tc_chunk_out"): (35.329792e6, "state_space_sequence_scan_b200/csrc/ssd_scan_tc.cu",
-                                  "a0afdb27d5acb42a"),
+    ("c3_long", "tc_chunk_out"): (2318.40512e6, "state_space_sequence_scan_b200/csrc/ssd_scan_tc.cu",
+                                  "452ad04813b5ea59"),
+    ("c2_2p7b", "tc_chunk_out"): (1018.312704e6, "state_space_sequence_scan_b200/csrc/ssd_scan_tc.cu",
+                                  "452ad04813b5ea59"),
     ("c4_decode", "decode_step"): (1291.7568e6, "state_space_sequence_scan_b200/csrc/ssd_step.cu",
                                    "a5f3c2cec738b994"),
 }
