@@ -248,7 +248,8 @@ SSD_API ssd_status ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seql
  * mamba kernels is not; this one has no atomics and sums in a fixed order, so
  * repeated calls on the same inputs give the same bits).
  *
- * Given the forward's inputs (as for ssd_chunk_scan_fwd, no packed rows) and
+ * Given the forward's inputs (as for ssd_chunk_scan_fwd; packed rows through
+ * ssd_chunk_scan_bwd_varlen) and
  * the gradients dy of y and dfinal_state of final_state, writes the gradient
  * of <dy, y> + <dfinal_state, final_state> with respect to every input:
  *   dy           [batch, seqlen, nheads, head_dim] float32 in
@@ -278,6 +279,23 @@ SSD_API ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const 
                               int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
                               int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi,
                               int in_dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ssd_chunk_scan_bwd over packed rows: the gradients of the forward of
+ * ssd_chunk_scan_fwd_varlen with the same seq_idx ([batch, seqlen] int32,
+ * 4-byte aligned; a token whose id differs from the previous token's starts a
+ * document and the state is zero before its update).  No gradient crosses a
+ * document start; dinit_state reaches only each row's first document.  NULL
+ * seq_idx makes the call ssd_chunk_scan_bwd.  Same workspace size,
+ * determinism and other arguments as ssd_chunk_scan_bwd. */
+SSD_API ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw, const float *dt_bias,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const float *init_state, const int32_t *seq_idx, const float *dy,
+                                     const float *dfinal_state, float *dx, float *ddt_raw, float *ddt_bias,
+                                     float *dA, float *dB, float *dC, float *dD, float *dinit_state,
+                                     int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
+                                     int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo,
+                                     float dt_hi, int in_dtype, void *workspace, size_t workspace_bytes,
+                                     void *stream);
 
 /* Waits for `stream`, then reads the device status word that the last
  * ssd_chunk_scan_fwd on this workspace left: SSD_OK, SSD_ERR_PRECONDITION or
@@ -316,7 +334,7 @@ SSD_API ssd_status ssd_set_test_fault(int kind);
 
 /* ABI version: (major << 16) | minor.  1.1 added the chunk-state, packed-row,
  * conv/norm and backward entry points to the 1.0 scan and step; 1.2 the test
- * hook ssd_set_test_fault. */
+ * hook ssd_set_test_fault and ssd_chunk_scan_bwd_varlen. */
 SSD_API int ssd_version(void);
 
 #ifdef __cplusplus

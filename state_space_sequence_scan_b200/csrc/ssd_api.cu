@@ -226,9 +226,9 @@ ssd_status ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int6
     return SSD_OK;
 }
 
-ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
-                              const void *B, const void *C, const float *D, const float *init_state,
-                              const float *dy, const float *dfinal_state, float *dx, float *ddt_raw,
+ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
+                                     const void *B, const void *C, const float *D, const float *init_state,
+                                     const int32_t *seq_idx, const float *dy, const float *dfinal_state, float *dx, float *ddt_raw,
                               float *ddt_bias, float *dA, float *dB, float *dC, float *dD, float *dinit_state,
                               int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim, int64_t state_dim,
                               int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype,
@@ -244,7 +244,9 @@ ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *d
     const void *al[] = {x, B, C, init_state, dy, dfinal_state, dx, dB, dC, dinit_state};
     for (const void *p : al)
         if (p && !aligned16(p)) return SSD_ERR_ALIGNMENT;
-    if ((reinterpret_cast<uintptr_t>(dt_raw) | reinterpret_cast<uintptr_t>(ddt_raw)) & 3u) return SSD_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(dt_raw) | reinterpret_cast<uintptr_t>(ddt_raw) |
+         reinterpret_cast<uintptr_t>(seq_idx)) & 3u)
+        return SSD_ERR_ALIGNMENT;
     const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
     if (!ssd::bwd_supported(d)) return SSD_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < ssd::bwd_workspace_bytes(d)) return SSD_ERR_WORKSPACE;
@@ -270,6 +272,7 @@ ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *d
     ssd::BwdArgs a;
     a.f.x = x; a.f.dt_raw = dt_raw; a.f.dt_bias = dt_bias; a.f.A = A; a.f.B = B; a.f.C = C; a.f.D = D;
     a.f.init_state = init_state; a.f.y = nullptr; a.f.final_state = nullptr;
+    a.f.seq_idx = seq_idx;
     a.f.dt_lo = dt_lo; a.f.dt_hi = dt_hi; a.f.bf16 = in_dtype == SSD_BF16;
     a.dy = dy; a.dfinal = dfinal_state;
     a.dx = dx; a.ddt_raw = ddt_raw; a.ddt_bias = ddt_bias; a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD;
@@ -277,6 +280,19 @@ ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *d
     e = ssd::bwd_scan(a, d, workspace, s);
     if (e != cudaSuccess) return cuda_fail(e);
     return SSD_OK;
+}
+
+ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
+                              const void *B, const void *C, const float *D, const float *init_state,
+                              const float *dy, const float *dfinal_state, float *dx, float *ddt_raw,
+                              float *ddt_bias, float *dA, float *dB, float *dC, float *dD, float *dinit_state,
+                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim, int64_t state_dim,
+                              int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    return ssd_chunk_scan_bwd_varlen(x, dt_raw, dt_bias, A, B, C, D, init_state, nullptr, dy, dfinal_state, dx,
+                                     ddt_raw, ddt_bias, dA, dB, dC, dD, dinit_state, batch, seqlen, nheads, head_dim,
+                                     state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, workspace,
+                                     workspace_bytes, stream);
 }
 
 ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_bias, const float *A,

@@ -8,7 +8,9 @@
 //   gated_rmsnorm      v = y * silu(z), RMS-normalised over groups of
 //                      channels, times a per-channel weight
 // Both are HBM-bound streams: coalesced vector loads and stores, one pass
-// over the data (the norm's second read of a group hits L1).
+// over the data (the norm holds a group in registers; groups that do not
+// split evenly over its CTA take a two-pass warp kernel, the second read
+// from L1/L2).
 #include "../../include/ssd.h"
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
@@ -22,7 +24,10 @@ constexpr int kConvCh = 4;      // channels per thread (one 8- or 16-byte access
 constexpr int kConvT = 16;      // tokens per thread (a sliding window in registers)
 constexpr int kConvMaxK = 4;
 
-__device__ __forceinline__ float silu_f(float u) { return u / (1.0f + expf(-u)); }
+// silu(u) = u / (1 + e^-u) with the fast exponential and division (relative
+// error about 1e-6: inside the fp32 bar of 1e-5 and one bf16 rounding).  For
+// u below about -87, e^-u is inf and the quotient is the limit, 0.
+__device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
 // 4 consecutive z values -> floats
 __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&v)[4]) {
@@ -46,16 +51,12 @@ __device__ __forceinline__ void store4(float *p, const float (&v)[4]) {
     *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
 }
 
-// grid (ceil(L/kConvT), ceil(Cd/4/256), b): thread = 4 channels x kConvT tokens.
-// out[t, c] = silu(bias[c] + sum_k w[c, k] in[t - (K-1) + k, c]), in[t < 0] = 0.
+// One token tile [t0, t0 + kConvT) of 4 channels from c0 (see conv1d_silu_kernel).
 template <typename T, int K>
-__global__ void __launch_bounds__(kConvThreads)
-conv1d_silu_kernel(const T *__restrict__ xbc, const float *__restrict__ w, const float *__restrict__ bias,
-                   T *__restrict__ x, T *__restrict__ Bo, T *__restrict__ Co, int L, int Cd, int HP, int GN) {
-    const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * kConvCh;
-    if (c0 >= Cd) return;
-    const int t0 = blockIdx.x * kConvT;
-    const size_t b = blockIdx.z;
+__device__ __forceinline__ void conv1d_silu_tile(const T *__restrict__ xbc, const float *__restrict__ w,
+                                                 const float *__restrict__ bias, T *__restrict__ x,
+                                                 T *__restrict__ Bo, T *__restrict__ Co, int L, int Cd, int HP,
+                                                 int GN, int c0, int t0, size_t b) {
     float wr[kConvCh][K], bs[kConvCh];
 #pragma unroll
     for (int e = 0; e < kConvCh; ++e) {
@@ -78,52 +79,108 @@ conv1d_silu_kernel(const T *__restrict__ xbc, const float *__restrict__ w, const
     }
     const T *src = xbc + b * L * (size_t)Cd + c0;
     dst += b * L * (size_t)ld;
-    // rows t-(K-1) .. t+kConvB-1: the K-1 rows before a batch of kConvB tokens
-    // and the batch, all loaded before any store (dst may not be proven apart
-    // from src, so the loads would otherwise wait for the stores before them)
-    constexpr int kConvB = 4;
-    float win[K - 1 + kConvB][kConvCh];
+    // rows t0-(K-1) .. t0+kConvT-1, all loaded before any arithmetic or store
+    // (dst may not be proven apart from src, so a load after a store would
+    // wait for it; 16 + K-1 independent loads keep enough bytes in flight)
+    float win[K - 1 + kConvT][kConvCh];
+    const int tn = min(kConvT, L - t0);
 #pragma unroll
-    for (int k = 0; k < K - 1; ++k) {
+    for (int k = 0; k < K - 1 + kConvT; ++k) {
         const int t = t0 - (K - 1) + k;
-        if (t >= 0) load4(src + (size_t)t * Cd, win[k]);
+        if (t >= 0 && k - (K - 1) < tn) load4(src + (size_t)t * Cd, win[k]);
         else {
 #pragma unroll
             for (int e = 0; e < kConvCh; ++e) win[k][e] = 0.f;
         }
     }
-    const int tn = min(kConvT, L - t0);
-    for (int i0 = 0; i0 < tn; i0 += kConvB) {
 #pragma unroll
-        for (int j = 0; j < kConvB; ++j) {
-            if (i0 + j < tn) load4(src + (size_t)(t0 + i0 + j) * Cd, win[K - 1 + j]);
-            else {
+    for (int j = 0; j < kConvT; ++j) {
+        if (j < tn) {
+            float o[kConvCh];
 #pragma unroll
-                for (int e = 0; e < kConvCh; ++e) win[K - 1 + j][e] = 0.f;
+            for (int e = 0; e < kConvCh; ++e) {
+                float acc = bs[e];
+#pragma unroll
+                for (int k = 0; k < K; ++k) acc = fmaf(wr[e][k], win[j + k][e], acc);
+                o[e] = silu_f(acc);
             }
+            store4(dst + (size_t)(t0 + j) * ld, o);
         }
-#pragma unroll
-        for (int j = 0; j < kConvB; ++j) {
-            if (i0 + j < tn) {
-                float o[kConvCh];
-#pragma unroll
-                for (int e = 0; e < kConvCh; ++e) {
-                    float acc = bs[e];
-#pragma unroll
-                    for (int k = 0; k < K; ++k) acc = fmaf(wr[e][k], win[j + k][e], acc);
-                    o[e] = silu_f(acc);
-                }
-                store4(dst + (size_t)(t0 + i0 + j) * ld, o);
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < K - 1; ++k)
-#pragma unroll
-            for (int e = 0; e < kConvCh; ++e) win[k][e] = win[kConvB + k][e];
     }
 }
 
-// one warp per (token, group); 8 warps per block.  Two passes over the group:
+// grid (ceil(L/kConvT), ceil(Cd/4/256), b): thread = 4 channels x kConvT tokens.
+// out[t, c] = silu(bias[c] + sum_k w[c, k] in[t - (K-1) + k, c]), in[t < 0] = 0.
+template <typename T, int K>
+__global__ void __launch_bounds__(kConvThreads)
+conv1d_silu_kernel(const T *__restrict__ xbc, const float *__restrict__ w, const float *__restrict__ bias,
+                   T *__restrict__ x, T *__restrict__ Bo, T *__restrict__ Co, int L, int Cd, int HP, int GN) {
+    const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * kConvCh;
+    if (c0 >= Cd) return;
+    conv1d_silu_tile<T, K>(xbc, w, bias, x, Bo, Co, L, Cd, HP, GN, c0, blockIdx.x * kConvT, blockIdx.z);
+}
+
+
+// One CTA of kNormThreads per (token, group) when the group splits evenly
+// into kNormThreads x V float4s: v = y silu(z) stays in registers, one read
+// of y and z.  The sum of squares runs in a fixed order (each thread's V
+// float4s, then a shuffle tree per warp, then the warps' partials by thread
+// 0 in warp order): deterministic.
+constexpr int kNormThreads = 128;
+constexpr int kNormMaxV = 10;
+
+template <typename Tz, int V>
+__global__ void __launch_bounds__(kNormThreads)
+gated_rmsnorm_block_kernel(const float *__restrict__ y, const Tz *__restrict__ z, const float *__restrict__ wt,
+                           float *__restrict__ out, int D, int group, float eps) {
+    __shared__ float s_part[kNormThreads / 32];
+    __shared__ float s_r;
+    const int ngr = D / group;
+    const int64_t t = blockIdx.x / ngr;
+    const int g0 = (int)(blockIdx.x % ngr) * group;
+    const float *yr = y + t * D + g0;
+    const Tz *zr = z + t * D + g0;
+    float v[V][4];
+    float yv[V][4], zv[V][4];
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+        const int j = (q * kNormThreads + threadIdx.x) * 4;
+        load4(yr + j, yv[q]);
+        load4(zr + j, zv[q]);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int q = 0; q < V; ++q)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            v[q][e] = yv[q][e] * silu_f(zv[q][e]);
+            ss = fmaf(v[q][e], v[q][e], ss);
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kNormThreads / 32; ++w) tot += s_part[w];
+        s_r = 1.0f / sqrtf(tot / (float)group + eps);
+    }
+    __syncthreads();
+    const float r = s_r;
+    float *orow = out + t * D + g0;
+    const float *wg = wt + g0;
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+        const int j = (q * kNormThreads + threadIdx.x) * 4;
+        const float4 wv = *reinterpret_cast<const float4 *>(wg + j);
+        *reinterpret_cast<float4 *>(orow + j) =
+            make_float4(v[q][0] * r * wv.x, v[q][1] * r * wv.y, v[q][2] * r * wv.z, v[q][3] * r * wv.w);
+    }
+}
+
+// Fallback for groups that do not split evenly: one warp per (token, group);
+// 8 warps per block.  Two passes over the group:
 // the sum of squares (fixed shuffle order: deterministic), then the output.
 template <typename Tz>
 __global__ void __launch_bounds__(256)
@@ -165,8 +222,8 @@ gated_rmsnorm_kernel(const float *__restrict__ y, const Tz *__restrict__ z, cons
 template <typename T>
 cudaError_t conv_launch(const void *xbc, const float *w, const float *bias, void *x, void *B, void *C, int64_t b,
                         int64_t L, int Cd, int HP, int GN, int K, cudaStream_t s) {
-    const dim3 g((unsigned)((L + kConvT - 1) / kConvT),
-                 (unsigned)((Cd / kConvCh + kConvThreads - 1) / kConvThreads), (unsigned)b);
+    const dim3 g((unsigned)((L + kConvT - 1) / kConvT), (unsigned)((Cd / kConvCh + kConvThreads - 1) / kConvThreads),
+                 (unsigned)b);
     TraceScope tr(s, kTrConv1d);
 #define SSD_CONV(KK)                                                                                           \
     conv1d_silu_kernel<T, KK><<<g, kConvThreads, 0, s>>>((const T *)xbc, w, bias, (T *)x, (T *)B, (T *)C,     \
@@ -196,7 +253,7 @@ extern "C" SSD_API ssd_status ssd_conv1d_silu_split(const void *xbc, const float
     if (kernel_width < 1 || kernel_width > ssd::kConvMaxK) return SSD_ERR_UNSUPPORTED;
     if (in_dtype != SSD_F32 && in_dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
     const int64_t HP = nheads * head_dim, GN = ngroups * state_dim, Cd = HP + 2 * GN;
-    // grid: token tiles in x, 256-thread channel blocks in y (<= 8192), batch in z
+    // grid: token tiles in x, 256-thread channel blocks in y (<= 65535), batch in z
     if (HP % 8 || GN % 8 || Cd > (1 << 24) || batch > 65535 || seqlen > (1ll << 31) - ssd::kConvT)
         return SSD_ERR_UNSUPPORTED;
     if (batch == 0 || seqlen == 0) return SSD_OK;
@@ -228,7 +285,35 @@ extern "C" SSD_API ssd_status ssd_gated_rmsnorm(const float *y, const void *z, c
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t warps = tokens * (dim / group_size);
     const unsigned blocks = (unsigned)((warps + 7) / 8);
-    {
+    // the single-pass block kernel when a group is kNormThreads x V float4s
+    const int64_t V = group_size / (4 * ssd::kNormThreads);
+    if (group_size % (4 * ssd::kNormThreads) == 0 && V >= 1 && V <= ssd::kNormMaxV && warps <= 0x7fffffffll) {
+        ssd::TraceScope tr(s, ssd::kTrGatedNorm);
+        const unsigned nb = (unsigned)warps;
+        const __nv_bfloat16 *zb = static_cast<const __nv_bfloat16 *>(z);
+        const float *zf = static_cast<const float *>(z);
+#define SSD_NORM(VV)                                                                                              \
+    if (z_dtype == SSD_BF16)                                                                                      \
+        ssd::gated_rmsnorm_block_kernel<__nv_bfloat16, VV><<<nb, ssd::kNormThreads, 0, s>>>(y, zb, weight, out,  \
+                                                                                            (int)dim,            \
+                                                                                            (int)group_size, eps); \
+    else                                                                                                          \
+        ssd::gated_rmsnorm_block_kernel<float, VV><<<nb, ssd::kNormThreads, 0, s>>>(y, zf, weight, out, (int)dim, \
+                                                                                    (int)group_size, eps)
+        switch (V) {
+            case 1: SSD_NORM(1); break;
+            case 2: SSD_NORM(2); break;
+            case 3: SSD_NORM(3); break;
+            case 4: SSD_NORM(4); break;
+            case 5: SSD_NORM(5); break;
+            case 6: SSD_NORM(6); break;
+            case 7: SSD_NORM(7); break;
+            case 8: SSD_NORM(8); break;
+            case 9: SSD_NORM(9); break;
+            default: SSD_NORM(10); break;
+        }
+#undef SSD_NORM
+    } else {
         ssd::TraceScope tr(s, ssd::kTrGatedNorm);
         if (z_dtype == SSD_BF16)
             ssd::gated_rmsnorm_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(

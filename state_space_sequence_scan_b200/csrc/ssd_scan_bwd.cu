@@ -62,21 +62,23 @@ struct BwdWs {
     float *dyx;        // [b, H, L]: dy_t . x_t
     float *part;       // [b, H, nc, 3]: dA, d(dt_bias), dD per chunk
     float *dBh, *dCh;  // [b, L, H, N] per head (null when G == H)
+    float *docc;       // [b, L] packed rows: document starts from the chunk's first token through t
 };
 
 int dpass_blocks(const ScanDims &d) { return (int)((d.N * d.P + kThreads - 1) / kThreads); }
 
 size_t bwd_extra_bytes(const ScanDims &d, size_t *offs) {
     const size_t bh = (size_t)d.b * d.H;
-    const size_t sizes[6] = {
+    const size_t sizes[7] = {
         bh * d.nc * d.N * d.P * sizeof(float),
         bh * d.nc * dpass_blocks(d) * sizeof(float),
         bh * d.L * sizeof(float) * 5,
         bh * d.nc * 3 * sizeof(float),
         d.G == d.H ? 0 : (size_t)d.b * d.L * d.H * d.N * sizeof(float),
-        d.G == d.H ? 0 : (size_t)d.b * d.L * d.H * d.N * sizeof(float)};
+        d.G == d.H ? 0 : (size_t)d.b * d.L * d.H * d.N * sizeof(float),
+        (size_t)d.b * d.L * sizeof(float)};
     size_t off = 0;
-    for (int i = 0; i < 6; ++i) {
+    for (int i = 0; i < 7; ++i) {
         if (offs) offs[i] = off;
         off += align256(sizes[i]);
     }
@@ -86,7 +88,7 @@ size_t bwd_extra_bytes(const ScanDims &d, size_t *offs) {
 BwdWs bwd_carve(const ScanDims &d, void *ws) {
     BwdWs w;
     w.f = simt_carve(d, ws);
-    size_t offs[6];
+    size_t offs[7];
     bwd_extra_bytes(d, offs);
     char *p = static_cast<char *>(ws) + simt_workspace_bytes(d);
     const size_t tok = (size_t)d.b * d.H * d.L;
@@ -101,6 +103,7 @@ BwdWs bwd_carve(const ScanDims &d, void *ws) {
     w.part = reinterpret_cast<float *>(p + offs[3]);
     w.dBh = d.G == d.H ? nullptr : reinterpret_cast<float *>(p + offs[4]);
     w.dCh = d.G == d.H ? nullptr : reinterpret_cast<float *>(p + offs[5]);
+    w.docc = reinterpret_cast<float *>(p + offs[6]);
     return w;
 }
 
@@ -117,11 +120,29 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
     return t;
 }
 
+// ---- 0. packed rows: document counters per chunk ---------------------------
+__global__ void __launch_bounds__(kThreads)
+docs_kernel(const int32_t *__restrict__ seq_idx, float *__restrict__ docc, int L, int Q) {
+    __shared__ float wtot[32];
+    const int c = blockIdx.x, b = blockIdx.y;
+    const int t0 = c * Q, q = min(Q, L - t0);
+    float carry = 0.f;
+    for (int base = 0; base < q; base += kThreads) {
+        const int i = base + threadIdx.x;
+        const int t = t0 + i;
+        const float f = (i < q && t > 0 && seq_idx[(size_t)b * L + t] != seq_idx[(size_t)b * L + t - 1]) ? 1.f : 0.f;
+        float tot;
+        const float v = block_inclusive_scan(f, wtot, tot) + carry;
+        if (i < q) docc[(size_t)b * L + t] = v;
+        carry += tot;
+    }
+}
+
 // ---- 1. sum_i e^{cum_i} C_i dy_i^T per chunk ------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 dstate_kernel(const T *__restrict__ Cm, const float *__restrict__ dy, BwdWs ws, int L, int H, int P, int N,
-              int G, int Q, int nc) {
+              int G, int Q, int nc, int packed) {
     extern __shared__ float sm[];
     float *s_C = sm;                 // kTK * N
     float *s_W = s_C + kTK * N;      // kTK * P
@@ -143,7 +164,9 @@ dstate_kernel(const T *__restrict__ Cm, const float *__restrict__ dy, BwdWs ws, 
         }
         for (int e = threadIdx.x; e < kk * P; e += kThreads) {
             const int k = e / P, pp = e - k * P;
-            const float w = expf(fminf(ws.f.cum[bh * L + t0 + k0 + k], 0.f));
+            // packed rows: only the chunk's first document reads the entering state
+            const bool first = !packed || ws.docc[(size_t)b * L + t0 + k0 + k] == 0.f;
+            const float w = first ? expf(fminf(ws.f.cum[bh * L + t0 + k0 + k], 0.f)) : 0.f;
             s_W[e] = w * dy[(((size_t)b * L + t0 + k0 + k) * H + h) * P + pp];
         }
         __syncthreads();
@@ -228,19 +251,19 @@ __device__ __forceinline__ void pair_dots(const float *sC, const float *sB, int 
 
 size_t cols_smem(const ScanDims &d) {
     const size_t ldn = d.N + 1, ldp = d.P + 1;
-    return sizeof(float) * (2 * kT * ldn + 2 * kT * ldp + 2 * kT * (kT + 1) + 2 * 16 * kT + 6 * kT);
+    return sizeof(float) * (2 * kT * ldn + 2 * kT * ldp + 2 * kT * (kT + 1) + 2 * 16 * kT + 8 * kT);
 }
 
 size_t rows_smem(const ScanDims &d) {
     const size_t ldn = d.N + 1, ldp = d.P + 1;
-    return sizeof(float) * (2 * kT * ldn + 2 * kT * ldp + kT * (kT + 1) + 5 * kT);
+    return sizeof(float) * (2 * kT * ldn + 2 * kT * ldp + kT * (kT + 1) + 7 * kT);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 cols_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restrict__ Cm,
             const float *__restrict__ D, const float *__restrict__ dy, BwdWs ws, float *__restrict__ dx,
-            float *__restrict__ dB, int L, int H, int P, int N, int G, int Q, int nc) {
+            float *__restrict__ dB, int L, int H, int P, int N, int G, int Q, int nc, int packed) {
     extern __shared__ float sm[];
     const int ldn = N + 1, ldp = P + 1;
     float *sB = sm;                        // kT x ldn   (j tile)
@@ -257,6 +280,8 @@ cols_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
     float *s_dst = s_cumi + kT;            // d(dt_j) from the state term
     float *s_E = s_dst + kT;               // E_j
     float *s_dyx = s_E + kT;               // dy_j . x_j
+    float *s_docj = s_dyx + kT;            // packed rows: document counters of the j tile
+    float *s_doci = s_docj + kT;           // and of the i tile
 
     const int tiles = (Q + kT - 1) / kT;
     const int c = blockIdx.x / tiles, jt = blockIdx.x - c * tiles;
@@ -282,9 +307,11 @@ cols_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
         sX[r * ldp + p] = r < tj ? to_f(x[(((size_t)b * L + t0 + j0 + r) * H + h) * P + p]) : 0.f;
     }
     const float cl = ws.f.cum[bh * L + t0 + q - 1];
+    const float dl = packed ? ws.docc[(size_t)b * L + t0 + q - 1] : 0.f;
     for (int r = tid; r < kT; r += kThreads) {
         s_cumj[r] = r < tj ? ws.f.cum[bh * L + t0 + j0 + r] : 0.f;
         s_dtj[r] = r < tj ? ws.f.dtv[bh * L + t0 + j0 + r] : 0.f;
+        s_docj[r] = (packed && r < tj) ? ws.docc[(size_t)b * L + t0 + j0 + r] : 0.f;
     }
     // G_c, the gradient of the state after this chunk
     float *sG = sC;
@@ -334,7 +361,8 @@ cols_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
         e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
         e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
         e1 += __shfl_xor_sync(0xffffffffu, e1, 4);
-        const float dec = jj < tj ? expf(fminf(cl - s_cumj[jj], 0.f)) : 0.f;
+        // packed rows: only the chunk's last document writes into the state it passes on
+        const float dec = (jj < tj && s_docj[jj] == dl) ? expf(fminf(cl - s_cumj[jj], 0.f)) : 0.f;
 #pragma unroll
         for (int k = 0; k < kMaxP / 8; ++k) adx[r][k] *= dec;
 #pragma unroll
@@ -358,7 +386,10 @@ cols_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
             const int r = e / P, p = e - r * P;
             sDY[r * ldp + p] = r < ti ? dy[(((size_t)b * L + t0 + i0 + r) * H + h) * P + p] : 0.f;
         }
-        for (int r = tid; r < kT; r += kThreads) s_cumi[r] = r < ti ? ws.f.cum[bh * L + t0 + i0 + r] : 0.f;
+        for (int r = tid; r < kT; r += kThreads) {
+            s_cumi[r] = r < ti ? ws.f.cum[bh * L + t0 + i0 + r] : 0.f;
+            s_doci[r] = (packed && r < ti) ? ws.docc[(size_t)b * L + t0 + i0 + r] : 0.f;
+        }
         __syncthreads();
         if (i0 == j0) {                    // the diagonal tile: dy_j . x_j
 #pragma unroll
@@ -383,7 +414,7 @@ cols_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
                 const int ii = ig + 16 * a;
-                const bool ok = ii < ti && jj < tj && i0 + ii >= j0 + jj;
+                const bool ok = ii < ti && jj < tj && i0 + ii >= j0 + jj && s_doci[ii] == s_docj[jj];
                 const float lw = ok ? expf(fminf(s_cumi[ii] - s_cumj[jj], 0.f)) : 0.f;
                 const float u = cb[a][bb] * lw, v = sx[a][bb] * lw;
                 sU[ii * (kT + 1) + jj] = u;
@@ -455,7 +486,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 rows_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restrict__ Cm,
             const float *__restrict__ dy, BwdWs ws, float *__restrict__ dC, int L, int H, int P, int N, int G,
-            int Q, int nc) {
+            int Q, int nc, int packed) {
     extern __shared__ float sm[];
     const int ldn = N + 1, ldp = P + 1;
     float *sC = sm;                        // kT x ldn   (i tile)
@@ -468,6 +499,8 @@ rows_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
     float *s_dtj = s_cumj + kT;
     float *s_T = s_dtj + kT;               // e^{cum_i} C_i^T H_in dy_i
     float *s_rs = s_T + kT;                // sum_{j<i} M_ij
+    float *s_doci = s_rs + kT;             // packed rows: document counters of the i tile
+    float *s_docj = s_doci + kT;           // and of the j tile
 
     const int tiles = (Q + kT - 1) / kT;
     const int c = blockIdx.x / tiles, it = blockIdx.x - c * tiles;
@@ -491,7 +524,10 @@ rows_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
         const int r = e / P, p = e - r * P;
         sDY[r * ldp + p] = r < ti ? dy[(((size_t)b * L + t0 + i0 + r) * H + h) * P + p] : 0.f;
     }
-    for (int r = tid; r < kT; r += kThreads) s_cumi[r] = r < ti ? ws.f.cum[bh * L + t0 + i0 + r] : 0.f;
+    for (int r = tid; r < kT; r += kThreads) {
+        s_cumi[r] = r < ti ? ws.f.cum[bh * L + t0 + i0 + r] : 0.f;
+        s_doci[r] = (packed && r < ti) ? ws.docc[(size_t)b * L + t0 + i0 + r] : 0.f;
+    }
     float *sH = sB;
     const float *Hin = ws.f.states + (bh * nc + c) * (size_t)N * P;
     for (int e = tid; e < N * P; e += kThreads) {
@@ -526,7 +562,8 @@ rows_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
         tv += __shfl_xor_sync(0xffffffffu, tv, 1);
         tv += __shfl_xor_sync(0xffffffffu, tv, 2);
         tv += __shfl_xor_sync(0xffffffffu, tv, 4);
-        const float dec = ii < ti ? expf(fminf(s_cumi[ii], 0.f)) : 0.f;
+        // packed rows: the entering state reaches only the chunk's first document
+        const float dec = (ii < ti && s_doci[ii] == 0.f) ? expf(fminf(s_cumi[ii], 0.f)) : 0.f;
 #pragma unroll
         for (int k = 0; k < kMaxN / 8; ++k) adc[r][k] *= dec;
         if (pc == 0) s_T[ii] = dec * tv;
@@ -547,6 +584,7 @@ rows_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
         for (int r = tid; r < kT; r += kThreads) {
             s_cumj[r] = r < tj ? ws.f.cum[bh * L + t0 + j0 + r] : 0.f;
             s_dtj[r] = r < tj ? ws.f.dtv[bh * L + t0 + j0 + r] : 0.f;
+            s_docj[r] = (packed && r < tj) ? ws.docc[(size_t)b * L + t0 + j0 + r] : 0.f;
         }
         __syncthreads();
         float cb[4][4], sx[4][4];
@@ -558,7 +596,7 @@ rows_kernel(const T *__restrict__ x, const T *__restrict__ Bm, const T *__restri
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
                 const int jj = jg + 16 * bb;
-                const bool ok = ii < ti && jj < tj && i0 + ii >= j0 + jj;
+                const bool ok = ii < ti && jj < tj && i0 + ii >= j0 + jj && s_doci[ii] == s_docj[jj];
                 const float v = ok ? sx[a][bb] * expf(fminf(s_cumi[ii] - s_cumj[jj], 0.f)) * s_dtj[jj] : 0.f;
                 sV[ii * (kT + 1) + jj] = v;
                 m += (i0 + ii > j0 + jj) ? cb[a][bb] * v : 0.f;
@@ -715,9 +753,14 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
     const int L = (int)d.L, H = (int)d.H, P = (int)d.P, N = (int)d.N, G = (int)d.G, Q = (int)d.Q;
     const int nc = (int)d.nc, NP = N * P;
     const dim3 gc((unsigned)nc, (unsigned)H, (unsigned)d.b);
+    const int packed = a.f.seq_idx ? 1 : 0;
+    if (packed) {
+        docs_kernel<<<dim3((unsigned)nc, (unsigned)d.b), kThreads, 0, s>>>(a.f.seq_idx, ws.docc, L, Q);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     {
         TraceScope tr(s, kTrBwdDstate);
-        dstate_kernel<T><<<gc, kThreads, smd, s>>>((const T *)a.f.C, a.dy, ws, L, H, P, N, G, Q, nc);
+        dstate_kernel<T><<<gc, kThreads, smd, s>>>((const T *)a.f.C, a.dy, ws, L, H, P, N, G, Q, nc, packed);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int nblk = dpass_blocks(d);
@@ -734,13 +777,13 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
     {
         TraceScope tr(s, kTrBwdCols);
         cols_kernel<T><<<gp, kThreads, smc, s>>>((const T *)a.f.x, (const T *)a.f.B, (const T *)a.f.C, a.f.D,
-                                                 a.dy, ws, a.dx, dBh, L, H, P, N, G, Q, nc);
+                                                 a.dy, ws, a.dx, dBh, L, H, P, N, G, Q, nc, packed);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
         TraceScope tr(s, kTrBwdRows);
         rows_kernel<T><<<gp, kThreads, smr, s>>>((const T *)a.f.x, (const T *)a.f.B, (const T *)a.f.C, a.dy, ws,
-                                                 dCh, L, H, P, N, G, Q, nc);
+                                                 dCh, L, H, P, N, G, Q, nc, packed);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {

@@ -31,7 +31,8 @@ EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_chunk_sc
             "ssd_read_device_status", "ssd_status_string", "ssd_last_cuda_error", "ssd_version",
             "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count",
             "ssd_conv1d_silu_split", "ssd_gated_rmsnorm", "ssd_chunk_scan_fwd_varlen",
-            "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd")
+            "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd", "ssd_chunk_scan_bwd_varlen",
+            "ssd_set_test_fault")
 
 _lib = None
 
@@ -66,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_chunk_scan_bwd_workspace_size.argtypes = [i64] * 7 + [i32, ctypes.POINTER(sz)]
     lib.ssd_chunk_scan_bwd.restype = i32
     lib.ssd_chunk_scan_bwd.argtypes = [vp] * 18 + [i64] * 7 + [f32, f32, i32, vp, sz, vp]
+    lib.ssd_chunk_scan_bwd_varlen.restype = i32
+    lib.ssd_chunk_scan_bwd_varlen.argtypes = [vp] * 19 + [i64] * 7 + [f32, f32, i32, vp, sz, vp]
     lib.ssd_step.restype = i32
     lib.ssd_step.argtypes = [vp] * 9 + [i64] * 5 + [f32, f32, i32, vp]
     lib.ssd_read_device_status.restype = i32
@@ -260,12 +263,14 @@ def chunk_scan_bwd(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor,
                    dfinal_state: Optional[torch.Tensor] = None, init_state: Optional[torch.Tensor] = None,
                    chunk_size: int = 256, dt_limit: Tuple[float, float] = (0.0, math.inf),
                    workspace: Optional[torch.Tensor] = None, want_dinit: bool = True,
-                   out: Optional[dict] = None) -> dict:
-    """Deterministic backward of chunk_scan_fwd (ssd_chunk_scan_bwd): the
-    gradients of <dy, y> + <dfinal_state, final_state> with respect to every
-    input, float32, keyed by input name ("x", "dt_raw", "dt_bias", "A", "B",
-    "C", "D", "init_state"; the last None unless want_dinit).  `out` may hold
-    preallocated outputs under the same keys."""
+                   out: Optional[dict] = None, seq_idx: Optional[torch.Tensor] = None) -> dict:
+    """Deterministic backward of chunk_scan_fwd (ssd_chunk_scan_bwd), or of
+    chunk_scan_fwd_varlen with the same seq_idx [b, L] int32 (packed rows,
+    ssd_chunk_scan_bwd_varlen): the gradients of <dy, y> + <dfinal_state,
+    final_state> with respect to every input, float32, keyed by input name
+    ("x", "dt_raw", "dt_bias", "A", "B", "C", "D", "init_state"; the last None
+    unless want_dinit).  `out` may hold preallocated outputs under the same
+    keys."""
     lib = load_library()
     if x.dim() != 4 or B.dim() != 4:
         raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
@@ -300,13 +305,16 @@ def chunk_scan_bwd(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor,
     need = bwd_workspace_size(b, L, H, P, N, G, Q, x.dtype)
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    st = lib.ssd_chunk_scan_bwd(
-        _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(dy),
+    if seq_idx is not None:
+        _need_cuda("seq_idx", seq_idx, torch.int32, (b, L))
+    st = lib.ssd_chunk_scan_bwd_varlen(
+        _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state), _ptr(seq_idx),
+        _ptr(dy),
         _ptr(dfinal_state), _ptr(g["x"]), _ptr(g["dt_raw"]), _ptr(g["dt_bias"]), _ptr(g["A"]), _ptr(g["B"]),
         _ptr(g["C"]), _ptr(g["D"]), _ptr(g["init_state"]), b, L, H, P, N, G, Q, float(dt_limit[0]),
         float(dt_limit[1]), DTYPES[x.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(dev))
-    _check("ssd_chunk_scan_bwd", st)
+    _check("ssd_chunk_scan_bwd_varlen" if seq_idx is not None else "ssd_chunk_scan_bwd", st)
     return g
 
 

@@ -136,3 +136,75 @@ def test_backward_130m_layer():
     got = run_bwd(inp, grads, cfg.chunk_size)
     ref = oracle_bwd(inp, grads)
     check_all(got, ref, "c1_130m", tol=TOL_BWD_FULL)
+
+
+# ---- packed rows (ssd_chunk_scan_bwd_varlen) ---------------------------------
+
+def _packed_ids(b, L, Q, rng, mean_len):
+    """Document ids with random lengths down to one token, a start exactly on
+    a chunk boundary and on a 64-token pair-tile edge, and a one-token
+    document at tokens 5..5."""
+    seq = np.zeros((b, L), np.int32)
+    for bi in range(b):
+        cuts = set(int(c) for c in rng.integers(1, L, size=max(1, L // mean_len)))
+        cuts.update({c for c in (Q, 64, 5, 6) if 0 < c < L})
+        doc = 0
+        for t in range(L):
+            if t in cuts:
+                doc += 1
+            seq[bi, t] = doc
+    return seq
+
+
+def run_bwd_packed(inp, grads, Q, seq):
+    d = to_dev(inp)
+    b, L, H, P = d["x"].shape
+    G, N = d["B"].shape[2], d["B"].shape[3]
+    ws = ssd.alloc_workspace(ssd.bwd_workspace_size(b, L, H, P, N, G, Q, d["x"].dtype), "cuda")
+    g = ssd.chunk_scan_bwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], grads["dy"].cuda(),
+                           dfinal_state=grads["dfinal"].cuda(), init_state=d["init_state"], chunk_size=Q,
+                           workspace=ws, seq_idx=torch.from_numpy(seq).cuda())
+    assert ssd.read_device_status(ws) == 0
+    torch.cuda.synchronize()
+    return {k: v.cpu().double().numpy() for k, v in g.items()}
+
+
+PACKED_CASES = [
+    # b, L, H, P, N, G, Q, dtype, mean document length
+    (2, 300, 4, 64, 128, 2, 64, "f32", 40),
+    (2, 300, 4, 64, 128, 2, 256, "bf16", 70),
+    (1, 200, 2, 32, 64, 2, 100, "f32", 25),
+    (2, 130, 3, 8, 8, 3, 7, "f32", 9),
+    (1, 257, 4, 64, 128, 1, 128, "f32", 3),      # documents of about three tokens
+]
+
+
+@pytest.mark.parametrize("case", PACKED_CASES, ids=lambda c: "b%d_L%d_H%d_P%d_N%d_G%d_Q%d_%s_doc%d" % c)
+def test_backward_packed_rows(case):
+    """Every gradient of a packed row against the oracle's reverse mode with
+    the same document ids (pinned by finite differences of the packed forward
+    and by 'a packed row's gradients are its documents' own')."""
+    b, L, H, P, N, G, Q, dt, mean_len = case
+    cfg = ScanConfig("bwdp", b, L, H, P, N, G, Q, dt, "normal", "normal", seed=sum(case[:7]) % 1009)
+    inp = make_scan_inputs(cfg)
+    grads = make_grad_inputs(cfg)
+    seq = _packed_ids(b, L, Q, np.random.default_rng(L + Q), mean_len)
+    got = run_bwd_packed(inp, grads, Q, seq)
+    ref = oracle.scan_bwd(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"],
+                          grads["dy"], dfinal=grads["dfinal"], init_state=inp["init_state"], seq_idx=seq)
+    check_all(got, ref, "packed %s" % (case,))
+
+
+def test_backward_packed_constant_ids_is_the_plain_backward():
+    """One document per row: the packed backward equals the plain one bit for
+    bit (every mask passes), and two packed calls give the same bits."""
+    cfg = ScanConfig("bwdc", 2, 300, 4, 64, 128, 2, 64, "bf16", "normal", "normal", seed=913)
+    inp = make_scan_inputs(cfg)
+    grads = make_grad_inputs(cfg)
+    seq = np.full((2, 300), 7, np.int32)
+    a = run_bwd_packed(inp, grads, 64, seq)
+    b_ = run_bwd_packed(inp, grads, 64, seq)
+    plain = run_bwd(inp, grads, 64)
+    for k in KEYS:
+        assert np.array_equal(a[k], plain[k]), "d%s differs from the plain backward" % k
+        assert np.array_equal(a[k], b_[k]), "d%s differs between two calls" % k

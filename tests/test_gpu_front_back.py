@@ -56,10 +56,10 @@ def test_conv1d_parity(K, dtype):
 
 
 @pytest.mark.parametrize("zdtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("group", [16, 64, 256])
+@pytest.mark.parametrize("group", [16, 64, 256, 512, 1536])   # 512, 1536: the single-pass block kernel
 def test_gated_rmsnorm_parity(group, zdtype):
     g = torch.Generator().manual_seed(group)
-    T, D = 300, 256
+    T, D = 300, 3072                           # a multiple of every group size above
     y = torch.randn(T, D, generator=g)
     z = torch.randn(T, D, generator=g).to(zdtype)
     w = torch.rand(D, generator=g) + 0.5
