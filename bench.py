@@ -511,6 +511,86 @@ def bench_stage(cfg, args, local, peaks, peak_kind):
             "clocks": clk}
 
 
+def bench_conv_scan(cfg, args, local, peaks, peak_kind):
+    """--stage conv_scan (and nested in the default scan line): the conv1d
+    (width 4, bf16) and the scan in the two arrangements on the workload's
+    shapes.  split: ssd_conv1d_silu_split writes x, B, C, then
+    ssd_chunk_scan_fwd reads them; combined: ssd_conv_scan_fwd reads xbc and
+    convolves inside the scan's kernels.  Same inputs, K steps of each in one
+    CUDA graph, inputs rotated past L2.  Bytes are the algorithmic HBM bytes
+    of each arrangement: the split one also writes and reads x, B and C."""
+    from state_space_sequence_scan_b200 import ssd
+    dev = torch.device("cuda", local)
+    b, L, H, P, N, G = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.ngroups
+    Q = cfg.chunk_size
+    Cd = H * P + 2 * G * N
+    xbc_bytes = 2.0 * b * L * Cd
+    scan_b = scan_bytes(cfg)
+    split_bytes = 2 * xbc_bytes + scan_b                 # conv reads xbc, writes x|B|C; the scan reads them
+    comb_bytes = scan_b                                  # xbc in place of x, B, C (the same bytes)
+    nsets = max(1, min(8, math.ceil(3 * L2_BYTES / split_bytes)))
+    gen = torch.Generator().manual_seed(cfg.seed + 91)
+    inp = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in make_scan_inputs(cfg).items()}
+    w = (torch.randn(Cd, 4, generator=gen) / 2).to(dev)
+    bias = (0.1 * torch.randn(Cd, generator=gen)).to(dev)
+    sets = [torch.randn(b, L, Cd, generator=gen).to(torch.bfloat16).to(dev) for _ in range(nsets)]
+    xs = [(torch.empty(b, L, H, P, dtype=torch.bfloat16, device=dev),
+           torch.empty(b, L, G, N, dtype=torch.bfloat16, device=dev),
+           torch.empty(b, L, G, N, dtype=torch.bfloat16, device=dev)) for _ in range(nsets)]
+    ys = [torch.empty(b, L, H, P, device=dev) for _ in range(nsets)]
+    fs = torch.empty(b, H, N, P, device=dev)
+    wsz = ssd.workspace_size(b, L, H, P, N, G, Q, torch.bfloat16, "tensor")
+    wsp = ssd.alloc_workspace(wsz, dev)
+    lib = ssd.load_library()
+    stream = torch.cuda.current_stream(dev)
+
+    def split(k):
+        x, B, C = xs[k % nsets]
+        st = lib.ssd_conv1d_silu_split(sets[k % nsets].data_ptr(), w.data_ptr(), bias.data_ptr(), x.data_ptr(),
+                                       B.data_ptr(), C.data_ptr(), b, L, H, P, G, N, 4, 1, stream.cuda_stream)
+        if st != 0:
+            raise RuntimeError("ssd_conv1d_silu_split: %d" % st)
+        ssd.chunk_scan_fwd(x, inp["dt_raw"], inp["dt_bias"], inp["A"], B, C, inp["D"], init_state=inp["init_state"],
+                           chunk_size=Q, path="tensor", workspace=wsp, y=ys[k % nsets], final_state=fs)
+
+    def combined(k):
+        ssd.conv_scan_fwd(sets[k % nsets], w, bias, inp["dt_raw"], inp["dt_bias"], inp["A"], inp["D"], H, P, G, N,
+                          init_state=inp["init_state"], chunk_size=Q, workspace=wsp, y=ys[k % nsets],
+                          final_state=fs)
+
+    res = {}
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for nm, fn in (("split", split), ("combined", combined)):
+        for k in range(args.warmup):
+            fn(k)
+        torch.cuda.synchronize()
+        graph = capture_steps(fn, args.steps)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        byt = split_bytes if nm == "split" else comb_bytes
+        res[nm] = {"ms_per_step": ms, "mtokens_per_s": b * L / (ms * 1e-3) / 1e6, "hbm_bytes": byt,
+                   "hbm_gbs": byt / (ms * 1e-3) / 1e9}
+        del graph
+    clk = clocks.stop()
+    if ssd.read_device_status(wsp) != 0 or ssd.read_device_status(None) != 0:
+        raise RuntimeError("conv_scan: device status not ok")
+    return {"stage": "conv_scan", "metric": "conv1d + scan Mtokens/s (combined arrangement)",
+            "value": res["combined"]["mtokens_per_s"], "unit": "Mtokens/s", "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "dtype": "bf16-in/f32",
+            "config": {"workload": cfg.name, "batch": b, "seqlen": L, "heads": H, "head_dim": P, "groups": G,
+                       "state_dim": N, "chunk_size": Q, "conv_width": 4, "l2": "rotating %d sets" % nsets},
+            "arrangements": res, "bytes_saved": split_bytes - comb_bytes,
+            "speedup_combined_over_split": res["split"]["ms_per_step"] / res["combined"]["ms_per_step"],
+            "clocks": clk}
+
+
 # fp32 FMA throughput of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 flop x
 # 1965 MHz (the clocks.max.sm of these B200s) = 74.45 TFLOP/s.
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
@@ -808,8 +888,11 @@ def main():
                     help="the scan also writes the chunk-boundary states [b, nc, H, N, P] (f32) every step")
     ap.add_argument("--packed", action="store_true",
                     help="rows packed with documents of about 512 tokens (seq_idx)")
-    ap.add_argument("--stage", default="scan", choices=["scan", "conv1d", "gated_norm", "backward"],
-                    help="time one of the steps either side of the scan instead (one GPU)")
+    ap.add_argument("--stage", default="scan", choices=["scan", "conv1d", "gated_norm", "backward", "conv_scan"],
+                    help="time one of the steps either side of the scan, the backward, or the conv and the "
+                         "scan in both arrangements instead (one GPU)")
+    ap.add_argument("--no-conv-scan", action="store_true",
+                    help="leave the conv + scan arrangements (split, combined) out of the default scan run")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -826,7 +909,7 @@ def main():
         cfg, is_step = pick(args.workload)
         if args.stage != "scan" and not is_step:
             if rank == 0:
-                fn = bench_backward if args.stage == "backward" else bench_stage
+                fn = {"backward": bench_backward, "conv_scan": bench_conv_scan}.get(args.stage, bench_stage)
                 print(json.dumps(fn(cfg, args, local, peaks, peak_kind)), flush=True)
             return
         if is_step:
@@ -864,6 +947,8 @@ def main():
         if not is_step and ws == 1 and not args.no_backward and out is not None:
             bcfg, _ = pick(args.backward_workload)
             out["backward"] = bench_backward(bcfg, args, local, peaks, peak_kind)
+        if not is_step and ws == 1 and not args.no_conv_scan and out is not None and cfg.dtype == "bf16":
+            out["conv_scan"] = bench_conv_scan(cfg, args, local, peaks, peak_kind)
         if rank == 0 and out is not None:
             if ws == 1 and not args.no_cpu_baseline:
                 cb = cpu_baseline_step(cfg) if is_step else cpu_baseline_scan(cfg)

@@ -218,11 +218,43 @@ SSD_API ssd_status ssd_chunk_scan_fwd_varlen(const void *x, const float *dt_raw,
  *   weight [Cd, K] and bias [Cd] float32; K = kernel_width, 1..4.
  *   in_dtype  ssd_dtype of xbc, x, B, C.
  * nheads*head_dim and ngroups*state_dim must be multiples of 8; xbc, x, B
- * and C 16-byte aligned and not overlapping.  Queued on `stream`. */
+ * and C 16-byte aligned and not overlapping; seqlen below 2^31 - 128 and
+ * seqlen*Cd*4 below 2^40 (SSD_ERR_UNSUPPORTED otherwise).  Queued on
+ * `stream`.  Its waits on its own copies are bounded: one that gives up
+ * (about 2 s) leaves SSD_ERR_DEVICE_TIMEOUT for ssd_read_device_status(NULL,
+ * stream), and the outputs undefined. */
 SSD_API ssd_status ssd_conv1d_silu_split(const void *xbc, const float *weight, const float *bias, void *x,
                                  void *B, void *C, int64_t batch, int64_t seqlen, int64_t nheads,
                                  int64_t head_dim, int64_t ngroups, int64_t state_dim,
                                  int64_t kernel_width, int in_dtype, void *stream);
+
+/* The conv1d and the scan in the combined arrangement (the HF transformers
+ * issue "mamba2 mixer different outputs" contrasts a fused
+ * mamba_split_conv1d_scan_combined with causal_conv1d_fn followed by
+ * mamba_chunk_scan_combined): y and final_state of ssd_chunk_scan_fwd on the
+ * x, B and C that ssd_conv1d_silu_split would write from xbc, without writing
+ * them.  The scan's kernels read xbc itself: each 128-token block's x tile
+ * arrives with the 3 rows before it and is convolved in shared memory, and
+ * the fp16 copies of B and C are convolved where they are made.  The
+ * arithmetic is the split conv's (each value rounded to bf16 as that conv
+ * stores it), so the two arrangements give the same bits.
+ *   xbc      [batch, seqlen, Cd] bf16, Cd = nheads*head_dim + 2*ngroups*state_dim
+ *            (channels x | B | C), 16-byte aligned
+ *   conv_w   [Cd, 4] float32, conv_b [Cd] float32, both 16-byte aligned
+ *   kernel_width  4 (else SSD_ERR_UNSUPPORTED)
+ *   the rest as for ssd_chunk_scan_fwd on the tensor-core path: in_dtype
+ *   SSD_BF16, head_dim 64, state_dim 128, chunk_size 64, 128 or 256 (else
+ *   SSD_ERR_UNSUPPORTED); workspace of ssd_chunk_scan_workspace_size(...,
+ *   SSD_PATH_TENSOR) bytes; status word as for ssd_chunk_scan_fwd.
+ * No packed rows and no chunk states here (use the split arrangement).
+ * Queued on `stream`. */
+SSD_API ssd_status ssd_conv_scan_fwd(const void *xbc, const float *conv_w, const float *conv_b,
+                                     int64_t kernel_width, const float *dt_raw, const float *dt_bias,
+                                     const float *A, const float *D, const float *init_state, float *y,
+                                     float *final_state, int64_t batch, int64_t seqlen, int64_t nheads,
+                                     int64_t head_dim, int64_t state_dim, int64_t ngroups, int64_t chunk_size,
+                                     float dt_lo, float dt_hi, int in_dtype, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /* The gated RMS norm that takes y after the scan (nnterp guide "Mamba-2",
  * table "The values": y is taken before the gated norm and out_proj):
@@ -299,7 +331,10 @@ SSD_API ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw,
 
 /* Waits for `stream`, then reads the device status word that the last
  * ssd_chunk_scan_fwd on this workspace left: SSD_OK, SSD_ERR_PRECONDITION or
- * SSD_ERR_DEVICE_TIMEOUT.  `workspace` is a device pointer. */
+ * SSD_ERR_DEVICE_TIMEOUT.  `workspace` is a device pointer.  With workspace
+ * NULL it reads, and then clears, the current device's status word of the
+ * kernels that take no workspace (ssd_conv1d_silu_split): SSD_OK or
+ * SSD_ERR_DEVICE_TIMEOUT since the last such read. */
 SSD_API ssd_status ssd_read_device_status(const void *workspace, void *stream);
 
 /* Text for a status code (static storage; never NULL). */
@@ -334,7 +369,8 @@ SSD_API ssd_status ssd_set_test_fault(int kind);
 
 /* ABI version: (major << 16) | minor.  1.1 added the chunk-state, packed-row,
  * conv/norm and backward entry points to the 1.0 scan and step; 1.2 the test
- * hook ssd_set_test_fault and ssd_chunk_scan_bwd_varlen. */
+ * hook ssd_set_test_fault and ssd_chunk_scan_bwd_varlen; 1.3
+ * ssd_conv_scan_fwd and the workspace-free status read. */
 SSD_API int ssd_version(void);
 
 #ifdef __cplusplus

@@ -83,7 +83,7 @@ size_t path_ws(const ssd::ScanDims &d, int chosen) {
 
 extern "C" {
 
-int ssd_version(void) { return (1 << 16) | 2; }
+int ssd_version(void) { return (1 << 16) | 3; }
 
 ssd_status ssd_set_test_fault(int kind) {
     if (kind != 0 && kind != 1) return SSD_ERR_INVALID_ARG;
@@ -129,14 +129,19 @@ ssd_status scan_fwd(const void *x, const float *dt_raw, const float *dt_bias, co
                     const void *C, const float *D, const float *init_state, const int32_t *seq_idx, float *y,
                     float *final_state, float *chunk_states, int64_t batch, int64_t seqlen, int64_t nheads,
                     int64_t head_dim, int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo,
-                    float dt_hi, int in_dtype, int path, void *workspace, size_t workspace_bytes, void *stream) {
+                    float dt_hi, int in_dtype, int path, void *workspace, size_t workspace_bytes, void *stream,
+                    const float *conv_w = nullptr, const float *conv_b = nullptr) {
     ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size,
                                     in_dtype, path);
     if (st != SSD_OK) return st;
     if (!limits_ok(dt_lo, dt_hi)) return SSD_ERR_INVALID_ARG;
     if (!dt_bias || !A || !D) return SSD_ERR_INVALID_ARG;
     const bool has_tokens = batch > 0 && seqlen > 0;
-    if (has_tokens && (!x || !dt_raw || !B || !C || !y)) return SSD_ERR_INVALID_ARG;
+    // the combined arrangement: x is xbc, B and C are inside it
+    const bool conv = conv_w != nullptr;
+    if (conv && (!conv_b || !aligned16(conv_w) || !aligned16(conv_b)))
+        return !conv_b ? SSD_ERR_INVALID_ARG : SSD_ERR_ALIGNMENT;
+    if (has_tokens && (!x || !dt_raw || (!conv && (!B || !C)) || !y)) return SSD_ERR_INVALID_ARG;
     if ((x && !aligned16(x)) || (B && !aligned16(B)) || (C && !aligned16(C)) || (y && !aligned16(y)) ||
         (init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)) ||
         (chunk_states && !aligned16(chunk_states)))
@@ -170,6 +175,11 @@ ssd_status scan_fwd(const void *x, const float *dt_raw, const float *dt_bias, co
     a.init_state = init_state; a.y = y; a.final_state = final_state; a.chunk_states = chunk_states;
     a.seq_idx = seq_idx;
     a.dt_lo = dt_lo; a.dt_hi = dt_hi; a.bf16 = in_dtype == SSD_BF16;
+    if (conv) {
+        a.conv_w = conv_w;
+        a.conv_b = conv_b;
+        a.Cd = nheads * head_dim + 2 * ngroups * state_dim;
+    }
     e = chosen == SSD_PATH_TENSOR ? ssd::tc_scan(a, d, workspace, s) : ssd::simt_scan(a, d, workspace, s);
     if (e != cudaSuccess) return cuda_fail(e);
     return SSD_OK;
@@ -211,6 +221,20 @@ ssd_status ssd_chunk_scan_fwd_varlen(const void *x, const float *dt_raw, const f
     return scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state, seq_idx, y, final_state, chunk_states, batch,
                     seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, path, workspace,
                     workspace_bytes, stream);
+}
+
+ssd_status ssd_conv_scan_fwd(const void *xbc, const float *conv_w, const float *conv_b, int64_t kernel_width,
+                             const float *dt_raw, const float *dt_bias, const float *A, const float *D,
+                             const float *init_state, float *y, float *final_state, int64_t batch, int64_t seqlen,
+                             int64_t nheads, int64_t head_dim, int64_t state_dim, int64_t ngroups,
+                             int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    if (!conv_w) return SSD_ERR_INVALID_ARG;
+    // the tensor path's shapes, bf16, width 4 (the conv runs inside its kernels)
+    if (kernel_width != 4 || in_dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
+    return scan_fwd(xbc, dt_raw, dt_bias, A, nullptr, nullptr, D, init_state, nullptr, y, final_state, nullptr, batch,
+                    seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, SSD_PATH_TENSOR,
+                    workspace, workspace_bytes, stream, conv_w, conv_b);
 }
 
 ssd_status ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
@@ -318,11 +342,15 @@ ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_bias, co
 }
 
 ssd_status ssd_read_device_status(const void *workspace, void *stream) {
-    if (!workspace) return SSD_ERR_INVALID_ARG;
     unsigned word = 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaError_t e;
+    if (!workspace) {
+        e = ssd::front_status_read(s, &word);
+    } else {
+        e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    }
     if (e != cudaSuccess) return cuda_fail(e);
     if (word & ssd::kStatusTimeout) return SSD_ERR_DEVICE_TIMEOUT;
     if (word & (ssd::kStatusPrecondition | ssd::kStatusRange)) return SSD_ERR_PRECONDITION;

@@ -25,6 +25,27 @@ __device__ __forceinline__ float dt_of(float raw, float bias, float lo, float hi
     return fminf(fmaxf(softplus_f(raw + bias), lo), hi);
 }
 
+// silu(u) = u / (1 + e^-u) with the fast exponential and division (relative
+// error about 1e-6: inside the fp32 bar of 1e-5 and one bf16 rounding).  For
+// u below about -87, e^-u is inf and the quotient is the limit, 0.
+__device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
+
+// The causal depthwise conv of one channel at one token, then SiLU:
+// silu(bias + sum_{k<K} w[k] x[k]), x[K-1] the current token's input and
+// x[0] the oldest.  Two chains of fmas (even k, odd k), added at the end.
+// Both arrangements of the conv (split and combined with the scan) evaluate
+// exactly this, so they agree bit for bit.
+template <int K>
+__device__ __forceinline__ float conv_silu(const float (&w)[K], const float (&x)[K], float bias) {
+    float a0 = bias, a1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        if (k & 1) a1 = fmaf(w[k], x[k], a1);
+        else a0 = fmaf(w[k], x[k], a0);
+    }
+    return silu_f(a0 + a1);
+}
+
 template <typename T> __device__ __forceinline__ float to_f(T v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {

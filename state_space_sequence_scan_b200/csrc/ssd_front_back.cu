@@ -7,27 +7,45 @@
 //                      separate x, B and C tensors (the split arrangement)
 //   gated_rmsnorm      v = y * silu(z), RMS-normalised over groups of
 //                      channels, times a per-channel weight
-// Both are HBM-bound streams: coalesced vector loads and stores, one pass
-// over the data (the norm holds a group in registers; groups that do not
-// split evenly over its CTA take a two-pass warp kernel, the second read
-// from L1/L2).
+// Both are HBM-bound streams with one pass over the data.  The conv stages
+// its input tiles in shared memory by TMA, several tiles in flight per CTA,
+// and stores from registers; its SiLU costs two special-function operations
+// an element, so it also needs enough warps to keep that unit busy.  The
+// norm holds a group in registers (groups that do not split evenly over its
+// CTA take a two-pass warp kernel, the second read from L1/L2).
+#include <cuda.h>
+
 #include "../../include/ssd.h"
 #include "ssd_common.cuh"
 #include "ssd_internal.h"
+#include "ssd_tc.cuh"
+#include "ssd_tmap.h"
 #include "ssd_trace.h"
 
 namespace ssd {
 namespace {
 
-constexpr int kConvThreads = 256;
-constexpr int kConvCh = 4;      // channels per thread (one 8- or 16-byte access per token)
-constexpr int kConvT = 16;      // tokens per thread (a sliding window in registers)
+constexpr int kConvCh = 4;                    // channels per lane (one 8- or 16-byte access per token)
 constexpr int kConvMaxK = 4;
+constexpr int kCvWarps = 16;
+constexpr int kCvThreads = 32 * kCvWarps;
+constexpr int kCvTC = 32 * kConvCh;           // channels per tile: one warp across
+constexpr int kCvTokPerWarp = 8;
+constexpr int kCvTT = kCvWarps * kCvTokPerWarp;  // tokens per tile
+constexpr int kCvHalo = kConvMaxK - 1;        // rows before the tile's first token
+constexpr int kCvRows = kCvHalo + kCvTT;      // rows per tile in shared memory
+constexpr long long kCvWaitBudget = 1ll << 32;  // clock cycles before a wait gives up (~2 s)
+// tiles in flight per CTA: 3 x 33.5 KB (bf16: two 16-warp CTAs per SM, the
+// most that 56 registers a thread allow), 3 x 67 KB (fp32: one CTA per SM)
+template <typename T> struct CvStages { static constexpr int value = 3; };
+template <typename T> constexpr size_t cv_smem_bytes() {
+    return (size_t)CvStages<T>::value * kCvRows * kCvTC * sizeof(T) + 8 * CvStages<T>::value;
+}
 
-// silu(u) = u / (1 + e^-u) with the fast exponential and division (relative
-// error about 1e-6: inside the fp32 bar of 1e-5 and one bf16 rounding).  For
-// u below about -87, e^-u is inf and the quotient is the limit, 0.
-__device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
+// Status word of the workspace-free kernels (conv1d): kStatusTimeout when a
+// bounded wait gave up.  Read and cleared by ssd_read_device_status(NULL, ...).
+__device__ unsigned g_front_status = 0;
+
 
 // 4 consecutive z values -> floats
 __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&v)[4]) {
@@ -51,25 +69,61 @@ __device__ __forceinline__ void store4(float *p, const float (&v)[4]) {
     *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
 }
 
-// One token tile [t0, t0 + kConvT) of 4 channels from c0 (see conv1d_silu_kernel).
+// Persistent conv1d + SiLU over tiles of kCvTT tokens x kCvTC channels.
+// Tile rows arrive in shared memory by TMA (a 3-D map over xbc [b, L, Cd],
+// box kCvTC x (kCvHalo + kCvTT) x 1, zero fill out of range: the rows before
+// token 0 and past L, and the channels past Cd, read as zeros), CvStages
+// tiles in flight per CTA.  Shared row r of a tile holds token
+// t0 - kCvHalo + r.  Warp w computes tokens [8w, 8w + 8) of the tile,
+// lane l channels [4l, 4l + 4), sliding a K-row window down shared memory,
+// and stores its outputs straight to x, B or C (8 or 16 bytes per lane, 256
+// or 512 bytes per warp and row).  CTA i keeps channel tile i % n_ct for its
+// whole life (its weights stay in registers) and walks the (batch, token
+// tile) rows i / n_ct, i / n_ct + rows_step, ...
+// out[t, c] = silu(bias[c] + sum_k w[c, k] in[t - (K-1) + k, c]), in[t < 0] = 0.
 template <typename T, int K>
-__device__ __forceinline__ void conv1d_silu_tile(const T *__restrict__ xbc, const float *__restrict__ w,
-                                                 const float *__restrict__ bias, T *__restrict__ x,
-                                                 T *__restrict__ Bo, T *__restrict__ Co, int L, int Cd, int HP,
-                                                 int GN, int c0, int t0, size_t b) {
+__global__ void __launch_bounds__(kCvThreads, 2)   // two CTAs per SM: at most 64 registers
+conv1d_silu_kernel(const __grid_constant__ CUtensorMap tm, const float *__restrict__ w,
+                   const float *__restrict__ bias, T *__restrict__ x, T *__restrict__ Bo, T *__restrict__ Co, int L,
+                   int Cd, int HP, int GN, int n_ct, int n_tt, long long n_rows, int rows_step,
+                   unsigned *__restrict__ status, long long wait_budget) {
+    constexpr int S = CvStages<T>::value;
+    constexpr uint32_t kStageBytes = (uint32_t)(kCvRows * kCvTC * sizeof(T));
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * kStageBytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ct = blockIdx.x % n_ct;
+    const long long row0 = blockIdx.x / n_ct;
+    if (tid == 0) {
+        tc::tma_prefetch_desc(&tm);
+        for (int i = 0; i < S; ++i) tc::mbar_init(&full[i], 1);
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    // request the tile of (batch, token tile) row `row` into stage `st`
+    auto request = [&](long long row, int st) {
+        const int tt = (int)(row % n_tt), bb = (int)(row / n_tt);
+        tc::mbar_arrive_expect_tx(&full[st], kStageBytes);
+        tc::tma_load_3d(smem + st * kStageBytes, &tm, &full[st], ct * kCvTC, tt * kCvTT - kCvHalo, bb);
+    };
+    if (tid == 0)
+        for (int i = 0; i < S; ++i)
+            if (row0 + (long long)i * rows_step < n_rows) request(row0 + (long long)i * rows_step, i);
+
+    // this lane's 4 channels, their weights and destination
+    const int c0 = ct * kCvTC + lane * kConvCh;
+    const bool live = c0 < Cd;
     float wr[kConvCh][K], bs[kConvCh];
 #pragma unroll
     for (int e = 0; e < kConvCh; ++e) {
-        bs[e] = bias[c0 + e];
+        bs[e] = live ? bias[c0 + e] : 0.f;
 #pragma unroll
-        for (int k = 0; k < K; ++k) wr[e][k] = w[(size_t)(c0 + e) * K + k];
+        for (int k = 0; k < K; ++k) wr[e][k] = live ? w[(size_t)(c0 + e) * K + k] : 0.f;
     }
-    // where these channels go: x [b,L,H*P], B or C [b,L,G*N] (H*P, G*N are multiples of 8)
-    T *dst;
-    int ld;
+    T *dst = x;
+    int ld = HP;
     if (c0 < HP) {
         dst = x + c0;
-        ld = HP;
     } else if (c0 < HP + GN) {
         dst = Bo + (c0 - HP);
         ld = GN;
@@ -77,49 +131,62 @@ __device__ __forceinline__ void conv1d_silu_tile(const T *__restrict__ xbc, cons
         dst = Co + (c0 - HP - GN);
         ld = GN;
     }
-    const T *src = xbc + b * L * (size_t)Cd + c0;
-    dst += b * L * (size_t)ld;
-    // rows t0-(K-1) .. t0+kConvT-1, all loaded before any arithmetic or store
-    // (dst may not be proven apart from src, so a load after a store would
-    // wait for it; 16 + K-1 independent loads keep enough bytes in flight)
-    float win[K - 1 + kConvT][kConvCh];
-    const int tn = min(kConvT, L - t0);
-#pragma unroll
-    for (int k = 0; k < K - 1 + kConvT; ++k) {
-        const int t = t0 - (K - 1) + k;
-        if (t >= 0 && k - (K - 1) < tn) load4(src + (size_t)t * Cd, win[k]);
-        else {
-#pragma unroll
-            for (int e = 0; e < kConvCh; ++e) win[k][e] = 0.f;
+
+    int it = 0;
+    bool timed_out = false;
+    for (long long row = row0; row < n_rows; row += rows_step, ++it) {
+        const int st = it % S;
+        const bool ok = tc::mbar_wait(&full[st], (uint32_t)(it / S) & 1u, wait_budget);
+        // one decision for the whole CTA; the barrier also says that every
+        // warp is done with the previous tile, whose stage is refilled now
+        if (!__syncthreads_and(ok)) {
+            timed_out = true;
+            break;
         }
-    }
+        if (tid == 0 && it > 0) {
+            const long long nxt = row + (long long)(S - 1) * rows_step;
+            if (nxt < n_rows) request(nxt, (it - 1) % S);
+        }
+        const int tt = (int)(row % n_tt);
+        const size_t bb = (size_t)(row / n_tt);
+        const int tbase = tt * kCvTT + warp * kCvTokPerWarp;     // first output token of this warp
+        const T *src = reinterpret_cast<const T *>(smem + st * kStageBytes) + lane * kConvCh;
+        // window of the K input rows of the current output token
+        float win[K][kConvCh];
 #pragma unroll
-    for (int j = 0; j < kConvT; ++j) {
-        if (j < tn) {
+        for (int k = 0; k < K - 1; ++k)
+            load4(src + (warp * kCvTokPerWarp + kCvHalo - (K - 1) + k) * kCvTC, win[k]);
+        T *out = dst + bb * (size_t)L * ld;
+#pragma unroll
+        for (int j = 0; j < kCvTokPerWarp; ++j) {
+            load4(src + (warp * kCvTokPerWarp + kCvHalo + j) * kCvTC, win[K - 1]);
             float o[kConvCh];
 #pragma unroll
             for (int e = 0; e < kConvCh; ++e) {
-                float acc = bs[e];
+                float xw[K];
 #pragma unroll
-                for (int k = 0; k < K; ++k) acc = fmaf(wr[e][k], win[j + k][e], acc);
-                o[e] = silu_f(acc);
+                for (int k = 0; k < K; ++k) xw[k] = win[k][e];
+                o[e] = conv_silu<K>(wr[e], xw, bs[e]);
             }
-            store4(dst + (size_t)(t0 + j) * ld, o);
+            if (live && tbase + j < L) store4(out + (size_t)(tbase + j) * ld, o);
+#pragma unroll
+            for (int k = 0; k < K - 1; ++k)
+#pragma unroll
+                for (int e = 0; e < kConvCh; ++e) win[k][e] = win[k + 1][e];
         }
     }
+    if (timed_out && tid == 0) {
+        atomicOr(status, kStatusTimeout);
+        // let this CTA's copies still in flight land before its shared memory
+        // goes away (each wait bounded again): iterations it .. last were
+        // requested and not consumed (the first S at the start, then one
+        // S - 1 ahead of each consumed iteration after the first)
+        const int last = it == 0 ? S - 1 : it + S - 2;
+        for (int j = it; j <= last; ++j)
+            if (row0 + (long long)j * rows_step < n_rows)
+                tc::mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, wait_budget);
+    }
 }
-
-// grid (ceil(L/kConvT), ceil(Cd/4/256), b): thread = 4 channels x kConvT tokens.
-// out[t, c] = silu(bias[c] + sum_k w[c, k] in[t - (K-1) + k, c]), in[t < 0] = 0.
-template <typename T, int K>
-__global__ void __launch_bounds__(kConvThreads)
-conv1d_silu_kernel(const T *__restrict__ xbc, const float *__restrict__ w, const float *__restrict__ bias,
-                   T *__restrict__ x, T *__restrict__ Bo, T *__restrict__ Co, int L, int Cd, int HP, int GN) {
-    const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * kConvCh;
-    if (c0 >= Cd) return;
-    conv1d_silu_tile<T, K>(xbc, w, bias, x, Bo, Co, L, Cd, HP, GN, c0, blockIdx.x * kConvT, blockIdx.z);
-}
-
 
 // One CTA of kNormThreads per (token, group) when the group splits evenly
 // into kNormThreads x V float4s: v = y silu(z) stays in registers, one read
@@ -219,28 +286,101 @@ gated_rmsnorm_kernel(const float *__restrict__ y, const Tz *__restrict__ z, cons
     }
 }
 
+constexpr int kCvMaxDevices = 64;
+
+// SM count and resident conv CTAs per SM on the current device, and the
+// shared-memory limit set for the kernel, once per (device, type, width)
+template <typename T, int K>
+cudaError_t conv_slots(int *slots) {
+    static int cached[kCvMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kCvMaxDevices) return cudaErrorInvalidDevice;
+    if (!cached[dev]) {
+        const int smem = (int)cv_smem_bytes<T>();
+        if ((e = cudaFuncSetAttribute(conv1d_silu_kernel<T, K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+            cudaSuccess)
+            return e;
+        int sms = 0, per_sm = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv1d_silu_kernel<T, K>, kCvThreads,
+                                                               smem)) != cudaSuccess)
+            return e;
+        cached[dev] = sms * (per_sm > 0 ? per_sm : 1);
+    }
+    *slots = cached[dev];
+    return cudaSuccess;
+}
+
+cudaError_t front_status_ptr(unsigned **p) {
+    static unsigned *cached[kCvMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kCvMaxDevices) return cudaErrorInvalidDevice;
+    if (!cached[dev]) {
+        void *q = nullptr;
+        if ((e = cudaGetSymbolAddress(&q, g_front_status)) != cudaSuccess) return e;
+        cached[dev] = static_cast<unsigned *>(q);
+    }
+    *p = cached[dev];
+    return cudaSuccess;
+}
+
+template <typename T, int K>
+cudaError_t conv_launch_k(const void *xbc, const float *w, const float *bias, void *x, void *B, void *C, int64_t b,
+                          int64_t L, int Cd, int HP, int GN, cudaStream_t s) {
+    CUtensorMap tm;
+    const uint64_t dims[3] = {(uint64_t)Cd, (uint64_t)L, (uint64_t)b};
+    const uint64_t strides[2] = {(uint64_t)Cd * sizeof(T), (uint64_t)L * Cd * sizeof(T)};
+    const uint32_t box[3] = {(uint32_t)kCvTC, (uint32_t)kCvRows, 1u};
+    if (!tmap_encode_3d_plain(&tm, xbc, sizeof(T) == 2 ? kTmapBF16 : kTmapF32, dims, strides, box))
+        return cudaErrorInvalidValue;
+    int slots = 0;
+    unsigned *status = nullptr;
+    cudaError_t e = conv_slots<T, K>(&slots);
+    if (e == cudaSuccess) e = front_status_ptr(&status);
+    if (e != cudaSuccess) return e;
+    const int n_ct = (Cd + kCvTC - 1) / kCvTC;
+    const int n_tt = (int)((L + kCvTT - 1) / kCvTT);
+    const long long n_rows = b * (long long)n_tt;
+    long long step = slots / n_ct;
+    if (step < 1) step = 1;
+    if (step > n_rows) step = n_rows;
+    const unsigned grid = (unsigned)(n_ct * step);
+    conv1d_silu_kernel<T, K><<<grid, kCvThreads, cv_smem_bytes<T>(), s>>>(
+        tm, w, bias, (T *)x, (T *)B, (T *)C, (int)L, Cd, HP, GN, n_ct, n_tt, n_rows, (int)step, status, kCvWaitBudget);
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t conv_launch(const void *xbc, const float *w, const float *bias, void *x, void *B, void *C, int64_t b,
                         int64_t L, int Cd, int HP, int GN, int K, cudaStream_t s) {
-    const dim3 g((unsigned)((L + kConvT - 1) / kConvT), (unsigned)((Cd / kConvCh + kConvThreads - 1) / kConvThreads),
-                 (unsigned)b);
     TraceScope tr(s, kTrConv1d);
-#define SSD_CONV(KK)                                                                                           \
-    conv1d_silu_kernel<T, KK><<<g, kConvThreads, 0, s>>>((const T *)xbc, w, bias, (T *)x, (T *)B, (T *)C,     \
-                                                         (int)L, Cd, HP, GN)
     switch (K) {
-        case 1: SSD_CONV(1); break;
-        case 2: SSD_CONV(2); break;
-        case 3: SSD_CONV(3); break;
-        default: SSD_CONV(4); break;
+        case 1: return conv_launch_k<T, 1>(xbc, w, bias, x, B, C, b, L, Cd, HP, GN, s);
+        case 2: return conv_launch_k<T, 2>(xbc, w, bias, x, B, C, b, L, Cd, HP, GN, s);
+        case 3: return conv_launch_k<T, 3>(xbc, w, bias, x, B, C, b, L, Cd, HP, GN, s);
+        default: return conv_launch_k<T, 4>(xbc, w, bias, x, B, C, b, L, Cd, HP, GN, s);
     }
-#undef SSD_CONV
-    return cudaGetLastError();
 }
 
 bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+// Reads and clears the workspace-free kernels' status word on the current
+// device (synchronises the stream).
+cudaError_t front_status_read(cudaStream_t s, unsigned *word) {
+    unsigned *p = nullptr;
+    cudaError_t e = front_status_ptr(&p);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemcpyAsync(word, p, sizeof(unsigned), cudaMemcpyDeviceToHost, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(p, 0, sizeof(unsigned), s)) != cudaSuccess) return e;
+    return cudaStreamSynchronize(s);
+}
+
 }  // namespace ssd
 
 extern "C" SSD_API ssd_status ssd_conv1d_silu_split(const void *xbc, const float *weight, const float *bias,
@@ -253,8 +393,9 @@ extern "C" SSD_API ssd_status ssd_conv1d_silu_split(const void *xbc, const float
     if (kernel_width < 1 || kernel_width > ssd::kConvMaxK) return SSD_ERR_UNSUPPORTED;
     if (in_dtype != SSD_F32 && in_dtype != SSD_BF16) return SSD_ERR_UNSUPPORTED;
     const int64_t HP = nheads * head_dim, GN = ngroups * state_dim, Cd = HP + 2 * GN;
-    // grid: token tiles in x, 256-thread channel blocks in y (<= 65535), batch in z
-    if (HP % 8 || GN % 8 || Cd > (1 << 24) || batch > 65535 || seqlen > (1ll << 31) - ssd::kConvT)
+    // TMA coordinates are 32-bit and the map's strides below 2^40 bytes
+    if (HP % 8 || GN % 8 || Cd > (1 << 24) || batch > (1 << 30) || seqlen > (1ll << 31) - 2 * ssd::kCvTT ||
+        seqlen * Cd * 4 >= (1ll << 40))
         return SSD_ERR_UNSUPPORTED;
     if (batch == 0 || seqlen == 0) return SSD_OK;
     if (!xbc || !weight || !bias || !x || !B || !C) return SSD_ERR_INVALID_ARG;

@@ -22,6 +22,12 @@ struct ScanArgs {
     const int32_t *seq_idx = nullptr;  // [b, L] document ids of packed rows, or null (SIMT path)
     float dt_lo, dt_hi;
     int bf16;                      // 1: x/B/C are bfloat16, 0: float32
+    // the combined arrangement (tensor path): x points at xbc [b, L, Cd] (the
+    // conv's input, channels x | B | C), B and C are unused, and x, B, C are
+    // conv1d + SiLU of xbc computed inside the scan's kernels (width 4)
+    const float *conv_w = nullptr;  // [Cd, 4]
+    const float *conv_b = nullptr;  // [Cd]
+    int64_t Cd = 0;
 };
 
 struct StepArgs {
@@ -81,5 +87,9 @@ int tc_test_fault();
 // ---- decode step ------------------------------------------------------------
 bool step_supported(int64_t P, int64_t N);
 cudaError_t step_launch(const StepArgs &a, cudaStream_t s);
+
+// Reads and clears the status word of the kernels that take no workspace
+// (conv1d); waits for `s`.
+cudaError_t front_status_read(cudaStream_t s, unsigned *word);
 
 }  // namespace ssd

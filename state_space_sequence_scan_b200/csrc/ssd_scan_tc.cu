@@ -80,6 +80,9 @@ constexpr double kCtaStartRel = 2.0;
 constexpr int64_t kMaxUnits = 4096;
 constexpr int kMaxAttrDevices = 64;
 constexpr uint32_t kTileBytes = 16384;          // one 128-row x 128-byte swizzled tile
+constexpr int kConvK = 4;                        // conv width of the combined arrangement
+constexpr int kXRaw = kBlk + kConvK - 1;         // input rows of a block's conv (3 before it)
+constexpr uint32_t kXRawBytes = kXRaw * 128;     // 16768: the raw X tile, 128 bytes a row
 
 struct TcWs {
     unsigned *status;
@@ -169,7 +172,15 @@ bool make_maps(const ScanArgs &a, const ScanDims &d, const TcPlan &p, const TcWs
     const uint64_t b = d.b, L = d.L, H = d.H, G = d.G, Lp = p.nblk * kBlk;
     const uint32_t box_h[4] = {64, 1, kBlk, 1};
     const uint32_t box_y[4] = {32, 1, kBlk, 1};
-    {
+    if (a.conv_w) {
+        // combined arrangement: the x channels of xbc [b, L, Cd], a block's 128
+        // tokens and the conv's 3 rows before them
+        const uint64_t Cd = a.Cd;
+        const uint32_t box_x[4] = {64, 1, (uint32_t)kXRaw, 1};
+        const uint64_t dims[4] = {kP, H, L, b};
+        const uint64_t st[3] = {kP * 2, Cd * 2, L * Cd * 2};
+        if (!tmap_encode_4d(&m->x, a.x, kTmapBF16, dims, st, box_x)) return false;
+    } else {
         const uint64_t dims[4] = {kP, H, L, b};
         const uint64_t st[3] = {kP * 2, H * kP * 2, L * H * kP * 2};
         if (!tmap_encode_4d(&m->x, a.x, kTmapBF16, dims, st, box_h)) return false;
@@ -212,6 +223,88 @@ __device__ __forceinline__ void bf16_chunk_to_f32(uint4 v, float *f) {
     f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
 }
 
+// ---- the combined arrangement: conv1d + SiLU inside the scan's kernels
+// A value the split conv would store as bf16, back in fp32.
+__device__ __forceinline__ float bf16_round(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+
+// Channels 4q..4q+3 of the bf16 row r of an X-type tile (128-byte-swizzled,
+// 64 channels a row): the 8-byte half (q & 1) of chunk q >> 1.
+__device__ __forceinline__ uint32_t xq_off(int r, int q) {
+    return (uint32_t)r * 128u + ((((uint32_t)q >> 1) ^ ((uint32_t)r & 7u)) << 4) + ((uint32_t)q & 1u) * 8u;
+}
+
+
+// In place on a 64-channel X tile that holds kXRaw raw input rows (row r' =
+// token t0 - 3 + r'): row r becomes conv1d + SiLU of token t0 + r, rounded to
+// bf16 (as the split conv stores x).  kScaled false (chunk_out): stored as
+// bf16; rows at or past L become 0 (as the TMA fills x there).  kScaled true
+// (unit_state): times w[r] in fp32, stored as fp16 (the w.X operand), the
+// largest magnitude tracked in `amax`.  256 threads take 4 channels x 8 rows
+// each: all read their 11 input rows, meet at named barrier 1, then write.
+// `wb` holds the 64 channels' weights (float4 each) then their biases.  Every
+// thread of the barrier calls this; `ok` false skips the reads and writes.
+template <bool kScaled>
+__device__ __forceinline__ void conv_x_tile(uint8_t *sx, const float4 *wb, int tid, int t0, int L, bool ok,
+                                            const float *w_row = nullptr, __half2 *amax = nullptr) {
+    const int q = tid & 15, rg = tid >> 4;
+    uint2 rw[8 + kConvK - 1];
+    if (ok) {
+#pragma unroll
+        for (int j = 0; j < 8 + kConvK - 1; ++j) rw[j] = *reinterpret_cast<const uint2 *>(sx + xq_off(8 * rg + j, q));
+    }
+    named_bar_sync(256);
+    if (!ok) return;
+    float w[4][kConvK], bias[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float4 v = wb[4 * q + e];
+        w[e][0] = v.x; w[e][1] = v.y; w[e][2] = v.z; w[e][3] = v.w;
+    }
+    {
+        const float4 v = wb[64 + q];
+        bias[0] = v.x; bias[1] = v.y; bias[2] = v.z; bias[3] = v.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int r = 8 * rg + j;
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float xw[kConvK];
+#pragma unroll
+            for (int k = 0; k < kConvK; ++k) {
+                const uint32_t u = (e < 2) ? rw[j + k].x : rw[j + k].y;
+                xw[k] = (e & 1) ? bf16hi(u) : bf16lo(u);
+            }
+            o[e] = conv_silu<kConvK>(w[e], xw, bias[e]);
+        }
+        uint2 out;
+        if (kScaled) {
+            const float wr = w_row[r];
+            const uint32_t h0 = pack_h2(bf16_round(o[0]) * wr, bf16_round(o[1]) * wr);
+            const uint32_t h1 = pack_h2(bf16_round(o[2]) * wr, bf16_round(o[3]) * wr);
+            *amax = __hmax2(*amax, __habs2(*reinterpret_cast<const __half2 *>(&h0)));
+            *amax = __hmax2(*amax, __habs2(*reinterpret_cast<const __half2 *>(&h1)));
+            out = make_uint2(h0, h1);
+        } else {
+            const bool live = t0 + r < L;
+            const __nv_bfloat162 a = __floats2bfloat162_rn(live ? o[0] : 0.f, live ? o[1] : 0.f);
+            const __nv_bfloat162 c = __floats2bfloat162_rn(live ? o[2] : 0.f, live ? o[3] : 0.f);
+            out = make_uint2(*reinterpret_cast<const uint32_t *>(&a), *reinterpret_cast<const uint32_t *>(&c));
+        }
+        *reinterpret_cast<uint2 *>(sx + xq_off(r, q)) = out;
+    }
+}
+
+// The 64 x channels of head h: weights [64][4] then biases [64] into `wb`
+// (a float4 each for the weights, 16 float4s of biases)
+__device__ __forceinline__ void conv_load_weights(float4 *wb, const float *cw, const float *cb, int h, int tid,
+                                                  int nthreads) {
+    for (int i = tid; i < 64 + 16; i += nthreads)
+        wb[i] = i < 64 ? *reinterpret_cast<const float4 *>(cw + ((size_t)h * kP + i) * kConvK)
+                       : *reinterpret_cast<const float4 *>(cb + (size_t)h * kP + 4 * (i - 64));
+}
+
 // ---------------------------------------------------------------------------
 // prep: grid (nblk, ceil(H/8) + 4 G, b), 256 threads.  y-slices below
 // ceil(H/8) do dt/cum for 8 heads of one 128-token block; the rest convert a
@@ -222,7 +315,8 @@ constexpr int kPrepHeads = 8;
 __global__ void __launch_bounds__(256)
 prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias, const float *__restrict__ A,
             const __nv_bfloat16 *__restrict__ Bm, const __nv_bfloat16 *__restrict__ Cm,
-            const int32_t *__restrict__ seq_idx, TcWs ws, int L, int H, int G, int nblk, float lo, float hi) {
+            const int32_t *__restrict__ seq_idx, TcWs ws, int L, int H, int G, int nblk, float lo, float hi,
+            const float *__restrict__ cw, const float *__restrict__ cb, int Cd) {
     __shared__ float s_dt[kPrepHeads][kBlk + 4];
     __shared__ float s_da[kPrepHeads][kBlk + 4];
     pdl_launch_dependents();                     // the next kernel waits for this one's writes itself
@@ -233,6 +327,47 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
         const int t0 = blk * kBlk + 32 * quarter;
         const size_t Lp = (size_t)nblk * kBlk;
         __half2 amax = __float2half2_rn(0.f);
+        if (cw) {
+            // combined arrangement: B and C are conv1d + SiLU of xbc's channels
+            // H*P + g*N.. (B) and H*P + G*N + g*N.. (C), rounded to bf16 as the
+            // split conv stores them.  Thread: one tensor, one 8-channel chunk,
+            // 4 consecutive rows, from a window of the 3 rows before them too
+            const int HP = Cd - 2 * G * kN;
+            const int which = threadIdx.x >> 7, kk = threadIdx.x & 15, r0 = 4 * ((threadIdx.x >> 4) & 7);
+            const size_t ch0 = (size_t)HP + (size_t)which * G * kN + (size_t)g * kN + kk * 8;
+            uint4 v[4 + kConvK - 1];
+#pragma unroll
+            for (int j = 0; j < 4 + kConvK - 1; ++j) {
+                const int tt = t0 + r0 - (kConvK - 1) + j;
+                v[j] = make_uint4(0u, 0u, 0u, 0u);
+                if (tt >= 0 && tt < L)
+                    v[j] = __ldg(reinterpret_cast<const uint4 *>(Bm + ((size_t)b * L + tt) * Cd + ch0));
+            }
+            float4 wv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) wv[e] = __ldg(reinterpret_cast<const float4 *>(cw + (ch0 + e) * kConvK));
+            const float4 b0 = __ldg(reinterpret_cast<const float4 *>(cb + ch0));
+            const float4 b1 = __ldg(reinterpret_cast<const float4 *>(cb + ch0 + 4));
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float xin[4 + kConvK - 1][8];
+#pragma unroll
+            for (int j = 0; j < 4 + kConvK - 1; ++j) bf16_chunk_to_f32(v[j], xin[j]);
+            __half *dst = which ? ws.Ch : ws.Bh;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = t0 + r0 + j;
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float w4[kConvK] = {wv[e].x, wv[e].y, wv[e].z, wv[e].w};
+                    const float xw[kConvK] = {xin[j][e], xin[j + 1][e], xin[j + 2][e], xin[j + 3][e]};
+                    f[e] = t < L ? bf16_round(conv_silu<kConvK>(w4, xw, bv[e])) : 0.f;
+                }
+                *reinterpret_cast<uint4 *>(dst + (((size_t)b * Lp + t) * G + g) * kN + kk * 8) = pack8(f, amax);
+            }
+            if (!in_f16_range(amax)) flag_status(ws.status, kStatusRange);
+            return;
+        }
         // 2 tensors x 32 rows x 16 chunks of 8: four chunks per thread, all loads first
         uint4 v[4];
 #pragma unroll
@@ -331,14 +466,23 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
 // is in the last unit), so every block here is a full 128 tokens.
 constexpr int kUsCompute = 256;
 constexpr int kUsThreads = kUsCompute + 32;
-constexpr uint32_t kUsStage = 3 * kTileBytes + 2 * kBlk * 4;  // B (2 tiles) + X (1 tile) + dt + cum
-constexpr uint32_t kUsOffW = 2 * kUsStage;                     // w [2][128]
-constexpr uint32_t kUsOffBar = kUsOffW + 2 * kBlk * 4;         // tma[2], mma[2], converted[2]
-constexpr size_t kUsSmem = 1024 + kUsOffBar + 6 * 8 + 16;
+// stage: B (2 tiles), X (1 tile; kXRaw rows in the combined arrangement), dt, cum
+template <bool kConv> struct UsLayout {
+    static constexpr uint32_t kXBytes = kConv ? kXRawBytes : kTileBytes;
+    static constexpr uint32_t kTx = 2 * kTileBytes + kXBytes + 2 * kBlk * 4;    // bytes a stage receives
+    static constexpr uint32_t kStage = (kTx + 1023) & ~1023u;                  // 1024-aligned stages
+    static constexpr uint32_t kOffW = 2 * kStage;                              // w [2][128]
+    static constexpr uint32_t kOffCw = kOffW + 2 * kBlk * 4;                   // conv weights [80] float4
+    static constexpr uint32_t kOffBar = kOffCw + (kConv ? 80 * 16 : 0);        // tma[2], mma[2], converted[2]
+    static constexpr size_t kSmem = 1024 + kOffBar + 6 * 8 + 16;
+};
 
+template <bool kConv>
 __global__ void __launch_bounds__(kUsThreads, 2)
 unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, int nblk, int U, int bpu,
-                  int packed) {
+                  int packed, const float *__restrict__ cw, const float *__restrict__ cb) {
+    using Lay = UsLayout<kConv>;
+    constexpr uint32_t kUsStage = Lay::kStage, kUsOffW = Lay::kOffW, kUsOffBar = Lay::kOffBar;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     // per stage: [0,1] TMA landed, [2,3] MMAs done, [4,5] X converted.  One barrier of
@@ -379,12 +523,12 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
             auto load = [&](int s, int k) {
                 uint8_t *st = stage(s);
                 const int t0 = k * kBlk;
-                mbar_arrive_expect_tx(bar + s, kUsStage);
+                mbar_arrive_expect_tx(bar + s, Lay::kTx);
                 tma_load_4d(st, &maps.B, bar + s, 0, g, t0, b);
                 tma_load_4d(st + kTileBytes, &maps.B, bar + s, 64, g, t0, b);
-                tma_load_4d(st + 2 * kTileBytes, &maps.x, bar + s, 0, h, t0, b);
-                bulk_load(st + 3 * kTileBytes, dtg + (size_t)t0, kBlk * 4, bar + s);
-                bulk_load(st + 3 * kTileBytes + kBlk * 4, cumg + (size_t)t0, kBlk * 4, bar + s);
+                tma_load_4d(st + 2 * kTileBytes, &maps.x, bar + s, 0, h, kConv ? t0 - (kConvK - 1) : t0, b);
+                bulk_load(st + 2 * kTileBytes + Lay::kXBytes, dtg + (size_t)t0, kBlk * 4, bar + s);
+                bulk_load(st + 2 * kTileBytes + Lay::kXBytes + kBlk * 4, cumg + (size_t)t0, kBlk * 4, bar + s);
             };
             const uint32_t idesc = idesc_f16(128, 64, 1, 1);
             bool ok = true;
@@ -411,6 +555,8 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
         // ------------------------------ compute warps -------------------------
         __half2 amax = __float2half2_rn(0.f);
         bool ok = true;
+        float4 *cwb = reinterpret_cast<float4 *>(sm + Lay::kOffCw);
+        if (kConv) conv_load_weights(cwb, cw, cb, h, tid, kUsCompute);   // visible after the first barrier below
         // the unit's log decay after the current block (sum of later block totals);
         // packed rows: how many later blocks of the unit hold a document start
         const int *rsb = ws.rs + (size_t)b * nblk * kBlk;
@@ -429,7 +575,7 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
         for (int i = 0; i < nk; ++i) {
             const int s = i & 1;
             uint8_t *st = stage(s);
-            const float *dt = reinterpret_cast<const float *>(st + 3 * kTileBytes);
+            const float *dt = reinterpret_cast<const float *>(st + 2 * kTileBytes + Lay::kXBytes);
             const float *cum = dt + kBlk;
             float *w = reinterpret_cast<float *>(sm + kUsOffW) + s * kBlk;
             ok = ok && mbar_wait_abortable(bar + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
@@ -443,7 +589,10 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
                 if (packed) later -= rsb[(size_t)(kb0 + i + 1) * kBlk + kBlk - 1] >= 0;
             }
             named_bar_sync(kUsCompute);                 // w[] visible
-            if (ok) {
+            if (kConv) {
+                // w.X (fp16) straight from the raw rows: conv1d + SiLU, bf16, times w
+                conv_x_tile<true>(st + 2 * kTileBytes, cwb, tid, 0, 0, ok, w, &amax);
+            } else if (ok) {
                 uint8_t *sx = st + 2 * kTileBytes;      // X (bf16) -> w.X (fp16); row = offset / 128
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
@@ -553,7 +702,8 @@ constexpr int kCoWarps = kCoCompute / 32;
 constexpr int kCoMmaWarp = kCoWarps, kCoTmaWarp = kCoWarps + 1;
 constexpr int kCoThreads = kCoCompute + 64;                     // + MMA warp + TMA warp
 constexpr uint32_t kCoCB = 4 * kTileBytes;                      // C(2 tiles) B(2 tiles) of one block
-constexpr uint32_t kCoXS = kTileBytes + 1024;                   // X tile, dt[128], cum[128]
+// x slot: X (kXRaw rows: room for the combined arrangement's raw rows), dt[128], cum[128]
+constexpr uint32_t kCoXS = (kXRawBytes + 1024 + 1023) & ~1023u;
 constexpr int kCoXSlots = 3;
 constexpr uint32_t kCoOffXS = 2 * kCoCB;                        // x ring
 constexpr uint32_t kCoOffWX = kCoOffXS + kCoXSlots * kCoXS;     // w.X fp16
@@ -563,7 +713,8 @@ constexpr uint32_t kCoOffF = kCoOffH16 + kTileBytes;            // factors [2][3
 constexpr uint32_t kCoOffG = kCoOffF + 2 * kCoFactors * 4;      // diagonal fast-path flags [2][4]
 constexpr uint32_t kCoOffMask = kCoOffG + 8 * 4;                // causal masks of the diagonal [4][32 lanes] x 16 B
 constexpr uint32_t kCoOffIss = kCoOffMask + 32 * 16 * 4;        // issue counters (drain after an abort)
-constexpr uint32_t kCoOffBar = kCoOffIss + 16 * 4;              // mbarriers, TMEM slot, abort flag
+constexpr uint32_t kCoOffCw = kCoOffIss + 16 * 4;               // conv weights [64] + biases [16] float4
+constexpr uint32_t kCoOffBar = kCoOffCw + 80 * 16;              // mbarriers, TMEM slot, abort flag
 constexpr int kCoBars = 13;
 constexpr size_t kCoSmem = 1024 + kCoOffBar + kCoBars * 8 + 16;
 constexpr float kDiagExpCap = 64.0f;                            // largest exponent on the diagonal fast path
@@ -595,7 +746,7 @@ struct CoSmem {
     __device__ uint8_t *C(int s) const { return base + s * kCoCB; }
     __device__ uint8_t *B(int s) const { return base + s * kCoCB + 2 * kTileBytes; }
     __device__ uint8_t *X(int r) const { return base + kCoOffXS + r * kCoXS; }
-    __device__ float *dt(int r) const { return reinterpret_cast<float *>(X(r) + kTileBytes); }
+    __device__ float *dt(int r) const { return reinterpret_cast<float *>(X(r) + kXRawBytes); }
     __device__ float *cum(int r) const { return dt(r) + kBlk; }
     __device__ uint8_t *WX() const { return base + kCoOffWX; }
     __device__ uint8_t *H16() const { return base + kCoOffH16; }
@@ -603,6 +754,7 @@ struct CoSmem {
     __device__ int *G(int s) const { return reinterpret_cast<int *>(base + kCoOffG) + s * 4; }
     __device__ uint4 *Mask() const { return reinterpret_cast<uint4 *>(base + kCoOffMask); }
     __device__ int *issued() const { return reinterpret_cast<int *>(base + kCoOffIss); }
+    __device__ float4 *Cw() const { return reinterpret_cast<float4 *>(base + kCoOffCw); }
     __device__ uint64_t *bar(int i) const { return reinterpret_cast<uint64_t *>(base + kCoOffBar) + i; }
     __device__ uint32_t *tslot() const { return reinterpret_cast<uint32_t *>(bar(kCoBars)); }
     __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(bar(kCoBars)) + 1; }
@@ -635,13 +787,16 @@ __device__ __forceinline__ void co_prefetch_cb(const TcMaps &maps, int k, int g,
     tma_prefetch_4d(&maps.B, 64, g, t0, b);
 }
 
-// TMA: X (bf16), dt and cum rows of block k into x slot r
+// TMA: X (bf16), dt and cum rows of block k into x slot r.  Combined
+// arrangement: the raw x channels of xbc for the block's tokens and the 3
+// before them (zero before token 0).
+template <bool kConv>
 __device__ __forceinline__ void co_load_x(const CoSmem &S, const TcMaps &maps, const float *dtv, const float *cum,
                                           int r, int k, int h, int b) {
     const int t0 = k * kBlk;
     uint64_t *bar = S.bar(kBarTx0 + r);
-    mbar_arrive_expect_tx(bar, kCoXS);
-    tma_load_4d(S.X(r), &maps.x, bar, 0, h, t0, b);
+    mbar_arrive_expect_tx(bar, (kConv ? kXRawBytes : kTileBytes) + 2 * kBlk * 4);
+    tma_load_4d(S.X(r), &maps.x, bar, 0, h, kConv ? t0 - (kConvK - 1) : t0, b);
     bulk_load(S.dt(r), dtv + (size_t)t0, kBlk * 4, bar);
     bulk_load(S.cum(r), cum + (size_t)t0, kBlk * 4, bar);
     ++S.issued()[kBarTx0 + r];
@@ -821,12 +976,13 @@ __device__ __forceinline__ void co_w_slice(const CoSmem &S, int r, int f, uint32
 
 // kPacked: packed rows (the document starts of ws.rs mask W, the C.H term,
 // w.X and the block decay); the unpacked instantiation carries none of it.
-template <bool kPacked>
+template <bool kPacked, bool kConv>
 __global__ void __launch_bounds__(kCoThreads, 1)
 chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ D,
                  const float *__restrict__ init, float *__restrict__ final_state, TcWs ws,
                  int L, int H, int G, int nblk, int U, int bpu, int states_from_ws, int prefetch_cb,
-                 float *__restrict__ chunk_states, int bpc, int nc, long long wait_budget, int test_fault) {
+                 float *__restrict__ chunk_states, int bpc, int nc, long long wait_budget, int test_fault,
+                 const float *__restrict__ cw, const float *__restrict__ cb) {
     extern __shared__ uint8_t smem_raw[];
     CoSmem S;
     S.base = align1024(smem_raw);
@@ -951,14 +1107,15 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
             // that depends on it runs out of budget (the timeout path)
             for (int q = 0; q < 2 && kb0 + q < kb1; ++q)
                 if (q > 0 || test_fault != 1) co_load_cb(S, maps, q, kb0 + q, g, b);
-            for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q) co_load_x(S, maps, dtg, cumg, q, kb0 + q, h, b);
+            for (int q = 0; q < kCoXSlots && kb0 + q < kb1; ++q)
+                co_load_x<kConv>(S, maps, dtg, cumg, q, kb0 + q, h, b);
             if (prefetch_cb && kb0 + 2 < kb1) co_prefetch_cb(maps, kb0 + 2, g, b);
             for (int k = kb0; k < kb1; ++k) {
                 const int i = k - kb0, s = i & 1;
                 if (!mbar_wait_abortable(S.bar(kBarFree0 + s), ((uint32_t)i >> 1) & 1u, wait_budget, abort_flag))
                     break;
                 // block k is done with its x slot; its y sits in its B tiles
-                if (k + kCoXSlots < kb1) co_load_x(S, maps, dtg, cumg, i % kCoXSlots, k + kCoXSlots, h, b);
+                if (k + kCoXSlots < kb1) co_load_x<kConv>(S, maps, dtg, cumg, i % kCoXSlots, k + kCoXSlots, h, b);
                 if (prefetch_cb && k + 3 < kb1) co_prefetch_cb(maps, k + 3, g, b);
                 tma_store_4d(&maps.y, S.B(s), 0, h, k * kBlk, b);
                 tma_store_4d(&maps.y, S.B(s) + kTileBytes, 32, h, k * kBlk, b);
@@ -1026,9 +1183,20 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 S.Mask()[q4 * 32 + ml] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
             }
         }
+        if (kConv) conv_load_weights(S.Cw(), cw, cb, h, tid, kCoCompute);
         // block kb0: x landed -> factors, w.X; then "state ready"
         ok = mbar_wait_abortable(S.bar(kBarTx0), 0, wait_budget, abort_flag);
         if (ok) co_factors(S, 0, 0, min(kBlk - 1, L - 1 - kb0 * kBlk), tid);
+        // combined arrangement: x of the first two blocks now, then each block's
+        // two blocks ahead while W.X runs (the conv weights are read after
+        // conv_x_tile's own barrier)
+        if (kConv) {
+            conv_x_tile<false>(S.X(0), S.Cw(), tid, kb0 * kBlk, L, ok);
+            if (kb0 + 1 < kb1) {
+                ok = ok && mbar_wait_abortable(S.bar(kBarTx0 + 1), 0, wait_budget, abort_flag);
+                conv_x_tile<false>(S.X(1), S.Cw(), tid, (kb0 + 1) * kBlk, L, ok);
+            }
+        }
         named_bar_sync(kCoCompute);                 // factors and masks visible to every compute warp
         // packed rows: document starts of each block (ws.rs, written by prep)
         const int *rsb = ws.rs + (size_t)b * nblk * kBlk;
@@ -1063,7 +1231,7 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 ok = ok && mbar_wait_abortable(S.bar(kBarTx0 + r1), ((uint32_t)(i + 1) / kCoXSlots) & 1u,
                                                wait_budget, abort_flag);
                 if (ok) co_factors(S, r1, f1, min(kBlk - 1, L - 1 - (k + 1) * kBlk), tid);
-                named_bar_sync(kCoCompute);          // factors of block k+1 visible
+                named_bar_sync(kCoCompute);          // factors (and x) of block k+1 visible
             }
 
             // [3] S(k) done (and Z(k), which read the fp16 copy) -> H_in(k+1), w.X(k+1)
@@ -1114,6 +1282,16 @@ chunk_out_kernel(const __grid_constant__ TcMaps maps, const float *__restrict__ 
                 }
             }
             if (k + 1 < kb1) co_arrive(S.bar(kBarH16), lane);
+
+            // [3b] combined arrangement: x of block k+2 (its slot was block k-1's)
+            // while Y(k) runs; read by the compute warps after the next [2]
+            // barrier, and by the MMAs after the next "state ready" arrival
+            if (kConv && k + 2 < kb1) {
+                const int r2 = (i + 2) % kCoXSlots;
+                ok = ok && mbar_wait_abortable(S.bar(kBarTx0 + r2), ((uint32_t)(i + 2) / kCoXSlots) & 1u, wait_budget,
+                                               abort_flag);
+                conv_x_tile<false>(S.X(r2), S.Cw(), tid, (k + 2) * kBlk, L, ok);
+            }
 
             // [4] Y(k) done -> y_i = Y_i + exp(cum_i) Z_i + D x_i -> staging in block k's B tiles
             ok = ok && mbar_wait_abortable(S.bar(kBarY), par, wait_budget, abort_flag);
@@ -1204,24 +1382,33 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxAttrDevices) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        if ((e = cudaFuncSetAttribute(unit_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kUsSmem)) != cudaSuccess)
+        if ((e = cudaFuncSetAttribute(unit_state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)UsLayout<false>::kSmem)) != cudaSuccess)
             return e;
-        if ((e = cudaFuncSetAttribute(chunk_out_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(unit_state_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)UsLayout<true>::kSmem)) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(chunk_out_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kCoSmem)) != cudaSuccess)
             return e;
-        if ((e = cudaFuncSetAttribute(chunk_out_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(chunk_out_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kCoSmem)) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(chunk_out_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kCoSmem)) != cudaSuccess)
             return e;
         attr_done[dev] = true;
     }
+    const bool conv = a.conv_w != nullptr;
     {
         TraceScope tr(s, kTrTcDtPrep);
         // a plain launch: it overwrites the workspace the previous call's kernels read
+        // (combined arrangement: B and C come from xbc, through the conv)
         const unsigned ny = (unsigned)((d.H + kPrepHeads - 1) / kPrepHeads + 4 * d.G);
         prep_kernel<<<dim3((unsigned)p.nblk, ny, (unsigned)d.b), 256, 0, s>>>(
-            a.dt_raw, a.dt_bias, a.A, static_cast<const __nv_bfloat16 *>(a.B), static_cast<const __nv_bfloat16 *>(a.C),
-            a.seq_idx, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk, a.dt_lo, a.dt_hi);
+            a.dt_raw, a.dt_bias, a.A, static_cast<const __nv_bfloat16 *>(conv ? a.x : a.B),
+            static_cast<const __nv_bfloat16 *>(a.C), a.seq_idx, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk,
+            a.dt_lo, a.dt_hi, a.conv_w, a.conv_b, (int)a.Cd);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // the kernels after prep may start their prologue while their predecessor
@@ -1242,9 +1429,12 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
     if (p.U > 1) {
         {
             TraceScope tr(s, kTrTcUnitState);
-            const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kUsThreads, kUsSmem);
-            if ((e = cudaLaunchKernelEx(&c, unit_state_kernel, maps, ws, (int)d.H, (int)d.G, (int)p.nblk, (int)p.U,
-                                        (int)p.bpu, a.seq_idx ? 1 : 0)) != cudaSuccess)
+            const cudaLaunchConfig_t c =
+                cfg(dim3((unsigned)d.H, (unsigned)(p.U - 1), (unsigned)d.b), kUsThreads,
+                    conv ? UsLayout<true>::kSmem : UsLayout<false>::kSmem);
+            if ((e = cudaLaunchKernelEx(&c, conv ? unit_state_kernel<true> : unit_state_kernel<false>, maps, ws,
+                                        (int)d.H, (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu, a.seq_idx ? 1 : 0,
+                                        a.conv_w, a.conv_b)) != cudaSuccess)
                 return e;
         }
         {
@@ -1264,10 +1454,13 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         const cudaLaunchConfig_t c = cfg(dim3((unsigned)d.H, (unsigned)p.U, (unsigned)d.b), kCoThreads, kCoSmem);
         // the caller checked that chunk_states come with chunk_size a multiple of kBlk
         const int bpc = (int)(d.Q / kBlk) > 0 ? (int)(d.Q / kBlk) : 1;
-        if ((e = cudaLaunchKernelEx(&c, a.seq_idx ? chunk_out_kernel<true> : chunk_out_kernel<false>, maps, a.D,
-                                    a.init_state, a.final_state, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk,
-                                    (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0, prefetch_cb, a.chunk_states, bpc,
-                                    (int)d.nc, fault ? kTestWaitBudget : kWaitBudget, fault)) != cudaSuccess)
+        // the combined arrangement takes no packed rows (the caller checked)
+        auto kern = conv ? chunk_out_kernel<false, true>
+                         : (a.seq_idx ? chunk_out_kernel<true, false> : chunk_out_kernel<false, false>);
+        if ((e = cudaLaunchKernelEx(&c, kern, maps, a.D, a.init_state, a.final_state, ws, (int)d.L, (int)d.H,
+                                    (int)d.G, (int)p.nblk, (int)p.U, (int)p.bpu, p.U > 1 ? 1 : 0, prefetch_cb,
+                                    a.chunk_states, bpc, (int)d.nc, fault ? kTestWaitBudget : kWaitBudget, fault,
+                                    a.conv_w, a.conv_b)) != cudaSuccess)
             return e;
     }
     return cudaGetLastError();

@@ -15,4 +15,9 @@ enum TmapElem { kTmapBF16 = 0, kTmapF16 = 1, kTmapF32 = 2 };
 bool tmap_encode_4d(CUtensorMap *map, const void *base, TmapElem elem, const uint64_t dims[4],
                     const uint64_t strides_bytes[3], const uint32_t box[4]);
 
+// 3-D tiled map without swizzle (the box lands in shared memory row after
+// row, box[0] elements per row), zero fill out of range.  Same conventions.
+bool tmap_encode_3d_plain(CUtensorMap *map, const void *base, TmapElem elem, const uint64_t dims[3],
+                          const uint64_t strides_bytes[2], const uint32_t box[3]);
+
 }  // namespace ssd

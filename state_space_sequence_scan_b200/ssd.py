@@ -32,7 +32,7 @@ EXPORTED = ("ssd_chunk_scan_workspace_size", "ssd_chunk_scan_fwd", "ssd_chunk_sc
             "ssd_trace_enable", "ssd_trace_read", "ssd_trace_kernel_name", "ssd_trace_kernel_count",
             "ssd_conv1d_silu_split", "ssd_gated_rmsnorm", "ssd_chunk_scan_fwd_varlen",
             "ssd_chunk_scan_bwd_workspace_size", "ssd_chunk_scan_bwd", "ssd_chunk_scan_bwd_varlen",
-            "ssd_set_test_fault")
+            "ssd_set_test_fault", "ssd_conv_scan_fwd")
 
 _lib = None
 
@@ -93,6 +93,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_conv1d_silu_split.argtypes = [vp] * 6 + [i64] * 7 + [i32, vp]
     lib.ssd_gated_rmsnorm.restype = i32
     lib.ssd_gated_rmsnorm.argtypes = [vp] * 4 + [i64] * 3 + [f32, i32, vp]
+    lib.ssd_conv_scan_fwd.restype = i32
+    lib.ssd_conv_scan_fwd.argtypes = [vp] * 3 + [i64] + [vp] * 7 + [i64] * 7 + [f32, f32, i32, vp, sz, vp]
     _lib = lib
     return lib
 
@@ -389,6 +391,52 @@ def conv1d_silu_split(xbc: torch.Tensor, weight: torch.Tensor, bias: torch.Tenso
     return x, B, C
 
 
+def conv_scan_fwd(xbc: torch.Tensor, conv_weight: torch.Tensor, conv_bias: torch.Tensor, dt_raw: torch.Tensor,
+                  dt_bias: torch.Tensor, A: torch.Tensor, D: torch.Tensor, nheads: int, head_dim: int,
+                  ngroups: int, state_dim: int, init_state: Optional[torch.Tensor] = None, chunk_size: int = 256,
+                  dt_limit: Tuple[float, float] = (0.0, math.inf), workspace: Optional[torch.Tensor] = None,
+                  y: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
+                  want_final_state: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """The conv1d and the scan in the combined arrangement (ssd_conv_scan_fwd):
+    y and final_state of chunk_scan_fwd(*conv1d_silu_split(xbc, ...)) without
+    writing x, B, C.  xbc [b, L, H*P + 2*G*N] bf16, conv_weight [Cd, 4] f32,
+    conv_bias [Cd] f32; the rest as for chunk_scan_fwd (tensor-core shapes)."""
+    lib = load_library()
+    if xbc.dim() != 3:
+        raise ValueError("xbc must be [b, L, Cd]")
+    b, L, Cd = xbc.shape
+    H, P, G, N = int(nheads), int(head_dim), int(ngroups), int(state_dim)
+    if Cd != H * P + 2 * G * N:
+        raise ValueError("xbc has %d channels, not H*P + 2*G*N" % Cd)
+    dev = xbc.device
+    _need_cuda("xbc", xbc, torch.bfloat16)
+    _need_cuda("conv_weight", conv_weight, torch.float32, (Cd, conv_weight.shape[-1]))
+    _need_cuda("conv_bias", conv_bias, torch.float32, (Cd,))
+    _need_cuda("dt_raw", dt_raw, torch.float32, (b, L, H))
+    for nm, t in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need_cuda(nm, t, torch.float32, (H,))
+    if init_state is not None:
+        _need_cuda("init_state", init_state, torch.float32, (b, H, N, P))
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
+    else:
+        _need_cuda("y", y, torch.float32, (b, L, H, P))
+    if want_final_state and final_state is None:
+        final_state = torch.empty((b, H, N, P), dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _need_cuda("final_state", final_state, torch.float32, (b, H, N, P))
+    need = workspace_size(b, L, H, P, N, G, chunk_size, torch.bfloat16, "tensor")
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    st = lib.ssd_conv_scan_fwd(
+        _ptr(xbc), _ptr(conv_weight), _ptr(conv_bias), conv_weight.shape[-1], _ptr(dt_raw), _ptr(dt_bias), _ptr(A),
+        _ptr(D), _ptr(init_state), _ptr(y), _ptr(final_state), b, L, H, P, N, G, int(chunk_size),
+        float(dt_limit[0]), float(dt_limit[1]), DTYPES[xbc.dtype], _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(dev))
+    _check("ssd_conv_scan_fwd", st)
+    return y, final_state
+
+
 def gated_rmsnorm(y: torch.Tensor, z: torch.Tensor, weight: torch.Tensor, group_size: int,
                   eps: float = 1e-5) -> torch.Tensor:
     """out = rmsnorm_over_groups(y * silu(z)) * weight, f32 (ssd_gated_rmsnorm).
@@ -407,9 +455,14 @@ def gated_rmsnorm(y: torch.Tensor, z: torch.Tensor, weight: torch.Tensor, group_
     return out
 
 
-def read_device_status(workspace: torch.Tensor) -> int:
-    """Synchronises the current stream and returns the device status code."""
+def read_device_status(workspace: Optional[torch.Tensor]) -> int:
+    """Synchronises the current stream and returns the device status code of
+    the calls on `workspace`; with None, reads and clears the current
+    device's status of the calls that take no workspace (conv1d)."""
     lib = load_library()
+    if workspace is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        return int(lib.ssd_read_device_status(None, _stream(dev)))
     return int(lib.ssd_read_device_status(_ptr(workspace), _stream(workspace.device)))
 
 

@@ -55,6 +55,26 @@ def test_conv1d_parity(K, dtype):
         _check_conv(got, r, dtype, "conv K=%d %s" % (K, nm))
 
 
+# (b, L, H, P, G, N): channel tiles of 128 with the x|B and B|C edges inside
+# a tile and a partial last tile (Cd = 152); token tiles of 64 with a ragged
+# tail; enough (batch, token tile) rows that each CTA walks its ring of
+# stages several times over
+TILE_CASES = [(3, 200, 3, 24, 1, 40), (2, 130, 2, 8, 3, 8), (4, 71040, 1, 64, 1, 32)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", TILE_CASES, ids=lambda c: "b%d_L%d_H%d_P%d_G%d_N%d" % c)
+def test_conv1d_tile_edges(shape, dtype):
+    b, L, H, P, G, N = shape
+    K = 4
+    xbc, w, bias = _conv_case(b, L, H, P, G, N, K, dtype, seed=L + H)
+    x, B, C = ssd.conv1d_silu_split(xbc.cuda(), w.cuda(), bias.cuda(), H, P, G, N)
+    assert ssd.read_device_status(None) == 0
+    ref = oracle.conv1d_silu(xbc.float().numpy(), w.numpy(), bias.numpy())
+    for got, r, nm in zip((x, B, C), _split(ref, b, L, H, P, G, N), "xBC"):
+        _check_conv(got, r, dtype, "conv %s %s" % (shape, nm))
+
+
 @pytest.mark.parametrize("zdtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("group", [16, 64, 256, 512, 1536])   # 512, 1536: the single-pass block kernel
 def test_gated_rmsnorm_parity(group, zdtype):
