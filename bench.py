@@ -546,8 +546,10 @@ def bench_conv_scan(cfg, args, local, peaks, peak_kind):
 
     def split(k):
         x, B, C = xs[k % nsets]
+        # the stream current at call time: under graph capture, the capturing one
         st = lib.ssd_conv1d_silu_split(sets[k % nsets].data_ptr(), w.data_ptr(), bias.data_ptr(), x.data_ptr(),
-                                       B.data_ptr(), C.data_ptr(), b, L, H, P, G, N, 4, 1, stream.cuda_stream)
+                                       B.data_ptr(), C.data_ptr(), b, L, H, P, G, N, 4, 1,
+                                       torch.cuda.current_stream(dev).cuda_stream)
         if st != 0:
             raise RuntimeError("ssd_conv1d_silu_split: %d" % st)
         ssd.chunk_scan_fwd(x, inp["dt_raw"], inp["dt_bias"], inp["A"], B, C, inp["D"], init_state=inp["init_state"],

@@ -25,9 +25,14 @@ __device__ __forceinline__ float dt_of(float raw, float bias, float lo, float hi
     return fminf(fmaxf(softplus_f(raw + bias), lo), hi);
 }
 
-// silu(u) = u / (1 + e^-u) with the fast exponential and division (relative
-// error about 1e-6: inside the fp32 bar of 1e-5 and one bf16 rounding).  For
-// u below about -87, e^-u is inf and the quotient is the limit, 0.
+// silu(u) = u / (1 + e^-u) with the fast exponential and division.  The
+// exponential's error grows with |u| (its argument u log2(e) is rounded to
+// fp32 first): about 6e-6 relative at |u| = 100, 1e-6 for |u| < 16; inside
+// the fp32 bar of 1e-5 and one bf16 rounding.  For u below about -87, e^-u
+// passes 2^126 and the quotient is 0 (silu itself is below 1e-35 there).
+// (A reciprocal by Newton steps on the FMA pipe instead of the special
+// function unit was measured slower: the conv is issue-bound, not bound by
+// that unit.)
 __device__ __forceinline__ float silu_f(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
 // The causal depthwise conv of one channel at one token, then SiLU:

@@ -55,6 +55,37 @@ def test_conv1d_parity(K, dtype):
         _check_conv(got, r, dtype, "conv K=%d %s" % (K, nm))
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_conv1d_silu_over_its_range(dtype):
+    """Weights (0, 0, 0, 1) and no bias make every output silu(x) of its own
+    input; x spans [-100, 100] (the SiLU's exponential saturates at both
+    ends) and tiny magnitudes.  fp32: within 1e-5 relative of the oracle (the
+    fast exponential's error grows with |x|: about 6e-6 at |x| = 100), and
+    1e-30 absolute where silu itself is below that; bf16: one rounding."""
+    H, P, G, N = 2, 64, 1, 64
+    Cd = H * P + 2 * G * N
+    vals = np.concatenate([np.linspace(-100, 100, 4001), np.geomspace(1e-20, 1, 500), -np.geomspace(1e-20, 1, 500)])
+    L = int(math.ceil(vals.size / Cd))
+    flat = np.zeros(L * Cd)
+    flat[:vals.size] = vals
+    xbc = torch.from_numpy(flat.reshape(1, L, Cd)).to(dtype)
+    w = torch.zeros(Cd, 4)
+    w[:, 3] = 1.0
+    bias = torch.zeros(Cd)
+    x, B, C = ssd.conv1d_silu_split(xbc.cuda(), w.cuda(), bias.cuda(), H, P, G, N)
+    ref = oracle.conv1d_silu(xbc.float().numpy(), w.numpy(), bias.numpy())
+    for got, r, nm in zip((x, B, C), _split(ref, 1, L, H, P, G, N), "xBC"):
+        g = got.float().cpu().double().numpy()
+        if dtype == torch.float32:
+            err = np.abs(g - r)
+            bad = err > 1e-5 * np.abs(r) + 1e-30
+            assert not bad.any(), "silu %s: %d values off, worst input %r (got %r, oracle %r)" % (
+                nm, int(bad.sum()), *(float(a[bad][np.argmax((err - 1e-5 * np.abs(r))[bad])])
+                                     for a in (_split(xbc.float().numpy(), 1, L, H, P, G, N)["xBC".index(nm)], g, r)))
+        else:
+            _check_conv(got, r, dtype, "silu range %s" % nm)
+
+
 # (b, L, H, P, G, N): channel tiles of 128 with the x|B and B|C edges inside
 # a tile and a partial last tile (Cd = 152); token tiles of 64 with a ragged
 # tail; enough (batch, token tile) rows that each CTA walks its ring of
