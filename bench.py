@@ -621,9 +621,12 @@ def bench_backward(cfg, args, local, peaks, peak_kind):
     the workload's shapes, inputs and upstream gradients rotated past L2, K
     calls in one CUDA graph, CUDA events on the launching stream; then the
     same K calls eagerly with the library's per-kernel event brackets for
-    the kernel shares.  The path runs on CUDA cores in fp32, so the roofline
-    is the fp32 ALU peak (FP32_ALU_TFLOPS); the HBM time of its algorithmic
-    bytes is reported beside it."""
+    the kernel shares.  bf16 layers with P 64, N 128 and Q a multiple of 128
+    take the tensor-core pair kernels (roofline: the dense bf16/fp16 tensor
+    peak), and the fp32 CUDA-core path is timed beside them under "simt";
+    other layers take the CUDA-core path (roofline: the fp32 ALU peak,
+    FP32_ALU_TFLOPS).  The HBM time of the algorithmic bytes is reported
+    beside it."""
     from state_space_sequence_scan_b200 import ssd
     from state_space_sequence_scan_b200.inputs import make_grad_inputs
     dev = torch.device("cuda", local)
@@ -647,58 +650,80 @@ def bench_backward(cfg, args, local, peaks, peak_kind):
                      "D": torch.empty(H, device=dev), "init_state": torch.empty(b, H, N, P, device=dev)})
     work = ssd.alloc_workspace(ssd.bwd_workspace_size(b, L, H, P, N, G, Q, sets[0][0]["x"].dtype), dev)
 
-    def step(k):
-        d, dy, df = sets[k % nsets]
-        ssd.chunk_scan_bwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], dy,
-                           dfinal_state=df, init_state=d["init_state"], chunk_size=Q, workspace=work,
-                           out=outs[k % nsets])
+    def timed(path):
+        def step(k):
+            d, dy, df = sets[k % nsets]
+            ssd.chunk_scan_bwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], dy,
+                               dfinal_state=df, init_state=d["init_state"], chunk_size=Q, workspace=work,
+                               out=outs[k % nsets], path=path)
 
-    for k in range(args.warmup):
-        step(k)
-    torch.cuda.synchronize()
-    if ssd.read_device_status(work) != 0:
-        raise RuntimeError("device status %d after warm-up" % ssd.read_device_status(work))
-    graph = capture_steps(step, args.steps)
-    stream = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    graph.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    del graph
-    ssd.trace_enable(min(8192, 16 * args.steps + 16))
-    for k in range(args.steps):
-        step(k)
-    torch.cuda.synchronize()
-    trace = ssd.trace_read()
-    ssd.trace_enable(0)
+        for k in range(args.warmup):
+            step(k)
+        torch.cuda.synchronize()
+        if ssd.read_device_status(work) != 0:
+            raise RuntimeError("device status %d after warm-up" % ssd.read_device_status(work))
+        graph = capture_steps(step, args.steps)
+        stream = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(local)
+        clocks.start()
+        time.sleep(0.3)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        ms = e0.elapsed_time(e1) / args.steps
+        del graph
+        ssd.trace_enable(min(8192, 16 * args.steps + 16))
+        for k in range(args.steps):
+            step(k)
+        torch.cuda.synchronize()
+        trace = ssd.trace_read()
+        ssd.trace_enable(0)
+        if ssd.read_device_status(work) != 0:
+            raise RuntimeError("device status %d after the %s backward" % (ssd.read_device_status(work), path))
+        return ms, trace, clk
+
+    # the tensor-core pair kernels where they apply (bf16, P 64, N 128, Q a multiple of 128), else SIMT
+    tensor = cfg.dtype == "bf16" and P == 64 and N == 128 and Q % 128 == 0
+    path = "tensor" if tensor else "simt"
+    ms, trace, clk = timed(path)
+    simt = None
+    if tensor:
+        sms, strace, _ = timed("simt")
+        simt = {"ms_per_step": sms, "mtokens_per_s": tok / (sms * 1e-3) / 1e6,
+                "shares": {k: round(v[1] / max(sum(x[1] for x in strace.values()), 1e-12), 4)
+                           for k, v in strace.items()}}
     tot_ms = sum(v[1] for v in trace.values())
     flops, cols_flops = bwd_flops(cfg)
     cols_ms = trace["bwd_cols"][1] / max(trace["bwd_cols"][0], 1)
     ach = cols_flops / (cols_ms * 1e-3) / 1e12
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     mtok = tok / (ms * 1e-3) / 1e6
+    if tensor:
+        # fp16 operands: the dense fp16 tensor peak equals the bf16 one (cuBLAS bf16, measured)
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS.get("bf16_tflops", 1590.0)))
+        roof_bound, roof_src = "tensor", "%s (MEASURED_PEAKS.json bf16_tflops; fp16 has the same rate)" % peak_kind
+    else:
+        peak = FP32_ALU_TFLOPS
+        roof_bound, roof_src = "alu", "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz"
     out = {"stage": "backward", "metric": "SSD chunked-scan backward Mtokens/s", "value": mtok,
            "unit": "Mtokens/s", "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
            "higher_is_better": True, "dtype": "%s-in/f32" % cfg.dtype, "data": "synthetic (seeded)",
            "config": {"workload": cfg.name, "batch": b, "seqlen": L, "heads": H, "head_dim": P, "state_dim": N,
                       "groups": G, "chunk_size": Q, "in_dtype": cfg.dtype, "grads": "f32",
                       "init_state": cfg.init == "normal", "l2": "rotating %d input/gradient sets" % nsets},
-           "roofline": {"bound": "alu", "kernel": "bwd_cols", "achieved": ach, "peak": FP32_ALU_TFLOPS,
-                        "unit": "TFLOP/s", "frac": ach / FP32_ALU_TFLOPS, "traffic": None,
-                        "kernel_ms_avg": cols_ms, "kernel_flops": cols_flops,
-                        "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz",
+           "roofline": {"bound": roof_bound, "kernel": "bwd_cols", "achieved": ach, "peak": peak,
+                        "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                        "kernel_ms_avg": cols_ms, "kernel_flops": cols_flops, "peak_source": roof_src,
                         "shares": {k: round(v[1] / max(tot_ms, 1e-12), 4) for k, v in trace.items()},
                         "path": {"algorithmic_flops": flops, "algorithmic_bytes": nbytes,
-                                 "alu_ms": flops / (FP32_ALU_TFLOPS * 1e12) * 1e3,
+                                 "compute_ms": flops / (peak * 1e12) * 1e3,
                                  "hbm_ms": nbytes / (hbm * 1e9) * 1e3,
-                                 "frac": flops / (FP32_ALU_TFLOPS * 1e12) * 1e3 / ms}},
+                                 "frac": flops / (peak * 1e12) * 1e3 / ms}},
+           "bwd_path": path, "simt": simt,
            "clocks": clk, "gpu_launches": int(sum(v[0] for v in trace.values()))}
     if not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_bwd(cfg)

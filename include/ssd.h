@@ -317,8 +317,21 @@ SSD_API ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const 
  * 4-byte aligned; a token whose id differs from the previous token's starts a
  * document and the state is zero before its update).  No gradient crosses a
  * document start; dinit_state reaches only each row's first document.  NULL
- * seq_idx makes the call ssd_chunk_scan_bwd.  Same workspace size,
- * determinism and other arguments as ssd_chunk_scan_bwd. */
+ * seq_idx makes the call ssd_chunk_scan_bwd (on the path chosen below).
+ * path (ssd_path):
+ *   SSD_PATH_SIMT    the fp32 CUDA-core kernels, as ssd_chunk_scan_bwd;
+ *   SSD_PATH_TENSOR  the products of two 128-token blocks (C.B^T, dy.x^T and
+ *                    the accumulations into dx, dB, dC) on the tcgen05
+ *                    tensor cores with fp16 operands and fp32 accumulation:
+ *                    bf16 inputs, head_dim 64, state_dim 128, chunk_size a
+ *                    multiple of 128 up to 1024, no packed rows (else
+ *                    SSD_ERR_UNSUPPORTED).  The gradients carry the forward
+ *                    tensor path's precision (about 1e-3 of their RMS), and
+ *                    a value outside fp16's range shows as
+ *                    SSD_ERR_PRECONDITION in the status word;
+ *   SSD_PATH_AUTO    the tensor path where it applies, else SIMT.
+ * Same workspace size and determinism, and the other arguments as
+ * ssd_chunk_scan_bwd. */
 SSD_API ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw, const float *dt_bias,
                                      const float *A, const void *B, const void *C, const float *D,
                                      const float *init_state, const int32_t *seq_idx, const float *dy,
@@ -326,8 +339,8 @@ SSD_API ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw,
                                      float *dA, float *dB, float *dC, float *dD, float *dinit_state,
                                      int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim,
                                      int64_t state_dim, int64_t ngroups, int64_t chunk_size, float dt_lo,
-                                     float dt_hi, int in_dtype, void *workspace, size_t workspace_bytes,
-                                     void *stream);
+                                     float dt_hi, int in_dtype, int path, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /* Waits for `stream`, then reads the device status word that the last
  * ssd_chunk_scan_fwd on this workspace left: SSD_OK, SSD_ERR_PRECONDITION or
@@ -370,7 +383,8 @@ SSD_API ssd_status ssd_set_test_fault(int kind);
 /* ABI version: (major << 16) | minor.  1.1 added the chunk-state, packed-row,
  * conv/norm and backward entry points to the 1.0 scan and step; 1.2 the test
  * hook ssd_set_test_fault and ssd_chunk_scan_bwd_varlen; 1.3
- * ssd_conv_scan_fwd and the workspace-free status read. */
+ * ssd_conv_scan_fwd, the workspace-free status read and the `path` argument
+ * of ssd_chunk_scan_bwd_varlen (the tensor-core backward). */
 SSD_API int ssd_version(void);
 
 #ifdef __cplusplus

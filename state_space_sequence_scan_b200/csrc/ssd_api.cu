@@ -256,9 +256,9 @@ ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw, const f
                               float *ddt_bias, float *dA, float *dB, float *dC, float *dD, float *dinit_state,
                               int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim, int64_t state_dim,
                               int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype,
-                              void *workspace, size_t workspace_bytes, void *stream) {
+                              int path, void *workspace, size_t workspace_bytes, void *stream) {
     ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, in_dtype,
-                                    SSD_PATH_SIMT);
+                                    path);
     if (st != SSD_OK) return st;
     if (!limits_ok(dt_lo, dt_hi)) return SSD_ERR_INVALID_ARG;
     if (!dt_bias || !A || !D || !ddt_bias || !dA || !dD) return SSD_ERR_INVALID_ARG;
@@ -273,6 +273,9 @@ ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw, const f
         return SSD_ERR_ALIGNMENT;
     const ssd::ScanDims d = make_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size);
     if (!ssd::bwd_supported(d)) return SSD_ERR_UNSUPPORTED;
+    const bool tc = ssd::bwd_tc_supported(d, in_dtype == SSD_BF16, seq_idx != nullptr);
+    if (path == SSD_PATH_TENSOR && !tc) return SSD_ERR_UNSUPPORTED;
+    const bool use_tc = tc && path != SSD_PATH_SIMT;
     if (!workspace || workspace_bytes < ssd::bwd_workspace_bytes(d)) return SSD_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
 
@@ -298,6 +301,7 @@ ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw, const f
     a.f.init_state = init_state; a.f.y = nullptr; a.f.final_state = nullptr;
     a.f.seq_idx = seq_idx;
     a.f.dt_lo = dt_lo; a.f.dt_hi = dt_hi; a.f.bf16 = in_dtype == SSD_BF16;
+    a.tensor = use_tc ? 1 : 0;
     a.dy = dy; a.dfinal = dfinal_state;
     a.dx = dx; a.ddt_raw = ddt_raw; a.ddt_bias = ddt_bias; a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD;
     a.dinit = dinit_state;
@@ -315,8 +319,8 @@ ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const float *d
                               void *workspace, size_t workspace_bytes, void *stream) {
     return ssd_chunk_scan_bwd_varlen(x, dt_raw, dt_bias, A, B, C, D, init_state, nullptr, dy, dfinal_state, dx,
                                      ddt_raw, ddt_bias, dA, dB, dC, dD, dinit_state, batch, seqlen, nheads, head_dim,
-                                     state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, workspace,
-                                     workspace_bytes, stream);
+                                     state_dim, ngroups, chunk_size, dt_lo, dt_hi, in_dtype, SSD_PATH_SIMT,
+                                     workspace, workspace_bytes, stream);
 }
 
 ssd_status ssd_step(const void *x, const float *dt_raw, const float *dt_bias, const float *A,

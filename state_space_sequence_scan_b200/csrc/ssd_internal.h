@@ -69,8 +69,27 @@ struct BwdArgs {
     ScanArgs f;                    // the forward's inputs (y, final_state, chunk_states unused)
     const float *dy, *dfinal;      // [b,L,H,P], [b,H,N,P] or null
     float *dx, *ddt_raw, *ddt_bias, *dA, *dB, *dC, *dD, *dinit;
+    int tensor = 0;                // 1: the tensor-core pair kernels (bwd_tc_supported)
 };
 bool bwd_supported(const ScanDims &d);
+
+// The tensor-core pair kernels of the backward (ssd_scan_bwd_tc.cu): the
+// same outputs as the CUDA-core `cols` and `rows` kernels, from the same
+// workspace (the forward recompute's dt, cum and entering states, the
+// reverse pass's G_c).  bf16 inputs, P 64, N 128, Q a multiple of 128, no
+// packed rows.
+struct BwdPairArgs {
+    const void *x, *B, *C;         // bf16 inputs
+    const float *D, *dy;
+    const float *dtv, *cum;        // [b, H, L]
+    const float *gst, *states;     // [b, H, nc, N, P]: G_c, H_in
+    float *ddt_dir, *dcum_col, *dcum_row, *E, *dyx;  // [b, H, L]
+    float *dx;                     // [b, L, H, P]
+    float *dBh, *dCh;              // [b, L, H, N] per head
+    unsigned *status;
+};
+bool bwd_tc_supported(const ScanDims &d, int bf16, int packed);
+cudaError_t bwd_tc_pairs(const BwdPairArgs &a, const ScanDims &d, cudaStream_t s);
 size_t bwd_workspace_bytes(const ScanDims &d);
 cudaError_t bwd_scan(const BwdArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
 

@@ -774,6 +774,15 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
     const dim3 gp((unsigned)(nc * tiles), (unsigned)H, (unsigned)d.b);
     float *dBh = ws.dBh ? ws.dBh : a.dB;
     float *dCh = ws.dCh ? ws.dCh : a.dC;
+    if (a.tensor) {
+        // the pair products on the tensor cores (ssd_scan_bwd_tc.cu)
+        BwdPairArgs pa;
+        pa.x = a.f.x; pa.B = a.f.B; pa.C = a.f.C; pa.D = a.f.D; pa.dy = a.dy;
+        pa.dtv = ws.f.dtv; pa.cum = ws.f.cum; pa.gst = ws.gst; pa.states = ws.f.states;
+        pa.ddt_dir = ws.ddt_dir; pa.dcum_col = ws.dcum_col; pa.dcum_row = ws.dcum_row; pa.E = ws.E;
+        pa.dyx = ws.dyx; pa.dx = a.dx; pa.dBh = dBh; pa.dCh = dCh; pa.status = ws.f.status;
+        if ((e = bwd_tc_pairs(pa, d, s)) != cudaSuccess) return e;
+    } else {
     {
         TraceScope tr(s, kTrBwdCols);
         cols_kernel<T><<<gp, kThreads, smc, s>>>((const T *)a.f.x, (const T *)a.f.B, (const T *)a.f.C, a.f.D,
@@ -786,6 +795,7 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
                                                  dCh, L, H, P, N, G, Q, nc, packed);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     {
         TraceScope tr(s, kTrBwdFinalize);
         finalize_kernel<<<gc, kThreads, 0, s>>>(a.f.dt_raw, a.f.dt_bias, a.f.A, ws, a.ddt_raw, L, H, Q, nc, nblk,

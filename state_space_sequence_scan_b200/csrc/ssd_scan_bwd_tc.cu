@@ -1,0 +1,620 @@
+// Tensor-core pair kernels of the backward (sm_100a: tcgen05 MMAs with TMEM
+// accumulators).  They take the place of the fp32 CUDA-core `cols` and
+// `rows` kernels of ssd_scan_bwd.cu (same inputs, same outputs in the same
+// workspace regions; the launches around them are unchanged), for bf16
+// inputs with head_dim 64, state_dim 128 and a chunk size that is a multiple
+// of 128.  The formulas are those of ssd_scan_bwd.cu's header (the chunked
+// form of the forward, "Mamba2" knowledge page); every product of two
+// 128-token blocks is an MMA:
+//
+// cols, per (j block J of a chunk, head, batch), TMEM lane = token j:
+//   dX_J  = e^{cl-cum_j} B_J G_c             (M=128 j, N=64 p,  K=128 n)
+//   dB_J  = e^{cl-cum_j} X_J G_c^T           (M=128 j, N=128 n, K=64 p)
+//           (before the scaling, a row dot with B_J gives E_j)
+//   for each i block I >= J of the chunk:
+//     CB^T = B_J C_I^T,  S^T = X_J dY_I^T    (M=128 j, N=128 i)
+//     U^T = CB^T L, V^T = S^T L  (L_ij = e^{cum_i-cum_j}, i >= j), as fp16
+//     dX_J += U^T dY_I,  dB_J += V^T C_I     (K=128 i; dB as two N=64 halves)
+//   dx_j = dt_j dX_j + D dy_j,  dB_j = dt_j dB_j, and per token the direct
+//   d(dt) (row sums of U^T.S^T), the column part of d(cum), E_j, dy_j.x_j.
+// rows, per (i block I, head, batch), TMEM lane = token i:
+//   dC_I  = e^{cum_i} dY_I H_in^T            (M=128 i, N=128 n, K=64 p)
+//           (before the scaling, a row dot with C_I gives T_i)
+//   for each j block J <= I: CB = C_I B_J^T, S = dY_I X_J^T,
+//     V = S L dt_j (j <= i) as fp16, dC_I += V B_J   (K=128 j; two N=64 halves)
+//   and the row part of d(cum): T_i + sum_{j<i} CB_ij V_ij.
+//
+// Operands are fp16 in 128-byte-swizzled shared-memory tiles, written by the
+// threads from the inputs (bf16 B, C, x widen to fp16 exactly inside its
+// range; dy, G_c and H_in round to fp16's 11 bits); accumulation is fp32.
+// The results carry the forward tensor path's precision: the bf16-input bar
+// (2e-2 of RMS) applies, not the fp32 CUDA-core backward's.  A value outside
+// fp16's range sets the workspace's range bit (SSD_ERR_PRECONDITION).  Each
+// CTA runs its phases in order (copy in, MMA, TMEM math, MMA, ...); every
+// wait on an MMA completion is bounded and a timeout sets the status word.
+// Sums run in a fixed order (no atomics): deterministic.
+#include "ssd_common.cuh"
+#include "ssd_internal.h"
+#include "ssd_tc.cuh"
+#include "ssd_trace.h"
+
+namespace ssd {
+namespace {
+using namespace tc;
+
+constexpr int kB = 128;                    // tokens per block (MMA M)
+constexpr int kNs = 128;                   // state_dim
+constexpr int kPh = 64;                    // head_dim
+constexpr uint32_t kT = 16384;             // one [128 rows x 64 fp16] swizzled tile
+constexpr int kThr = 256;                  // 8 warps: lane quarter w % 4, column half w / 4
+constexpr long long kBudget = 1ll << 32;   // clock cycles before an MMA wait gives up (~2 s)
+constexpr float kF16Max = 65504.0f;
+
+// K-step q (16 elements) of a K-major operand 128 wide (two 64-wide tiles)
+__device__ __forceinline__ uint32_t kofs128(int q) { return (uint32_t)((q >> 2) * kT + (q & 3) * 32); }
+
+// Rows 0..127 of a [128 x W] fp16 tile (W = 64 or 128: one or two swizzled
+// 64-wide tiles) from `nrows` source rows of `ld` elements (bf16 or fp32);
+// rows past nrows are zero.  All 256 threads; one 16-byte chunk (8 values)
+// per step, consecutive threads on consecutive chunks of a row.
+template <typename S>
+__device__ __forceinline__ void fill_tile(uint8_t *tile, const S *src, size_t ld, int nrows, int W, int tid,
+                                          __half2 &amax) {
+    const int cpr = W / 8;                 // chunks per row
+    for (int c = tid; c < kB * cpr; c += kThr) {
+        const int r = c / cpr, k = c - r * cpr;
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (r < nrows) {
+            float f[8];
+            if constexpr (sizeof(S) == 2) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * ld + 8 * k);
+                f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+                f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+            } else {
+                const float4 a = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k);
+                const float4 b = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k + 4);
+                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+            }
+            o = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
+            const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&w[i])));
+        }
+        *reinterpret_cast<uint4 *>(tile + (k >> 3) * kT + sw128_off(r, k & 7)) = o;
+    }
+}
+
+// Dot of 32 fp32 accumulator values with row `r`, chunks c0..c0+3 of tile
+// `half` (32 fp16 values) of a 128-wide swizzled tile
+__device__ __forceinline__ float row_dot32(const uint8_t *tile, int r, int half, int c0, const float (&a)[32]) {
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(tile + half * kT + sw128_off(r, c0 + k));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_h2(w[e]);
+            s = fmaf(f.x, a[8 * k + 2 * e], s);
+            s = fmaf(f.y, a[8 * k + 2 * e + 1], s);
+        }
+    }
+    return s;
+}
+
+// 32 fp32 values -> fp16 into row `r`, chunks c0..c0+3 of a swizzled tile
+__device__ __forceinline__ void store_row32(uint8_t *tile, int r, int c0, const float (&v)[32], __half2 &amax) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            w[e] = pack_h2(v[8 * k + 2 * e], v[8 * k + 2 * e + 1]);
+            amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&w[e])));
+        }
+        *reinterpret_cast<uint4 *>(tile + sw128_off(r, c0 + k)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// Waits for the next completion of `bar` (phase `ph`, then advances it).
+// Bounded: false after the budget.
+__device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t &ph) {
+    const bool ok = mbar_wait(bar, ph & 1u, kBudget);
+    ++ph;
+    tc_fence_after();
+    return ok;
+}
+
+__device__ __forceinline__ void finish_range(unsigned *status, __half2 amax) {
+    const float2 m = __half22float2(amax);
+    if (!(m.x <= kF16Max && m.y <= kF16Max)) flag_status(status, kStatusRange);
+}
+
+// ---- cols -----------------------------------------------------------------
+// shared memory (offsets from a 1024-aligned base)
+constexpr uint32_t kCBj = 0, kCXj = 2 * kT, kCG = 3 * kT, kCCi = 4 * kT, kCDYi = 6 * kT, kCU = 7 * kT,
+                   kCV = 9 * kT, kCScal = 11 * kT;
+// scalars: cum_j, dt_j, dec_j, cum_i, e1[2], zs[2], zo[2], dyx[2] (128 floats each)
+constexpr uint32_t kCBar = kCScal + 13 * kB * 4;
+constexpr size_t kColsSmem = 1024 + kCBar + 16;
+// TMEM columns (each accumulator starts on a multiple of its width, as in
+// the forward kernels)
+constexpr uint32_t kTmCBt = 0, kTmSt = 128, kTmDB = 256, kTmDX = 384;
+
+__global__ void __launch_bounds__(kThr, 1)
+tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *s_cumj = reinterpret_cast<float *>(sm + kCScal);
+    float *s_dtj = s_cumj + kB, *s_dec = s_dtj + kB, *s_cumi = s_dec + kB;
+    float *s_e1 = s_cumi + kB, *s_zs = s_e1 + 2 * kB, *s_zo = s_zs + 2 * kB, *s_dyx = s_zo + 2 * kB;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kCBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
+
+    const int nJ = Q / kB;
+    const int c = blockIdx.x / nJ, Jb = blockIdx.x - c * nJ;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (H / G);
+    const int t0 = c * Q, q = min(Q, L - t0);
+    const int j0 = Jb * kB;
+    if (j0 >= q) return;                               // uniform over the CTA
+    const int tj = min(kB, q - j0);
+    const size_t bh = (size_t)b * H + h;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lg = warp & 3, ch = warp >> 2, row = 32 * lg + lane;
+    __half2 amax = __float2half2_rn(0.f);
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    // j block: B_J, X_J (fp16), G_c (fp16 [n][p]); per-token scalars
+    const size_t tokj = (size_t)b * L + t0 + j0;
+    fill_tile(sm + kCBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs, (size_t)G * kNs, tj, 128,
+              tid, amax);
+    fill_tile(sm + kCXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh, (size_t)H * kPh, tj, 64,
+              tid, amax);
+    fill_tile(sm + kCG, a.gst + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, 64, tid, amax);
+    const float cl = a.cum[bh * L + t0 + q - 1];
+    if (tid < kB) {
+        const bool v = tid < tj;
+        const float cj = v ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
+        s_cumj[tid] = cj;
+        s_dtj[tid] = v ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
+        s_dec[tid] = v ? expf(fminf(cl - cj, 0.f)) : 0.f;
+    }
+    // dy_j . x_j exactly in fp32 (thread: token row, half ch of p)
+    {
+        float d = 0.f;
+        if (row < tj) {
+            const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(a.x) + ((tokj + row) * H + h) * kPh + 32 * ch;
+            const float *dr = a.dy + ((tokj + row) * H + h) * kPh + 32 * ch;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xr + 8 * k);
+                const float4 d0 = *reinterpret_cast<const float4 *>(dr + 8 * k);
+                const float4 d1 = *reinterpret_cast<const float4 *>(dr + 8 * k + 4);
+                d = fmaf(bf16lo(xv.x), d0.x, d); d = fmaf(bf16hi(xv.x), d0.y, d);
+                d = fmaf(bf16lo(xv.y), d0.z, d); d = fmaf(bf16hi(xv.y), d0.w, d);
+                d = fmaf(bf16lo(xv.z), d1.x, d); d = fmaf(bf16hi(xv.z), d1.y, d);
+                d = fmaf(bf16lo(xv.w), d1.z, d); d = fmaf(bf16hi(xv.w), d1.w, d);
+            }
+        }
+        s_dyx[ch * kB + row] = d;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * lg) << 16);
+    const uint32_t sbase = smem_u32(sm);
+    uint32_t ph = 0, commits = 0;            // completions waited for; commits issued (thread 0)
+    bool ok = true;
+
+    // G_c terms: dX = B_J G_c, dB = X_J G_c^T
+    if (tid == 0) {
+        const uint64_t dBj = sdesc_sw128(sbase + kCBj, 16, 1024), dXj = sdesc_sw128(sbase + kCXj, 16, 1024);
+        const uint64_t dGmn = sdesc_sw128(sbase + kCG, kT, 1024), dGk = sdesc_sw128(sbase + kCG, 16, 1024);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            mma_f16(tmem + kTmDX, dBj + (kofs128(s) >> 4), dGmn + ((s * 2048) >> 4), idesc_f16(128, 64, 0, 1), s > 0);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_f16(tmem + kTmDB, dXj + ((s * 32) >> 4), dGk + ((s * 32) >> 4), idesc_f16(128, 128, 0, 0), s > 0);
+        mma_commit(bar);
+        ++commits;
+    }
+    ok = wait_mma(bar, ph);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+        // E_j's dot (B_J row j with the unscaled dB row), then both accumulators times dec_j
+        const float dec = s_dec[row];
+        float e1 = 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+            float t32[32];
+            tmem_ld32(lane_addr + kTmDB + 64 * ch + 32 * hh, t32);
+            e1 += row_dot32(sm + kCBj, row, ch, 4 * hh, t32);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) t32[k] *= dec;
+            tmem_st32(lane_addr + kTmDB + 64 * ch + 32 * hh, t32);
+        }
+        s_e1[ch * kB + row] = e1;
+        float t32[32];
+        tmem_ld32(lane_addr + kTmDX + 32 * ch, t32);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) t32[k] *= dec;
+        tmem_st32(lane_addr + kTmDX + 32 * ch, t32);
+    }
+    float zs = 0.f, zo = 0.f;                          // this thread's i half
+    const int nIb = (q + kB - 1) / kB;
+    for (int Ib = Jb; Ib < nIb; ++Ib) {
+        const int i0 = Ib * kB, ti = min(kB, q - i0);
+        const size_t toki = (size_t)b * L + t0 + i0;
+        // the previous pair's MMAs (which read C_I, DY_I, U, V) are complete
+        fill_tile(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs, (size_t)G * kNs, ti,
+                  128, tid, amax);
+        fill_tile(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, 64, tid, amax);
+        if (tid < kB) s_cumi[tid] = tid < ti ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            const uint64_t dBj = sdesc_sw128(sbase + kCBj, 16, 1024), dCi = sdesc_sw128(sbase + kCCi, 16, 1024);
+            const uint64_t dXj = sdesc_sw128(sbase + kCXj, 16, 1024), dDY = sdesc_sw128(sbase + kCDYi, 16, 1024);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_f16(tmem + kTmCBt, dBj + (kofs128(s) >> 4), dCi + (kofs128(s) >> 4), idesc_f16(128, 128, 0, 0),
+                        s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_f16(tmem + kTmSt, dXj + ((s * 32) >> 4), dDY + ((s * 32) >> 4), idesc_f16(128, 128, 0, 0), s > 0);
+            mma_commit(bar);
+            ++commits;
+        }
+        ok = ok && wait_mma(bar, ph);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            const float cj = s_cumj[row];
+            const int gj = j0 + row;
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                const int ib = 64 * ch + 32 * hh;      // first i of this group of 32
+                float cb[32], sv[32];
+                tmem_ld32(lane_addr + kTmCBt + ib, cb);
+                tmem_ld32(lane_addr + kTmSt + ib, sv);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int il = ib + k, gi = i0 + il;
+                    const bool v = il < ti && row < tj && gi >= gj;
+                    const float lw = v ? expf(fminf(s_cumi[il] - cj, 0.f)) : 0.f;
+                    const float u = cb[k] * lw, w = sv[k] * lw;
+                    const float z = u * sv[k];
+                    zs += z;
+                    zo += gi > gj ? z : 0.f;
+                    cb[k] = u;
+                    sv[k] = w;
+                }
+                store_row32(sm + kCU + ch * kT, row, 4 * hh, cb, amax);
+                store_row32(sm + kCV + ch * kT, row, 4 * hh, sv, amax);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            const uint64_t dU = sdesc_sw128(sbase + kCU, 16, 1024), dV = sdesc_sw128(sbase + kCV, 16, 1024);
+            const uint64_t dDYmn = sdesc_sw128(sbase + kCDYi, kT, 1024);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_f16(tmem + kTmDX, dU + (kofs128(s) >> 4), dDYmn + ((s * 2048) >> 4), idesc_f16(128, 64, 0, 1), 1u);
+            // dB's two 64-column halves, each with one 64-wide MN-major tile of C_I
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+                const uint64_t dCmn = sdesc_sw128(sbase + kCCi + nh * kT, kT, 1024);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_f16(tmem + kTmDB + 64 * nh, dV + (kofs128(s) >> 4), dCmn + ((s * 2048) >> 4),
+                            idesc_f16(128, 64, 0, 1), 1u);
+            }
+            mma_commit(bar);
+            ++commits;
+        }
+        ok = ok && wait_mma(bar, ph);
+        ok = __all_sync(0xffffffffu, ok);
+    }
+    s_zs[ch * kB + row] = zs;
+    s_zo[ch * kB + row] = zo;
+    __syncthreads();
+    // (tcgen05.ld is warp-collective: every lane loads, only the block's own
+    // tokens store; `ok` is warp-uniform)
+    if (ok) {
+        const bool mine = row < tj;
+        const float dtj = s_dtj[row];
+        const size_t tok = tokj + row;
+        const float Dh = a.D[h];
+        float t32[32];
+        tmem_ld32(lane_addr + kTmDX + 32 * ch, t32);
+        float *dxr = a.dx + (tok * H + h) * kPh + 32 * ch;
+        const float *dyr = a.dy + (tok * H + h) * kPh + 32 * ch;
+        if (mine) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(dyr + 4 * k);
+                *reinterpret_cast<float4 *>(dxr + 4 * k) =
+                    make_float4(fmaf(dtj, t32[4 * k], Dh * d4.x), fmaf(dtj, t32[4 * k + 1], Dh * d4.y),
+                                fmaf(dtj, t32[4 * k + 2], Dh * d4.z), fmaf(dtj, t32[4 * k + 3], Dh * d4.w));
+            }
+        }
+        float *dbr = a.dBh + (tok * H + h) * kNs + 64 * ch;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            tmem_ld32(lane_addr + kTmDB + 64 * ch + 32 * hh, t32);
+            if (mine) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<float4 *>(dbr + 32 * hh + 4 * k) = make_float4(
+                        dtj * t32[4 * k], dtj * t32[4 * k + 1], dtj * t32[4 * k + 2], dtj * t32[4 * k + 3]);
+            }
+        }
+        if (mine && ch == 0) {
+            const float dec = s_dec[row];
+            const float e1 = s_e1[row] + s_e1[kB + row];
+            const float sdst = dec * e1, E = dtj * sdst;
+            const size_t o = bh * L + t0 + j0 + row;
+            a.ddt_dir[o] = sdst + (s_zs[row] + s_zs[kB + row]);
+            a.dcum_col[o] = -(dtj * (s_zo[row] + s_zo[kB + row])) - E;
+            a.E[o] = E;
+            a.dyx[o] = s_dyx[row] + s_dyx[kB + row];
+        }
+    }
+    if (__any_sync(0xffffffffu, !ok) && lane == 0) flag_status(a.status, kStatusTimeout);
+    if (lane == 0) finish_range(a.status, amax);
+    // after a timeout, let the last MMAs this CTA issued finish (bounded)
+    // before its tensor memory is released
+    if (tid == 0 && commits > ph) mbar_wait(bar, (commits - 1) & 1u, kBudget);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---- rows -----------------------------------------------------------------
+constexpr uint32_t kRCi = 0, kRDYi = 2 * kT, kRH = 3 * kT, kRBj = 4 * kT, kRXj = 6 * kT, kRV = 7 * kT,
+                   kRScal = 9 * kT;
+// scalars: cum_i, dec_i, cum_j, dt_j, tv[2], rs[2] (128 floats each)
+constexpr uint32_t kRBar = kRScal + 8 * kB * 4;
+constexpr size_t kRowsSmem = 1024 + kRBar + 16;
+constexpr uint32_t kTmCB = 0, kTmS = 128, kTmDC = 256;
+
+__global__ void __launch_bounds__(kThr, 1)
+tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *s_cumi = reinterpret_cast<float *>(sm + kRScal);
+    float *s_dec = s_cumi + kB, *s_cumj = s_dec + kB, *s_dtj = s_cumj + kB;
+    float *s_tv = s_dtj + kB, *s_rs = s_tv + 2 * kB;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kRBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
+
+    const int nI = Q / kB;
+    const int c = blockIdx.x / nI, Ib = blockIdx.x - c * nI;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (H / G);
+    const int t0 = c * Q, q = min(Q, L - t0);
+    const int i0 = Ib * kB;
+    if (i0 >= q) return;                               // uniform over the CTA
+    const int ti = min(kB, q - i0);
+    const size_t bh = (size_t)b * H + h;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lg = warp & 3, ch = warp >> 2, row = 32 * lg + lane;
+    __half2 amax = __float2half2_rn(0.f);
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    const size_t toki = (size_t)b * L + t0 + i0;
+    fill_tile(sm + kRCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs, (size_t)G * kNs, ti, 128,
+              tid, amax);
+    fill_tile(sm + kRDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, 64, tid, amax);
+    fill_tile(sm + kRH, a.states + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, 64, tid, amax);
+    if (tid < kB) {
+        const bool v = tid < ti;
+        const float ci = v ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
+        s_cumi[tid] = ci;
+        s_dec[tid] = v ? expf(fminf(ci, 0.f)) : 0.f;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * lg) << 16);
+    const uint32_t sbase = smem_u32(sm);
+    uint32_t ph = 0, commits = 0;            // completions waited for; commits issued (thread 0)
+    bool ok = true;
+
+    // H_in term: dC = dY_I H_in^T (M=i, N=n, K=p)
+    if (tid == 0) {
+        const uint64_t dDY = sdesc_sw128(sbase + kRDYi, 16, 1024), dH = sdesc_sw128(sbase + kRH, 16, 1024);
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_f16(tmem + kTmDC, dDY + ((s * 32) >> 4), dH + ((s * 32) >> 4), idesc_f16(128, 128, 0, 0), s > 0);
+        mma_commit(bar);
+        ++commits;
+    }
+    ok = wait_mma(bar, ph);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+        // T_i's dot (C_I row i with the unscaled dC row), then the accumulator times dec_i
+        const float dec = s_dec[row];
+        float tv = 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+            float t32[32];
+            tmem_ld32(lane_addr + kTmDC + 64 * ch + 32 * hh, t32);
+            tv += row_dot32(sm + kRCi, row, ch, 4 * hh, t32);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) t32[k] *= dec;
+            tmem_st32(lane_addr + kTmDC + 64 * ch + 32 * hh, t32);
+        }
+        s_tv[ch * kB + row] = tv;
+    }
+    float rs = 0.f;                                    // sum over this thread's j half of CB_ij V_ij, j < i
+    const float ci = s_cumi[row];
+    const int gi = i0 + row;
+    for (int Jb = 0; Jb <= Ib; ++Jb) {
+        const int j0 = Jb * kB, tj = min(kB, q - j0);
+        const size_t tokj = (size_t)b * L + t0 + j0;
+        fill_tile(sm + kRBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs, (size_t)G * kNs, tj,
+                  128, tid, amax);
+        fill_tile(sm + kRXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh, (size_t)H * kPh, tj,
+                  64, tid, amax);
+        if (tid < kB) {
+            s_cumj[tid] = tid < tj ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
+            s_dtj[tid] = tid < tj ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            const uint64_t dCi = sdesc_sw128(sbase + kRCi, 16, 1024), dBj = sdesc_sw128(sbase + kRBj, 16, 1024);
+            const uint64_t dDY = sdesc_sw128(sbase + kRDYi, 16, 1024), dXj = sdesc_sw128(sbase + kRXj, 16, 1024);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_f16(tmem + kTmCB, dCi + (kofs128(s) >> 4), dBj + (kofs128(s) >> 4), idesc_f16(128, 128, 0, 0),
+                        s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_f16(tmem + kTmS, dDY + ((s * 32) >> 4), dXj + ((s * 32) >> 4), idesc_f16(128, 128, 0, 0), s > 0);
+            mma_commit(bar);
+            ++commits;
+        }
+        ok = ok && wait_mma(bar, ph);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                const int jb = 64 * ch + 32 * hh;
+                float cb[32], sv[32];
+                tmem_ld32(lane_addr + kTmCB + jb, cb);
+                tmem_ld32(lane_addr + kTmS + jb, sv);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int jl = jb + k, gj = j0 + jl;
+                    const bool v = jl < tj && row < ti && gi >= gj;
+                    const float w = v ? sv[k] * expf(fminf(ci - s_cumj[jl], 0.f)) * s_dtj[jl] : 0.f;
+                    rs += gi > gj ? cb[k] * w : 0.f;
+                    sv[k] = w;
+                }
+                store_row32(sm + kRV + ch * kT, row, 4 * hh, sv, amax);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            const uint64_t dV = sdesc_sw128(sbase + kRV, 16, 1024);
+            // dC's two 64-column halves, each with one 64-wide MN-major tile of B_J
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+                const uint64_t dBmn = sdesc_sw128(sbase + kRBj + nh * kT, kT, 1024);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_f16(tmem + kTmDC + 64 * nh, dV + (kofs128(s) >> 4), dBmn + ((s * 2048) >> 4),
+                            idesc_f16(128, 64, 0, 1), 1u);
+            }
+            mma_commit(bar);
+            ++commits;
+        }
+        ok = ok && wait_mma(bar, ph);
+        ok = __all_sync(0xffffffffu, ok);
+    }
+    s_rs[ch * kB + row] = rs;
+    __syncthreads();
+    // (tcgen05.ld is warp-collective: every lane loads, only the block's own
+    // tokens store; `ok` is warp-uniform)
+    if (ok) {
+        const bool mine = row < ti;
+        const size_t tok = toki + row;
+        float *dcr = a.dCh + (tok * H + h) * kNs + 64 * ch;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float t32[32];
+            tmem_ld32(lane_addr + kTmDC + 64 * ch + 32 * hh, t32);
+            if (mine) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<float4 *>(dcr + 32 * hh + 4 * k) =
+                        make_float4(t32[4 * k], t32[4 * k + 1], t32[4 * k + 2], t32[4 * k + 3]);
+            }
+        }
+        if (mine && ch == 0) {
+            const float tv = s_dec[row] * (s_tv[row] + s_tv[kB + row]);
+            a.dcum_row[bh * L + t0 + i0 + row] = tv + (s_rs[row] + s_rs[kB + row]);
+        }
+    }
+    if (__any_sync(0xffffffffu, !ok) && lane == 0) flag_status(a.status, kStatusTimeout);
+    if (lane == 0) finish_range(a.status, amax);
+    // after a timeout, let the last MMAs this CTA issued finish (bounded)
+    // before its tensor memory is released
+    if (tid == 0 && commits > ph) mbar_wait(bar, (commits - 1) & 1u, kBudget);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+bool bwd_tc_supported(const ScanDims &d, int bf16, int packed) {
+    if (!bf16 || packed || d.P != kPh || d.N != kNs || d.Q % kB != 0 || d.Q > 1024) return false;
+    if (d.H > 65535 || d.b > 65535 || d.nc * (d.Q / kB) > 0x7fffffffll) return false;
+    return true;
+}
+
+cudaError_t bwd_tc_pairs(const BwdPairArgs &a, const ScanDims &d, cudaStream_t s) {
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        if ((e = cudaFuncSetAttribute(tc_cols_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColsSmem)) !=
+            cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(tc_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowsSmem)) !=
+            cudaSuccess)
+            return e;
+        attr_done[dev] = true;
+    }
+    const dim3 grid((unsigned)(d.nc * (d.Q / kB)), (unsigned)d.H, (unsigned)d.b);
+    {
+        TraceScope tr(s, kTrBwdCols);
+        tc_cols_kernel<<<grid, kThr, kColsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        TraceScope tr(s, kTrBwdRows);
+        tc_rows_kernel<<<grid, kThr, kRowsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

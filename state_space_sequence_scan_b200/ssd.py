@@ -68,7 +68,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ssd_chunk_scan_bwd.restype = i32
     lib.ssd_chunk_scan_bwd.argtypes = [vp] * 18 + [i64] * 7 + [f32, f32, i32, vp, sz, vp]
     lib.ssd_chunk_scan_bwd_varlen.restype = i32
-    lib.ssd_chunk_scan_bwd_varlen.argtypes = [vp] * 19 + [i64] * 7 + [f32, f32, i32, vp, sz, vp]
+    lib.ssd_chunk_scan_bwd_varlen.argtypes = [vp] * 19 + [i64] * 7 + [f32, f32, i32, i32, vp, sz, vp]
     lib.ssd_step.restype = i32
     lib.ssd_step.argtypes = [vp] * 9 + [i64] * 5 + [f32, f32, i32, vp]
     lib.ssd_read_device_status.restype = i32
@@ -265,14 +265,17 @@ def chunk_scan_bwd(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor,
                    dfinal_state: Optional[torch.Tensor] = None, init_state: Optional[torch.Tensor] = None,
                    chunk_size: int = 256, dt_limit: Tuple[float, float] = (0.0, math.inf),
                    workspace: Optional[torch.Tensor] = None, want_dinit: bool = True,
-                   out: Optional[dict] = None, seq_idx: Optional[torch.Tensor] = None) -> dict:
+                   out: Optional[dict] = None, seq_idx: Optional[torch.Tensor] = None,
+                   path: str = "simt") -> dict:
     """Deterministic backward of chunk_scan_fwd (ssd_chunk_scan_bwd), or of
     chunk_scan_fwd_varlen with the same seq_idx [b, L] int32 (packed rows,
     ssd_chunk_scan_bwd_varlen): the gradients of <dy, y> + <dfinal_state,
     final_state> with respect to every input, float32, keyed by input name
     ("x", "dt_raw", "dt_bias", "A", "B", "C", "D", "init_state"; the last None
     unless want_dinit).  `out` may hold preallocated outputs under the same
-    keys."""
+    keys.  path "simt" (fp32 CUDA cores), "tensor" (the block products on the
+    tensor cores, bf16 inputs: the forward tensor path's precision) or
+    "auto" (tensor where it applies)."""
     lib = load_library()
     if x.dim() != 4 or B.dim() != 4:
         raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
@@ -314,9 +317,9 @@ def chunk_scan_bwd(x: torch.Tensor, dt_raw: torch.Tensor, dt_bias: torch.Tensor,
         _ptr(dy),
         _ptr(dfinal_state), _ptr(g["x"]), _ptr(g["dt_raw"]), _ptr(g["dt_bias"]), _ptr(g["A"]), _ptr(g["B"]),
         _ptr(g["C"]), _ptr(g["D"]), _ptr(g["init_state"]), b, L, H, P, N, G, Q, float(dt_limit[0]),
-        float(dt_limit[1]), DTYPES[x.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(dev))
-    _check("ssd_chunk_scan_bwd_varlen" if seq_idx is not None else "ssd_chunk_scan_bwd", st)
+        float(dt_limit[1]), DTYPES[x.dtype], PATHS[path], _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(dev))
+    _check("ssd_chunk_scan_bwd_varlen", st)
     return g
 
 

@@ -208,3 +208,93 @@ def test_backward_packed_constant_ids_is_the_plain_backward():
     for k in KEYS:
         assert np.array_equal(a[k], plain[k]), "d%s differs from the plain backward" % k
         assert np.array_equal(a[k], b_[k]), "d%s differs between two calls" % k
+
+
+# ---- the tensor-core pair kernels (path "tensor") ----------------------------
+# bf16 inputs, P 64, N 128, chunk sizes that are multiples of 128.  The block
+# products run with fp16 operands: dy, the decay-weighted U = (C.B^T) L and
+# V = (dy.x^T) L, G_c and H_in are rounded to 11 bits, so every product term
+# carries up to 2^-10 relative error.  Derived bar: an output's error is
+# about 2^-11 of its own size, and the gradients are heavy-tailed (dx on the
+# 130m layer reaches 60x its RMS; an fp64 emulation of the kernels' roundings
+# on it gives 1.2e-2 max/RMS on 8 heads), so the largest elements reach
+# 2^-11 x 60 = 3e-2 of the RMS: max|gpu - oracle| / RMS <= 5e-2 per gradient,
+# and relative L2 <= 2e-3 for the per-element ones (the emulation gives
+# 2.2e-4, about 2^-12).
+TOL_TC = 5e-2
+TOL_TC_L2 = 2e-3
+
+TC_CASES = [
+    # b, L, H, G, Q, init, dfinal
+    (2, 300, 4, 2, 256, True, True),
+    (1, 128, 2, 1, 128, False, True),
+    (1, 129, 2, 2, 128, True, False),
+    (2, 640, 3, 3, 256, True, True),
+    (1, 1000, 4, 1, 512, True, True),
+]
+
+
+def _tc_case(b, L, H, G, Q, init, seed):
+    cfg = ScanConfig("bwdtc", b, L, H, 64, 128, G, Q, "bf16", "normal", "normal" if init else "zero", seed=seed)
+    return cfg, make_scan_inputs(cfg), make_grad_inputs(cfg)
+
+
+def run_bwd_tc(inp, grads, Q, with_dfinal=True, dt_limit=(0.0, math.inf)):
+    d = to_dev(inp)
+    b, L, H, P = d["x"].shape
+    G, N = d["B"].shape[2], d["B"].shape[3]
+    ws = ssd.alloc_workspace(ssd.bwd_workspace_size(b, L, H, P, N, G, Q, d["x"].dtype), "cuda")
+    g = ssd.chunk_scan_bwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], grads["dy"].cuda(),
+                           dfinal_state=grads["dfinal"].cuda() if with_dfinal else None, init_state=d["init_state"],
+                           chunk_size=Q, dt_limit=dt_limit, workspace=ws, path="tensor")
+    assert ssd.read_device_status(ws) == 0
+    torch.cuda.synchronize()
+    return {k: v.cpu().double().numpy() for k, v in g.items()}
+
+
+def check_tc(got, ref, what):
+    for k in KEYS:
+        if ref[k] is None:
+            continue
+        rel_max, rel_l2 = compare(got[k], ref[k], TOL_TC, "%s d%s" % (what, k))
+        if k in ("x", "dt_raw", "B", "C", "init_state"):
+            assert rel_l2 <= TOL_TC_L2, "%s d%s: relative L2 %.3e" % (what, k, rel_l2)
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "b%d_L%d_H%d_G%d_Q%d_init%d_df%d" % c)
+def test_backward_tensor_path(case):
+    b, L, H, G, Q, init, dfin = case
+    cfg, inp, grads = _tc_case(b, L, H, G, Q, init, seed=L + 11 * H + G)
+    got = run_bwd_tc(inp, grads, Q, with_dfinal=dfin)
+    ref = oracle_bwd(inp, grads, with_dfinal=dfin)
+    check_tc(got, ref, "tensor %s" % (case,))
+
+
+def test_backward_tensor_path_clamped_dt():
+    cfg, inp, grads = _tc_case(2, 300, 4, 2, 256, True, seed=77)
+    lim = (0.002, 0.05)
+    got = run_bwd_tc(inp, grads, 256, dt_limit=lim)
+    ref = oracle_bwd(inp, grads, dt_limit=lim)
+    check_tc(got, ref, "tensor clamped")
+
+
+def test_backward_tensor_path_130m_layer_and_determinism():
+    """The full-size 130m layer on the tensor path against the oracle, and two
+    calls give the same bits."""
+    cfg = SCAN_CONFIGS["c1_130m"]
+    inp = make_scan_inputs(cfg)
+    grads = make_grad_inputs(cfg)
+    a = run_bwd_tc(inp, grads, cfg.chunk_size)
+    b_ = run_bwd_tc(inp, grads, cfg.chunk_size)
+    for k in KEYS:
+        if a[k] is not None:
+            assert np.array_equal(a[k], b_[k]), "d%s differs between two calls" % k
+    check_tc(a, oracle_bwd(inp, grads), "tensor c1_130m")
+
+
+def test_backward_tensor_path_rejects_what_it_does_not_take():
+    for dtype, P, Q in (("f32", 64, 256), ("bf16", 32, 256), ("bf16", 64, 64)):
+        cfg = ScanConfig("bwdtcx", 1, 200, 2, P, 128, 1, Q, dtype, "normal", "zero", seed=3)
+        inp, grads = make_scan_inputs(cfg), make_grad_inputs(cfg)
+        with pytest.raises(ssd.SSDError, match="SSD_ERR_UNSUPPORTED"):
+            run_bwd_tc(inp, grads, Q)
