@@ -63,6 +63,9 @@ cudaError_t simt_scan(const ScanArgs &a, const ScanDims &d, void *workspace, cud
 // The first two launches of simt_scan alone (no y): fills dtv, cum, ell and
 // the entering states; writes final_state / chunk_states when not null.
 cudaError_t simt_scan_states(const ScanArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
+// Launch 2 of simt_scan alone: the chunk states already in the workspace
+// (with dtv, cum, ell) become the states entering each chunk.
+cudaError_t simt_state_pass(const ScanArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
 
 // ---- backward of the scan (SIMT fp32, deterministic) -----------------------
 struct BwdArgs {
@@ -90,6 +93,20 @@ struct BwdPairArgs {
 };
 bool bwd_tc_supported(const ScanDims &d, int bf16, int packed);
 cudaError_t bwd_tc_pairs(const BwdPairArgs &a, const ScanDims &d, cudaStream_t s);
+// The forward recompute's first launch and the backward's per-chunk sums on
+// the tensor cores, for the same shapes: dt, cum and the chunk log decay
+// (ell), the chunk state S_c = sum_j e^{cl-cum_j} dt_j B_j x_j^T into
+// `states`, and sum_i e^{cum_i} C_i dy_i^T into `gst`, per (chunk, head,
+// batch).  The state passes run after it as before.
+struct BwdStatesArgs {
+    const void *x, *B, *C;          // bf16
+    const float *dt_raw, *dt_bias, *A, *dy;
+    float dt_lo, dt_hi;
+    float *dtv, *cum, *ell;         // [b, H, L], [b, H, L], [b, H, nc]
+    float *states, *gst;            // [b, H, nc, N, P]
+    unsigned *status;
+};
+cudaError_t bwd_tc_states(const BwdStatesArgs &a, const ScanDims &d, cudaStream_t s);
 size_t bwd_workspace_bytes(const ScanDims &d);
 cudaError_t bwd_scan(const BwdArgs &a, const ScanDims &d, void *workspace, cudaStream_t s);
 

@@ -749,20 +749,31 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
     if ((e = cudaFuncSetAttribute(rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr)) !=
         cudaSuccess)
         return e;
-    if ((e = simt_scan_states(a.f, d, wsp, s)) != cudaSuccess) return e;
     const int L = (int)d.L, H = (int)d.H, P = (int)d.P, N = (int)d.N, G = (int)d.G, Q = (int)d.Q;
     const int nc = (int)d.nc, NP = N * P;
     const dim3 gc((unsigned)nc, (unsigned)H, (unsigned)d.b);
     const int packed = a.f.seq_idx ? 1 : 0;
-    if (packed) {
-        docs_kernel<<<dim3((unsigned)nc, (unsigned)d.b), kThreads, 0, s>>>(a.f.seq_idx, ws.docc, L, Q);
+    if (a.tensor) {
+        // the chunk states and the per-chunk dy sums on the tensor cores
+        // (ssd_scan_bwd_tc.cu), then the forward's state pass
+        BwdStatesArgs sa;
+        sa.x = a.f.x; sa.B = a.f.B; sa.C = a.f.C; sa.dt_raw = a.f.dt_raw; sa.dt_bias = a.f.dt_bias; sa.A = a.f.A;
+        sa.dy = a.dy; sa.dt_lo = a.f.dt_lo; sa.dt_hi = a.f.dt_hi; sa.dtv = ws.f.dtv; sa.cum = ws.f.cum;
+        sa.ell = ws.f.ell; sa.states = ws.f.states; sa.gst = ws.gst; sa.status = ws.f.status;
+        if ((e = bwd_tc_states(sa, d, s)) != cudaSuccess) return e;
+        if ((e = simt_state_pass(a.f, d, wsp, s)) != cudaSuccess) return e;
+    } else {
+        if ((e = simt_scan_states(a.f, d, wsp, s)) != cudaSuccess) return e;
+        if (packed) {
+            docs_kernel<<<dim3((unsigned)nc, (unsigned)d.b), kThreads, 0, s>>>(a.f.seq_idx, ws.docc, L, Q);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        {
+            TraceScope tr(s, kTrBwdDstate);
+            dstate_kernel<T><<<gc, kThreads, smd, s>>>((const T *)a.f.C, a.dy, ws, L, H, P, N, G, Q, nc, packed);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    {
-        TraceScope tr(s, kTrBwdDstate);
-        dstate_kernel<T><<<gc, kThreads, smd, s>>>((const T *)a.f.C, a.dy, ws, L, H, P, N, G, Q, nc, packed);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int nblk = dpass_blocks(d);
     {
         TraceScope tr(s, kTrBwdDpass);

@@ -581,12 +581,190 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     }
 }
 
+// ---- states ---------------------------------------------------------------
+// per (chunk, head, batch): dt, cum, ell, and the two per-chunk N x P sums,
+// block by block of 128 tokens:
+//   S_c  += B_k^T (w x)_k     w_j = e^{min(cl-cum_j,0)} dt_j   (M=128 n, N=64 p, K=128 j)
+//   dS_c += C_k^T (e dy)_k    e_i = e^{min(cum_i,0)}            (M=128 n, N=64 p, K=128 i)
+// (the operand forms of the forward's unit-state MMA: B and C tiles read
+// MN-major, the scaled x and dy tiles MN-major).  TMEM lane = state row n.
+constexpr int kQMax = 1024;
+constexpr uint32_t kSB = 0, kSWX = 2 * kT, kSC = 3 * kT, kSEDY = 5 * kT, kSScal = 6 * kT;
+// scalars: dt[kQMax], cum[kQMax], w[128], e[128], warp totals[32]
+constexpr uint32_t kSBar = kSScal + (2 * kQMax + 2 * kB + 32) * 4;
+constexpr size_t kStatesSmem = 1024 + kSBar + 16;
+
+// Rows 0..127 of a [128 x 64] fp16 tile: row r of `src` (bf16 or fp32, 64
+// values) times scale[r]; rows past nrows zero
+template <typename S>
+__device__ __forceinline__ void fill_scaled64(uint8_t *tile, const S *src, size_t ld, int nrows, const float *scale,
+                                              int tid, __half2 &amax) {
+    for (int c = tid; c < kB * 8; c += kThr) {
+        const int r = c >> 3, k = c & 7;
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (r < nrows) {
+            float f[8];
+            if constexpr (sizeof(S) == 2) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * ld + 8 * k);
+                f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+                f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+            } else {
+                const float4 a = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k);
+                const float4 b = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k + 4);
+                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+            }
+            const float w = scale[r];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= w;
+            o = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
+            const uint32_t wv[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&wv[i])));
+        }
+        *reinterpret_cast<uint4 *>(tile + sw128_off(r, k)) = o;
+    }
+}
+
+__global__ void __launch_bounds__(kThr, 2)
+tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *s_dt = reinterpret_cast<float *>(sm + kSScal);
+    float *s_cum = s_dt + kQMax, *s_w = s_cum + kQMax, *s_e = s_w + kB, *s_wt = s_e + kB;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kSBar);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
+
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (H / G);
+    const int t0 = c * Q, q = min(Q, L - t0);
+    const size_t bh = (size_t)b * H + h;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lg = warp & 3, ch = warp >> 2, row = 32 * lg + lane;
+    const float Ah = a.A[h], bias = a.dt_bias[h];
+    __half2 amax = __float2half2_rn(0.f);
+    if (tid == 0 && Ah > 0.f) flag_status(a.status, kStatusPrecondition);
+    if (warp == 0) {
+        tmem_alloc(tslot, 128);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    // dt = clamp(softplus(dt_raw + dt_bias)) and its inclusive cumsum times A (fixed order)
+    float carry = 0.f;
+    for (int base = 0; base < q; base += kThr) {
+        const int i = base + tid;
+        const float d = i < q ? dt_of(a.dt_raw[((size_t)b * L + t0 + i) * H + h], bias, a.dt_lo, a.dt_hi) : 0.f;
+        float tot;
+        const float sc = block_inclusive_scan(d * Ah, s_wt, tot) + carry;
+        if (i < q) {
+            s_dt[i] = d;
+            s_cum[i] = sc;
+            a.dtv[bh * L + t0 + i] = d;
+            a.cum[bh * L + t0 + i] = sc;
+        }
+        carry += tot;
+    }
+    __syncthreads();
+    const float cl = s_cum[q - 1];
+    if (tid == 0) a.ell[bh * nc + c] = cl;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * lg) << 16);
+    const uint32_t sbase = smem_u32(sm);
+    uint32_t ph = 0, commits = 0;
+    bool ok = true;
+    const int nk = (q + kB - 1) / kB;
+    for (int kb = 0; kb < nk; ++kb) {
+        const int j0 = kb * kB, nr = min(kB, q - j0);
+        const size_t tok = (size_t)b * L + t0 + j0;
+        if (tid < kB) {
+            const bool v = tid < nr;
+            s_w[tid] = v ? expf(fminf(cl - s_cum[j0 + tid], 0.f)) * s_dt[j0 + tid] : 0.f;
+            s_e[tid] = v ? expf(fminf(s_cum[j0 + tid], 0.f)) : 0.f;
+        }
+        __syncthreads();                               // the previous block's MMAs are complete
+        fill_tile(sm + kSB, static_cast<const __nv_bfloat16 *>(a.B) + (tok * G + g) * kNs, (size_t)G * kNs, nr, 128,
+                  tid, amax);
+        fill_tile(sm + kSC, static_cast<const __nv_bfloat16 *>(a.C) + (tok * G + g) * kNs, (size_t)G * kNs, nr, 128,
+                  tid, amax);
+        fill_scaled64(sm + kSWX, static_cast<const __nv_bfloat16 *>(a.x) + (tok * H + h) * kPh, (size_t)H * kPh, nr,
+                      s_w, tid, amax);
+        fill_scaled64(sm + kSEDY, a.dy + (tok * H + h) * kPh, (size_t)H * kPh, nr, s_e, tid, amax);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            const uint64_t dB = sdesc_sw128(sbase + kSB, kT, 1024), dWX = sdesc_sw128(sbase + kSWX, kT, 1024);
+            const uint64_t dC = sdesc_sw128(sbase + kSC, kT, 1024), dE = sdesc_sw128(sbase + kSEDY, kT, 1024);
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8)
+                mma_f16(tmem, dB + ((s8 * 2048) >> 4), dWX + ((s8 * 2048) >> 4), idesc_f16(128, 64, 1, 1),
+                        (kb > 0 || s8 > 0) ? 1u : 0u);
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8)
+                mma_f16(tmem + 64, dC + ((s8 * 2048) >> 4), dE + ((s8 * 2048) >> 4), idesc_f16(128, 64, 1, 1),
+                        (kb > 0 || s8 > 0) ? 1u : 0u);
+            mma_commit(bar);
+            ++commits;
+        }
+        ok = ok && wait_mma(bar, ph);
+        ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+        // lane n of TMEM is state row n; this thread's 32 of the 64 p columns
+        float t32[32];
+        const size_t off = (bh * nc + c) * (size_t)(kNs * kPh) + (size_t)row * kPh + 32 * ch;
+        tmem_ld32(lane_addr + 32 * ch, t32);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4 *>(a.states + off + 4 * k) =
+                make_float4(t32[4 * k], t32[4 * k + 1], t32[4 * k + 2], t32[4 * k + 3]);
+        tmem_ld32(lane_addr + 64 + 32 * ch, t32);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4 *>(a.gst + off + 4 * k) =
+                make_float4(t32[4 * k], t32[4 * k + 1], t32[4 * k + 2], t32[4 * k + 3]);
+    }
+    if (__any_sync(0xffffffffu, !ok) && lane == 0) flag_status(a.status, kStatusTimeout);
+    if (lane == 0) finish_range(a.status, amax);
+    if (tid == 0 && commits > ph) mbar_wait(bar, (commits - 1) & 1u, kBudget);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
 }  // namespace
 
 bool bwd_tc_supported(const ScanDims &d, int bf16, int packed) {
-    if (!bf16 || packed || d.P != kPh || d.N != kNs || d.Q % kB != 0 || d.Q > 1024) return false;
+    if (!bf16 || packed || d.P != kPh || d.N != kNs || d.Q % kB != 0 || d.Q > kQMax) return false;
     if (d.H > 65535 || d.b > 65535 || d.nc * (d.Q / kB) > 0x7fffffffll) return false;
     return true;
+}
+
+cudaError_t bwd_tc_states(const BwdStatesArgs &a, const ScanDims &d, cudaStream_t s) {
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        if ((e = cudaFuncSetAttribute(tc_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kStatesSmem)) != cudaSuccess)
+            return e;
+        attr_done[dev] = true;
+    }
+    TraceScope tr(s, kTrBwdStates);
+    tc_states_kernel<<<dim3((unsigned)d.nc, (unsigned)d.H, (unsigned)d.b), kThr, kStatesSmem, s>>>(
+        a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+    return cudaGetLastError();
 }
 
 cudaError_t bwd_tc_pairs(const BwdPairArgs &a, const ScanDims &d, cudaStream_t s) {

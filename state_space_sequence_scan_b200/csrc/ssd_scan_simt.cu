@@ -392,6 +392,18 @@ cudaError_t simt_scan(const ScanArgs &a, const ScanDims &d, void *ws, cudaStream
     return a.bf16 ? run<__nv_bfloat16>(a, d, ws, s) : run<float>(a, d, ws, s);
 }
 
+cudaError_t simt_state_pass(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) {
+    const SimtWs ws = simt_carve(d, wsp);
+    const int NP = (int)(d.N * d.P);
+    const dim3 g2((unsigned)((NP + kThreads - 1) / kThreads), (unsigned)d.H, (unsigned)d.b);
+    {
+        TraceScope tr(s, kTrSimtStatePass);
+        state_pass_kernel<<<g2, kThreads, 0, s>>>(ws, a.init_state, a.final_state, a.chunk_states, (int)d.H, NP,
+                                                  (int)d.nc);
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t simt_scan_states(const ScanArgs &a, const ScanDims &d, void *ws, cudaStream_t s) {
     const SimtWs w = simt_carve(d, ws);
     return a.bf16 ? run_states<__nv_bfloat16>(a, d, w, s) : run_states<float>(a, d, w, s);

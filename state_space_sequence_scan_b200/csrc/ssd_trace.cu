@@ -31,7 +31,7 @@ struct Tracer {
 const char *kNames[kKernelCount] = {
     "simt_chunk_state", "simt_state_pass", "simt_chunk_out", "decode_step",
     "tc_unit_state", "tc_state_pass", "tc_chunk_out", "tc_dt_prep", "conv1d_silu", "gated_rmsnorm",
-    "bwd_dstate", "bwd_dpass", "bwd_cols", "bwd_rows", "bwd_finalize", "bwd_reduce",
+    "bwd_dstate", "bwd_dpass", "bwd_cols", "bwd_rows", "bwd_finalize", "bwd_reduce", "bwd_states",
 };
 
 }  // namespace

@@ -22,7 +22,8 @@ enum TraceKernel {
     kTrBwdRows = 13,
     kTrBwdFinalize = 14,
     kTrBwdReduce = 15,
-    kKernelCount = 16,
+    kTrBwdStates = 16,
+    kKernelCount = 17,
 };
 
 bool trace_on();
