@@ -317,51 +317,78 @@ def capture_steps(step, steps):
 
 
 def e2e_scan(inp, cfg, args, dev, work):
-    """Same metric through the public call with host buffers: pinned host
-    inputs copied in, the scan, y and final_state (and with --chunk-states the
-    chunk-boundary states) copied back, every step."""
+    """Same metric through the public call with host buffers: every step
+    copies its inputs in from pinned host memory, runs the scan and copies y
+    and final_state (and with --chunk-states the chunk-boundary states) back.
+    Steps are pipelined the way a caller streaming batches would run them:
+    two device and two pinned host buffer sets, the copies in on one stream,
+    the scans on another, the copies out on a third, so that step k+1's
+    inputs cross PCIe while step k computes and step k-1's results come back
+    (the link is full duplex).  Timed with CUDA events from the first copy in
+    to the last copy out."""
     from state_space_sequence_scan_b200 import ssd
-    host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
-    d = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in inp.items()}
     b, L, H, P, N, Q = cfg.batch, cfg.seqlen, cfg.nheads, cfg.head_dim, cfg.state_dim, cfg.chunk_size
-    y = torch.empty(b, L, H, P, device=dev)
-    fs = torch.empty(b, H, N, P, device=dev)
-    y_h = torch.empty(b, L, H, P).pin_memory()
-    fs_h = torch.empty(b, H, N, P).pin_memory()
     nc = math.ceil(L / Q)
-    cs = torch.empty(b, nc, H, N, P, device=dev) if args.chunk_states else None
-    cs_h = torch.empty(b, nc, H, N, P).pin_memory() if args.chunk_states else None
-    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = y_h.numel() * 4 + fs_h.numel() * 4 + (cs_h.numel() * 4 if cs_h is not None else 0)
-    steps = max(3, min(args.steps, 20))
-
-    def one():
-        for k, v in host.items():
-            if v is not None:
-                d[k].copy_(v, non_blocking=True)
-        if cs is None:
-            ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
-                               init_state=d["init_state"], chunk_size=Q, path=args.path, workspace=work, y=y,
-                               final_state=fs)
-        else:
-            ssd.chunk_scan_fwd_states(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
-                                      init_state=d["init_state"], chunk_size=Q, path=args.path, workspace=work,
-                                      y=y, final_state=fs, chunk_states=cs)
-            cs_h.copy_(cs, non_blocking=True)
-        y_h.copy_(y, non_blocking=True)
-        fs_h.copy_(fs, non_blocking=True)
-
+    host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+    slots = []
     for _ in range(2):
-        one()
+        sl = {"d": {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in inp.items()},
+              "y": torch.empty(b, L, H, P, device=dev), "fs": torch.empty(b, H, N, P, device=dev),
+              "y_h": torch.empty(b, L, H, P).pin_memory(), "fs_h": torch.empty(b, H, N, P).pin_memory(),
+              "cs": torch.empty(b, nc, H, N, P, device=dev) if args.chunk_states else None,
+              "cs_h": torch.empty(b, nc, H, N, P).pin_memory() if args.chunk_states else None}
+        slots.append(sl)
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = (slots[0]["y_h"].numel() * 4 + slots[0]["fs_h"].numel() * 4 +
+           (slots[0]["cs_h"].numel() * 4 if args.chunk_states else 0))
+    steps = max(3, min(args.steps, 20))
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "cmp", "out")}
+
+    def one(k):
+        sl = slots[k % 2]
+        e_in, e_cmp, e_out = ev["in"][k % 2], ev["cmp"][k % 2], ev["out"][k % 2]
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(e_out)          # step k-2 is done with this slot (its scan and its copy out)
+            for kk, v in host.items():
+                if v is not None:
+                    sl["d"][kk].copy_(v, non_blocking=True)
+            e_in.record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(e_in)
+            d = sl["d"]
+            if sl["cs"] is None:
+                ssd.chunk_scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                                   init_state=d["init_state"], chunk_size=Q, path=args.path, workspace=work,
+                                   y=sl["y"], final_state=sl["fs"])
+            else:
+                ssd.chunk_scan_fwd_states(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                                          init_state=d["init_state"], chunk_size=Q, path=args.path,
+                                          workspace=work, y=sl["y"], final_state=sl["fs"], chunk_states=sl["cs"])
+            e_cmp.record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(e_cmp)
+            sl["y_h"].copy_(sl["y"], non_blocking=True)
+            sl["fs_h"].copy_(sl["fs"], non_blocking=True)
+            if sl["cs"] is not None:
+                sl["cs_h"].copy_(sl["cs"], non_blocking=True)
+            e_out.record(s_out)
+
+    for k in range(2):
+        one(k)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(s_in)
+    for k in range(steps):
+        one(k)
+    s_out.synchronize()
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    return dict(ms_per_step=ms, h2d=h2d, d2h=d2h, steps=steps)
+    if ssd.read_device_status(work) != 0:
+        raise RuntimeError("device status %d after the end-to-end steps" % ssd.read_device_status(work))
+    return dict(ms_per_step=ms, h2d=h2d, d2h=d2h, steps=steps, pipelined="2 buffer sets, 3 streams")
 
 
 def bench_step(cfg, args, ws, rank, local):
@@ -1027,7 +1054,8 @@ def finish(cfg, is_step, r, args, ws, rank, peaks, peak_kind, sub=False):
                                       (not is_step) and args.packed),
             "roofline": roof, "clocks": r["clocks"],
             "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": r["e2e"]["h2d"],
-                    "d2h_bytes_per_step": r["e2e"]["d2h"]},
+                    "d2h_bytes_per_step": r["e2e"]["d2h"], "ms_per_step": r["e2e"]["ms_per_step"],
+                    **({"pipelined": r["e2e"]["pipelined"]} if "pipelined" in r["e2e"] else {})},
             "gpu_launches": r["launches"]}
     if sub:
         for k in ("metric", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "vs_baseline", "data"):

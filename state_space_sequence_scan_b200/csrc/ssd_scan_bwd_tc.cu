@@ -229,6 +229,17 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         mma_commit(bar);
         ++commits;
     }
+    // the first i block's operands while the G_c MMAs run (they read other tiles)
+    const int nIb = (q + kB - 1) / kB;
+    auto fill_i = [&](int Ib) {
+        const int i0 = Ib * kB, ti = min(kB, q - i0);
+        const size_t toki = (size_t)b * L + t0 + i0;
+        fill_tile(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs, (size_t)G * kNs, ti,
+                  128, tid, amax);
+        fill_tile(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, 64, tid, amax);
+        if (tid < kB) s_cumi[tid] = tid < ti ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
+    };
+    fill_i(Jb);
     ok = wait_mma(bar, ph);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
@@ -251,15 +262,10 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         tmem_st32(lane_addr + kTmDX + 32 * ch, t32);
     }
     float zs = 0.f, zo = 0.f;                          // this thread's i half
-    const int nIb = (q + kB - 1) / kB;
     for (int Ib = Jb; Ib < nIb; ++Ib) {
         const int i0 = Ib * kB, ti = min(kB, q - i0);
-        const size_t toki = (size_t)b * L + t0 + i0;
         // the previous pair's MMAs (which read C_I, DY_I, U, V) are complete
-        fill_tile(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs, (size_t)G * kNs, ti,
-                  128, tid, amax);
-        fill_tile(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, 64, tid, amax);
-        if (tid < kB) s_cumi[tid] = tid < ti ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
+        if (Ib > Jb) fill_i(Ib);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -456,6 +462,20 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         mma_commit(bar);
         ++commits;
     }
+    // the first j block's operands while the H_in MMAs run (they read other tiles)
+    auto fill_j = [&](int Jb) {
+        const int j0 = Jb * kB, tj = min(kB, q - j0);
+        const size_t tokj = (size_t)b * L + t0 + j0;
+        fill_tile(sm + kRBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs, (size_t)G * kNs, tj,
+                  128, tid, amax);
+        fill_tile(sm + kRXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh, (size_t)H * kPh, tj,
+                  64, tid, amax);
+        if (tid < kB) {
+            s_cumj[tid] = tid < tj ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
+            s_dtj[tid] = tid < tj ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
+        }
+    };
+    fill_j(0);
     ok = wait_mma(bar, ph);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
@@ -477,15 +497,8 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     const int gi = i0 + row;
     for (int Jb = 0; Jb <= Ib; ++Jb) {
         const int j0 = Jb * kB, tj = min(kB, q - j0);
-        const size_t tokj = (size_t)b * L + t0 + j0;
-        fill_tile(sm + kRBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs, (size_t)G * kNs, tj,
-                  128, tid, amax);
-        fill_tile(sm + kRXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh, (size_t)H * kPh, tj,
-                  64, tid, amax);
-        if (tid < kB) {
-            s_cumj[tid] = tid < tj ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
-            s_dtj[tid] = tid < tj ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
-        }
+        // the previous pair's MMAs (which read B_J, V) are complete
+        if (Jb > 0) fill_j(Jb);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();

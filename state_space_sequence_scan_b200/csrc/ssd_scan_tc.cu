@@ -312,6 +312,7 @@ __device__ __forceinline__ void conv_load_weights(float4 *wb, const float *cw, c
 // CTAs in flight: every thread issues its few loads before any arithmetic.
 constexpr int kPrepHeads = 8;
 
+template <bool kConv>
 __global__ void __launch_bounds__(256)
 prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias, const float *__restrict__ A,
             const __nv_bfloat16 *__restrict__ Bm, const __nv_bfloat16 *__restrict__ Cm,
@@ -327,7 +328,7 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
         const int t0 = blk * kBlk + 32 * quarter;
         const size_t Lp = (size_t)nblk * kBlk;
         __half2 amax = __float2half2_rn(0.f);
-        if (cw) {
+        if constexpr (kConv) {
             // combined arrangement: B and C are conv1d + SiLU of xbc's channels
             // H*P + g*N.. (B) and H*P + G*N + g*N.. (C), rounded to bf16 as the
             // split conv stores them.  Thread: one tensor, one 8-channel chunk,
@@ -1405,7 +1406,8 @@ cudaError_t tc_scan(const ScanArgs &a, const ScanDims &d, void *wsp, cudaStream_
         // a plain launch: it overwrites the workspace the previous call's kernels read
         // (combined arrangement: B and C come from xbc, through the conv)
         const unsigned ny = (unsigned)((d.H + kPrepHeads - 1) / kPrepHeads + 4 * d.G);
-        prep_kernel<<<dim3((unsigned)p.nblk, ny, (unsigned)d.b), 256, 0, s>>>(
+        auto prep = conv ? prep_kernel<true> : prep_kernel<false>;   // the split path compiles without the conv
+        prep<<<dim3((unsigned)p.nblk, ny, (unsigned)d.b), 256, 0, s>>>(
             a.dt_raw, a.dt_bias, a.A, static_cast<const __nv_bfloat16 *>(conv ? a.x : a.B),
             static_cast<const __nv_bfloat16 *>(a.C), a.seq_idx, ws, (int)d.L, (int)d.H, (int)d.G, (int)p.nblk,
             a.dt_lo, a.dt_hi, a.conv_w, a.conv_b, (int)a.Cd);
