@@ -53,33 +53,61 @@ constexpr float kF16Max = 65504.0f;
 // K-step q (16 elements) of a K-major operand 128 wide (two 64-wide tiles)
 __device__ __forceinline__ uint32_t kofs128(int q) { return (uint32_t)((q >> 2) * kT + (q & 3) * 32); }
 
+// 8 source values (one 16-byte fp16 chunk's worth) -> floats
+template <typename S> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) { v = *reinterpret_cast<const uint4 *>(p); }
+    __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void get(float (&f)[8]) const {
+        f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+        f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float *p) {
+        a = *reinterpret_cast<const float4 *>(p);
+        b = *reinterpret_cast<const float4 *>(p + 4);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void get(float (&f)[8]) const {
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    }
+};
+
 // Rows 0..127 of a [128 x W] fp16 tile (W = 64 or 128: one or two swizzled
-// 64-wide tiles) from `nrows` source rows of `ld` elements (bf16 or fp32);
-// rows past nrows are zero.  All 256 threads; one 16-byte chunk (8 values)
-// per step, consecutive threads on consecutive chunks of a row.
-template <typename S>
-__device__ __forceinline__ void fill_tile(uint8_t *tile, const S *src, size_t ld, int nrows, int W, int tid,
-                                          __half2 &amax) {
-    const int cpr = W / 8;                 // chunks per row
-    for (int c = tid; c < kB * cpr; c += kThr) {
-        const int r = c / cpr, k = c - r * cpr;
-        uint4 o = make_uint4(0u, 0u, 0u, 0u);
-        if (r < nrows) {
-            float f[8];
-            if constexpr (sizeof(S) == 2) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * ld + 8 * k);
-                f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
-                f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
-            } else {
-                const float4 a = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k);
-                const float4 b = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k + 4);
-                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-            }
-            o = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
-            const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+// 64-wide tiles) from `nrows` source rows of `ld` elements (bf16 or fp32),
+// each row times scale[r] when `scale` is given; rows past nrows are zero.
+// All 256 threads; one 16-byte chunk (8 values) per step, consecutive
+// threads on consecutive chunks of a row, every load issued before the
+// first conversion.
+template <int W, typename S>
+__device__ __forceinline__ void fill_tile(uint8_t *tile, const S *src, size_t ld, int nrows, int tid, __half2 &amax,
+                                          const float *scale = nullptr) {
+    constexpr int cpr = W / 8;             // chunks per row
+    constexpr int kIt = kB * cpr / kThr;   // chunks per thread
+    Raw8<S> raw[kIt];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&w[i])));
+    for (int it = 0; it < kIt; ++it) {
+        const int c = tid + it * kThr, r = c / cpr, k = c - r * cpr;
+        if (r < nrows) raw[it].load(src + (size_t)r * ld + 8 * k);
+        else raw[it].zero();
+    }
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+        const int c = tid + it * kThr, r = c / cpr, k = c - r * cpr;
+        float f[8];
+        raw[it].get(f);
+        if (scale) {
+            const float w = scale[r];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= w;
         }
+        const uint4 o = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
+        const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&w4[i])));
         *reinterpret_cast<uint4 *>(tile + (k >> 3) * kT + sw128_off(r, k & 7)) = o;
     }
 }
@@ -174,11 +202,11 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     }
     // j block: B_J, X_J (fp16), G_c (fp16 [n][p]); per-token scalars
     const size_t tokj = (size_t)b * L + t0 + j0;
-    fill_tile(sm + kCBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs, (size_t)G * kNs, tj, 128,
-              tid, amax);
-    fill_tile(sm + kCXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh, (size_t)H * kPh, tj, 64,
-              tid, amax);
-    fill_tile(sm + kCG, a.gst + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, 64, tid, amax);
+    fill_tile<128>(sm + kCBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs,
+                   (size_t)G * kNs, tj, tid, amax);
+    fill_tile<64>(sm + kCXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh,
+                  (size_t)H * kPh, tj, tid, amax);
+    fill_tile<64>(sm + kCG, a.gst + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, tid, amax);
     const float cl = a.cum[bh * L + t0 + q - 1];
     if (tid < kB) {
         const bool v = tid < tj;
@@ -234,9 +262,9 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     auto fill_i = [&](int Ib) {
         const int i0 = Ib * kB, ti = min(kB, q - i0);
         const size_t toki = (size_t)b * L + t0 + i0;
-        fill_tile(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs, (size_t)G * kNs, ti,
-                  128, tid, amax);
-        fill_tile(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, 64, tid, amax);
+        fill_tile<128>(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs,
+                       (size_t)G * kNs, ti, tid, amax);
+        fill_tile<64>(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, tid, amax);
         if (tid < kB) s_cumi[tid] = tid < ti ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
     };
     fill_i(Jb);
@@ -433,10 +461,10 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         fence_mbar_init();
     }
     const size_t toki = (size_t)b * L + t0 + i0;
-    fill_tile(sm + kRCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs, (size_t)G * kNs, ti, 128,
-              tid, amax);
-    fill_tile(sm + kRDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, 64, tid, amax);
-    fill_tile(sm + kRH, a.states + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, 64, tid, amax);
+    fill_tile<128>(sm + kRCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs,
+                   (size_t)G * kNs, ti, tid, amax);
+    fill_tile<64>(sm + kRDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, tid, amax);
+    fill_tile<64>(sm + kRH, a.states + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, tid, amax);
     if (tid < kB) {
         const bool v = tid < ti;
         const float ci = v ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
@@ -466,10 +494,10 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     auto fill_j = [&](int Jb) {
         const int j0 = Jb * kB, tj = min(kB, q - j0);
         const size_t tokj = (size_t)b * L + t0 + j0;
-        fill_tile(sm + kRBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs, (size_t)G * kNs, tj,
-                  128, tid, amax);
-        fill_tile(sm + kRXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh, (size_t)H * kPh, tj,
-                  64, tid, amax);
+        fill_tile<128>(sm + kRBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs,
+                       (size_t)G * kNs, tj, tid, amax);
+        fill_tile<64>(sm + kRXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh,
+                      (size_t)H * kPh, tj, tid, amax);
         if (tid < kB) {
             s_cumj[tid] = tid < tj ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
             s_dtj[tid] = tid < tj ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
@@ -607,37 +635,6 @@ constexpr uint32_t kSB = 0, kSWX = 2 * kT, kSC = 3 * kT, kSEDY = 5 * kT, kSScal 
 constexpr uint32_t kSBar = kSScal + (2 * kQMax + 2 * kB + 32) * 4;
 constexpr size_t kStatesSmem = 1024 + kSBar + 16;
 
-// Rows 0..127 of a [128 x 64] fp16 tile: row r of `src` (bf16 or fp32, 64
-// values) times scale[r]; rows past nrows zero
-template <typename S>
-__device__ __forceinline__ void fill_scaled64(uint8_t *tile, const S *src, size_t ld, int nrows, const float *scale,
-                                              int tid, __half2 &amax) {
-    for (int c = tid; c < kB * 8; c += kThr) {
-        const int r = c >> 3, k = c & 7;
-        uint4 o = make_uint4(0u, 0u, 0u, 0u);
-        if (r < nrows) {
-            float f[8];
-            if constexpr (sizeof(S) == 2) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(src + (size_t)r * ld + 8 * k);
-                f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
-                f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
-            } else {
-                const float4 a = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k);
-                const float4 b = *reinterpret_cast<const float4 *>(src + (size_t)r * ld + 8 * k + 4);
-                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-            }
-            const float w = scale[r];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] *= w;
-            o = make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
-            const uint32_t wv[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) amax = __hmax2(amax, __habs2(*reinterpret_cast<const __half2 *>(&wv[i])));
-        }
-        *reinterpret_cast<uint4 *>(tile + sw128_off(r, k)) = o;
-    }
-}
-
 __global__ void __launch_bounds__(kThr, 2)
 tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
     extern __shared__ uint8_t smem_raw[];
@@ -700,13 +697,13 @@ tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
             s_e[tid] = v ? expf(fminf(s_cum[j0 + tid], 0.f)) : 0.f;
         }
         __syncthreads();                               // the previous block's MMAs are complete
-        fill_tile(sm + kSB, static_cast<const __nv_bfloat16 *>(a.B) + (tok * G + g) * kNs, (size_t)G * kNs, nr, 128,
-                  tid, amax);
-        fill_tile(sm + kSC, static_cast<const __nv_bfloat16 *>(a.C) + (tok * G + g) * kNs, (size_t)G * kNs, nr, 128,
-                  tid, amax);
-        fill_scaled64(sm + kSWX, static_cast<const __nv_bfloat16 *>(a.x) + (tok * H + h) * kPh, (size_t)H * kPh, nr,
-                      s_w, tid, amax);
-        fill_scaled64(sm + kSEDY, a.dy + (tok * H + h) * kPh, (size_t)H * kPh, nr, s_e, tid, amax);
+        fill_tile<128>(sm + kSB, static_cast<const __nv_bfloat16 *>(a.B) + (tok * G + g) * kNs,
+                       (size_t)G * kNs, nr, tid, amax);
+        fill_tile<128>(sm + kSC, static_cast<const __nv_bfloat16 *>(a.C) + (tok * G + g) * kNs,
+                       (size_t)G * kNs, nr, tid, amax);
+        fill_tile<64>(sm + kSWX, static_cast<const __nv_bfloat16 *>(a.x) + (tok * H + h) * kPh, (size_t)H * kPh, nr,
+                      tid, amax, s_w);
+        fill_tile<64>(sm + kSEDY, a.dy + (tok * H + h) * kPh, (size_t)H * kPh, nr, tid, amax, s_e);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
