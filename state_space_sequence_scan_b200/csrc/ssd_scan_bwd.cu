@@ -54,7 +54,7 @@ constexpr int kMaxP = 64, kMaxN = 128;
 struct BwdWs {
     SimtWs f;          // forward: dtv, cum, ell, entering states
     float *gst;        // [b, H, nc, N, P]: 1's output, then G_c
-    float *ghp;        // [b, H, nc, nblk]: partial <G_c, H_in>
+    float *ghp;        // [b, H, nc, nblk * 8]: partial <G_c, H_in> per dpass warp
     float *ddt_dir;    // [b, H, L]
     float *dcum_col;   // [b, H, L]
     float *dcum_row;   // [b, H, L]
@@ -71,7 +71,7 @@ size_t bwd_extra_bytes(const ScanDims &d, size_t *offs) {
     const size_t bh = (size_t)d.b * d.H;
     const size_t sizes[7] = {
         bh * d.nc * d.N * d.P * sizeof(float),
-        bh * d.nc * dpass_blocks(d) * sizeof(float),
+        bh * d.nc * dpass_blocks(d) * (kThreads / 32) * sizeof(float),
         bh * d.L * sizeof(float) * 5,
         bh * d.nc * 3 * sizeof(float),
         d.G == d.H ? 0 : (size_t)d.b * d.L * d.H * d.N * sizeof(float),
@@ -189,24 +189,45 @@ dstate_kernel(const T *__restrict__ Cm, const float *__restrict__ dy, BwdWs ws, 
 }
 
 // ---- 2. reverse state pass --------------------------------------------------
+// Thread = one state element, serial over chunks from the last; the inputs
+// of kDpBatch chunks are loaded together before their steps run.  Each
+// warp's share of <G_c, H_in> goes to its own slot (a shuffle tree, fixed
+// order); finalize adds the slots in index order.
+constexpr int kDpBatch = 8;
 __global__ void __launch_bounds__(kThreads)
 dpass_kernel(BwdWs ws, const float *__restrict__ dfinal, float *__restrict__ dinit, int H, int NP, int nc) {
-    __shared__ float red[32];
     const int e = blockIdx.x * kThreads + threadIdx.x;
     const bool live = e < NP;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t bh = (size_t)blockIdx.z * H + blockIdx.y;
+    const int nparts = gridDim.x * (kThreads / 32);
     float gcur = (live && dfinal) ? dfinal[bh * NP + e] : 0.f;
-    for (int c = nc - 1; c >= 0; --c) {
-        const size_t off = (bh * nc + c) * (size_t)NP + e;
-        float ds = 0.f, hin = 0.f;
-        if (live) {
-            ds = ws.gst[off];
-            hin = ws.f.states[off];
-            ws.gst[off] = gcur;                     // gradient of the state after chunk c
+    for (int c1 = nc - 1; c1 >= 0; c1 -= kDpBatch) {
+        float ds[kDpBatch], hin[kDpBatch], dec[kDpBatch];
+#pragma unroll
+        for (int k = 0; k < kDpBatch; ++k) {
+            const int c = c1 - k;
+            ds[k] = hin[k] = dec[k] = 0.f;
+            if (c >= 0) {
+                dec[k] = expf(fminf(ws.f.ell[bh * nc + c], 0.f));
+                if (live) {
+                    const size_t off = (bh * nc + c) * (size_t)NP + e;
+                    ds[k] = ws.gst[off];
+                    hin[k] = ws.f.states[off];
+                }
+            }
         }
-        const float tot = block_sum(gcur * hin, red);
-        if (threadIdx.x == 0) ws.ghp[(bh * nc + c) * gridDim.x + blockIdx.x] = tot;
-        gcur = fmaf(expf(fminf(ws.f.ell[bh * nc + c], 0.f)), gcur, ds);
+#pragma unroll
+        for (int k = 0; k < kDpBatch; ++k) {
+            const int c = c1 - k;
+            if (c < 0) break;                       // uniform over the block
+            if (live) ws.gst[(bh * nc + c) * (size_t)NP + e] = gcur;   // gradient of the state after chunk c
+            float v = gcur * hin[k];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) ws.ghp[(bh * nc + c) * (size_t)nparts + blockIdx.x * (kThreads / 32) + warp] = v;
+            gcur = fmaf(dec[k], gcur, ds[k]);
+        }
     }
     if (live && dinit) dinit[bh * NP + e] = gcur;
 }
@@ -651,8 +672,11 @@ finalize_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_b
     float e_part = 0.f;
     for (int i = threadIdx.x; i < q; i += kThreads) e_part += ws.E[bh * L + t0 + i];
     const float etot = block_sum(e_part, red);
-    float gh = 0.f;
-    for (int k = 0; k < nblk; ++k) gh += ws.ghp[(bh * nc + c) * nblk + k];
+    // the reverse pass's per-warp partials of <G_c, H_in>, in a fixed order
+    const int nparts = nblk * (kThreads / 32);
+    float g_part = 0.f;
+    for (int k = threadIdx.x; k < nparts; k += kThreads) g_part += ws.ghp[(bh * nc + c) * (size_t)nparts + k];
+    const float gh = block_sum(g_part, red);
     const float extra = etot + expf(fminf(ws.f.ell[bh * nc + c], 0.f)) * gh;
 
     float carry = 0.f, pa = 0.f, pb = 0.f, pd = 0.f;
