@@ -740,21 +740,36 @@ heads_kernel(BwdWs ws, float *__restrict__ dA, float *__restrict__ ddt_bias, flo
 
 // ---- 7. dB, dC: the heads of each group in head order -----------------------
 __global__ void __launch_bounds__(kThreads)
-groups_kernel(const float *__restrict__ dBh, const float *__restrict__ dCh, float *__restrict__ dB,
+groups_kernel(const float *__restrict__ dBh, const float *__restrict__ dC_h, float *__restrict__ dB,
               float *__restrict__ dC, int64_t total, int H, int G, int N) {
+    // 4 consecutive state elements per thread (N % 8 == 0); the heads of the
+    // group are added in head order, the loads of 8 heads issued together
     const int hpg = H / G;
-    for (int64_t e = blockIdx.x * (int64_t)kThreads + threadIdx.x; e < total;
-         e += (int64_t)gridDim.x * kThreads) {
+    const int64_t total4 = total / 4;
+    for (int64_t e4 = blockIdx.x * (int64_t)kThreads + threadIdx.x; e4 < total4;
+         e4 += (int64_t)gridDim.x * kThreads) {
+        const int64_t e = 4 * e4;
         const int64_t n = e % N, r = e / N;          // r = (b*L + t)*G + g
         const int64_t g = r % G, tok = r / G;
         const size_t src = ((size_t)tok * H + g * hpg) * N + n;
-        float sb = 0.f, sc = 0.f;
-        for (int k = 0; k < hpg; ++k) {
-            sb += dBh[src + (size_t)k * N];
-            sc += dCh[src + (size_t)k * N];
+        float4 sb = make_float4(0.f, 0.f, 0.f, 0.f), sc = sb;
+        for (int k0 = 0; k0 < hpg; k0 += 8) {
+            float4 vb[8], vc[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k0 + k < hpg) {
+                    vb[k] = *reinterpret_cast<const float4 *>(dBh + src + (size_t)(k0 + k) * N);
+                    vc[k] = *reinterpret_cast<const float4 *>(dC_h + src + (size_t)(k0 + k) * N);
+                }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k0 + k < hpg) {
+                    sb.x += vb[k].x; sb.y += vb[k].y; sb.z += vb[k].z; sb.w += vb[k].w;
+                    sc.x += vc[k].x; sc.y += vc[k].y; sc.z += vc[k].z; sc.w += vc[k].w;
+                }
         }
-        dB[e] = sb;
-        dC[e] = sc;
+        *reinterpret_cast<float4 *>(dB + e) = sb;
+        *reinterpret_cast<float4 *>(dC + e) = sc;
     }
 }
 
@@ -843,7 +858,7 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (ws.dBh) {
             const int64_t total = d.b * d.L * d.G * d.N;
-            const int64_t blocks = (total + kThreads - 1) / kThreads;
+            const int64_t blocks = (total / 4 + kThreads - 1) / kThreads;
             groups_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), kThreads, 0, s>>>(
                 ws.dBh, ws.dCh, a.dB, a.dC, total, H, G, N);
         }
