@@ -7,7 +7,8 @@
 // form of the forward, "Mamba2" knowledge page); every product of two
 // 128-token blocks is an MMA:
 //
-// cols, per (j block J of a chunk, head, batch), TMEM lane = token j:
+// cols, per (j block J of a chunk, head, batch), TMEM lane = token j (16 warps:
+// lane quarter w % 4, column quarter w / 4):
 //   dX_J  = e^{cl-cum_j} B_J G_c             (M=128 j, N=64 p,  K=128 n)
 //   dB_J  = e^{cl-cum_j} X_J G_c^T           (M=128 j, N=128 n, K=64 p)
 //           (before the scaling, a row dot with B_J gives E_j)
@@ -46,7 +47,8 @@ constexpr int kB = 128;                    // tokens per block (MMA M)
 constexpr int kNs = 128;                   // state_dim
 constexpr int kPh = 64;                    // head_dim
 constexpr uint32_t kT = 16384;             // one [128 rows x 64 fp16] swizzled tile
-constexpr int kThr = 256;                  // 8 warps: lane quarter w % 4, column half w / 4
+constexpr int kThr = 256;                  // tc_states: 8 warps, lane quarter w % 4, column half w / 4
+constexpr int kThrP = 512;                 // pair kernels: 16 warps, lane quarter w % 4, column quarter w / 4
 constexpr long long kBudget = 1ll << 32;   // clock cycles before an MMA wait gives up (~2 s)
 constexpr float kF16Max = 65504.0f;
 
@@ -79,24 +81,24 @@ template <> struct Raw8<float> {
 // Rows 0..127 of a [128 x W] fp16 tile (W = 64 or 128: one or two swizzled
 // 64-wide tiles) from `nrows` source rows of `ld` elements (bf16 or fp32),
 // each row times scale[r] when `scale` is given; rows past nrows are zero.
-// All 256 threads; one 16-byte chunk (8 values) per step, consecutive
+// All NT threads; one 16-byte chunk (8 values) per step, consecutive
 // threads on consecutive chunks of a row, every load issued before the
 // first conversion.
-template <int W, typename S>
+template <int W, int NT, typename S>
 __device__ __forceinline__ void fill_tile(uint8_t *tile, const S *src, size_t ld, int nrows, int tid, __half2 &amax,
                                           const float *scale = nullptr) {
     constexpr int cpr = W / 8;             // chunks per row
-    constexpr int kIt = kB * cpr / kThr;   // chunks per thread
+    constexpr int kIt = kB * cpr / NT;     // chunks per thread
     Raw8<S> raw[kIt];
 #pragma unroll
     for (int it = 0; it < kIt; ++it) {
-        const int c = tid + it * kThr, r = c / cpr, k = c - r * cpr;
+        const int c = tid + it * NT, r = c / cpr, k = c - r * cpr;
         if (r < nrows) raw[it].load(src + (size_t)r * ld + 8 * k);
         else raw[it].zero();
     }
 #pragma unroll
     for (int it = 0; it < kIt; ++it) {
-        const int c = tid + it * kThr, r = c / cpr, k = c - r * cpr;
+        const int c = tid + it * NT, r = c / cpr, k = c - r * cpr;
         float f[8];
         raw[it].get(f);
         if (scale) {
@@ -162,20 +164,20 @@ __device__ __forceinline__ void finish_range(unsigned *status, __half2 amax) {
 // shared memory (offsets from a 1024-aligned base)
 constexpr uint32_t kCBj = 0, kCXj = 2 * kT, kCG = 3 * kT, kCCi = 4 * kT, kCDYi = 6 * kT, kCU = 7 * kT,
                    kCV = 9 * kT, kCScal = 11 * kT;
-// scalars: cum_j, dt_j, dec_j, cum_i, e1[2], zs[2], zo[2], dyx[2] (128 floats each)
-constexpr uint32_t kCBar = kCScal + 13 * kB * 4;
+// scalars: cum_j, dt_j, dec_j, cum_i, then per column quarter e1[4], zs[4], zo[4], dyx[4] (128 floats each)
+constexpr uint32_t kCBar = kCScal + 20 * kB * 4;
 constexpr size_t kColsSmem = 1024 + kCBar + 16;
 // TMEM columns (each accumulator starts on a multiple of its width, as in
 // the forward kernels)
 constexpr uint32_t kTmCBt = 0, kTmSt = 128, kTmDB = 256, kTmDX = 384;
 
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThrP, 1)
 tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *s_cumj = reinterpret_cast<float *>(sm + kCScal);
     float *s_dtj = s_cumj + kB, *s_dec = s_dtj + kB, *s_cumi = s_dec + kB;
-    float *s_e1 = s_cumi + kB, *s_zs = s_e1 + 2 * kB, *s_zo = s_zs + 2 * kB, *s_dyx = s_zo + 2 * kB;
+    float *s_e1 = s_cumi + kB, *s_zs = s_e1 + 4 * kB, *s_zo = s_zs + 4 * kB, *s_dyx = s_zo + 4 * kB;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kCBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
 
@@ -202,11 +204,11 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     }
     // j block: B_J, X_J (fp16), G_c (fp16 [n][p]); per-token scalars
     const size_t tokj = (size_t)b * L + t0 + j0;
-    fill_tile<128>(sm + kCBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs,
+    fill_tile<128, kThrP>(sm + kCBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs,
                    (size_t)G * kNs, tj, tid, amax);
-    fill_tile<64>(sm + kCXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh,
+    fill_tile<64, kThrP>(sm + kCXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh,
                   (size_t)H * kPh, tj, tid, amax);
-    fill_tile<64>(sm + kCG, a.gst + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, tid, amax);
+    fill_tile<64, kThrP>(sm + kCG, a.gst + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, tid, amax);
     const float cl = a.cum[bh * L + t0 + q - 1];
     if (tid < kB) {
         const bool v = tid < tj;
@@ -215,14 +217,14 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         s_dtj[tid] = v ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
         s_dec[tid] = v ? expf(fminf(cl - cj, 0.f)) : 0.f;
     }
-    // dy_j . x_j exactly in fp32 (thread: token row, half ch of p)
+    // dy_j . x_j exactly in fp32 (thread: token row, quarter ch of p)
     {
         float d = 0.f;
         if (row < tj) {
-            const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(a.x) + ((tokj + row) * H + h) * kPh + 32 * ch;
-            const float *dr = a.dy + ((tokj + row) * H + h) * kPh + 32 * ch;
+            const __nv_bfloat16 *xr = static_cast<const __nv_bfloat16 *>(a.x) + ((tokj + row) * H + h) * kPh + 16 * ch;
+            const float *dr = a.dy + ((tokj + row) * H + h) * kPh + 16 * ch;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 2; ++k) {
                 const uint4 xv = *reinterpret_cast<const uint4 *>(xr + 8 * k);
                 const float4 d0 = *reinterpret_cast<const float4 *>(dr + 8 * k);
                 const float4 d1 = *reinterpret_cast<const float4 *>(dr + 8 * k + 4);
@@ -262,9 +264,9 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     auto fill_i = [&](int Ib) {
         const int i0 = Ib * kB, ti = min(kB, q - i0);
         const size_t toki = (size_t)b * L + t0 + i0;
-        fill_tile<128>(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs,
+        fill_tile<128, kThrP>(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs,
                        (size_t)G * kNs, ti, tid, amax);
-        fill_tile<64>(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, tid, amax);
+        fill_tile<64, kThrP>(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, tid, amax);
         if (tid < kB) s_cumi[tid] = tid < ti ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
     };
     fill_i(Jb);
@@ -272,24 +274,21 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
         // E_j's dot (B_J row j with the unscaled dB row), then both accumulators times dec_j
+        // (this thread: dB columns [32ch, 32ch+32), dX columns [16ch, 16ch+16))
         const float dec = s_dec[row];
-        float e1 = 0.f;
-        for (int hh = 0; hh < 2; ++hh) {
-            float t32[32];
-            tmem_ld32(lane_addr + kTmDB + 64 * ch + 32 * hh, t32);
-            e1 += row_dot32(sm + kCBj, row, ch, 4 * hh, t32);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) t32[k] *= dec;
-            tmem_st32(lane_addr + kTmDB + 64 * ch + 32 * hh, t32);
-        }
-        s_e1[ch * kB + row] = e1;
         float t32[32];
-        tmem_ld32(lane_addr + kTmDX + 32 * ch, t32);
+        tmem_ld32(lane_addr + kTmDB + 32 * ch, t32);
+        s_e1[ch * kB + row] = row_dot32(sm + kCBj, row, ch >> 1, 4 * (ch & 1), t32);
 #pragma unroll
         for (int k = 0; k < 32; ++k) t32[k] *= dec;
-        tmem_st32(lane_addr + kTmDX + 32 * ch, t32);
+        tmem_st32(lane_addr + kTmDB + 32 * ch, t32);
+        float t16[16];
+        tmem_ld16(lane_addr + kTmDX + 16 * ch, t16);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) t16[k] *= dec;
+        tmem_st16(lane_addr + kTmDX + 16 * ch, t16);
     }
-    float zs = 0.f, zo = 0.f;                          // this thread's i half
+    float zs = 0.f, zo = 0.f;                          // this thread's i quarter
     for (int Ib = Jb; Ib < nIb; ++Ib) {
         const int i0 = Ib * kB, ti = min(kB, q - i0);
         // the previous pair's MMAs (which read C_I, DY_I, U, V) are complete
@@ -316,9 +315,8 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         if (ok) {
             const float cj = s_cumj[row];
             const int gj = j0 + row;
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                const int ib = 64 * ch + 32 * hh;      // first i of this group of 32
+            {
+                const int ib = 32 * ch;                // first i of this thread's quarter
                 float cb[32], sv[32];
                 tmem_ld32(lane_addr + kTmCBt + ib, cb);
                 tmem_ld32(lane_addr + kTmSt + ib, sv);
@@ -334,8 +332,8 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
                     cb[k] = u;
                     sv[k] = w;
                 }
-                store_row32(sm + kCU + ch * kT, row, 4 * hh, cb, amax);
-                store_row32(sm + kCV + ch * kT, row, 4 * hh, sv, amax);
+                store_row32(sm + kCU + (ch >> 1) * kT, row, 4 * (ch & 1), cb, amax);
+                store_row32(sm + kCV + (ch >> 1) * kT, row, 4 * (ch & 1), sv, amax);
             }
         }
         fence_proxy_async_smem();
@@ -373,39 +371,40 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         const float dtj = s_dtj[row];
         const size_t tok = tokj + row;
         const float Dh = a.D[h];
-        float t32[32];
-        tmem_ld32(lane_addr + kTmDX + 32 * ch, t32);
-        float *dxr = a.dx + (tok * H + h) * kPh + 32 * ch;
-        const float *dyr = a.dy + (tok * H + h) * kPh + 32 * ch;
+        // this thread: dx columns [16ch, 16ch+16), dB columns [32ch, 32ch+32)
+        float t16[16];
+        tmem_ld16(lane_addr + kTmDX + 16 * ch, t16);
+        float *dxr = a.dx + (tok * H + h) * kPh + 16 * ch;
+        const float *dyr = a.dy + (tok * H + h) * kPh + 16 * ch;
         if (mine) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 4; ++k) {
                 const float4 d4 = *reinterpret_cast<const float4 *>(dyr + 4 * k);
                 *reinterpret_cast<float4 *>(dxr + 4 * k) =
-                    make_float4(fmaf(dtj, t32[4 * k], Dh * d4.x), fmaf(dtj, t32[4 * k + 1], Dh * d4.y),
-                                fmaf(dtj, t32[4 * k + 2], Dh * d4.z), fmaf(dtj, t32[4 * k + 3], Dh * d4.w));
+                    make_float4(fmaf(dtj, t16[4 * k], Dh * d4.x), fmaf(dtj, t16[4 * k + 1], Dh * d4.y),
+                                fmaf(dtj, t16[4 * k + 2], Dh * d4.z), fmaf(dtj, t16[4 * k + 3], Dh * d4.w));
             }
         }
-        float *dbr = a.dBh + (tok * H + h) * kNs + 64 * ch;
+        float t32[32];
+        tmem_ld32(lane_addr + kTmDB + 32 * ch, t32);
+        float *dbr = a.dBh + (tok * H + h) * kNs + 32 * ch;
+        if (mine) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            tmem_ld32(lane_addr + kTmDB + 64 * ch + 32 * hh, t32);
-            if (mine) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<float4 *>(dbr + 32 * hh + 4 * k) = make_float4(
-                        dtj * t32[4 * k], dtj * t32[4 * k + 1], dtj * t32[4 * k + 2], dtj * t32[4 * k + 3]);
-            }
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4 *>(dbr + 4 * k) =
+                    make_float4(dtj * t32[4 * k], dtj * t32[4 * k + 1], dtj * t32[4 * k + 2], dtj * t32[4 * k + 3]);
         }
         if (mine && ch == 0) {
+            // the four column quarters' partials, in quarter order
+            auto sum4 = [&](const float *v) { return ((v[row] + v[kB + row]) + v[2 * kB + row]) + v[3 * kB + row]; };
             const float dec = s_dec[row];
-            const float e1 = s_e1[row] + s_e1[kB + row];
+            const float e1 = sum4(s_e1);
             const float sdst = dec * e1, E = dtj * sdst;
             const size_t o = bh * L + t0 + j0 + row;
-            a.ddt_dir[o] = sdst + (s_zs[row] + s_zs[kB + row]);
-            a.dcum_col[o] = -(dtj * (s_zo[row] + s_zo[kB + row])) - E;
+            a.ddt_dir[o] = sdst + sum4(s_zs);
+            a.dcum_col[o] = -(dtj * sum4(s_zo)) - E;
             a.E[o] = E;
-            a.dyx[o] = s_dyx[row] + s_dyx[kB + row];
+            a.dyx[o] = sum4(s_dyx);
         }
     }
     if (__any_sync(0xffffffffu, !ok) && lane == 0) flag_status(a.status, kStatusTimeout);
@@ -424,18 +423,18 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
 // ---- rows -----------------------------------------------------------------
 constexpr uint32_t kRCi = 0, kRDYi = 2 * kT, kRH = 3 * kT, kRBj = 4 * kT, kRXj = 6 * kT, kRV = 7 * kT,
                    kRScal = 9 * kT;
-// scalars: cum_i, dec_i, cum_j, dt_j, tv[2], rs[2] (128 floats each)
-constexpr uint32_t kRBar = kRScal + 8 * kB * 4;
+// scalars: cum_i, dec_i, cum_j, dt_j, then per column quarter tv[4], rs[4] (128 floats each)
+constexpr uint32_t kRBar = kRScal + 12 * kB * 4;
 constexpr size_t kRowsSmem = 1024 + kRBar + 16;
 constexpr uint32_t kTmCB = 0, kTmS = 128, kTmDC = 256;
 
-__global__ void __launch_bounds__(kThr, 1)
+__global__ void __launch_bounds__(kThrP, 1)
 tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *s_cumi = reinterpret_cast<float *>(sm + kRScal);
     float *s_dec = s_cumi + kB, *s_cumj = s_dec + kB, *s_dtj = s_cumj + kB;
-    float *s_tv = s_dtj + kB, *s_rs = s_tv + 2 * kB;
+    float *s_tv = s_dtj + kB, *s_rs = s_tv + 4 * kB;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kRBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
 
@@ -461,10 +460,10 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         fence_mbar_init();
     }
     const size_t toki = (size_t)b * L + t0 + i0;
-    fill_tile<128>(sm + kRCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs,
+    fill_tile<128, kThrP>(sm + kRCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs,
                    (size_t)G * kNs, ti, tid, amax);
-    fill_tile<64>(sm + kRDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, tid, amax);
-    fill_tile<64>(sm + kRH, a.states + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, tid, amax);
+    fill_tile<64, kThrP>(sm + kRDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, tid, amax);
+    fill_tile<64, kThrP>(sm + kRH, a.states + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, tid, amax);
     if (tid < kB) {
         const bool v = tid < ti;
         const float ci = v ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
@@ -494,9 +493,9 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     auto fill_j = [&](int Jb) {
         const int j0 = Jb * kB, tj = min(kB, q - j0);
         const size_t tokj = (size_t)b * L + t0 + j0;
-        fill_tile<128>(sm + kRBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs,
+        fill_tile<128, kThrP>(sm + kRBj, static_cast<const __nv_bfloat16 *>(a.B) + (tokj * G + g) * kNs,
                        (size_t)G * kNs, tj, tid, amax);
-        fill_tile<64>(sm + kRXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh,
+        fill_tile<64, kThrP>(sm + kRXj, static_cast<const __nv_bfloat16 *>(a.x) + (tokj * H + h) * kPh,
                       (size_t)H * kPh, tj, tid, amax);
         if (tid < kB) {
             s_cumj[tid] = tid < tj ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
@@ -508,19 +507,16 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
         // T_i's dot (C_I row i with the unscaled dC row), then the accumulator times dec_i
+        // (this thread: dC columns [32ch, 32ch+32))
         const float dec = s_dec[row];
-        float tv = 0.f;
-        for (int hh = 0; hh < 2; ++hh) {
-            float t32[32];
-            tmem_ld32(lane_addr + kTmDC + 64 * ch + 32 * hh, t32);
-            tv += row_dot32(sm + kRCi, row, ch, 4 * hh, t32);
+        float t32[32];
+        tmem_ld32(lane_addr + kTmDC + 32 * ch, t32);
+        s_tv[ch * kB + row] = row_dot32(sm + kRCi, row, ch >> 1, 4 * (ch & 1), t32);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) t32[k] *= dec;
-            tmem_st32(lane_addr + kTmDC + 64 * ch + 32 * hh, t32);
-        }
-        s_tv[ch * kB + row] = tv;
+        for (int k = 0; k < 32; ++k) t32[k] *= dec;
+        tmem_st32(lane_addr + kTmDC + 32 * ch, t32);
     }
-    float rs = 0.f;                                    // sum over this thread's j half of CB_ij V_ij, j < i
+    float rs = 0.f;                                    // sum over this thread's j quarter of CB_ij V_ij, j < i
     const float ci = s_cumi[row];
     const int gi = i0 + row;
     for (int Jb = 0; Jb <= Ib; ++Jb) {
@@ -547,9 +543,8 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         ok = ok && wait_mma(bar, ph);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                const int jb = 64 * ch + 32 * hh;
+            {
+                const int jb = 32 * ch;
                 float cb[32], sv[32];
                 tmem_ld32(lane_addr + kTmCB + jb, cb);
                 tmem_ld32(lane_addr + kTmS + jb, sv);
@@ -561,7 +556,7 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
                     rs += gi > gj ? cb[k] * w : 0.f;
                     sv[k] = w;
                 }
-                store_row32(sm + kRV + ch * kT, row, 4 * hh, sv, amax);
+                store_row32(sm + kRV + (ch >> 1) * kT, row, 4 * (ch & 1), sv, amax);
             }
         }
         fence_proxy_async_smem();
@@ -592,21 +587,20 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     if (ok) {
         const bool mine = row < ti;
         const size_t tok = toki + row;
-        float *dcr = a.dCh + (tok * H + h) * kNs + 64 * ch;
+        float *dcr = a.dCh + (tok * H + h) * kNs + 32 * ch;
+        float t32[32];
+        tmem_ld32(lane_addr + kTmDC + 32 * ch, t32);
+        if (mine) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float t32[32];
-            tmem_ld32(lane_addr + kTmDC + 64 * ch + 32 * hh, t32);
-            if (mine) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<float4 *>(dcr + 32 * hh + 4 * k) =
-                        make_float4(t32[4 * k], t32[4 * k + 1], t32[4 * k + 2], t32[4 * k + 3]);
-            }
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4 *>(dcr + 4 * k) =
+                    make_float4(t32[4 * k], t32[4 * k + 1], t32[4 * k + 2], t32[4 * k + 3]);
         }
         if (mine && ch == 0) {
-            const float tv = s_dec[row] * (s_tv[row] + s_tv[kB + row]);
-            a.dcum_row[bh * L + t0 + i0 + row] = tv + (s_rs[row] + s_rs[kB + row]);
+            // the four column quarters' partials, in quarter order
+            auto sum4 = [&](const float *v) { return ((v[row] + v[kB + row]) + v[2 * kB + row]) + v[3 * kB + row]; };
+            const float tv = s_dec[row] * sum4(s_tv);
+            a.dcum_row[bh * L + t0 + i0 + row] = tv + sum4(s_rs);
         }
     }
     if (__any_sync(0xffffffffu, !ok) && lane == 0) flag_status(a.status, kStatusTimeout);
@@ -697,13 +691,14 @@ tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
             s_e[tid] = v ? expf(fminf(s_cum[j0 + tid], 0.f)) : 0.f;
         }
         __syncthreads();                               // the previous block's MMAs are complete
-        fill_tile<128>(sm + kSB, static_cast<const __nv_bfloat16 *>(a.B) + (tok * G + g) * kNs,
+        fill_tile<128, kThr>(sm + kSB, static_cast<const __nv_bfloat16 *>(a.B) + (tok * G + g) * kNs,
                        (size_t)G * kNs, nr, tid, amax);
-        fill_tile<128>(sm + kSC, static_cast<const __nv_bfloat16 *>(a.C) + (tok * G + g) * kNs,
+        fill_tile<128, kThr>(sm + kSC, static_cast<const __nv_bfloat16 *>(a.C) + (tok * G + g) * kNs,
                        (size_t)G * kNs, nr, tid, amax);
-        fill_tile<64>(sm + kSWX, static_cast<const __nv_bfloat16 *>(a.x) + (tok * H + h) * kPh, (size_t)H * kPh, nr,
+        fill_tile<64, kThr>(sm + kSWX, static_cast<const __nv_bfloat16 *>(a.x) + (tok * H + h) * kPh,
+                            (size_t)H * kPh, nr,
                       tid, amax, s_w);
-        fill_tile<64>(sm + kSEDY, a.dy + (tok * H + h) * kPh, (size_t)H * kPh, nr, tid, amax, s_e);
+        fill_tile<64, kThr>(sm + kSEDY, a.dy + (tok * H + h) * kPh, (size_t)H * kPh, nr, tid, amax, s_e);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -795,12 +790,12 @@ cudaError_t bwd_tc_pairs(const BwdPairArgs &a, const ScanDims &d, cudaStream_t s
     const dim3 grid((unsigned)(d.nc * (d.Q / kB)), (unsigned)d.H, (unsigned)d.b);
     {
         TraceScope tr(s, kTrBwdCols);
-        tc_cols_kernel<<<grid, kThr, kColsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+        tc_cols_kernel<<<grid, kThrP, kColsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
         TraceScope tr(s, kTrBwdRows);
-        tc_rows_kernel<<<grid, kThr, kRowsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+        tc_rows_kernel<<<grid, kThrP, kRowsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
     }
     return cudaGetLastError();
 }
