@@ -324,8 +324,8 @@ SSD_API ssd_status ssd_chunk_scan_bwd(const void *x, const float *dt_raw, const 
  *                    the accumulations into dx, dB, dC) on the tcgen05
  *                    tensor cores with fp16 operands and fp32 accumulation:
  *                    bf16 inputs, head_dim 64, state_dim 128, chunk_size a
- *                    multiple of 128 up to 1024, no packed rows (else
- *                    SSD_ERR_UNSUPPORTED).  The gradients carry the forward
+ *                    multiple of 128 up to 1024 (else SSD_ERR_UNSUPPORTED);
+ *                    packed rows included.  The gradients carry the forward
  *                    tensor path's precision (about 1e-3 of their RMS), and
  *                    a value outside fp16's range shows as
  *                    SSD_ERR_PRECONDITION in the status word;

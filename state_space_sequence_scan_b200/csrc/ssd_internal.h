@@ -79,8 +79,7 @@ bool bwd_supported(const ScanDims &d);
 // The tensor-core pair kernels of the backward (ssd_scan_bwd_tc.cu): the
 // same outputs as the CUDA-core `cols` and `rows` kernels, from the same
 // workspace (the forward recompute's dt, cum and entering states, the
-// reverse pass's G_c).  bf16 inputs, P 64, N 128, Q a multiple of 128, no
-// packed rows.
+// reverse pass's G_c).  bf16 inputs, P 64, N 128, Q a multiple of 128.
 struct BwdPairArgs {
     const void *x, *B, *C;         // bf16 inputs
     const float *D, *dy;
@@ -90,6 +89,8 @@ struct BwdPairArgs {
     float *dx;                     // [b, L, H, P]
     float *dBh, *dCh;              // [b, L, H, N] per head
     unsigned *status;
+    const float *docc = nullptr;   // [b, L] packed rows: document starts from the chunk's first token
+                                   // through each token (null: one document per row)
 };
 bool bwd_tc_supported(const ScanDims &d, int bf16, int packed);
 cudaError_t bwd_tc_pairs(const BwdPairArgs &a, const ScanDims &d, cudaStream_t s);
@@ -105,6 +106,7 @@ struct BwdStatesArgs {
     float *dtv, *cum, *ell;         // [b, H, L], [b, H, L], [b, H, nc]
     float *states, *gst;            // [b, H, nc, N, P]
     unsigned *status;
+    const float *docc = nullptr;    // as in BwdPairArgs
 };
 cudaError_t bwd_tc_states(const BwdStatesArgs &a, const ScanDims &d, cudaStream_t s);
 size_t bwd_workspace_bytes(const ScanDims &d);

@@ -795,10 +795,15 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
     if (a.tensor) {
         // the chunk states and the per-chunk dy sums on the tensor cores
         // (ssd_scan_bwd_tc.cu), then the forward's state pass
+        if (packed) {
+            docs_kernel<<<dim3((unsigned)nc, (unsigned)d.b), kThreads, 0, s>>>(a.f.seq_idx, ws.docc, L, Q);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
         BwdStatesArgs sa;
         sa.x = a.f.x; sa.B = a.f.B; sa.C = a.f.C; sa.dt_raw = a.f.dt_raw; sa.dt_bias = a.f.dt_bias; sa.A = a.f.A;
         sa.dy = a.dy; sa.dt_lo = a.f.dt_lo; sa.dt_hi = a.f.dt_hi; sa.dtv = ws.f.dtv; sa.cum = ws.f.cum;
         sa.ell = ws.f.ell; sa.states = ws.f.states; sa.gst = ws.gst; sa.status = ws.f.status;
+        sa.docc = packed ? ws.docc : nullptr;
         if ((e = bwd_tc_states(sa, d, s)) != cudaSuccess) return e;
         if ((e = simt_state_pass(a.f, d, wsp, s)) != cudaSuccess) return e;
     } else {
@@ -831,6 +836,7 @@ cudaError_t run(const BwdArgs &a, const ScanDims &d, void *wsp, cudaStream_t s) 
         pa.dtv = ws.f.dtv; pa.cum = ws.f.cum; pa.gst = ws.gst; pa.states = ws.f.states;
         pa.ddt_dir = ws.ddt_dir; pa.dcum_col = ws.dcum_col; pa.dcum_row = ws.dcum_row; pa.E = ws.E;
         pa.dyx = ws.dyx; pa.dx = a.dx; pa.dBh = dBh; pa.dCh = dCh; pa.status = ws.f.status;
+        pa.docc = packed ? ws.docc : nullptr;
         if ((e = bwd_tc_pairs(pa, d, s)) != cudaSuccess) return e;
     } else {
     {

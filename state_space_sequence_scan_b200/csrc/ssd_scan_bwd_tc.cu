@@ -3,7 +3,8 @@
 // `rows` kernels of ssd_scan_bwd.cu (same inputs, same outputs in the same
 // workspace regions; the launches around them are unchanged), for bf16
 // inputs with head_dim 64, state_dim 128 and a chunk size that is a multiple
-// of 128.  The formulas are those of ssd_scan_bwd.cu's header (the chunked
+// of 128, packed rows included (the fp32 kernels' document masks, applied to
+// values).  The formulas are those of ssd_scan_bwd.cu's header (the chunked
 // form of the forward, "Mamba2" knowledge page); every product of two
 // 128-token blocks is an MMA:
 //
@@ -164,13 +165,15 @@ __device__ __forceinline__ void finish_range(unsigned *status, __half2 amax) {
 // shared memory (offsets from a 1024-aligned base)
 constexpr uint32_t kCBj = 0, kCXj = 2 * kT, kCG = 3 * kT, kCCi = 4 * kT, kCDYi = 6 * kT, kCU = 7 * kT,
                    kCV = 9 * kT, kCScal = 11 * kT;
-// scalars: cum_j, dt_j, dec_j, cum_i, then per column quarter e1[4], zs[4], zo[4], dyx[4] (128 floats each)
-constexpr uint32_t kCBar = kCScal + 20 * kB * 4;
+// scalars: cum_j, dt_j, dec_j, cum_i, then per column quarter e1[4], zs[4], zo[4], dyx[4], then the
+// document counters doc_j, doc_i of packed rows (128 floats each)
+constexpr uint32_t kCBar = kCScal + 22 * kB * 4;
 constexpr size_t kColsSmem = 1024 + kCBar + 16;
 // TMEM columns (each accumulator starts on a multiple of its width, as in
 // the forward kernels)
 constexpr uint32_t kTmCBt = 0, kTmSt = 128, kTmDB = 256, kTmDX = 384;
 
+template <bool kPacked>
 __global__ void __launch_bounds__(kThrP, 1)
 tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     extern __shared__ uint8_t smem_raw[];
@@ -178,6 +181,7 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     float *s_cumj = reinterpret_cast<float *>(sm + kCScal);
     float *s_dtj = s_cumj + kB, *s_dec = s_dtj + kB, *s_cumi = s_dec + kB;
     float *s_e1 = s_cumi + kB, *s_zs = s_e1 + 4 * kB, *s_zo = s_zs + 4 * kB, *s_dyx = s_zo + 4 * kB;
+    float *s_docj = s_dyx + 4 * kB, *s_doci = s_docj + kB;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kCBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
 
@@ -210,12 +214,17 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
                   (size_t)H * kPh, tj, tid, amax);
     fill_tile<64, kThrP>(sm + kCG, a.gst + (bh * nc + c) * (size_t)(kNs * kPh), (size_t)kPh, kNs, tid, amax);
     const float cl = a.cum[bh * L + t0 + q - 1];
+    // packed rows: dl counts the chunk's document starts; only the last
+    // document's tokens write into the state the chunk passes on
+    const float dl = kPacked ? a.docc[(size_t)b * L + t0 + q - 1] : 0.f;
     if (tid < kB) {
         const bool v = tid < tj;
         const float cj = v ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
+        const float dj = (kPacked && v) ? a.docc[(size_t)b * L + t0 + j0 + tid] : 0.f;
         s_cumj[tid] = cj;
         s_dtj[tid] = v ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
-        s_dec[tid] = v ? expf(fminf(cl - cj, 0.f)) : 0.f;
+        s_dec[tid] = (v && dj == dl) ? expf(fminf(cl - cj, 0.f)) : 0.f;
+        s_docj[tid] = dj;
     }
     // dy_j . x_j exactly in fp32 (thread: token row, quarter ch of p)
     {
@@ -267,7 +276,10 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         fill_tile<128, kThrP>(sm + kCCi, static_cast<const __nv_bfloat16 *>(a.C) + (toki * G + g) * kNs,
                        (size_t)G * kNs, ti, tid, amax);
         fill_tile<64, kThrP>(sm + kCDYi, a.dy + (toki * H + h) * kPh, (size_t)H * kPh, ti, tid, amax);
-        if (tid < kB) s_cumi[tid] = tid < ti ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
+        if (tid < kB) {
+            s_cumi[tid] = tid < ti ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
+            s_doci[tid] = (kPacked && tid < ti) ? a.docc[(size_t)b * L + t0 + i0 + tid] : 0.f;
+        }
     };
     fill_i(Jb);
     ok = wait_mma(bar, ph);
@@ -323,7 +335,7 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
                     const int il = ib + k, gi = i0 + il;
-                    const bool v = il < ti && row < tj && gi >= gj;
+                    const bool v = il < ti && row < tj && gi >= gj && (!kPacked || s_doci[il] == s_docj[row]);
                     const float lw = v ? expf(fminf(s_cumi[il] - cj, 0.f)) : 0.f;
                     const float u = cb[k] * lw, w = sv[k] * lw;
                     const float z = u * sv[k];
@@ -423,11 +435,13 @@ tc_cols_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
 // ---- rows -----------------------------------------------------------------
 constexpr uint32_t kRCi = 0, kRDYi = 2 * kT, kRH = 3 * kT, kRBj = 4 * kT, kRXj = 6 * kT, kRV = 7 * kT,
                    kRScal = 9 * kT;
-// scalars: cum_i, dec_i, cum_j, dt_j, then per column quarter tv[4], rs[4] (128 floats each)
-constexpr uint32_t kRBar = kRScal + 12 * kB * 4;
+// scalars: cum_i, dec_i, cum_j, dt_j, then per column quarter tv[4], rs[4], then the document
+// counters doc_i, doc_j of packed rows (128 floats each)
+constexpr uint32_t kRBar = kRScal + 14 * kB * 4;
 constexpr size_t kRowsSmem = 1024 + kRBar + 16;
 constexpr uint32_t kTmCB = 0, kTmS = 128, kTmDC = 256;
 
+template <bool kPacked>
 __global__ void __launch_bounds__(kThrP, 1)
 tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     extern __shared__ uint8_t smem_raw[];
@@ -435,6 +449,7 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     float *s_cumi = reinterpret_cast<float *>(sm + kRScal);
     float *s_dec = s_cumi + kB, *s_cumj = s_dec + kB, *s_dtj = s_cumj + kB;
     float *s_tv = s_dtj + kB, *s_rs = s_tv + 4 * kB;
+    float *s_doci = s_rs + 4 * kB, *s_docj = s_doci + kB;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kRBar);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
 
@@ -467,8 +482,11 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
     if (tid < kB) {
         const bool v = tid < ti;
         const float ci = v ? a.cum[bh * L + t0 + i0 + tid] : 0.f;
+        // packed rows: the entering state reaches only the chunk's first document
+        const float di = (kPacked && v) ? a.docc[(size_t)b * L + t0 + i0 + tid] : 0.f;
         s_cumi[tid] = ci;
-        s_dec[tid] = v ? expf(fminf(ci, 0.f)) : 0.f;
+        s_dec[tid] = (v && di == 0.f) ? expf(fminf(ci, 0.f)) : 0.f;
+        s_doci[tid] = di;
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -500,6 +518,7 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
         if (tid < kB) {
             s_cumj[tid] = tid < tj ? a.cum[bh * L + t0 + j0 + tid] : 0.f;
             s_dtj[tid] = tid < tj ? a.dtv[bh * L + t0 + j0 + tid] : 0.f;
+            s_docj[tid] = (kPacked && tid < tj) ? a.docc[(size_t)b * L + t0 + j0 + tid] : 0.f;
         }
     };
     fill_j(0);
@@ -551,7 +570,7 @@ tc_rows_kernel(BwdPairArgs a, int L, int H, int G, int Q, int nc) {
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
                     const int jl = jb + k, gj = j0 + jl;
-                    const bool v = jl < tj && row < ti && gi >= gj;
+                    const bool v = jl < tj && row < ti && gi >= gj && (!kPacked || s_doci[row] == s_docj[jl]);
                     const float w = v ? sv[k] * expf(fminf(ci - s_cumj[jl], 0.f)) * s_dtj[jl] : 0.f;
                     rs += gi > gj ? cb[k] * w : 0.f;
                     sv[k] = w;
@@ -629,6 +648,7 @@ constexpr uint32_t kSB = 0, kSWX = 2 * kT, kSC = 3 * kT, kSEDY = 5 * kT, kSScal 
 constexpr uint32_t kSBar = kSScal + (2 * kQMax + 2 * kB + 32) * 4;
 constexpr size_t kStatesSmem = 1024 + kSBar + 16;
 
+template <bool kPacked>
 __global__ void __launch_bounds__(kThr, 2)
 tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
     extern __shared__ uint8_t smem_raw[];
@@ -672,7 +692,9 @@ tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
     }
     __syncthreads();
     const float cl = s_cum[q - 1];
-    if (tid == 0) a.ell[bh * nc + c] = cl;
+    // packed rows: a chunk that holds a document start passes no decayed state on
+    const float dl = kPacked ? a.docc[(size_t)b * L + t0 + q - 1] : 0.f;
+    if (tid == 0) a.ell[bh * nc + c] = dl > 0.f ? -INFINITY : cl;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -687,8 +709,11 @@ tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
         const size_t tok = (size_t)b * L + t0 + j0;
         if (tid < kB) {
             const bool v = tid < nr;
-            s_w[tid] = v ? expf(fminf(cl - s_cum[j0 + tid], 0.f)) * s_dt[j0 + tid] : 0.f;
-            s_e[tid] = v ? expf(fminf(s_cum[j0 + tid], 0.f)) : 0.f;
+            // packed rows: only the last document writes the chunk state, only the
+            // first reads the entering state
+            const float dj = (kPacked && v) ? a.docc[(size_t)b * L + t0 + j0 + tid] : 0.f;
+            s_w[tid] = (v && dj == dl) ? expf(fminf(cl - s_cum[j0 + tid], 0.f)) * s_dt[j0 + tid] : 0.f;
+            s_e[tid] = (v && dj == 0.f) ? expf(fminf(s_cum[j0 + tid], 0.f)) : 0.f;
         }
         __syncthreads();                               // the previous block's MMAs are complete
         fill_tile<128, kThr>(sm + kSB, static_cast<const __nv_bfloat16 *>(a.B) + (tok * G + g) * kNs,
@@ -749,7 +774,8 @@ tc_states_kernel(BwdStatesArgs a, int L, int H, int G, int Q, int nc) {
 }  // namespace
 
 bool bwd_tc_supported(const ScanDims &d, int bf16, int packed) {
-    if (!bf16 || packed || d.P != kPh || d.N != kNs || d.Q % kB != 0 || d.Q > kQMax) return false;
+    (void)packed;                      // packed rows: value masks from the document counters
+    if (!bf16 || d.P != kPh || d.N != kNs || d.Q % kB != 0 || d.Q > kQMax) return false;
     if (d.H > 65535 || d.b > 65535 || d.nc * (d.Q / kB) > 0x7fffffffll) return false;
     return true;
 }
@@ -761,14 +787,19 @@ cudaError_t bwd_tc_states(const BwdStatesArgs &a, const ScanDims &d, cudaStream_
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        if ((e = cudaFuncSetAttribute(tc_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(tc_states_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kStatesSmem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(tc_states_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kStatesSmem)) != cudaSuccess)
             return e;
         attr_done[dev] = true;
     }
     TraceScope tr(s, kTrBwdStates);
-    tc_states_kernel<<<dim3((unsigned)d.nc, (unsigned)d.H, (unsigned)d.b), kThr, kStatesSmem, s>>>(
-        a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+    const dim3 grid((unsigned)d.nc, (unsigned)d.H, (unsigned)d.b);
+    if (a.docc)
+        tc_states_kernel<true><<<grid, kThr, kStatesSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+    else
+        tc_states_kernel<false><<<grid, kThr, kStatesSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
     return cudaGetLastError();
 }
 
@@ -779,23 +810,27 @@ cudaError_t bwd_tc_pairs(const BwdPairArgs &a, const ScanDims &d, cudaStream_t s
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        if ((e = cudaFuncSetAttribute(tc_cols_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColsSmem)) !=
-            cudaSuccess)
-            return e;
-        if ((e = cudaFuncSetAttribute(tc_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowsSmem)) !=
-            cudaSuccess)
-            return e;
+        for (auto k : {tc_cols_kernel<false>, tc_cols_kernel<true>})
+            if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kColsSmem)) !=
+                cudaSuccess)
+                return e;
+        for (auto k : {tc_rows_kernel<false>, tc_rows_kernel<true>})
+            if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowsSmem)) !=
+                cudaSuccess)
+                return e;
         attr_done[dev] = true;
     }
     const dim3 grid((unsigned)(d.nc * (d.Q / kB)), (unsigned)d.H, (unsigned)d.b);
     {
         TraceScope tr(s, kTrBwdCols);
-        tc_cols_kernel<<<grid, kThrP, kColsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+        auto k = a.docc ? tc_cols_kernel<true> : tc_cols_kernel<false>;
+        k<<<grid, kThrP, kColsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
         TraceScope tr(s, kTrBwdRows);
-        tc_rows_kernel<<<grid, kThrP, kRowsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
+        auto k = a.docc ? tc_rows_kernel<true> : tc_rows_kernel<false>;
+        k<<<grid, kThrP, kRowsSmem, s>>>(a, (int)d.L, (int)d.H, (int)d.G, (int)d.Q, (int)d.nc);
     }
     return cudaGetLastError();
 }

@@ -298,3 +298,47 @@ def test_backward_tensor_path_rejects_what_it_does_not_take():
         inp, grads = make_scan_inputs(cfg), make_grad_inputs(cfg)
         with pytest.raises(ssd.SSDError, match="SSD_ERR_UNSUPPORTED"):
             run_bwd_tc(inp, grads, Q)
+
+
+TC_PACKED_CASES = [
+    # b, L, H, G, Q, mean document length
+    (2, 300, 4, 2, 256, 40),
+    (1, 257, 4, 1, 128, 3),          # documents of about three tokens
+    (2, 640, 3, 3, 256, 100),
+]
+
+
+def run_bwd_packed_tc(inp, grads, Q, seq):
+    d = to_dev(inp)
+    b, L, H, P = d["x"].shape
+    G, N = d["B"].shape[2], d["B"].shape[3]
+    ws = ssd.alloc_workspace(ssd.bwd_workspace_size(b, L, H, P, N, G, Q, d["x"].dtype), "cuda")
+    g = ssd.chunk_scan_bwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"], grads["dy"].cuda(),
+                           dfinal_state=grads["dfinal"].cuda(), init_state=d["init_state"], chunk_size=Q,
+                           workspace=ws, seq_idx=torch.from_numpy(seq).cuda(), path="tensor")
+    assert ssd.read_device_status(ws) == 0
+    torch.cuda.synchronize()
+    return {k: v.cpu().double().numpy() for k, v in g.items()}
+
+
+@pytest.mark.parametrize("case", TC_PACKED_CASES, ids=lambda c: "b%d_L%d_H%d_G%d_Q%d_doc%d" % c)
+def test_backward_tensor_path_packed_rows(case):
+    """Packed rows on the tensor path against the oracle's reverse mode with
+    the same document ids, at the tensor path's bar."""
+    b, L, H, G, Q, mean_len = case
+    cfg, inp, grads = _tc_case(b, L, H, G, Q, True, seed=L + Q + mean_len)
+    seq = _packed_ids(b, L, Q, np.random.default_rng(L + 3 * Q), mean_len)
+    got = run_bwd_packed_tc(inp, grads, Q, seq)
+    ref = oracle.scan_bwd(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"],
+                          grads["dy"], dfinal=grads["dfinal"], init_state=inp["init_state"], seq_idx=seq)
+    check_tc(got, ref, "tensor packed %s" % (case,))
+
+
+def test_backward_tensor_path_constant_ids_is_unpacked():
+    """One document per row: the packed tensor path equals the unpacked one
+    bit for bit (every mask passes)."""
+    cfg, inp, grads = _tc_case(2, 300, 4, 2, 256, True, seed=915)
+    a = run_bwd_packed_tc(inp, grads, 256, np.full((2, 300), 3, np.int32))
+    plain = run_bwd_tc(inp, grads, 256)
+    for k in KEYS:
+        assert np.array_equal(a[k], plain[k]), "d%s differs from the unpacked tensor path" % k
