@@ -116,3 +116,14 @@ def test_combined_rejects_what_it_does_not_take():
         ssd.conv_scan_fwd(xbc.cuda(), w[:, :3].contiguous().cuda(), bias.cuda(), *args)   # width 3
     with pytest.raises(ssd.SSDError, match="SSD_ERR_UNSUPPORTED"):
         ssd.conv_scan_fwd(xbc.cuda(), w.cuda(), bias.cuda(), *args, chunk_size=100)       # SIMT-only chunk
+
+
+def test_combined_long_context_layer_full_size():
+    """The long-context layer (b 1, L 65536, H 80, G 8: 11 units of 47 blocks,
+    so unit_state convolves too and every unit's first block reads its 3
+    earlier rows from the unit before), bit for bit against the split
+    arrangement."""
+    inp, xbc, w, bias = _layer(1, 65536, 80, 8, seed=65)
+    ys, fs, yc, fc = _both(inp, xbc, w, bias, 80, 8, 256)
+    assert np.array_equal(yc, ys), "combined y differs from split: max %.3e" % float(np.max(np.abs(yc - ys)))
+    assert np.array_equal(fc, fs)
