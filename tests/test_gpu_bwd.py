@@ -227,6 +227,8 @@ TOL_TC_L2 = 2e-3
 TC_CASES = [
     # b, L, H, G, Q, init, dfinal
     (2, 300, 4, 2, 256, True, True),
+    (1, 1, 2, 1, 128, True, True),          # one token
+    (2, 2, 2, 2, 256, False, True),         # two tokens
     (1, 128, 2, 1, 128, False, True),
     (1, 129, 2, 2, 128, True, False),
     (2, 640, 3, 3, 256, True, True),

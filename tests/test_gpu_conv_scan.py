@@ -60,6 +60,8 @@ def _both(inp, xbc, w, bias, H, G, Q):
 # 3 earlier rows from the unit before)
 CASES = [
     (2, 300, 4, 2, 256),
+    (1, 1, 2, 1, 128),
+    (2, 2, 2, 2, 64),
     (1, 128, 2, 1, 128),
     (1, 129, 2, 2, 64),
     (2, 77, 3, 3, 256),

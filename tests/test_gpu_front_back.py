@@ -90,7 +90,8 @@ def test_conv1d_silu_over_its_range(dtype):
 # a tile and a partial last tile (Cd = 152); token tiles of 64 with a ragged
 # tail; enough (batch, token tile) rows that each CTA walks its ring of
 # stages several times over
-TILE_CASES = [(3, 200, 3, 24, 1, 40), (2, 130, 2, 8, 3, 8), (4, 71040, 1, 64, 1, 32)]
+TILE_CASES = [(3, 200, 3, 24, 1, 40), (2, 130, 2, 8, 3, 8), (4, 71040, 1, 64, 1, 32),
+              (2, 1, 2, 8, 1, 8), (1, 2, 2, 8, 1, 8)]      # one and two tokens: all of the window is halo
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
