@@ -467,31 +467,29 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
 // is in the last unit), so every block here is a full 128 tokens.
 constexpr int kUsCompute = 256;
 constexpr int kUsThreads = kUsCompute + 32;
-constexpr int kUsStages = 2;                                   // TMA ring depth (2 CTAs per SM at 2)
 // stage: B (2 tiles), X (1 tile; kXRaw rows in the combined arrangement), dt, cum
 template <bool kConv> struct UsLayout {
     static constexpr uint32_t kXBytes = kConv ? kXRawBytes : kTileBytes;
     static constexpr uint32_t kTx = 2 * kTileBytes + kXBytes + 2 * kBlk * 4;    // bytes a stage receives
     static constexpr uint32_t kStage = (kTx + 1023) & ~1023u;                  // 1024-aligned stages
-    static constexpr uint32_t kOffW = kUsStages * kStage;                      // w [stages][128]
-    static constexpr uint32_t kOffCw = kOffW + kUsStages * kBlk * 4;           // conv weights [80] float4
-    static constexpr uint32_t kOffBar = kOffCw + (kConv ? 80 * 16 : 0);        // tma, mma, converted [stages]
-    static constexpr size_t kSmem = 1024 + kOffBar + 3 * kUsStages * 8 + 16;
+    static constexpr uint32_t kOffW = 2 * kStage;                              // w [2][128]
+    static constexpr uint32_t kOffCw = kOffW + 2 * kBlk * 4;                   // conv weights [80] float4
+    static constexpr uint32_t kOffBar = kOffCw + (kConv ? 80 * 16 : 0);        // tma[2], mma[2], converted[2]
+    static constexpr size_t kSmem = 1024 + kOffBar + 6 * 8 + 16;
 };
 
 template <bool kConv>
-__global__ void __launch_bounds__(kUsThreads, kUsStages == 2 ? 2 : 1)
+__global__ void __launch_bounds__(kUsThreads, 2)
 unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, int nblk, int U, int bpu,
                   int packed, const float *__restrict__ cw, const float *__restrict__ cb) {
     using Lay = UsLayout<kConv>;
     constexpr uint32_t kUsStage = Lay::kStage, kUsOffW = Lay::kOffW, kUsOffBar = Lay::kOffBar;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    // per stage s: bar[s] TMA landed, bar[S + s] MMAs done, bar[2S + s] X converted.  One
-    // barrier of each kind per stage keeps every waiter within one phase of its signaller.
-    constexpr int S = kUsStages;
+    // per stage: [0,1] TMA landed, [2,3] MMAs done, [4,5] X converted.  One barrier of
+    // each kind per stage keeps every waiter within one phase of its signaller.
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kUsOffBar);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 3 * S);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 6);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tslot + 1);
 
     const int h = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
@@ -509,7 +507,7 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 3 * S; ++i) mbar_init(bar + i, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(bar + i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -535,11 +533,10 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
             };
             const uint32_t idesc = idesc_f16(128, 64, 1, 1);
             bool ok = true;
-            for (int i = 0; i < S && i < nk; ++i) load(i, kb0 + i);
+            for (int i = 0; i < 2 && i < nk; ++i) load(i, kb0 + i);
             for (int i = 0; i < nk && ok; ++i) {
-                const int s = i % S;
-                const uint32_t par = (uint32_t)(i / S) & 1u;
-                ok = mbar_wait_abortable(bar + 2 * S + s, par, kWaitBudget, abort_flag);
+                const int s = i & 1;
+                ok = mbar_wait_abortable(bar + 4 + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t b_base = smem_u32(stage(s)), x_base = smem_u32(stage(s) + 2 * kTileBytes);
@@ -547,10 +544,10 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
                 for (int q = 0; q < 8; ++q)
                     mma_f16(tmem, sdesc_sw128(b_base + q * 2048, kTileBytes, 1024),
                             sdesc_sw128(x_base + q * 2048, kTileBytes, 1024), idesc, (i > 0 || q > 0) ? 1u : 0u);
-                mma_commit(bar + S + s);
-                if (i + S < nk) {       // refill stage s once these MMAs have read it
-                    ok = mbar_wait_abortable(bar + S + s, par, kWaitBudget, abort_flag);
-                    if (ok) load(s, kb0 + i + S);
+                mma_commit(bar + 2 + s);
+                if (i + 2 < nk) {       // refill stage s once these MMAs have read it
+                    ok = mbar_wait_abortable(bar + 2 + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
+                    if (ok) load(s, kb0 + i + 2);
                 }
             }
         }
@@ -577,12 +574,12 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
             ws.ell[bh * U + u] = starts ? -INFINITY : suffix + cumg[(size_t)kb0 * kBlk + kBlk - 1];
         }
         for (int i = 0; i < nk; ++i) {
-            const int s = i % S;
+            const int s = i & 1;
             uint8_t *st = stage(s);
             const float *dt = reinterpret_cast<const float *>(st + 2 * kTileBytes + Lay::kXBytes);
             const float *cum = dt + kBlk;
             float *w = reinterpret_cast<float *>(sm + kUsOffW) + s * kBlk;
-            ok = ok && mbar_wait_abortable(bar + s, (uint32_t)(i / S) & 1u, kWaitBudget, abort_flag);
+            ok = ok && mbar_wait_abortable(bar + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
             if (ok && tid < kBlk) {
                 // packed rows: only the unit's last document writes into its state
                 const bool cut = packed && (later > 0 || tid < rsb[(size_t)(kb0 + i) * kBlk + kBlk - 1]);
@@ -612,11 +609,11 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
             }
             fence_proxy_async_smem();
             named_bar_sync(kUsCompute);
-            if (tid == 0) mbar_arrive(bar + 2 * S + s);
+            if (tid == 0) mbar_arrive(bar + 4 + s);
         }
         // the accumulated state: wait for the last block's MMAs
-        const int sl = (nk - 1) % S;
-        ok = __all_sync(0xffffffffu, ok && mbar_wait_abortable(bar + S + sl, (uint32_t)((nk - 1) / S) & 1u,
+        const int sl = (nk - 1) & 1;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_abortable(bar + 2 + sl, ((uint32_t)(nk - 1) >> 1) & 1u,
                                                                    kWaitBudget, abort_flag));
         tc_fence_after();
         if (ok) {
