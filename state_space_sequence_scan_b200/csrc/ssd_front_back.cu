@@ -35,8 +35,9 @@ constexpr int kCvTT = kCvWarps * kCvTokPerWarp;  // tokens per tile
 constexpr int kCvHalo = kConvMaxK - 1;        // rows before the tile's first token
 constexpr int kCvRows = kCvHalo + kCvTT;      // rows per tile in shared memory
 constexpr long long kCvWaitBudget = 1ll << 32;  // clock cycles before a wait gives up (~2 s)
-// tiles in flight per CTA: 3 x 33.5 KB (bf16: two 16-warp CTAs per SM, the
-// most that 56 registers a thread allow), 3 x 67 KB (fp32: one CTA per SM)
+// tiles in flight per CTA: 3 x 33.5 KB (bf16: two 16-warp CTAs per SM, as
+// the register file allows at 64 registers a thread), 3 x 67 KB (fp32: one
+// CTA per SM by shared memory)
 template <typename T> struct CvStages { static constexpr int value = 3; };
 template <typename T> constexpr size_t cv_smem_bytes() {
     return (size_t)CvStages<T>::value * kCvRows * kCvTC * sizeof(T) + 8 * CvStages<T>::value;
@@ -45,7 +46,6 @@ template <typename T> constexpr size_t cv_smem_bytes() {
 // Status word of the workspace-free kernels (conv1d): kStatusTimeout when a
 // bounded wait gave up.  Read and cleared by ssd_read_device_status(NULL, ...).
 __device__ unsigned g_front_status = 0;
-
 
 // 4 consecutive z values -> floats
 __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&v)[4]) {
