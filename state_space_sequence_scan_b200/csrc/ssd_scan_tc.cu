@@ -461,11 +461,13 @@ prep_kernel(const float *__restrict__ dt_raw, const float *__restrict__ dt_bias,
 
 // ---------------------------------------------------------------------------
 // unit_state: grid (H, U-1, b), 8 compute warps + 1 control warp, 2 CTAs per
-// SM, two TMA stages of (B fp16, X bf16, dt, cum).  The control warp's lane 0
+// SM, two TMA stages of (B fp16, X bf16, dt, cum), and x of the two blocks
+// after them requested into L2.  The control warp's lane 0
 // issues the TMA copies and the MMAs; the compute warps only widen X (scaled
 // by w) and signal.  Units 0..U-2 never hold the sequence's ragged tail (it
 // is in the last unit), so every block here is a full 128 tokens.
 constexpr int kUsCompute = 256;
+constexpr int kUsPrefetch = 2;   // blocks of x requested into L2 ahead of the two stages
 constexpr int kUsThreads = kUsCompute + 32;
 // stage: B (2 tiles), X (1 tile; kXRaw rows in the combined arrangement), dt, cum
 template <bool kConv> struct UsLayout {
@@ -531,9 +533,16 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
                 bulk_load(st + 2 * kTileBytes + Lay::kXBytes, dtg + (size_t)t0, kBlk * 4, bar + s);
                 bulk_load(st + 2 * kTileBytes + Lay::kXBytes + kBlk * 4, cumg + (size_t)t0, kBlk * 4, bar + s);
             };
+            // x of block k into L2 (x is the kernel's DRAM stream; B comes from L2, where
+            // the group's heads share it): two blocks beyond the two stages, so more of
+            // the row's reads are in flight than the stages hold
+            auto prefetch_x = [&](int k) {
+                if (k < kb1) tma_prefetch_4d(&maps.x, 0, h, kConv ? k * kBlk - (kConvK - 1) : k * kBlk, b);
+            };
             const uint32_t idesc = idesc_f16(128, 64, 1, 1);
             bool ok = true;
             for (int i = 0; i < 2 && i < nk; ++i) load(i, kb0 + i);
+            for (int i = 2; i < 2 + kUsPrefetch; ++i) prefetch_x(kb0 + i);
             for (int i = 0; i < nk && ok; ++i) {
                 const int s = i & 1;
                 ok = mbar_wait_abortable(bar + 4 + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
@@ -547,7 +556,10 @@ unit_state_kernel(const __grid_constant__ TcMaps maps, TcWs ws, int H, int G, in
                 mma_commit(bar + 2 + s);
                 if (i + 2 < nk) {       // refill stage s once these MMAs have read it
                     ok = mbar_wait_abortable(bar + 2 + s, ((uint32_t)i >> 1) & 1u, kWaitBudget, abort_flag);
-                    if (ok) load(s, kb0 + i + 2);
+                    if (ok) {
+                        load(s, kb0 + i + 2);
+                        prefetch_x(kb0 + i + 2 + kUsPrefetch);
+                    }
                 }
             }
         }
