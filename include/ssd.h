@@ -241,6 +241,7 @@ SSD_API ssd_status ssd_conv1d_silu_split(const void *xbc, const float *weight, c
  *   xbc      [batch, seqlen, Cd] bf16, Cd = nheads*head_dim + 2*ngroups*state_dim
  *            (channels x | B | C), 16-byte aligned
  *   conv_w   [Cd, 4] float32, conv_b [Cd] float32, both 16-byte aligned
+ *            (SSD_ERR_ALIGNMENT) and neither NULL (SSD_ERR_INVALID_ARG)
  *   kernel_width  4 (else SSD_ERR_UNSUPPORTED)
  *   the rest as for ssd_chunk_scan_fwd on the tensor-core path: in_dtype
  *   SSD_BF16, head_dim 64, state_dim 128, chunk_size 64, 128 or 256 (else

@@ -252,11 +252,12 @@ ssd_status ssd_chunk_scan_bwd_workspace_size(int64_t batch, int64_t seqlen, int6
 
 ssd_status ssd_chunk_scan_bwd_varlen(const void *x, const float *dt_raw, const float *dt_bias, const float *A,
                                      const void *B, const void *C, const float *D, const float *init_state,
-                                     const int32_t *seq_idx, const float *dy, const float *dfinal_state, float *dx, float *ddt_raw,
-                              float *ddt_bias, float *dA, float *dB, float *dC, float *dD, float *dinit_state,
-                              int64_t batch, int64_t seqlen, int64_t nheads, int64_t head_dim, int64_t state_dim,
-                              int64_t ngroups, int64_t chunk_size, float dt_lo, float dt_hi, int in_dtype,
-                              int path, void *workspace, size_t workspace_bytes, void *stream) {
+                                     const int32_t *seq_idx, const float *dy, const float *dfinal_state,
+                                     float *dx, float *ddt_raw, float *ddt_bias, float *dA, float *dB, float *dC,
+                                     float *dD, float *dinit_state, int64_t batch, int64_t seqlen, int64_t nheads,
+                                     int64_t head_dim, int64_t state_dim, int64_t ngroups, int64_t chunk_size,
+                                     float dt_lo, float dt_hi, int in_dtype, int path, void *workspace,
+                                     size_t workspace_bytes, void *stream) {
     ssd_status st = check_scan_dims(batch, seqlen, nheads, head_dim, state_dim, ngroups, chunk_size, in_dtype,
                                     path);
     if (st != SSD_OK) return st;
