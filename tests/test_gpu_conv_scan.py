@@ -79,6 +79,18 @@ def test_combined_equals_split_bit_for_bit(case):
     assert np.array_equal(fc, fs), "combined final_state differs from split"
 
 
+@pytest.mark.parametrize("case", [CASES[0], CASES[6]], ids=lambda c: "b%d_L%d_H%d_G%d_Q%d" % c)
+def test_combined_equals_split_without_an_initial_state(case):
+    """No initial state (the 130m and 2.7B layers' case): both arrangements
+    start every chain from zeros, bit for bit alike."""
+    b, L, H, G, Q = case
+    inp, xbc, w, bias = _layer(b, L, H, G, seed=L + 5 * H + G, init="zero")
+    assert inp["init_state"] is None
+    ys, fs, yc, fc = _both(inp, xbc, w, bias, H, G, Q)
+    assert np.array_equal(yc, ys), "combined y differs from split: max %.3e" % float(np.max(np.abs(yc - ys)))
+    assert np.array_equal(fc, fs), "combined final_state differs from split"
+
+
 @pytest.mark.parametrize("case", CASES[:4], ids=lambda c: "b%d_L%d_H%d_G%d_Q%d" % c)
 def test_combined_against_the_oracle_chain(case):
     """The oracle's conv (fp64, rounded to bf16 as both arrangements store
